@@ -1,0 +1,385 @@
+#!/usr/bin/env python
+"""Benchmark of the tensor-parallel two-projection MLP on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--config decode_bs1|decode_bs32|prefill|sweep|tiny] [--tokens T] [--tp P]
+                    [--plan auto|gemv|simt|tc]
+
+One step = one forward of the whole hot path (first projection + activation,
+second projection with the ranks' partial sums reduced on the device) over one
+batch of seeded synthetic input, on weights packed once before timing.  The
+default workload is decode at batch 1 (bf16 SwiGLU, d_model 8192, d_ff 28672,
+8 ranks' shards on one GPU).  The weights (1.41 GB) are far larger than L2, so
+every step re-reads them from HBM; no L2 flush is needed.
+
+Rank 0 prints one JSON line.  With N > 1 (torchrun) each GPU runs an
+independent replica on its own batch (data-parallel replicas: no collective on
+the data path); the reported time is the max over ranks.
+
+--impl reference times the oracle (plain fp64 C loops on the host cores) on a
+bounded sample of the same workload; under torchrun only rank 0 runs it.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "sharded-MLP tokens/s; decode HBM GB/s & prefill TFLOP/s vs B200 peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default="decode_bs1")
+    ap.add_argument("--tokens", type=int, default=None)
+    ap.add_argument("--tp", type=int, default=None)
+    ap.add_argument("--plan", default="auto")
+    ap.add_argument("--d-model", type=int, default=None, help="override (small cases for profiling)")
+    ap.add_argument("--d-ff", type=int, default=None, help="override (small cases for profiling)")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def resolve(args):
+    from tensor_sharded_mlp_b200 import inputs
+    c = dict(inputs.CONFIGS[args.config])
+    T = c["tokens"]
+    if isinstance(T, tuple):
+        T = args.tokens if args.tokens is not None else T[-1]
+    elif args.tokens is not None:
+        T = args.tokens
+    tp = c["tp"]
+    if isinstance(tp, tuple):
+        tp = args.tp if args.tp is not None else tp[-1]
+    elif args.tp is not None:
+        tp = args.tp
+    c.update(tokens=T, tp=tp)
+    small = ""
+    if args.d_model is not None or args.d_ff is not None:
+        c["d_model"] = args.d_model or c["d_model"]
+        c["d_ff"] = args.d_ff or c["d_ff"]
+        small = " [reduced size for profiling]"
+    c["workload"] = (f"{args.config}{small}: {c['dtype']} {c['act']} MLP, tokens={T}, d_model={c['d_model']}, "
+                     f"d_ff={c['d_ff']}, tp={tp} shards on one GPU, X~N(0,1), "
+                     f"weights~N(0,{'1/fan_in' if c['init'] == 'fan_in' else str(c['init']) + '^2'}), "
+                     f"seed {c['seed']}")
+    return c
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def csrc_hash() -> str:
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "tensor_sharded_mlp_b200", "csrc")
+    for n in sorted(os.listdir(d)):
+        with open(os.path.join(d, n), "rb") as f:
+            h.update(n.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if taken on this exact source."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    e = rec.get(f"{kernel}|{workload}")
+    if not e or e.get("csrc_hash") != csrc_hash():
+        return None
+    return e.get("bytes_per_launch")
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML in a thread."""
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int, period_s: float = 0.02):
+        self.samples = []
+        self.period = period_s
+        self.ok = False
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # NVML missing: report no clocks rather than invent them
+            self.err = str(e)
+        self.window = None
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((time.perf_counter(), sm, rs))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+
+    def mark(self, t0, t1):
+        self.window = (t0, t1)
+
+    def stop(self):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "note": getattr(self, "err", "no samples")}
+        sel = self.samples
+        if self.window:
+            w = [s for s in self.samples if self.window[0] <= s[0] <= self.window[1]]
+            if len(w) >= 3:
+                sel = w
+        mask = 0
+        for s in sel:
+            mask |= s[2]
+        reasons = [n for b, n in self.REASONS.items() if mask & b and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(s[1] for s in sel), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(sel),
+                "window": "timed region" if sel is not self.samples else "warm-up + timed region"}
+
+
+def oracle_baseline(p, A, Bs, act, budget_s=12.0, max_calls=50):
+    """Time the oracle as it stands on a bounded sample: whole calls until the budget is spent."""
+    import oracle
+    T = p.tokens
+    calls, t_total = 0, 0.0
+    while calls < max_calls and t_total < budget_s:
+        t0 = time.perf_counter()
+        oracle.tp_mlp_sharded(p.x, A, Bs, act)
+        t_total += time.perf_counter() - t0
+        calls += 1
+    threads = min(oracle.max_threads(), T)
+    return {"value": T * calls / t_total, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{calls} full forward(s) of this workload ({T} token(s) each) on the host, "
+                      f"{t_total:.1f} s; the oracle runs OpenMP over tokens"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", 0))
+    if rank != 0:
+        return 0
+    import oracle
+    from tensor_sharded_mlp_b200 import inputs
+    c = resolve(args)
+    p = inputs.generate(c["tokens"], c["d_model"], c["d_ff"], c["act"], c["dtype"], c["seed"], c["init"])
+    A, Bs = p.shards(c["tp"])
+    T, P = c["tokens"], c["tp"]
+    # sample: the first t_s tokens and the first r_s of the P ranks (work is linear in both)
+    t_s = min(T, 64)
+    oracle.tp_mlp_sharded(p.x[:t_s], A[:1], Bs[:1], c["act"])          # warm the code path
+    t0 = time.perf_counter()
+    oracle.tp_mlp_sharded(p.x[:t_s], A[:1], Bs[:1], c["act"])
+    per_rank = time.perf_counter() - t0
+    budget = 150.0 / max(1, args.steps + args.warmup)
+    r_s = max(1, min(P, int(budget / max(per_rank, 1e-6))))
+    for _ in range(args.warmup):
+        oracle.tp_mlp_sharded(p.x[:t_s], A[:r_s], Bs[:r_s], c["act"])
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.tp_mlp_sharded(p.x[:t_s], A[:r_s], Bs[:r_s], c["act"])
+    dt = time.perf_counter() - t0
+    work_tokens = t_s * r_s / P * args.steps
+    value = work_tokens / dt
+    cores = min(oracle.max_threads(), t_s)
+    sample = (f"each step: the oracle on the first {t_s} of {T} token(s) and {r_s} of {P} ranks' shards "
+              f"({r_s}/{P} of the weights); tokens/s counts {t_s}*{r_s}/{P} tokens per step")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": c["workload"], "tokens": T, "d_model": c["d_model"],
+                                             "d_ff": c["d_ff"], "tp": P, "act": c["act"],
+                                             "parallelism": "host oracle"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from tensor_sharded_mlp_b200 import binding, counts, inputs
+
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local = int(os.environ.get("LOCAL_RANK", 0))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    c = resolve(args)
+    T, d, f, tp, act, dt = c["tokens"], c["d_model"], c["d_ff"], c["tp"], c["act"], c["dtype"]
+    p = inputs.generate(T, d, f, act, dt, c["seed"], c["init"])
+    A, Bs = p.shards(tp)
+    tdt = torch.bfloat16 if dt == "bf16" else torch.float32
+
+    def up(a):
+        return torch.from_numpy(a).cuda().to(tdt).contiguous()
+
+    m = binding.TpMlp(d, f, tp, act, dt, max_tokens=T)
+    m.set_plan(args.plan)
+    Ad, Bd = [up(a) for a in A], [up(b) for b in Bs]
+    packed = m.pack(Ad, Bd)
+    del Ad, Bd
+    x = up(p.x)
+    out = torch.empty(T, d, dtype=tdt, device="cuda")
+    torch.cuda.synchronize()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    K, W = args.steps, max(3, args.warmup)
+    for _ in range(W):
+        m.forward_packed(x, packed, out=out)
+    nk = m.last_launches
+    plan = m.last_plan
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)] for _ in range(K)]
+    stream = torch.cuda.current_stream()
+    for row in ev:
+        for e in row:
+            e.record(stream)
+    sampler = ClockSampler(torch.cuda.current_device())
+    sampler.start()
+    time.sleep(0.1)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    t0 = time.perf_counter()
+    start.record(stream)
+    for i in range(K):
+        binding.tp_mlp_set_profile_events(m.h, ev[i])
+        m.forward_packed(x, packed, out=out)
+    end.record(stream)
+    barrier()
+    t1 = time.perf_counter()
+    sampler.mark(t0, t1)
+    binding.tp_mlp_set_profile_events(m.h, None)
+    elapsed_ms = start.elapsed_time(end)
+    kern_ms = [statistics.fmean(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(K)) for j in range(nk)]
+    if world > 1:
+        t = torch.tensor([elapsed_ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+
+    # end to end through the public API with host buffers (pinned), copies inside the region
+    e2e = None
+    if not args.no_e2e:
+        x_host = x.cpu().pin_memory()
+        out_host = torch.empty(out.shape, dtype=tdt).pin_memory()
+        x_dev = torch.empty_like(x)
+        for _ in range(W):
+            x_dev.copy_(x_host, non_blocking=True)
+            m.forward_packed(x_dev, packed, out=out)
+            out_host.copy_(out, non_blocking=True)
+            stream.synchronize()
+        barrier()
+        s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s2.record(stream)
+        for _ in range(K):
+            x_dev.copy_(x_host, non_blocking=True)
+            m.forward_packed(x_dev, packed, out=out)
+            out_host.copy_(out, non_blocking=True)
+            stream.synchronize()      # the caller reads the result every step
+        e2.record(stream)
+        barrier()
+        e2e_ms = s2.elapsed_time(e2)
+        if world > 1:
+            t = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        e2e = {"value": world * T * K / (e2e_ms / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
+               "d2h_bytes_per_step": out_host.numel() * out_host.element_size()}
+    sampler.stop()
+
+    value = world * T * K / (elapsed_ms / 1e3)
+    peaks, src = load_peaks()
+    # roofline of the dominant kernel (largest share of the step)
+    j = int(np.argmax(kern_ms))
+    names = ["first projection + activation", "second projection + rank sum"]
+    if plan == "tc":
+        bound, unit = "tensor", "TFLOP/s"
+        work = counts.gemm1_flops(T, d, f, act) if j == 0 else counts.gemm2_flops(T, f, d)
+        achieved = work / (kern_ms[j] / 1e3) / 1e12
+        peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+        peak_note = f"bf16_tflops_sustained ({src})"
+    else:
+        bound, unit = "hbm", "GB/s"
+        work = counts.gemm1_bytes(T, d, f, act, dt) if j == 0 else counts.gemm2_bytes(T, f, d, dt)
+        achieved = work / (kern_ms[j] / 1e3) / 1e9
+        peak = peaks["hbm_gbs"]
+        peak_note = f"hbm_gbs ({src})"
+    kname = f"{plan}:{'first' if j == 0 else 'second'}"
+    roofline = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
+                "traffic": recorded_traffic(kname, args.config), "kernel": names[j] if j < 2 else str(j),
+                "kernel_ms": kern_ms[j], "algorithmic_per_launch": work, "peak_source": peak_note,
+                "kernel_ms_all": kern_ms}
+    step_bytes = counts.algorithmic_bytes(T, d, f, d, act, dt)
+    step_flops = counts.forward_flops(T, d, f, d, act)
+    ms = elapsed_ms / K
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W,
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": dt, "data": "synthetic",
+            "config": {"workload": c["workload"], "tokens": T, "d_model": d, "d_ff": f, "tp": tp, "act": act,
+                       "plan": plan, "parallelism": "replicas" if world > 1 else "single GPU",
+                       "l2": "inputs larger than L2: every step re-reads %.2f GB of weights" % (step_bytes / 1e9)},
+            "step_hbm_gbs": step_bytes / (ms / 1e3) / 1e9, "step_tflops": step_flops / (ms / 1e3) / 1e12,
+            "roofline": roofline, "gpu_launches": K * nk, "clocks": sampler.summary(), "e2e": e2e}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = oracle_baseline(p, A, Bs, act)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,202 @@
+/*
+ * tp_mlp.h -- C ABI of the tensor-parallel two-projection MLP on one B200.
+ *
+ * The operation (sources by page title and section):
+ *   "LLM 推理并行化：先找瓶颈，再决定怎么切", §三 2) 张量并行（TP）: the first
+ *   weight is split by columns and the second by rows; rank i computes
+ *   hidden_i = act(x @ A_i) and partial_i = hidden_i @ B_i, and the layer
+ *   output is the sum of the partials (an all-reduce across ranks).  The
+ *   default activation is tanh.
+ *   "大模型推理系统揭秘（07）：Multi-GPU：一张卡不够时如何扩展？", §1.2.2 (column-
+ *   and row-parallel linears), §1.2.3 (Z = [Y_0|..|Y_P-1][W_20;..] = sum_i
+ *   Y_i W_2i), §1.2.4 (gate/up column-parallel, activation local, down
+ *   row-parallel) and §1.4.3 (SwiGLU: W_2[SiLU(W_1 x) ⊙ (W_3 x)]).
+ *
+ * Here every rank's shards live in the memory of ONE GPU, so the all-reduce
+ * is a sum on the device, fused into the second projection's accumulation.
+ *
+ * Conventions for every entry point
+ *   - Matrices are row-major and densely packed (row stride = row length).
+ *   - "device pointer" = memory of the current CUDA device; "host" = CPU memory.
+ *   - Every pointer argument must be 16-byte aligned (TP_MLP_ERR_ALIGNMENT).
+ *   - All calls that take a stream are asynchronous on it; arguments are
+ *     checked on the host first and, on any error, nothing is launched and no
+ *     output is written.  Errors of earlier asynchronous work surface as
+ *     TP_MLP_ERR_CUDA on a later call or at the caller's synchronisation.
+ *   - The library never allocates device memory.  The caller owns x, the
+ *     shards, out, partials, the packed buffer and the workspace; the handle
+ *     owns host metadata only.
+ *   - A handle must not be used from two host threads or two streams at once:
+ *     its workspace is shared by the calls made on it.
+ *   - Accumulation is always fp32.  x, the weights and out share the handle's
+ *     dtype; partials are fp32.
+ */
+#ifndef TP_MLP_H
+#define TP_MLP_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Opaque handle (host memory, owned by the library). */
+typedef struct tp_mlp_s *tp_mlp_t;
+
+/* A CUDA stream; the same type as cudaStream_t.  NULL = the legacy default stream. */
+typedef struct CUstream_st *tp_mlp_stream_t;
+
+/* Activation applied to the first projection.
+ *   TANH:     H = tanh(X A)                 (the pages' default activation)
+ *   SWIGLU:   H = SiLU(X gate) * (X up), SiLU(g) = g / (1 + e^{-g})
+ *   IDENTITY: H = X A                       (no activation; exact-integer tests) */
+typedef enum { TP_MLP_ACT_TANH = 0, TP_MLP_ACT_SWIGLU = 1, TP_MLP_ACT_IDENTITY = 2 } tp_mlp_act;
+
+/* Element type of x, the weights and out. */
+typedef enum { TP_MLP_F32 = 0, TP_MLP_BF16 = 1 } tp_mlp_dtype;
+
+typedef enum {
+    TP_MLP_OK = 0,
+    TP_MLP_ERR_INVALID_ARG = 1,  /* NULL handle/pointer, unknown enum value            */
+    TP_MLP_ERR_SHAPE = 2,        /* sizes, shard count, d_ff % tp, tokens > max_tokens */
+    TP_MLP_ERR_ALIGNMENT = 3,    /* a pointer is not 16-byte aligned                   */
+    TP_MLP_ERR_UNSUPPORTED = 4,  /* valid request this build cannot serve              */
+    TP_MLP_ERR_CUDA = 5,         /* a CUDA runtime call failed (launch or earlier work) */
+    TP_MLP_ERR_TIMEOUT = 6,      /* reserved: a bounded device-side wait ran out       */
+    TP_MLP_ERR_WORKSPACE = 7     /* no workspace set, or smaller than required         */
+} tp_mlp_status;
+
+/* Kernel family used for a forward (for tests and measurements). */
+typedef enum {
+    TP_MLP_PLAN_AUTO = 0,   /* let the library choose (default)                      */
+    TP_MLP_PLAN_SIMT = 1,   /* tiled CUDA-core kernels, any shape and layout          */
+    TP_MLP_PLAN_GEMV = 2,   /* packed bf16, 1-4 tokens: streaming split-K GEMV        */
+    TP_MLP_PLAN_TC = 3      /* packed bf16: tcgen05 tensor-core GEMMs (TMA + TMEM)    */
+} tp_mlp_plan;
+
+/*
+ * Create a handle for one MLP shape.
+ *   d_model    input width (columns of x, rows of every A_i), >= 1
+ *   d_ff       intermediate width summed over ranks; d_ff % tp_degree == 0
+ *   d_out      output width (columns of every B_i); pass d_model for the usual
+ *              square layer (the §1.2.3 example maps 8 -> 8 -> 4)
+ *   tp_degree  number of ranks (shards), 1..8
+ *   act, dtype see the enums above
+ *   max_tokens largest token count a call will pass, >= 1
+ * Allocates host memory only.  Returns TP_MLP_OK and sets *handle, or an
+ * error and leaves *handle untouched.
+ */
+int tp_mlp_create(tp_mlp_t *handle, int d_model, int d_ff, int d_out, int tp_degree,
+                  int act, int dtype, int max_tokens);
+
+/* Free the handle (host memory).  NULL is accepted. */
+int tp_mlp_destroy(tp_mlp_t handle);
+
+/*
+ * Device workspace (bytes) the forward / partials / packed calls need for
+ * `tokens` tokens (0 <= tokens <= max_tokens).  It holds the intermediate
+ * activation H (tokens x d_ff, dtype) and split-K scratch.  Returns 0 for an
+ * invalid handle or token count.
+ */
+size_t tp_mlp_workspace_bytes(tp_mlp_t handle, int tokens);
+
+/*
+ * Give the handle a device workspace of `bytes` bytes (owned by the caller,
+ * kept until replaced or the handle is destroyed).  Zeroes the split-K
+ * counters inside it synchronously (cudaMemset).  bytes must be at least
+ * tp_mlp_workspace_bytes(handle, max_tokens) -- or pass the size for the
+ * largest token count you will use: each call checks its own need.
+ */
+int tp_mlp_set_workspace(tp_mlp_t handle, void *dev_ptr, size_t bytes);
+
+/*
+ * Forward pass on per-rank shards, the pages' interface
+ * tensor_parallel_output(x, a_shards, b_shards, activation):
+ *   out = sum_{i<tp} act(x @ A_i) @ B_i
+ *   x          device, tokens x d_model
+ *   A_shards   host array of tp_degree device pointers.
+ *              tanh / identity: A_i is d_model x f_s (columns i*f_s.. of A);
+ *              SwiGLU: A_i is d_model x 2*f_s laid out [gate_i | up_i]
+ *              (gate and up columns of the same intermediate features).
+ *   B_shards   host array of tp_degree device pointers; B_i is f_s x d_out
+ *              (rows i*f_s.. of B).           f_s = d_ff / tp_degree.
+ *   tp_degree  must equal the handle's (the shard arrays are paired strictly)
+ *   act        must equal the handle's
+ *   out        device, tokens x d_out
+ *   stream     CUDA stream
+ * tokens == 0 is a no-op.  Uses the workspace.
+ */
+int tp_mlp_forward(tp_mlp_t handle, const void *x, int tokens, const void *const *A_shards,
+                   const void *const *B_shards, int tp_degree, int act, void *out,
+                   tp_mlp_stream_t stream);
+
+/*
+ * Per-rank partials without the final sum: partials[i] = act(x @ A_i) @ B_i,
+ * fp32, laid out tp_degree x tokens x d_out (device).  Other arguments as
+ * tp_mlp_forward.  Summing them over i gives the forward's result (before
+ * rounding to the output dtype).
+ */
+int tp_mlp_partials(tp_mlp_t handle, const void *x, int tokens, const void *const *A_shards,
+                    const void *const *B_shards, int tp_degree, int act, float *partials,
+                    tp_mlp_stream_t stream);
+
+/*
+ * Size in bytes of the packed weight buffer (the shard-layout packer's output).
+ * Layout (element = the handle's dtype; each part starts 256-byte aligned):
+ *   part 1, first projection, K-major: one row of d_model elements per
+ *     intermediate feature (a column of A).  tanh / identity: row n holds
+ *     A[:, n] for n = 0..d_ff-1 in rank order (n = i*f_s + j).  SwiGLU: the
+ *     features go in blocks of 128 (the last block may be shorter, nb rows):
+ *     block b holds the nb gate rows of features 128b.. then their nb up rows.
+ *   part 2, second projection, K-major: row c (0..d_out-1) holds column c of
+ *     B, i.e. d_ff elements B[k][c] with k running over rank 0's rows, then
+ *     rank 1's, and so on -- so one K loop over a row sums the ranks.
+ */
+size_t tp_mlp_packed_bytes(tp_mlp_t handle);
+
+/* Pack the shards (same arrays as tp_mlp_forward) into `packed` (device,
+ * tp_mlp_packed_bytes bytes).  A bit-exact copy in a new order.  The handle's
+ * tp_degree fixes how many pointers each array holds. */
+int tp_mlp_pack(tp_mlp_t handle, const void *const *A_shards, const void *const *B_shards,
+                void *packed, tp_mlp_stream_t stream);
+
+/* Inverse of tp_mlp_pack: write the shards back from `packed` (bit-exact). */
+int tp_mlp_unpack(tp_mlp_t handle, const void *packed, void *const *A_shards,
+                  void *const *B_shards, tp_mlp_stream_t stream);
+
+/*
+ * Forward pass on packed weights (the fast path; weights are packed once).
+ *   x device tokens x d_model, out device tokens x d_out, packed from
+ *   tp_mlp_pack.  Same result as tp_mlp_forward up to fp32 summation order.
+ */
+int tp_mlp_forward_packed(tp_mlp_t handle, const void *x, int tokens, const void *packed,
+                          void *out, tp_mlp_stream_t stream);
+
+/* Force a kernel family (tp_mlp_plan) for later forwards; AUTO restores the
+ * library's choice.  A forced plan that cannot serve a call returns
+ * TP_MLP_ERR_UNSUPPORTED from that call. */
+int tp_mlp_set_plan(tp_mlp_t handle, int plan);
+
+/*
+ * Timing hook: with n > 0, later forward / forward_packed / partials calls
+ * record events[0] on their stream before their first kernel and events[j]
+ * after their j-th kernel (j = 1 .. n-1; kernels beyond that are not
+ * marked).  The events are caller-owned cudaEvent_t handles (created with
+ * timing enabled) and must stay valid while calls use them; n = 0 (or
+ * events = NULL) turns the hook off.  At most 8 events.
+ */
+int tp_mlp_set_profile_events(tp_mlp_t handle, void *const *events, int n);
+
+/* Plan (tp_mlp_plan) and number of kernel launches of the last successful
+ * forward / partials call on this handle; -1 before the first. */
+int tp_mlp_last_plan(tp_mlp_t handle);
+int tp_mlp_last_launches(tp_mlp_t handle);
+
+/* Human-readable name of a status code (static string). */
+const char *tp_mlp_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TP_MLP_H */

@@ -1,0 +1,276 @@
+"""Thin Python binding of ``libtp_mlp.so`` (argument marshalling only).
+
+The functions carry the C ABI's names (``include/tp_mlp.h``) and take torch
+tensors where the C call takes device pointers; every step of the MLP runs in
+the library's CUDA kernels.  Tensors supply device memory and
+``torch.cuda.current_stream()`` (or an explicit stream) supplies the stream.
+
+If the library is missing this module raises on import: there is no fallback.
+``TpMlp`` is a small convenience wrapper that owns the handle and a
+torch-allocated workspace.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libtp_mlp.so")
+if not os.path.exists(_LIB_PATH):
+    raise ImportError(f"CUDA library not built: {_LIB_PATH} is missing "
+                      "(run python -m tensor_sharded_mlp_b200.build)")
+_lib = ctypes.CDLL(_LIB_PATH)
+
+ACT = {"tanh": 0, "swiglu": 1, "identity": 2}
+DTYPE = {"f32": 0, "bf16": 1}
+TORCH_DTYPE = {"f32": torch.float32, "bf16": torch.bfloat16}
+PLAN = {"auto": 0, "simt": 1, "gemv": 2, "tc": 3}
+PLAN_NAME = {v: k for k, v in PLAN.items()}
+STATUS = {0: "OK", 1: "ERR_INVALID_ARG", 2: "ERR_SHAPE", 3: "ERR_ALIGNMENT", 4: "ERR_UNSUPPORTED",
+          5: "ERR_CUDA", 6: "ERR_TIMEOUT", 7: "ERR_WORKSPACE"}
+
+_vp = ctypes.c_void_p
+_i = ctypes.c_int
+_sz = ctypes.c_size_t
+_vpp = ctypes.POINTER(ctypes.c_void_p)
+
+_SIGS = {
+    "tp_mlp_create": (_i, [ctypes.POINTER(_vp), _i, _i, _i, _i, _i, _i, _i]),
+    "tp_mlp_destroy": (_i, [_vp]),
+    "tp_mlp_workspace_bytes": (_sz, [_vp, _i]),
+    "tp_mlp_set_workspace": (_i, [_vp, _vp, _sz]),
+    "tp_mlp_forward": (_i, [_vp, _vp, _i, _vpp, _vpp, _i, _i, _vp, _vp]),
+    "tp_mlp_partials": (_i, [_vp, _vp, _i, _vpp, _vpp, _i, _i, _vp, _vp]),
+    "tp_mlp_packed_bytes": (_sz, [_vp]),
+    "tp_mlp_pack": (_i, [_vp, _vpp, _vpp, _vp, _vp]),
+    "tp_mlp_unpack": (_i, [_vp, _vp, _vpp, _vpp, _vp]),
+    "tp_mlp_forward_packed": (_i, [_vp, _vp, _i, _vp, _vp, _vp]),
+    "tp_mlp_set_plan": (_i, [_vp, _i]),
+    "tp_mlp_set_profile_events": (_i, [_vp, _vpp, _i]),
+    "tp_mlp_last_plan": (_i, [_vp]),
+    "tp_mlp_last_launches": (_i, [_vp]),
+    "tp_mlp_status_string": (ctypes.c_char_p, [_i]),
+}
+for _name, (_res, _args) in _SIGS.items():
+    _f = getattr(_lib, _name)
+    _f.restype = _res
+    _f.argtypes = _args
+
+EXPORTED = tuple(_SIGS)
+
+
+class TpMlpError(RuntimeError):
+    def __init__(self, call: str, status: int):
+        self.status = status
+        self.name = STATUS.get(status, str(status))
+        super().__init__(f"{call} failed: {self.name} "
+                         f"({_lib.tp_mlp_status_string(status).decode()})")
+
+
+def _check(call: str, status: int) -> None:
+    if status != 0:
+        raise TpMlpError(call, status)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _ptr_array(ts: Sequence[torch.Tensor], n: int):
+    # the C call reads exactly n pointers from this array
+    if len(ts) != n:
+        raise ValueError(f"{len(ts)} shards given for tp_degree={n}")
+    for t in ts:
+        if not t.is_contiguous():
+            raise ValueError("shards must be contiguous")
+    arr = (ctypes.c_void_p * max(1, len(ts)))(*[t.data_ptr() for t in ts])
+    return ctypes.cast(arr, _vpp), arr
+
+
+# --- functions with the C ABI's names ------------------------------------------
+
+def tp_mlp_create(d_model: int, d_ff: int, d_out: int, tp_degree: int, act: str, dtype: str,
+                  max_tokens: int) -> ctypes.c_void_p:
+    h = ctypes.c_void_p()
+    _check("tp_mlp_create", _lib.tp_mlp_create(ctypes.byref(h), d_model, d_ff, d_out, tp_degree,
+                                               ACT[act], DTYPE[dtype], max_tokens))
+    return h
+
+
+def tp_mlp_destroy(h) -> None:
+    _check("tp_mlp_destroy", _lib.tp_mlp_destroy(h))
+
+
+def tp_mlp_workspace_bytes(h, tokens: int) -> int:
+    return int(_lib.tp_mlp_workspace_bytes(h, tokens))
+
+
+def tp_mlp_set_workspace(h, ws: Optional[torch.Tensor]) -> None:
+    nbytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check("tp_mlp_set_workspace", _lib.tp_mlp_set_workspace(h, _ptr(ws), nbytes))
+
+
+def tp_mlp_forward(h, x: torch.Tensor, A_shards, B_shards, tp_degree: int, act: str,
+                   out: torch.Tensor, stream=None) -> None:
+    a, _ka = _ptr_array(A_shards, tp_degree)
+    b, _kb = _ptr_array(B_shards, tp_degree)
+    _check("tp_mlp_forward", _lib.tp_mlp_forward(h, _ptr(x), x.shape[0], a, b, tp_degree, ACT[act],
+                                                 _ptr(out), _stream(stream)))
+
+
+def tp_mlp_partials(h, x: torch.Tensor, A_shards, B_shards, tp_degree: int, act: str,
+                    partials: torch.Tensor, stream=None) -> None:
+    a, _ka = _ptr_array(A_shards, tp_degree)
+    b, _kb = _ptr_array(B_shards, tp_degree)
+    _check("tp_mlp_partials", _lib.tp_mlp_partials(h, _ptr(x), x.shape[0], a, b, tp_degree,
+                                                   ACT[act], _ptr(partials), _stream(stream)))
+
+
+def tp_mlp_packed_bytes(h) -> int:
+    return int(_lib.tp_mlp_packed_bytes(h))
+
+
+def tp_mlp_pack(h, A_shards, B_shards, packed: torch.Tensor, tp_degree: int, stream=None) -> None:
+    a, _ka = _ptr_array(A_shards, tp_degree)
+    b, _kb = _ptr_array(B_shards, tp_degree)
+    _check("tp_mlp_pack", _lib.tp_mlp_pack(h, a, b, _ptr(packed), _stream(stream)))
+
+
+def tp_mlp_unpack(h, packed: torch.Tensor, A_shards, B_shards, tp_degree: int, stream=None) -> None:
+    a, _ka = _ptr_array(A_shards, tp_degree)
+    b, _kb = _ptr_array(B_shards, tp_degree)
+    _check("tp_mlp_unpack", _lib.tp_mlp_unpack(h, _ptr(packed), a, b, _stream(stream)))
+
+
+def tp_mlp_forward_packed(h, x: torch.Tensor, packed: torch.Tensor, out: torch.Tensor,
+                          stream=None) -> None:
+    _check("tp_mlp_forward_packed", _lib.tp_mlp_forward_packed(h, _ptr(x), x.shape[0], _ptr(packed),
+                                                               _ptr(out), _stream(stream)))
+
+
+def tp_mlp_set_plan(h, plan: str) -> None:
+    _check("tp_mlp_set_plan", _lib.tp_mlp_set_plan(h, PLAN[plan]))
+
+
+def tp_mlp_set_profile_events(h, events) -> None:
+    """events: torch.cuda.Event objects (timing enabled, already recorded once so
+    that they exist), or None to turn the hook off."""
+    if not events:
+        _check("tp_mlp_set_profile_events", _lib.tp_mlp_set_profile_events(h, None, 0))
+        return
+    arr = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
+    _check("tp_mlp_set_profile_events",
+           _lib.tp_mlp_set_profile_events(h, ctypes.cast(arr, _vpp), len(events)))
+
+
+def tp_mlp_last_plan(h) -> str:
+    return PLAN_NAME.get(_lib.tp_mlp_last_plan(h), "none")
+
+
+def tp_mlp_last_launches(h) -> int:
+    return int(_lib.tp_mlp_last_launches(h))
+
+
+def tp_mlp_status_string(status: int) -> str:
+    return _lib.tp_mlp_status_string(status).decode()
+
+
+# --- convenience wrapper -----------------------------------------------------------
+
+class TpMlp:
+    """One MLP shape: handle + workspace.  Tensors must live on the current CUDA device."""
+
+    def __init__(self, d_model: int, d_ff: int, tp: int, act: str = "tanh", dtype: str = "bf16",
+                 max_tokens: int = 32, d_out: Optional[int] = None, device=None):
+        self.d_model, self.d_ff, self.tp, self.act, self.dtype = d_model, d_ff, tp, act, dtype
+        self.d_out = d_model if d_out is None else d_out
+        self.max_tokens = max_tokens
+        self.device = torch.device("cuda" if device is None else device)
+        self.h = tp_mlp_create(d_model, d_ff, self.d_out, tp, act, dtype, max_tokens)
+        nbytes = tp_mlp_workspace_bytes(self.h, max_tokens)
+        self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
+        tp_mlp_set_workspace(self.h, self.workspace)
+
+    def __del__(self):
+        h = getattr(self, "h", None)
+        if h is not None:
+            _lib.tp_mlp_destroy(h)
+            self.h = None
+
+    @property
+    def torch_dtype(self):
+        return TORCH_DTYPE[self.dtype]
+
+    def _out(self, x, out):
+        if out is None:
+            out = torch.empty(x.shape[0], self.d_out, dtype=self.torch_dtype, device=x.device)
+        return out
+
+    def _check_x(self, x):
+        if x.dtype != self.torch_dtype or x.dim() != 2 or x.shape[1] != self.d_model or \
+                not x.is_contiguous() or not x.is_cuda:
+            raise ValueError(f"x must be a contiguous CUDA {self.torch_dtype} tensor (T, {self.d_model})")
+
+    def _check_shards(self, A_shards, B_shards):
+        if len(A_shards) != len(B_shards):
+            raise ValueError(f"{len(A_shards)} first-projection shards but {len(B_shards)} "
+                             "second-projection shards")
+        for t in list(A_shards) + list(B_shards):
+            if t.dtype != self.torch_dtype or not t.is_cuda:
+                raise ValueError(f"shards must be CUDA {self.torch_dtype} tensors")
+
+    def forward(self, x, A_shards, B_shards, out=None, stream=None):
+        self._check_x(x)
+        self._check_shards(A_shards, B_shards)
+        out = self._out(x, out)
+        tp_mlp_forward(self.h, x, A_shards, B_shards, len(A_shards), self.act, out, stream)
+        return out
+
+    def partials(self, x, A_shards, B_shards, out=None, stream=None):
+        if out is None:
+            out = torch.empty(self.tp, x.shape[0], self.d_out, dtype=torch.float32, device=x.device)
+        self._check_x(x)
+        self._check_shards(A_shards, B_shards)
+        tp_mlp_partials(self.h, x, A_shards, B_shards, len(A_shards), self.act, out, stream)
+        return out
+
+    def pack(self, A_shards, B_shards, stream=None):
+        self._check_shards(A_shards, B_shards)
+        packed = torch.empty(tp_mlp_packed_bytes(self.h), dtype=torch.uint8, device=self.device)
+        tp_mlp_pack(self.h, A_shards, B_shards, packed, self.tp, stream)
+        return packed
+
+    def unpack(self, packed, stream=None):
+        fs = self.d_ff // self.tp
+        wa = 2 * fs if self.act == "swiglu" else fs
+        A = [torch.empty(self.d_model, wa, dtype=self.torch_dtype, device=self.device)
+             for _ in range(self.tp)]
+        B = [torch.empty(fs, self.d_out, dtype=self.torch_dtype, device=self.device)
+             for _ in range(self.tp)]
+        tp_mlp_unpack(self.h, packed, A, B, self.tp, stream)
+        return A, B
+
+    def forward_packed(self, x, packed, out=None, stream=None):
+        self._check_x(x)
+        out = self._out(x, out)
+        tp_mlp_forward_packed(self.h, x, packed, out, stream)
+        return out
+
+    def set_plan(self, plan: str):
+        tp_mlp_set_plan(self.h, plan)
+
+    @property
+    def last_plan(self) -> str:
+        return tp_mlp_last_plan(self.h)
+
+    @property
+    def last_launches(self) -> int:
+        return tp_mlp_last_launches(self.h)

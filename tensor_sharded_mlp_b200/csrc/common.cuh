@@ -1,0 +1,83 @@
+// common.cuh -- small device/host helpers shared by the CUDA kernels of the
+// tensor-parallel MLP library.  No MLP arithmetic lives here.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/tp_mlp.h"
+
+namespace tpmlp {
+
+constexpr int kMaxTp = 8;
+constexpr int kSwigluBlock = 128;   // gate/up interleave granularity of the packed layout
+
+// Per-rank shard pointers, passed to kernels by value.
+struct ShardPtrs {
+    const void *p[kMaxTp];
+};
+
+// Problem description shared by every launcher.
+struct Problem {
+    int T;        // tokens
+    int d_in;     // d_model
+    int d_ff;     // sum of shard widths
+    int d_out;
+    int tp;
+    int fs;       // d_ff / tp
+    int act;      // tp_mlp_act
+    int dtype;    // tp_mlp_dtype
+};
+
+// --- element conversion ------------------------------------------------------
+__device__ __forceinline__ float to_f32(float v) { return v; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
+template <typename E> __device__ __forceinline__ E from_f32(float v);
+template <> __device__ __forceinline__ float from_f32<float>(float v) { return v; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float v) {
+    return __float2bfloat16_rn(v);
+}
+
+// Two bf16 packed in a 32-bit word -> two floats (exact: bf16 is the top half of fp32).
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// --- activations ---------------------------------------------------------------
+// SiLU(g) = g * sigma(g) = g / (1 + e^{-g}).  Large negative g: e^{-g} -> inf, result -> -0.
+__device__ __forceinline__ float silu_precise(float g) { return g / (1.0f + expf(-g)); }
+__device__ __forceinline__ float silu_fast(float g) { return g / (1.0f + __expf(-g)); }
+
+template <bool kFast>
+__device__ __forceinline__ float activate(int act, float u, float v) {
+    if (act == TP_MLP_ACT_TANH) return tanhf(u);
+    if (act == TP_MLP_ACT_SWIGLU) return (kFast ? silu_fast(u) : silu_precise(u)) * v;
+    return u;
+}
+
+// --- packed-layout index maps (shard-layout packer) ----------------------------
+// Row of the K-major first-projection part holding feature n (0 <= n < d_ff);
+// `up` selects the up row of a SwiGLU feature.
+__host__ __device__ __forceinline__ long w1p_row(int n, bool up, int d_ff, int act) {
+    if (act != TP_MLP_ACT_SWIGLU) return n;
+    const int b = n / kSwigluBlock;
+    const int r = n - b * kSwigluBlock;
+    const int nb = min(kSwigluBlock, d_ff - b * kSwigluBlock);
+    return 2L * kSwigluBlock * b + (up ? nb : 0) + r;
+}
+__host__ __device__ __forceinline__ long w1p_rows(int d_ff, int act) {
+    return act == TP_MLP_ACT_SWIGLU ? 2L * d_ff : (long)d_ff;
+}
+__host__ __device__ __forceinline__ size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+// --- cache-hinted loads ----------------------------------------------------------
+// 16-byte streaming load: read-only, not kept in L1 (weights are read once).
+__device__ __forceinline__ uint4 ld_stream_v4(const void *p) {
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+
+}  // namespace tpmlp

@@ -1,0 +1,42 @@
+// internal.h -- launchers shared between the library's translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+namespace tpmlp {
+
+struct Problem;
+struct ShardPtrs;
+
+// Caller-owned events recorded around the kernels of one call (timing hook).
+struct Marks {
+    cudaEvent_t ev[8];
+    int n;
+    void mark(int i, cudaStream_t s) const {
+        if (i < n && ev[i]) cudaEventRecord(ev[i], s);
+    }
+};
+
+// simt.cu: tiled CUDA-core path, any shape, both dtypes, shard or packed layout.
+// h: T x d_ff scratch (dtype).  partials != nullptr selects the per-rank output.
+cudaError_t launch_simt(const Problem &p, bool packed, const void *x, const ShardPtrs &w1,
+                        const ShardPtrs &w2, void *h, void *out, float *partials, cudaStream_t s,
+                        const Marks &marks);
+
+// pack.cu: shard-layout packer.
+size_t packed_part2_offset(const Problem &p);
+size_t packed_total_bytes(const Problem &p);
+cudaError_t launch_pack(const Problem &p, const ShardPtrs &a, const ShardPtrs &b, void *packed,
+                        bool unpack, cudaStream_t s);
+
+// gemv.cu: decode path, packed bf16, 1..kGemvMaxTokens tokens.
+constexpr int kGemvMaxTokens = 4;
+bool gemv_supported(const Problem &p);
+size_t gemv_workspace_bytes(const Problem &p, int num_sms);
+size_t gemv_counter_slots(const Problem &p);
+cudaError_t launch_gemv(const Problem &p, const void *x, const void *w1p, const void *w2p, void *h,
+                        void *out, float *part, unsigned *counters, int num_sms, cudaStream_t st,
+                        const Marks &marks, int *launches);
+
+}  // namespace tpmlp

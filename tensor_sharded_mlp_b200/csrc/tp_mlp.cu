@@ -1,0 +1,359 @@
+// tp_mlp.cu -- the C ABI: handle, argument checks, workspace layout, plan choice.
+//
+// Every call checks its arguments on the host before launching anything:
+// sizes and enums, 16-byte alignment, and that each device pointer lies inside
+// one device allocation large enough for what the kernels will touch (so a
+// wrong pointer is an error code, never an out-of-bounds access on the GPU).
+#include <cuda.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <new>
+
+#include "common.cuh"
+#include "internal.h"
+
+using namespace tpmlp;
+
+struct tp_mlp_s {
+    int d_model, d_ff, d_out, tp, act, dtype, max_tokens;
+    int num_sms;
+    void *ws;
+    size_t ws_bytes;
+    int plan;            // forced tp_mlp_plan
+    int last_plan, last_launches;
+    Marks marks;         // timing hook
+};
+
+namespace {
+
+typedef CUresult (*PFN_getAddressRange)(CUdeviceptr *, size_t *, CUdeviceptr);
+
+PFN_getAddressRange address_range_fn() {
+    static PFN_getAddressRange fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        tried = true;
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuMemGetAddressRange", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_getAddressRange>(p);
+    }
+    return fn;
+}
+
+size_t elem_bytes(int dtype) { return dtype == TP_MLP_F32 ? 4 : 2; }
+
+// A device pointer, 16-byte aligned, inside an allocation holding `bytes` from it.
+int check_dev(const void *p, size_t bytes) {
+    if (!p) return TP_MLP_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(p) & 15u) return TP_MLP_ERR_ALIGNMENT;
+    PFN_getAddressRange fn = address_range_fn();
+    if (!fn) return TP_MLP_ERR_CUDA;
+    CUdeviceptr base = 0;
+    size_t size = 0;
+    if (fn(&base, &size, reinterpret_cast<CUdeviceptr>(p)) != CUDA_SUCCESS)
+        return TP_MLP_ERR_INVALID_ARG;   // not memory of the current device's context
+    if (reinterpret_cast<uintptr_t>(p) + bytes > base + size) return TP_MLP_ERR_SHAPE;
+    return TP_MLP_OK;
+}
+
+Problem problem_of(const tp_mlp_s *h, int tokens) {
+    Problem p;
+    p.T = tokens;
+    p.d_in = h->d_model;
+    p.d_ff = h->d_ff;
+    p.d_out = h->d_out;
+    p.tp = h->tp;
+    p.fs = h->d_ff / h->tp;
+    p.act = h->act;
+    p.dtype = h->dtype;
+    return p;
+}
+
+// Workspace layout: [counters | H (tokens x d_ff) | split-K partial sums].
+size_t counters_bytes(const tp_mlp_s *h) {
+    Problem p = problem_of(h, 1);
+    return align256(gemv_counter_slots(p) * sizeof(unsigned));
+}
+size_t h_bytes(const tp_mlp_s *h, int tokens) {
+    return align256((size_t)tokens * h->d_ff * elem_bytes(h->dtype));
+}
+// Largest split-K scratch any call with <= tokens tokens needs, so that a
+// workspace sized for max_tokens serves every smaller call too.
+size_t part_bytes(const tp_mlp_s *h, int tokens) {
+    size_t m = 0;
+    for (int t = 1; t <= tokens && t <= kGemvMaxTokens; ++t) {
+        const size_t v = gemv_workspace_bytes(problem_of(h, t), h->num_sms);
+        m = v > m ? v : m;
+    }
+    return m;
+}
+size_t need_bytes(const tp_mlp_s *h, int tokens) {
+    return counters_bytes(h) + h_bytes(h, tokens) + part_bytes(h, tokens);
+}
+
+int from_cuda(cudaError_t e) { return e == cudaSuccess ? TP_MLP_OK : TP_MLP_ERR_CUDA; }
+
+// Checks shared by forward and partials (shard form).
+int check_common(tp_mlp_t h, const void *x, int tokens, int tp_degree, int act) {
+    if (!h) return TP_MLP_ERR_INVALID_ARG;
+    if (tokens < 0 || tokens > h->max_tokens) return TP_MLP_ERR_SHAPE;
+    if (tp_degree != h->tp) return TP_MLP_ERR_SHAPE;   // shards pair strictly, rank for rank
+    if (act != h->act) return TP_MLP_ERR_INVALID_ARG;
+    (void)x;
+    return TP_MLP_OK;
+}
+
+int check_shards(tp_mlp_t h, const void *const *A, const void *const *B) {
+    if (!A || !B) return TP_MLP_ERR_INVALID_ARG;
+    const size_t e = elem_bytes(h->dtype);
+    const size_t fs = (size_t)h->d_ff / h->tp;
+    const size_t lda = h->act == TP_MLP_ACT_SWIGLU ? 2 * fs : fs;
+    for (int i = 0; i < h->tp; ++i) {
+        if (!A[i] || !B[i]) return TP_MLP_ERR_INVALID_ARG;
+        if (((uintptr_t)A[i] | (uintptr_t)B[i]) & 15u) return TP_MLP_ERR_ALIGNMENT;
+    }
+    for (int i = 0; i < h->tp; ++i) {
+        int s = check_dev(A[i], (size_t)h->d_model * lda * e);
+        if (s) return s;
+        s = check_dev(B[i], fs * h->d_out * e);
+        if (s) return s;
+    }
+    return TP_MLP_OK;
+}
+
+int check_workspace(tp_mlp_t h, int tokens) {
+    if (!h->ws || h->ws_bytes < need_bytes(h, tokens)) return TP_MLP_ERR_WORKSPACE;
+    return TP_MLP_OK;
+}
+
+ShardPtrs to_ptrs(const void *const *arr, int n) {
+    ShardPtrs s;
+    memset(&s, 0, sizeof(s));
+    for (int i = 0; i < n; ++i) s.p[i] = arr[i];
+    return s;
+}
+
+}  // namespace
+
+extern "C" {
+
+int tp_mlp_create(tp_mlp_t *handle, int d_model, int d_ff, int d_out, int tp_degree, int act,
+                  int dtype, int max_tokens) {
+    if (!handle) return TP_MLP_ERR_INVALID_ARG;
+    if (act != TP_MLP_ACT_TANH && act != TP_MLP_ACT_SWIGLU && act != TP_MLP_ACT_IDENTITY)
+        return TP_MLP_ERR_INVALID_ARG;
+    if (dtype != TP_MLP_F32 && dtype != TP_MLP_BF16) return TP_MLP_ERR_INVALID_ARG;
+    if (d_model < 1 || d_ff < 1 || d_out < 1 || max_tokens < 1) return TP_MLP_ERR_SHAPE;
+    if (tp_degree < 1 || tp_degree > kMaxTp || d_ff % tp_degree != 0) return TP_MLP_ERR_SHAPE;
+    // keep every index inside 32-bit ints where the kernels use them
+    if ((long long)max_tokens * d_ff > (1LL << 31) || (long long)max_tokens * d_model > (1LL << 31) ||
+        (long long)max_tokens * d_out > (1LL << 31))
+        return TP_MLP_ERR_SHAPE;
+    tp_mlp_s *h = new (std::nothrow) tp_mlp_s;
+    if (!h) return TP_MLP_ERR_INVALID_ARG;
+    h->d_model = d_model;
+    h->d_ff = d_ff;
+    h->d_out = d_out;
+    h->tp = tp_degree;
+    h->act = act;
+    h->dtype = dtype;
+    h->max_tokens = max_tokens;
+    h->ws = nullptr;
+    h->ws_bytes = 0;
+    h->plan = TP_MLP_PLAN_AUTO;
+    h->last_plan = -1;
+    h->last_launches = -1;
+    memset(&h->marks, 0, sizeof(h->marks));
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess &&
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && sms > 0)
+        h->num_sms = sms;
+    else {
+        cudaGetLastError();
+        h->num_sms = 148;   // B200; only sizes split-K scratch
+    }
+    *handle = h;
+    return TP_MLP_OK;
+}
+
+int tp_mlp_destroy(tp_mlp_t h) {
+    delete h;
+    return TP_MLP_OK;
+}
+
+size_t tp_mlp_workspace_bytes(tp_mlp_t h, int tokens) {
+    if (!h || tokens < 0 || tokens > h->max_tokens) return 0;
+    return need_bytes(h, tokens);
+}
+
+int tp_mlp_set_workspace(tp_mlp_t h, void *dev_ptr, size_t bytes) {
+    if (!h) return TP_MLP_ERR_INVALID_ARG;
+    if (!dev_ptr) {
+        h->ws = nullptr;
+        h->ws_bytes = 0;
+        return TP_MLP_OK;
+    }
+    if (bytes < need_bytes(h, 0)) return TP_MLP_ERR_WORKSPACE;
+    int s = check_dev(dev_ptr, bytes);
+    if (s) return s;
+    if (cudaMemset(dev_ptr, 0, counters_bytes(h)) != cudaSuccess) return TP_MLP_ERR_CUDA;
+    h->ws = dev_ptr;
+    h->ws_bytes = bytes;
+    return TP_MLP_OK;
+}
+
+static int run_shard_form(tp_mlp_t h, const void *x, int tokens, const void *const *A,
+                          const void *const *B, int tp_degree, int act, void *out, float *partials,
+                          tp_mlp_stream_t stream) {
+    int s = check_common(h, x, tokens, tp_degree, act);
+    if (s) return s;
+    if (h->plan != TP_MLP_PLAN_AUTO && h->plan != TP_MLP_PLAN_SIMT) return TP_MLP_ERR_UNSUPPORTED;
+    if (tokens == 0) {
+        h->last_plan = TP_MLP_PLAN_SIMT;
+        h->last_launches = 0;
+        return TP_MLP_OK;
+    }
+    const size_t e = elem_bytes(h->dtype);
+    if ((s = check_dev(x, (size_t)tokens * h->d_model * e))) return s;
+    if (partials) {
+        if ((s = check_dev(partials, (size_t)h->tp * tokens * h->d_out * sizeof(float)))) return s;
+    } else if ((s = check_dev(out, (size_t)tokens * h->d_out * e))) {
+        return s;
+    }
+    if ((s = check_shards(h, A, B))) return s;
+    if ((s = check_workspace(h, tokens))) return s;
+    Problem p = problem_of(h, tokens);
+    void *hbuf = static_cast<char *>(h->ws) + counters_bytes(h);
+    cudaError_t ce = launch_simt(p, false, x, to_ptrs(A, h->tp), to_ptrs(B, h->tp), hbuf, out,
+                                 partials, reinterpret_cast<cudaStream_t>(stream), h->marks);
+    if (ce != cudaSuccess) return TP_MLP_ERR_CUDA;
+    h->last_plan = TP_MLP_PLAN_SIMT;
+    h->last_launches = 2;
+    return TP_MLP_OK;
+}
+
+int tp_mlp_forward(tp_mlp_t h, const void *x, int tokens, const void *const *A_shards,
+                   const void *const *B_shards, int tp_degree, int act, void *out,
+                   tp_mlp_stream_t stream) {
+    return run_shard_form(h, x, tokens, A_shards, B_shards, tp_degree, act, out, nullptr, stream);
+}
+
+int tp_mlp_partials(tp_mlp_t h, const void *x, int tokens, const void *const *A_shards,
+                    const void *const *B_shards, int tp_degree, int act, float *partials,
+                    tp_mlp_stream_t stream) {
+    if (!partials && h && tokens > 0) return TP_MLP_ERR_INVALID_ARG;
+    return run_shard_form(h, x, tokens, A_shards, B_shards, tp_degree, act, nullptr, partials, stream);
+}
+
+size_t tp_mlp_packed_bytes(tp_mlp_t h) {
+    if (!h) return 0;
+    return packed_total_bytes(problem_of(h, 0));
+}
+
+static int pack_common(tp_mlp_t h, const void *const *A, const void *const *B, const void *packed,
+                       bool unpack, tp_mlp_stream_t stream) {
+    if (!h) return TP_MLP_ERR_INVALID_ARG;
+    int s = check_shards(h, A, B);
+    if (s) return s;
+    if ((s = check_dev(packed, tp_mlp_packed_bytes(h)))) return s;
+    Problem p = problem_of(h, 0);
+    return from_cuda(launch_pack(p, to_ptrs(A, h->tp), to_ptrs(B, h->tp), const_cast<void *>(packed),
+                                 unpack, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int tp_mlp_pack(tp_mlp_t h, const void *const *A_shards, const void *const *B_shards, void *packed,
+                tp_mlp_stream_t stream) {
+    return pack_common(h, A_shards, B_shards, packed, false, stream);
+}
+
+int tp_mlp_unpack(tp_mlp_t h, const void *packed, void *const *A_shards, void *const *B_shards,
+                  tp_mlp_stream_t stream) {
+    return pack_common(h, A_shards, B_shards, packed, true, stream);
+}
+
+int tp_mlp_forward_packed(tp_mlp_t h, const void *x, int tokens, const void *packed, void *out,
+                          tp_mlp_stream_t stream) {
+    if (!h) return TP_MLP_ERR_INVALID_ARG;
+    if (tokens < 0 || tokens > h->max_tokens) return TP_MLP_ERR_SHAPE;
+    Problem p = problem_of(h, tokens);
+    // plan choice
+    int plan = h->plan;
+    if (plan == TP_MLP_PLAN_AUTO) plan = gemv_supported(p) ? TP_MLP_PLAN_GEMV : TP_MLP_PLAN_SIMT;
+    if (plan == TP_MLP_PLAN_GEMV && !gemv_supported(p) && tokens > 0) return TP_MLP_ERR_UNSUPPORTED;
+    if (plan == TP_MLP_PLAN_TC) return TP_MLP_ERR_UNSUPPORTED;
+    if (tokens == 0) {
+        h->last_plan = plan;
+        h->last_launches = 0;
+        return TP_MLP_OK;
+    }
+    const size_t e = elem_bytes(h->dtype);
+    int s;
+    if ((s = check_dev(x, (size_t)tokens * h->d_model * e))) return s;
+    if ((s = check_dev(out, (size_t)tokens * h->d_out * e))) return s;
+    if ((s = check_dev(packed, tp_mlp_packed_bytes(h)))) return s;
+    if ((s = check_workspace(h, tokens))) return s;
+    char *ws = static_cast<char *>(h->ws);
+    unsigned *counters = reinterpret_cast<unsigned *>(ws);
+    void *hbuf = ws + counters_bytes(h);
+    float *part = reinterpret_cast<float *>(ws + counters_bytes(h) + h_bytes(h, tokens));
+    const void *w1p = packed;
+    const void *w2p = static_cast<const char *>(packed) + packed_part2_offset(p);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t ce;
+    int launches = 2;
+    if (plan == TP_MLP_PLAN_GEMV) {
+        ce = launch_gemv(p, x, w1p, w2p, hbuf, out, part, counters, h->num_sms, st, h->marks,
+                         &launches);
+    } else {
+        ShardPtrs a, b;
+        memset(&a, 0, sizeof(a));
+        memset(&b, 0, sizeof(b));
+        a.p[0] = w1p;
+        b.p[0] = w2p;
+        ce = launch_simt(p, true, x, a, b, hbuf, out, nullptr, st, h->marks);
+    }
+    if (ce != cudaSuccess) return TP_MLP_ERR_CUDA;
+    h->last_plan = plan;
+    h->last_launches = launches;
+    return TP_MLP_OK;
+}
+
+int tp_mlp_set_plan(tp_mlp_t h, int plan) {
+    if (!h) return TP_MLP_ERR_INVALID_ARG;
+    if (plan < TP_MLP_PLAN_AUTO || plan > TP_MLP_PLAN_TC) return TP_MLP_ERR_INVALID_ARG;
+    h->plan = plan;
+    return TP_MLP_OK;
+}
+
+int tp_mlp_set_profile_events(tp_mlp_t h, void *const *events, int n) {
+    if (!h || n < 0 || n > 8) return TP_MLP_ERR_INVALID_ARG;
+    memset(&h->marks, 0, sizeof(h->marks));
+    if (!events || n == 0) return TP_MLP_OK;
+    for (int i = 0; i < n; ++i) h->marks.ev[i] = static_cast<cudaEvent_t>(events[i]);
+    h->marks.n = n;
+    return TP_MLP_OK;
+}
+
+int tp_mlp_last_plan(tp_mlp_t h) { return h ? h->last_plan : -1; }
+int tp_mlp_last_launches(tp_mlp_t h) { return h ? h->last_launches : -1; }
+
+const char *tp_mlp_status_string(int status) {
+    switch (status) {
+        case TP_MLP_OK: return "ok";
+        case TP_MLP_ERR_INVALID_ARG: return "invalid argument";
+        case TP_MLP_ERR_SHAPE: return "shape mismatch";
+        case TP_MLP_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+        case TP_MLP_ERR_UNSUPPORTED: return "unsupported by this build";
+        case TP_MLP_ERR_CUDA: return "CUDA error";
+        case TP_MLP_ERR_TIMEOUT: return "device wait timed out";
+        case TP_MLP_ERR_WORKSPACE: return "workspace missing or too small";
+    }
+    return "unknown status";
+}
+
+}  // extern "C"

@@ -1,0 +1,151 @@
+"""C ABI checks that need no GPU: exports, header validity, host-side validation.
+
+No call here launches a kernel: every argument error is detected on the host
+before the library touches the device.
+"""
+import ctypes
+import glob
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADERS = sorted(glob.glob(os.path.join(ROOT, "include", "*.h")))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from tensor_sharded_mlp_b200 import build
+    path = build.build()
+    return ctypes.CDLL(path)
+
+
+@pytest.fixture(scope="module")
+def b(lib):
+    from tensor_sharded_mlp_b200 import binding
+    return binding
+
+
+def _declared():
+    names = []
+    for h in HEADERS:
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names += re.findall(r"\b(tp_mlp_\w+)\s*\(", text)
+    return sorted(set(names))
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for n in ("tp_mlp_create", "tp_mlp_forward", "tp_mlp_partials", "tp_mlp_destroy",
+              "tp_mlp_pack", "tp_mlp_unpack", "tp_mlp_forward_packed", "tp_mlp_workspace_bytes",
+              "tp_mlp_set_workspace", "tp_mlp_packed_bytes", "tp_mlp_status_string"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    nm = subprocess.run(["nm", "-D", "--defined-only", lib._name], capture_output=True, text=True,
+                        check=True).stdout
+    exported = set(re.findall(r"\s[TW]\s+(\w+)$", nm, flags=re.M))
+    missing = [n for n in _declared() if n not in exported]
+    assert not missing, missing
+
+
+def test_binding_covers_every_symbol(b):
+    assert set(_declared()) <= set(b.EXPORTED)
+
+
+def test_header_compiles_as_c(tmp_path, lib):
+    src = tmp_path / "use.c"
+    src.write_text('#include "tp_mlp.h"\n#include <stdio.h>\n'
+                   'int main(void){ tp_mlp_t h = 0;\n'
+                   ' int s = tp_mlp_create(&h, 64, 256, 64, 2, TP_MLP_ACT_TANH, TP_MLP_F32, 4);\n'
+                   ' printf("%d %zu %s\\n", s, tp_mlp_packed_bytes(h), tp_mlp_status_string(s));\n'
+                   ' tp_mlp_destroy(h); return s; }\n')
+    exe = tmp_path / "use"
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    str(src), "-o", str(exe), lib._name, "-Wl,-rpath," + os.path.dirname(lib._name)],
+                   check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()
+    assert out[0] == "0" and int(out[1]) == 64 * 256 * 4 + 256 * 64 * 4
+
+
+def test_create_argument_errors(b):
+    E = b.STATUS
+    cases = [((64, 256, 64, 3, "tanh", "f32", 4), "ERR_SHAPE"),     # d_ff % tp
+             ((64, 256, 64, 0, "tanh", "f32", 4), "ERR_SHAPE"),
+             ((64, 256, 64, 16, "tanh", "f32", 4), "ERR_SHAPE"),    # tp > 8
+             ((0, 256, 64, 2, "tanh", "f32", 4), "ERR_SHAPE"),
+             ((64, 256, 64, 2, "tanh", "f32", 0), "ERR_SHAPE"),
+             ((64, 256, 0, 2, "tanh", "f32", 4), "ERR_SHAPE")]
+    for args, want in cases:
+        with pytest.raises(b.TpMlpError) as ei:
+            b.tp_mlp_create(*args)
+        assert ei.value.name == want, args
+    h = ctypes.c_void_p()
+    assert b._lib.tp_mlp_create(ctypes.byref(h), 64, 256, 64, 2, 7, 0, 4) == 1   # bad act
+    assert b._lib.tp_mlp_create(ctypes.byref(h), 64, 256, 64, 2, 0, 5, 4) == 1   # bad dtype
+    assert b._lib.tp_mlp_create(None, 64, 256, 64, 2, 0, 0, 4) == 1
+
+
+def test_sizes_follow_the_documented_layout(b):
+    def a256(v):
+        return (v + 255) // 256 * 256
+    for act, dtype, d, f, dout, tp in [("tanh", "f32", 64, 256, 64, 2), ("swiglu", "bf16", 8192, 28672, 8192, 8),
+                                       ("swiglu", "bf16", 40, 200, 24, 4), ("identity", "bf16", 8, 8, 4, 4)]:
+        h = b.tp_mlp_create(d, f, dout, tp, act, dtype, 32)
+        e = 4 if dtype == "f32" else 2
+        rows1 = 2 * f if act == "swiglu" else f
+        assert b.tp_mlp_packed_bytes(h) == a256(rows1 * d * e) + a256(dout * f * e)
+        w = [b.tp_mlp_workspace_bytes(h, t) for t in range(0, 33)]
+        assert all(x > 0 for x in w) and all(w[i] <= w[i + 1] for i in range(32))
+        assert w[32] >= 32 * f * e            # holds H
+        assert b.tp_mlp_workspace_bytes(h, 33) == 0
+        b.tp_mlp_destroy(h)
+
+
+def test_call_argument_errors_before_any_launch(b):
+    """Each bad argument is rejected on the host (no device is present here)."""
+    L = b._lib
+    h = b.tp_mlp_create(64, 256, 64, 2, "tanh", "f32", 4)
+    vp = ctypes.c_void_p
+    arr = (ctypes.c_void_p * 2)(0x10000, 0x20000)
+    A = ctypes.cast(arr, b._vpp)
+    ok_ptr = vp(0x100000)
+    bad_ptr = vp(0x100004)         # not 16-byte aligned
+    assert L.tp_mlp_forward(None, ok_ptr, 1, A, A, 2, 0, ok_ptr, None) == 1
+    assert L.tp_mlp_forward(h, ok_ptr, 5, A, A, 2, 0, ok_ptr, None) == 2       # tokens > max
+    assert L.tp_mlp_forward(h, ok_ptr, -1, A, A, 2, 0, ok_ptr, None) == 2
+    assert L.tp_mlp_forward(h, ok_ptr, 1, A, A, 4, 0, ok_ptr, None) == 2       # tp mismatch
+    assert L.tp_mlp_forward(h, ok_ptr, 1, A, A, 2, 1, ok_ptr, None) == 1       # act mismatch
+    assert L.tp_mlp_forward(h, None, 1, A, A, 2, 0, ok_ptr, None) == 1          # null x
+    assert L.tp_mlp_forward(h, bad_ptr, 1, A, A, 2, 0, ok_ptr, None) == 3       # misaligned
+    assert L.tp_mlp_forward(h, ok_ptr, 0, A, A, 2, 0, ok_ptr, None) == 0        # 0 tokens: no-op
+    assert L.tp_mlp_partials(h, ok_ptr, 1, A, A, 2, 0, None, None) == 1
+    assert L.tp_mlp_forward_packed(h, ok_ptr, 5, ok_ptr, ok_ptr, None) == 2
+    assert L.tp_mlp_forward_packed(h, bad_ptr, 1, ok_ptr, ok_ptr, None) == 3
+    assert L.tp_mlp_pack(None, A, A, ok_ptr, None) == 1
+    assert L.tp_mlp_set_plan(h, 9) == 1
+    assert L.tp_mlp_set_plan(h, 3) == 0
+    assert L.tp_mlp_forward_packed(h, ok_ptr, 1, ok_ptr, ok_ptr, None) == 4     # tcgen05 needs bf16
+    assert L.tp_mlp_set_plan(h, 2) == 0
+    assert L.tp_mlp_forward_packed(h, ok_ptr, 1, ok_ptr, ok_ptr, None) == 4     # GEMV needs bf16
+    assert L.tp_mlp_set_plan(h, 0) == 0
+    assert L.tp_mlp_set_workspace(h, ok_ptr, 16) == 7                           # too small
+    assert L.tp_mlp_set_profile_events(h, None, 9) == 1
+    assert L.tp_mlp_last_plan(h) == 1 and L.tp_mlp_last_launches(h) == 0        # the 0-token no-op
+    b.tp_mlp_destroy(h)
+    for s in range(8):
+        assert b.tp_mlp_status_string(s) not in ("", "unknown status")
+    assert b.tp_mlp_status_string(99) == "unknown status"
+
+
+def test_binding_pairs_shards_strictly(b):
+    import torch
+    h = b.tp_mlp_create(8, 8, 4, 2, "tanh", "f32", 2)
+    t = torch.zeros(8, 4)
+    with pytest.raises(ValueError):
+        b.tp_mlp_forward(h, torch.zeros(1, 8), [t, t], [t], 2, "tanh", torch.zeros(1, 4))
+    b.tp_mlp_destroy(h)
