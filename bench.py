@@ -288,19 +288,26 @@ def main():
     sampler = ClockSampler(torch.cuda.current_device())
     sampler.start()
     time.sleep(0.1)
+    # Timed region: K clean steps (kernels back to back, so each may overlap the
+    # previous one's tail through programmatic dependent launch).
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     t0 = time.perf_counter()
     start.record(stream)
     for i in range(K):
-        binding.tp_mlp_set_profile_events(m.h, ev[i])
         m.forward_packed(x, packed, out=out)
     end.record(stream)
     barrier()
     t1 = time.perf_counter()
     sampler.mark(t0, t1)
-    binding.tp_mlp_set_profile_events(m.h, None)
     elapsed_ms = start.elapsed_time(end)
+    # Per-kernel durations: the same K steps again with the library recording
+    # events on the launch stream before, between and after its kernels.
+    for i in range(K):
+        binding.tp_mlp_set_profile_events(m.h, ev[i])
+        m.forward_packed(x, packed, out=out)
+    binding.tp_mlp_set_profile_events(m.h, None)
+    barrier()
     kern_ms = [statistics.fmean(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(K)) for j in range(nk)]
     if world > 1:
         t = torch.tensor([elapsed_ms], dtype=torch.float64, device="cuda")

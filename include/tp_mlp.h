@@ -71,7 +71,11 @@ typedef enum {
     TP_MLP_PLAN_AUTO = 0,   /* let the library choose (default)                      */
     TP_MLP_PLAN_SIMT = 1,   /* tiled CUDA-core kernels, any shape and layout          */
     TP_MLP_PLAN_GEMV = 2,   /* packed bf16, 1-4 tokens: streaming split-K GEMV        */
-    TP_MLP_PLAN_TC = 3      /* packed bf16: tcgen05 tensor-core GEMMs (TMA + TMEM)    */
+    TP_MLP_PLAN_TC = 3,     /* packed bf16: tcgen05 tensor-core GEMMs (TMA + TMEM);
+                               the library picks the tiling from the token count      */
+    TP_MLP_PLAN_TC_WIDE = 4,   /* tcgen05, tiles of 128 tokens x 256 weight rows      */
+    TP_MLP_PLAN_TC_SKINNY = 5  /* tcgen05, weights as the MMA's M, 1..128 tokens as N,
+                                  weight stream split evenly over the SMs             */
 } tp_mlp_plan;
 
 /*
@@ -186,6 +190,14 @@ int tp_mlp_set_plan(tp_mlp_t handle, int plan);
  * events = NULL) turns the hook off.  At most 8 events.
  */
 int tp_mlp_set_profile_events(tp_mlp_t handle, void *const *events, int n);
+
+/*
+ * Device-side status of the work issued so far on this handle's workspace:
+ * synchronises the device, returns TP_MLP_ERR_TIMEOUT if a kernel gave up a
+ * bounded internal wait (its results are then invalid) and clears the flag,
+ * TP_MLP_OK otherwise.  Needs a workspace.
+ */
+int tp_mlp_get_device_status(tp_mlp_t handle);
 
 /* Plan (tp_mlp_plan) and number of kernel launches of the last successful
  * forward / partials call on this handle; -1 before the first. */

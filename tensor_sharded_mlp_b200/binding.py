@@ -26,7 +26,7 @@ _lib = ctypes.CDLL(_LIB_PATH)
 ACT = {"tanh": 0, "swiglu": 1, "identity": 2}
 DTYPE = {"f32": 0, "bf16": 1}
 TORCH_DTYPE = {"f32": torch.float32, "bf16": torch.bfloat16}
-PLAN = {"auto": 0, "simt": 1, "gemv": 2, "tc": 3}
+PLAN = {"auto": 0, "simt": 1, "gemv": 2, "tc": 3, "tc_wide": 4, "tc_skinny": 5}
 PLAN_NAME = {v: k for k, v in PLAN.items()}
 STATUS = {0: "OK", 1: "ERR_INVALID_ARG", 2: "ERR_SHAPE", 3: "ERR_ALIGNMENT", 4: "ERR_UNSUPPORTED",
           5: "ERR_CUDA", 6: "ERR_TIMEOUT", 7: "ERR_WORKSPACE"}
@@ -49,6 +49,7 @@ _SIGS = {
     "tp_mlp_forward_packed": (_i, [_vp, _vp, _i, _vp, _vp, _vp]),
     "tp_mlp_set_plan": (_i, [_vp, _i]),
     "tp_mlp_set_profile_events": (_i, [_vp, _vpp, _i]),
+    "tp_mlp_get_device_status": (_i, [_vp]),
     "tp_mlp_last_plan": (_i, [_vp]),
     "tp_mlp_last_launches": (_i, [_vp]),
     "tp_mlp_status_string": (ctypes.c_char_p, [_i]),
@@ -169,6 +170,10 @@ def tp_mlp_set_profile_events(h, events) -> None:
     arr = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
     _check("tp_mlp_set_profile_events",
            _lib.tp_mlp_set_profile_events(h, ctypes.cast(arr, _vpp), len(events)))
+
+
+def tp_mlp_get_device_status(h) -> None:
+    _check("tp_mlp_get_device_status", _lib.tp_mlp_get_device_status(h))
 
 
 def tp_mlp_last_plan(h) -> str:

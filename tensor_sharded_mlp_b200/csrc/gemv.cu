@@ -94,7 +94,42 @@ __global__ void __launch_bounds__(NTHR) gemv_kernel(GemvArgs a) {
     const int klen = (int)min((long)a.Kc, (long)a.K - kbase);
     const int kpad = (klen + KSTEP - 1) / KSTEP * KSTEP;
 
-    // stage X[:, kbase : kbase + klen] (zero-padded to a whole step) as fp32
+    const int g0 = blockIdx.x * a.gpb;
+    const int g1 = min(a.groups, g0 + a.gpb);
+    auto rows_of = [&](int g, const __nv_bfloat16 *(&row)[R]) {
+        if (MODE == 0) {
+            row[0] = a.w + w1p_row(g, false, a.d_ff, a.act) * a.ldw + kbase;
+            if (R > 1) row[R - 1] = a.w + w1p_row(g, true, a.d_ff, a.act) * a.ldw + kbase;
+        } else {
+            row[0] = a.w + (long)g * a.ldw + kbase;
+        }
+    };
+    auto load_bundle = [&](const __nv_bfloat16 *const (&row)[R], int k0, uint4 (&wv)[U][R]) {
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int k = k0 + u * KSTEP + lane * 8;
+#pragma unroll
+            for (int r = 0; r < R; ++r)
+                wv[u][r] = (k < klen) ? ld_stream_v4(row[r] + k) : make_uint4(0, 0, 0, 0);
+        }
+    };
+
+    // Prologue, independent of the previous kernel: let the next kernel launch,
+    // pull this warp's first rows towards L2 and issue its first weight loads.
+    pdl_allow_dependents();
+    uint4 wv[U][R];
+    {
+        const int g = g0 + warp;
+        if (g < g1) {
+            const __nv_bfloat16 *row[R];
+            rows_of(g, row);
+            if (lane < R) prefetch_l2(row[lane], (uint32_t)klen * 2u);
+            load_bundle(row, 0, wv);
+        }
+    }
+    // X (or H) is produced by the previous kernel: wait for it, then stage
+    // X[:, kbase : kbase + klen] (zero-padded to a whole step) as fp32.
+    pdl_wait_previous();
     for (int t = 0; t < T; ++t) {
         const __nv_bfloat16 *xr = a.x + (long)t * a.K + kbase;
         for (int k = threadIdx.x; k < kpad; k += NTHR)
@@ -102,16 +137,10 @@ __global__ void __launch_bounds__(NTHR) gemv_kernel(GemvArgs a) {
     }
     __syncthreads();
 
-    const int g0 = blockIdx.x * a.gpb;
-    const int g1 = min(a.groups, g0 + a.gpb);
+    bool first = true;
     for (int g = g0 + warp; g < g1; g += WARPS) {
         const __nv_bfloat16 *row[R];
-        if (MODE == 0) {
-            row[0] = a.w + w1p_row(g, false, a.d_ff, a.act) * a.ldw + kbase;
-            if (R > 1) row[R - 1] = a.w + w1p_row(g, true, a.d_ff, a.act) * a.ldw + kbase;
-        } else {
-            row[0] = a.w + (long)g * a.ldw + kbase;
-        }
+        rows_of(g, row);
         float acc[R][T];
 #pragma unroll
         for (int r = 0; r < R; ++r)
@@ -119,14 +148,8 @@ __global__ void __launch_bounds__(NTHR) gemv_kernel(GemvArgs a) {
             for (int t = 0; t < T; ++t) acc[r][t] = 0.f;
 
         for (int k0 = 0; k0 < klen; k0 += KSTEP * U) {
-            uint4 wv[U][R];
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int k = k0 + u * KSTEP + lane * 8;
-#pragma unroll
-                for (int r = 0; r < R; ++r)
-                    wv[u][r] = (k < klen) ? ld_stream_v4(row[r] + k) : make_uint4(0, 0, 0, 0);
-            }
+            if (!first) load_bundle(row, k0, wv);
+            first = false;
 #pragma unroll
             for (int u = 0; u < U; ++u) {
                 const int kk = k0 + u * KSTEP;
@@ -199,8 +222,7 @@ cudaError_t launch_one(const GemvArgs &a, cudaStream_t st) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const dim3 grid((a.groups + a.gpb - 1) / a.gpb, a.S);
-    kern<<<grid, NTHR, smem, st>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(kern, grid, dim3(NTHR), smem, st, a);
 }
 
 template <int R, int MODE>
@@ -215,8 +237,8 @@ cudaError_t launch_T(int T, const GemvArgs &a, cudaStream_t st) {
 }
 
 // Split count: keep the staged chunk <= kSmemBudget and give the grid enough blocks.
-constexpr size_t kSmemBudget = 64 * 1024;
-constexpr int kGpb = 32;
+constexpr size_t kSmemBudget = 48 * 1024;
+constexpr int kGpb = 16;
 
 void plan_split(int T, int K, int groups, int num_sms, int &S, int &Kc) {
     const long steps = (K + KSTEP - 1) / KSTEP;

@@ -39,4 +39,13 @@ cudaError_t launch_gemv(const Problem &p, const void *x, const void *w1p, const 
                         void *out, float *part, unsigned *counters, int num_sms, cudaStream_t st,
                         const Marks &marks, int *launches);
 
+// tc_gemm.cu: tcgen05 path, packed bf16.  skinny: tokens <= kTcSkinnyMaxTokens.
+constexpr int kTcSkinnyMaxTokens = 128;
+bool tc_supported(const Problem &p);
+size_t tc_counter_slots(const Problem &p);
+size_t tc_workspace_bytes(const Problem &p, int num_sms);
+cudaError_t launch_tc(const Problem &p, bool skinny, const void *x, const void *w1p, const void *w2p, void *h,
+                      void *out, float *part, unsigned *counters, int *status, int num_sms, cudaStream_t st,
+                      const Marks &marks);
+
 }  // namespace tpmlp

@@ -1,0 +1,661 @@
+// tc_gemm.cu -- tensor-core path for bf16: tcgen05 MMA with TMEM accumulators,
+// operands streamed by TMA through a shared-memory ring, warp-specialised.
+//
+// Both projections are GEMMs over the packed K-major weights W (rows x K):
+//   first  ("大模型推理系统揭秘（07）", §1.2.2 column-parallel):  U = X W1^T,
+//          H = tanh(U) or SiLU(U_gate) * U_up (§1.4.3), fused in the epilogue;
+//   second (§1.2.2 row-parallel + §1.2.3 sum of partials):  Z = H W2^T, one
+//          K loop over every rank's rows, so the ranks' partial sums accumulate
+//          in TMEM and never reach HBM.
+//
+// Two tilings share the pipeline code:
+//   wide   (many tokens, compute-bound): the MMA's M is 128 tokens and its N is
+//          256 weight rows; persistent CTAs walk the tiles in groups of
+//          kGroupM token tiles so a weight tile is reused from L2;
+//   skinny (few tokens, memory-bound, the decode case "7.4 推理侧并行" §7.4.1
+//          describes): operands swapped -- M is 128 weight rows (two MMAs per
+//          256-row weight tile), N is the token count rounded up to BT.  The
+//          weight stream is cut into equal contiguous shares, one per CTA
+//          ("stream-K"); a tile split between CTAs is finished by the last CTA
+//          to arrive, which adds the fp32 partial slots in a fixed order.
+//          Nothing waits on another CTA.
+//
+// Roles: warp 0 lane 0 issues TMA loads, warp 1 allocates TMEM and lane 0
+// issues the MMAs, warps 2..5 run the epilogue (TMEM lanes 32*(warp%4)...).
+// Every mbarrier wait is bounded (tc_ptx.cuh); a wait that runs out raises an
+// abort flag that every role checks, and the CTA records it in a status word.
+#include <cuda.h>
+
+#include <algorithm>
+
+#include "common.cuh"
+#include "internal.h"
+#include "tc_ptx.cuh"
+
+namespace tpmlp {
+namespace {
+
+using namespace tc;
+
+constexpr int BK = 64;              // K per stage: one 128-byte swizzle row of bf16
+constexpr int NTHREADS = 192;
+constexpr int kGroupM = 8;          // wide tiling: token tiles per raster group
+constexpr int kWideStages = 4;
+
+enum { EPI_H_TANH = 0, EPI_H_SWIGLU = 1, EPI_H_IDENT = 2, EPI_OUT = 3 };
+
+struct TcArgs {
+    int rows_x;          // X rows (tokens)
+    int rows_w;          // W rows
+    int K, KB;           // K and ceil(K / BK)
+    int epi;
+    __nv_bfloat16 *out;  // H (T x d_ff) or out (T x d_out)
+    int ldo;             // row stride of out = out_cols
+    int out_cols;
+    // skinny tiling (stream-K)
+    long long total_iters;
+    int slots;           // partial slots per weight tile
+    float *part;         // [tile][slot][256][BT] fp32
+    unsigned *tile_cnt;  // k-blocks done per weight tile, zero between launches
+    int *status;         // set to 1 if a bounded wait ran out
+};
+
+__device__ __forceinline__ float act_out(int epi, float u) {
+    if (epi == EPI_H_TANH) return tanhf(u);
+    return u;   // identity / plain output
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t *>(&v);
+}
+
+// Shared-memory carve-up common to both tilings.
+struct Smem {
+    uint8_t *a, *b;           // stage rings (1024-aligned)
+    uint64_t *full, *empty;   // per stage
+    uint64_t *tfull, *tempty; // per accumulator buffer (2)
+    uint64_t *drain;          // abort path: waits for the MMAs in flight
+    uint32_t *tmem_slot;
+    volatile int *abort;
+    int *flag;
+};
+
+template <int STAGES>
+__device__ __forceinline__ Smem carve(uint8_t *raw, uint32_t a_bytes, uint32_t b_bytes) {
+    Smem s;
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
+    s.a = base;
+    s.b = base + STAGES * a_bytes;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(s.b + STAGES * b_bytes);
+    s.full = bars;
+    s.empty = bars + STAGES;
+    s.tfull = bars + 2 * STAGES;
+    s.tempty = bars + 2 * STAGES + 2;
+    s.drain = bars + 2 * STAGES + 4;
+    s.tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 5);
+    s.abort = reinterpret_cast<volatile int *>(s.tmem_slot + 1);
+    s.flag = reinterpret_cast<int *>(s.tmem_slot + 2);
+    return s;
+}
+
+template <int STAGES>
+constexpr size_t smem_bytes(uint32_t a_bytes, uint32_t b_bytes) {
+    return 1024 + STAGES * (size_t)(a_bytes + b_bytes) + (2 * STAGES + 5) * 8 + 16;
+}
+
+// Setup shared by both kernels: barriers, TMEM (512 columns), descriptor prefetch.
+template <int STAGES>
+__device__ __forceinline__ uint32_t setup(const Smem &s, const CUtensorMap *m0, const CUtensorMap *m1) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < STAGES; ++i) {
+            mbar_init(smem_u32(&s.full[i]), 1);
+            mbar_init(smem_u32(&s.empty[i]), 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(smem_u32(&s.tfull[i]), 1);
+            mbar_init(smem_u32(&s.tempty[i]), 4);
+        }
+        mbar_init(smem_u32(s.drain), 1);
+        *s.abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(m0);
+        tma_prefetch_desc(m1);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(s.tmem_slot), 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    return *s.tmem_slot;
+}
+
+__device__ __forceinline__ void teardown(const Smem &s, uint32_t tmem_base, int *status) {
+    if (*s.abort) {
+        // A bounded wait gave up somewhere.  Before TMEM and shared memory are
+        // released: let the MMA issuer's MMAs finish, and give TMA copies in
+        // flight time to land (both bounded).
+        if (threadIdx.x == 32) {
+            mma_commit(smem_u32(s.drain));
+            volatile int never = 0;
+            mbar_wait(smem_u32(s.drain), 0, &never);
+        }
+        if (threadIdx.x == 0) {
+            const unsigned long long t0 = globaltimer();
+            while (globaltimer() - t0 < 100000ull) {
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if ((threadIdx.x >> 5) == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem_base, 512);
+    }
+    if (threadIdx.x == 0 && *s.abort) atomicExch(status, 1);
+}
+
+// ======================= wide tiling: 128 tokens x 256 weight rows ======================
+
+__device__ __forceinline__ void wide_tile(int u, int MT, int NT, int &mt, int &nt) {
+    const int per_group = kGroupM * NT;
+    const int g = u / per_group;
+    const int gm = min(kGroupM, MT - g * kGroupM);
+    const int r = u - g * per_group;
+    nt = r / gm;
+    mt = g * kGroupM + r % gm;
+}
+
+__global__ void __launch_bounds__(NTHREADS, 1)
+    tc_wide_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW, TcArgs a) {
+    constexpr int STAGES = kWideStages;
+    constexpr uint32_t A_BYTES = 128 * BK * 2;   // X tile: 128 tokens
+    constexpr uint32_t B_BYTES = 256 * BK * 2;   // W tile: 256 rows
+    extern __shared__ uint8_t smem_raw[];
+    const Smem s = carve<STAGES>(smem_raw, A_BYTES, B_BYTES);
+    const uint32_t tmem_base = setup<STAGES>(s, &tmX, &tmW);
+    pdl_allow_dependents();
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int MT = (a.rows_x + 127) / 128, NT = (a.rows_w + 255) / 256;
+    const int units = MT * NT;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            pdl_wait_previous();   // X / H come from the previous kernel
+            int stage = 0;
+            uint32_t phase = 0;
+            for (int u = blockIdx.x; u < units; u += gridDim.x) {
+                int mt, nt;
+                wide_tile(u, MT, NT, mt, nt);
+                for (int kb = 0; kb < a.KB; ++kb) {
+                    if (!mbar_wait(smem_u32(&s.empty[stage]), phase ^ 1, s.abort)) goto done;
+                    const uint32_t fb = smem_u32(&s.full[stage]);
+                    mbar_arrive_expect_tx(fb, A_BYTES + B_BYTES);
+                    tma_load_2d(smem_u32(s.a + stage * A_BYTES), &tmX, kb * BK, mt * 128, fb);
+                    tma_load_2d(smem_u32(s.b + stage * B_BYTES), &tmW, kb * BK, nt * 256, fb);
+                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t idesc = idesc_bf16_f32(128, 256);
+            int stage = 0, acc = 0;
+            uint32_t phase = 0, acc_phase = 0;
+            for (int u = blockIdx.x; u < units; u += gridDim.x) {
+                if (!mbar_wait(smem_u32(&s.tempty[acc]), acc_phase ^ 1, s.abort)) goto done;
+                tc_fence_after();
+                const uint32_t d = tmem_base + acc * 256;
+                for (int kb = 0; kb < a.KB; ++kb) {
+                    if (!mbar_wait(smem_u32(&s.full[stage]), phase, s.abort)) goto done;
+                    tc_fence_after();
+                    const uint64_t da = smem_desc_kmajor_sw128(smem_u32(s.a + stage * A_BYTES));
+                    const uint64_t db = smem_desc_kmajor_sw128(smem_u32(s.b + stage * B_BYTES));
+#pragma unroll
+                    for (int k = 0; k < BK / 16; ++k)   // +32 bytes along K = +2 in the address field
+                        mma_bf16(d, da + 2 * k, db + 2 * k, idesc, (kb | k) != 0);
+                    mma_commit(smem_u32(&s.empty[stage]));
+                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                }
+                mma_commit(smem_u32(&s.tfull[acc]));
+                acc ^= 1;
+                if (acc == 0) acc_phase ^= 1;
+            }
+        }
+    } else {
+        // epilogue: TMEM lane quadrant q holds tokens 32q..32q+31 of the tile
+        pdl_wait_previous();   // outputs may still be read by the previous kernel
+        const int q = warp & 3;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int u = blockIdx.x; u < units; u += gridDim.x) {
+            int mt, nt;
+            wide_tile(u, MT, NT, mt, nt);
+            if (!mbar_wait(smem_u32(&s.tfull[acc]), acc_phase, s.abort)) break;
+            tc_fence_after();
+            const int row = mt * 128 + q * 32 + lane;
+            const bool row_ok = row < a.rows_x;
+            __nv_bfloat16 *orow = a.out + (long)row * a.ldo;
+            const uint32_t taddr = tmem_base + acc * 256 + ((uint32_t)(q * 32) << 16);
+            if (a.epi == EPI_H_SWIGLU) {
+                // columns 0..127 = gate rows, 128..255 = up rows of features 128*nt ..
+                const int c0 = nt * 128;
+#pragma unroll 1
+                for (int j = 0; j < 8; ++j) {
+                    float g[16], v[16];
+                    tmem_ld16(taddr + 16 * j, g);
+                    tmem_ld16(taddr + 128 + 16 * j, v);
+                    tmem_ld_wait();
+                    if (row_ok) {
+                        uint32_t w[8];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            w[i] = pack_bf16x2(silu_fast(g[2 * i]) * v[2 * i], silu_fast(g[2 * i + 1]) * v[2 * i + 1]);
+                        uint4 *dst = reinterpret_cast<uint4 *>(orow + c0 + 16 * j);
+                        dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+                        dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+                    }
+                }
+            } else {
+                const int c0 = nt * 256;
+#pragma unroll 1
+                for (int j = 0; j < 16; ++j) {
+                    float v[16];
+                    tmem_ld16(taddr + 16 * j, v);
+                    tmem_ld_wait();
+                    const int col = c0 + 16 * j;
+                    if (row_ok && col < a.out_cols) {
+                        if (col + 16 <= a.out_cols) {
+                            uint32_t w[8];
+#pragma unroll
+                            for (int i = 0; i < 8; ++i)
+                                w[i] = pack_bf16x2(act_out(a.epi, v[2 * i]), act_out(a.epi, v[2 * i + 1]));
+                            uint4 *dst = reinterpret_cast<uint4 *>(orow + col);
+                            dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+                            dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+                        } else {
+                            for (int i = 0; i < 16 && col + i < a.out_cols; ++i)
+                                orow[col + i] = __float2bfloat16_rn(act_out(a.epi, v[i]));
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&s.tempty[acc]));
+            acc ^= 1;
+            if (acc == 0) acc_phase ^= 1;
+        }
+    }
+done:
+    teardown(s, tmem_base, a.status);
+}
+
+// ================== skinny tiling: 256 weight rows x BT tokens, stream-K ==================
+
+__device__ __forceinline__ long long share_begin(long long c, long long total, long long G) {
+    return c * total / G;
+}
+// CTA whose share holds iteration `it`.
+__device__ __forceinline__ int share_owner(long long it, long long total, long long G) {
+    return (int)(((it + 1) * G - 1) / total);
+}
+
+// Final epilogue of a skinny tile for 16 tokens t0..t0+15: v0 = rows r, v1 = rows 128 + r.
+__device__ __forceinline__ void skinny_final16(const TcArgs &a, int tile, int r, int t0, const float (&v0)[16],
+                                               const float (&v1)[16]) {
+    const int T = a.rows_x;
+    if (a.epi == EPI_H_SWIGLU) {
+        const int n = tile * 128 + r;
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            if (t0 + i < T) a.out[(long)(t0 + i) * a.ldo + n] = __float2bfloat16_rn(silu_fast(v0[i]) * v1[i]);
+    } else {
+        const int n0 = tile * 256 + r, n1 = n0 + 128;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            if (t0 + i >= T) break;
+            if (n0 < a.out_cols) a.out[(long)(t0 + i) * a.ldo + n0] = __float2bfloat16_rn(act_out(a.epi, v0[i]));
+            if (n1 < a.out_cols) a.out[(long)(t0 + i) * a.ldo + n1] = __float2bfloat16_rn(act_out(a.epi, v1[i]));
+        }
+    }
+}
+
+template <int BT, int STAGES>
+__global__ void __launch_bounds__(NTHREADS, 1)
+    tc_skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX, TcArgs a) {
+    constexpr uint32_t W_BYTES = 256 * BK * 2;   // 256 weight rows (two M=128 halves)
+    constexpr uint32_t X_BYTES = BT * BK * 2;
+    extern __shared__ uint8_t smem_raw[];
+    const Smem s = carve<STAGES>(smem_raw, W_BYTES, X_BYTES);
+    const uint32_t tmem_base = setup<STAGES>(s, &tmW, &tmX);
+    pdl_allow_dependents();
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long total = a.total_iters, G = gridDim.x, c = blockIdx.x;
+    const long long it_b = share_begin(c, total, G), it_e = share_begin(c + 1, total, G);
+    const int KB = a.KB;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            bool waited = false;
+            for (long long it = it_b; it < it_e;) {
+                const int tile = (int)(it / KB);
+                const int kb0 = (int)(it - (long long)tile * KB);
+                const int kb1 = (int)min((long long)KB, it_e - (long long)tile * KB);
+                for (int kb = kb0; kb < kb1; ++kb) {
+                    if (!mbar_wait(smem_u32(&s.empty[stage]), phase ^ 1, s.abort)) goto done;
+                    const uint32_t fb = smem_u32(&s.full[stage]);
+                    mbar_arrive_expect_tx(fb, W_BYTES + X_BYTES);
+                    tma_load_2d(smem_u32(s.a + stage * W_BYTES), &tmW, kb * BK, tile * 256, fb);
+                    if (!waited) {   // weights do not depend on the previous kernel; X does
+                        pdl_wait_previous();
+                        waited = true;
+                    }
+                    tma_load_2d(smem_u32(s.b + stage * X_BYTES), &tmX, kb * BK, 0, fb);
+                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                }
+                it = (long long)tile * KB + kb1;
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t idesc = idesc_bf16_f32(128, BT);
+            int stage = 0, acc = 0;
+            uint32_t phase = 0, acc_phase = 0;
+            for (long long it = it_b; it < it_e;) {
+                const int tile = (int)(it / KB);
+                const int kb0 = (int)(it - (long long)tile * KB);
+                const int kb1 = (int)min((long long)KB, it_e - (long long)tile * KB);
+                if (!mbar_wait(smem_u32(&s.tempty[acc]), acc_phase ^ 1, s.abort)) goto done;
+                tc_fence_after();
+                const uint32_t d0 = tmem_base + acc * (2 * BT), d1 = d0 + BT;
+                for (int kb = kb0; kb < kb1; ++kb) {
+                    if (!mbar_wait(smem_u32(&s.full[stage]), phase, s.abort)) goto done;
+                    tc_fence_after();
+                    const uint32_t wa = smem_u32(s.a + stage * W_BYTES);
+                    const uint64_t dw0 = smem_desc_kmajor_sw128(wa);
+                    const uint64_t dw1 = smem_desc_kmajor_sw128(wa + 128 * 128);   // rows 128..255
+                    const uint64_t dx = smem_desc_kmajor_sw128(smem_u32(s.b + stage * X_BYTES));
+#pragma unroll
+                    for (int k = 0; k < BK / 16; ++k) {
+                        const uint32_t accum = (kb != kb0 || k != 0) ? 1u : 0u;
+                        mma_bf16(d0, dw0 + 2 * k, dx + 2 * k, idesc, accum);
+                        mma_bf16(d1, dw1 + 2 * k, dx + 2 * k, idesc, accum);
+                    }
+                    mma_commit(smem_u32(&s.empty[stage]));
+                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                }
+                mma_commit(smem_u32(&s.tfull[acc]));
+                acc ^= 1;
+                if (acc == 0) acc_phase ^= 1;
+                it = (long long)tile * KB + kb1;
+            }
+        }
+    } else {
+        pdl_wait_previous();
+        const int q = warp & 3;
+        const int r = q * 32 + lane;   // row within each 128-row half
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (long long it = it_b; it < it_e;) {
+            const int tile = (int)(it / KB);
+            const int kb0 = (int)(it - (long long)tile * KB);
+            const int kb1 = (int)min((long long)KB, it_e - (long long)tile * KB);
+            it = (long long)tile * KB + kb1;
+            if (!mbar_wait(smem_u32(&s.tfull[acc]), acc_phase, s.abort)) break;
+            tc_fence_after();
+            const uint32_t taddr = tmem_base + acc * (2 * BT) + ((uint32_t)(q * 32) << 16);
+            const bool whole = (kb0 == 0 && kb1 == KB);
+            if (whole) {
+#pragma unroll 1
+                for (int t0 = 0; t0 < BT; t0 += 16) {
+                    float v0[16], v1[16];
+                    tmem_ld16(taddr + t0, v0);
+                    tmem_ld16(taddr + BT + t0, v1);
+                    tmem_ld_wait();
+                    skinny_final16(a, tile, r, t0, v0, v1);
+                }
+            } else {
+                // this CTA's share of the tile -> its partial slot
+                const int c_first = share_owner((long long)tile * KB, total, G);
+                const int c_last = share_owner((long long)tile * KB + KB - 1, total, G);
+                const int slot = (int)c - c_first;
+                float *base = a.part + ((long long)tile * a.slots + slot) * 256 * BT;
+#pragma unroll 1
+                for (int t0 = 0; t0 < BT; t0 += 16) {
+                    float v0[16], v1[16];
+                    tmem_ld16(taddr + t0, v0);
+                    tmem_ld16(taddr + BT + t0, v1);
+                    tmem_ld_wait();
+                    float4 *p0 = reinterpret_cast<float4 *>(base + (long)r * BT + t0);
+                    float4 *p1 = reinterpret_cast<float4 *>(base + (long)(128 + r) * BT + t0);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        p0[i] = make_float4(v0[4 * i], v0[4 * i + 1], v0[4 * i + 2], v0[4 * i + 3]);
+                        p1[i] = make_float4(v1[4 * i], v1[4 * i + 1], v1[4 * i + 2], v1[4 * i + 3]);
+                    }
+                }
+                __threadfence();
+                named_bar(1, 128);
+                if (threadIdx.x == 64) {
+                    const unsigned done_kb = atomicAdd(&a.tile_cnt[tile], (unsigned)(kb1 - kb0)) + (kb1 - kb0);
+                    *s.flag = (done_kb == (unsigned)KB);
+                }
+                named_bar(1, 128);
+                if (*s.flag) {
+                    __threadfence();
+                    const float *tb = a.part + (long long)tile * a.slots * 256 * BT;
+                    const int n = c_last - c_first + 1;
+#pragma unroll 1
+                    for (int t0 = 0; t0 < BT; t0 += 16) {
+                        float v0[16], v1[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) v0[i] = v1[i] = 0.f;
+                        for (int sl = 0; sl < n; ++sl) {
+                            const float *sb = tb + (long long)sl * 256 * BT;
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) {
+                                v0[i] += __ldcg(sb + (long)r * BT + t0 + i);
+                                v1[i] += __ldcg(sb + (long)(128 + r) * BT + t0 + i);
+                            }
+                        }
+                        skinny_final16(a, tile, r, t0, v0, v1);
+                    }
+                    if (threadIdx.x == 64) a.tile_cnt[tile] = 0u;
+                }
+                named_bar(1, 128);   // the flag is reused by the next split tile
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&s.tempty[acc]));
+            acc ^= 1;
+            if (acc == 0) acc_phase ^= 1;
+        }
+    }
+done:
+    teardown(s, tmem_base, a.status);
+}
+
+// ======================================= host side =======================================
+
+typedef CUresult (*PFN_encodeTiled)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                    const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
+                                    CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                    CUtensorMapFloatOOBfill);
+
+PFN_encodeTiled encode_fn() {
+    static PFN_encodeTiled fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        tried = true;
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_encodeTiled>(p);
+    }
+    return fn;
+}
+
+// K-major bf16 matrix (rows x K, row stride K), box = 64 (K) x box_rows, 128-byte swizzle,
+// out-of-range elements read as zero.
+bool make_map(CUtensorMap *m, const void *base, int K, int rows, int box_rows) {
+    PFN_encodeTiled enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int skinny_bt(int T) { return T <= 16 ? 16 : T <= 32 ? 32 : T <= 64 ? 64 : 128; }
+
+struct SkinnyGeom {
+    int tiles, KB, grid, slots;
+    long long total;
+};
+
+SkinnyGeom skinny_geom(int rows_w, int K, int num_sms) {
+    SkinnyGeom g;
+    g.tiles = (rows_w + 255) / 256;
+    g.KB = (K + BK - 1) / BK;
+    g.total = (long long)g.tiles * g.KB;
+    g.grid = (int)std::min<long long>(num_sms, g.total);
+    g.slots = 1;
+    for (int t = 0; t < g.tiles; ++t) {
+        const long long b = (long long)t * g.KB, e = b + g.KB - 1;
+        const int c0 = (int)(((b + 1) * g.grid - 1) / g.total), c1 = (int)(((e + 1) * g.grid - 1) / g.total);
+        g.slots = std::max(g.slots, c1 - c0 + 1);
+    }
+    return g;
+}
+
+template <typename K>
+cudaError_t set_smem(K kern, size_t bytes) {
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
+template <int BT, int STAGES>
+cudaError_t launch_skinny_bt(const CUtensorMap &mw, const CUtensorMap &mx, const TcArgs &a, int grid,
+                             cudaStream_t st) {
+    auto kern = tc_skinny_kernel<BT, STAGES>;
+    const size_t smem = smem_bytes<STAGES>(256 * BK * 2, BT * BK * 2);
+    cudaError_t e = set_smem(kern, smem);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(kern, dim3(grid), dim3(NTHREADS), smem, st, mw, mx, a);
+}
+
+// One projection with the skinny tiling.  w: rows_w x K packed weights; x: T x K.
+cudaError_t run_skinny(const void *w, int rows_w, const void *x, int T, int K, int epi, void *out, int out_cols,
+                       float *part, unsigned *cnt, int *status, int num_sms, cudaStream_t st) {
+    const int BT = skinny_bt(T);
+    CUtensorMap mw, mx;
+    if (!make_map(&mw, w, K, rows_w, 256) || !make_map(&mx, x, K, T, BT)) return cudaErrorInvalidValue;
+    const SkinnyGeom g = skinny_geom(rows_w, K, num_sms);
+    TcArgs a{};
+    a.rows_x = T;
+    a.rows_w = rows_w;
+    a.K = K;
+    a.KB = g.KB;
+    a.epi = epi;
+    a.out = static_cast<__nv_bfloat16 *>(out);
+    a.ldo = out_cols;
+    a.out_cols = out_cols;
+    a.total_iters = g.total;
+    a.slots = g.slots;
+    a.part = part;
+    a.tile_cnt = cnt;
+    a.status = status;
+    switch (BT) {
+        case 16: return launch_skinny_bt<16, 6>(mw, mx, a, g.grid, st);
+        case 32: return launch_skinny_bt<32, 6>(mw, mx, a, g.grid, st);
+        case 64: return launch_skinny_bt<64, 5>(mw, mx, a, g.grid, st);
+        default: return launch_skinny_bt<128, 4>(mw, mx, a, g.grid, st);
+    }
+}
+
+cudaError_t run_wide(const void *x, int T, const void *w, int rows_w, int K, int epi, void *out, int out_cols,
+                     int *status, int num_sms, cudaStream_t st) {
+    CUtensorMap mx, mw;
+    if (!make_map(&mx, x, K, T, 128) || !make_map(&mw, w, K, rows_w, 256)) return cudaErrorInvalidValue;
+    TcArgs a{};
+    a.rows_x = T;
+    a.rows_w = rows_w;
+    a.K = K;
+    a.KB = (K + BK - 1) / BK;
+    a.epi = epi;
+    a.out = static_cast<__nv_bfloat16 *>(out);
+    a.ldo = out_cols;
+    a.out_cols = out_cols;
+    a.status = status;
+    const int units = ((T + 127) / 128) * ((rows_w + 255) / 256);
+    const int grid = std::min(units, num_sms);
+    const size_t smem = smem_bytes<kWideStages>(128 * BK * 2, 256 * BK * 2);
+    cudaError_t e = set_smem(tc_wide_kernel, smem);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(tc_wide_kernel, dim3(grid), dim3(NTHREADS), smem, st, mx, mw, a);
+}
+
+int first_epi(int act) {
+    return act == TP_MLP_ACT_SWIGLU ? EPI_H_SWIGLU : act == TP_MLP_ACT_TANH ? EPI_H_TANH : EPI_H_IDENT;
+}
+
+}  // namespace
+
+bool tc_supported(const Problem &p) {
+    return p.dtype == TP_MLP_BF16 && p.d_in % 8 == 0 && p.d_ff % 8 == 0 && p.d_out % 8 == 0 &&
+           (p.act != TP_MLP_ACT_SWIGLU || p.d_ff % 128 == 0) && encode_fn() != nullptr;
+}
+
+size_t tc_counter_slots(const Problem &p) {
+    const long rows1 = w1p_rows(p.d_ff, p.act);
+    return (size_t)((rows1 + 255) / 256 + (p.d_out + 255) / 256);
+}
+
+size_t tc_workspace_bytes(const Problem &p, int num_sms) {
+    if (p.T < 1 || p.T > kTcSkinnyMaxTokens) return 0;
+    const int BT = skinny_bt(p.T);
+    const SkinnyGeom g1 = skinny_geom((int)w1p_rows(p.d_ff, p.act), p.d_in, num_sms);
+    const SkinnyGeom g2 = skinny_geom(p.d_out, p.d_ff, num_sms);
+    const size_t s1 = (size_t)g1.tiles * g1.slots * 256 * BT * 4;
+    const size_t s2 = (size_t)g2.tiles * g2.slots * 256 * BT * 4;
+    return align256(s1 > s2 ? s1 : s2);
+}
+
+cudaError_t launch_tc(const Problem &p, bool skinny, const void *x, const void *w1p, const void *w2p, void *h,
+                      void *out, float *part, unsigned *counters, int *status, int num_sms, cudaStream_t st,
+                      const Marks &marks) {
+    const int rows1 = (int)w1p_rows(p.d_ff, p.act);
+    cudaError_t e;
+    marks.mark(0, st);
+    if (skinny) {
+        unsigned *cnt1 = counters, *cnt2 = counters + (rows1 + 255) / 256;
+        e = run_skinny(w1p, rows1, x, p.T, p.d_in, first_epi(p.act), h, p.d_ff, part, cnt1, status, num_sms, st);
+        if (e != cudaSuccess) return e;
+        marks.mark(1, st);
+        e = run_skinny(w2p, p.d_out, h, p.T, p.d_ff, EPI_OUT, out, p.d_out, part, cnt2, status, num_sms, st);
+    } else {
+        e = run_wide(x, p.T, w1p, rows1, p.d_in, first_epi(p.act), h, p.d_ff, status, num_sms, st);
+        if (e != cudaSuccess) return e;
+        marks.mark(1, st);
+        e = run_wide(h, p.T, w2p, p.d_out, p.d_ff, EPI_OUT, out, p.d_out, status, num_sms, st);
+    }
+    marks.mark(2, st);
+    return e;
+}
+
+}  // namespace tpmlp

@@ -24,6 +24,10 @@ struct tp_mlp_s {
     int plan;            // forced tp_mlp_plan
     int last_plan, last_launches;
     Marks marks;         // timing hook
+    // split-K scratch each token count needs, precomputed at creation:
+    // gemv_part[t] for t = 1..kGemvMaxTokens, tc_part[i] for skinny widths 16/32/64/128
+    size_t gemv_part[kGemvMaxTokens + 1];
+    size_t tc_part[4];
 };
 
 namespace {
@@ -74,10 +78,17 @@ Problem problem_of(const tp_mlp_s *h, int tokens) {
     return p;
 }
 
-// Workspace layout: [counters | H (tokens x d_ff) | split-K partial sums].
+// Workspace layout:
+//   [GEMV counters | tcgen05 tile counters | status word]  (zeroed by set_workspace)
+//   [H: tokens x d_ff]
+//   [split-K partial sums]
+size_t gemv_counters_n(const tp_mlp_s *h) { return gemv_counter_slots(problem_of(h, 1)); }
+size_t tc_counters_n(const tp_mlp_s *h) { return tc_counter_slots(problem_of(h, 1)); }
 size_t counters_bytes(const tp_mlp_s *h) {
-    Problem p = problem_of(h, 1);
-    return align256(gemv_counter_slots(p) * sizeof(unsigned));
+    return align256((gemv_counters_n(h) + tc_counters_n(h) + 1) * sizeof(unsigned));
+}
+int *status_word(const tp_mlp_s *h) {
+    return reinterpret_cast<int *>(static_cast<unsigned *>(h->ws) + gemv_counters_n(h) + tc_counters_n(h));
 }
 size_t h_bytes(const tp_mlp_s *h, int tokens) {
     return align256((size_t)tokens * h->d_ff * elem_bytes(h->dtype));
@@ -86,9 +97,11 @@ size_t h_bytes(const tp_mlp_s *h, int tokens) {
 // workspace sized for max_tokens serves every smaller call too.
 size_t part_bytes(const tp_mlp_s *h, int tokens) {
     size_t m = 0;
-    for (int t = 1; t <= tokens && t <= kGemvMaxTokens; ++t) {
-        const size_t v = gemv_workspace_bytes(problem_of(h, t), h->num_sms);
-        m = v > m ? v : m;
+    for (int t = 1; t <= tokens && t <= kGemvMaxTokens; ++t) m = h->gemv_part[t] > m ? h->gemv_part[t] : m;
+    const int widths[4] = {16, 32, 64, 128};
+    for (int i = 0; i < 4; ++i) {
+        if (tokens >= 1 && (i == 0 || tokens > widths[i - 1]))
+            m = h->tc_part[i] > m ? h->tc_part[i] : m;
     }
     return m;
 }
@@ -176,6 +189,14 @@ int tp_mlp_create(tp_mlp_t *handle, int d_model, int d_ff, int d_out, int tp_deg
     else {
         cudaGetLastError();
         h->num_sms = 148;   // B200; only sizes split-K scratch
+    }
+    h->gemv_part[0] = 0;
+    for (int t = 1; t <= kGemvMaxTokens; ++t)
+        h->gemv_part[t] = t <= max_tokens ? gemv_workspace_bytes(problem_of(h, t), h->num_sms) : 0;
+    const int widths[4] = {16, 32, 64, 128};
+    for (int i = 0; i < 4; ++i) {
+        const int t = widths[i] < max_tokens ? widths[i] : max_tokens;
+        h->tc_part[i] = (i == 0 || max_tokens > widths[i - 1]) ? tc_workspace_bytes(problem_of(h, t), h->num_sms) : 0;
     }
     *handle = h;
     return TP_MLP_OK;
@@ -281,11 +302,21 @@ int tp_mlp_forward_packed(tp_mlp_t h, const void *x, int tokens, const void *pac
     if (!h) return TP_MLP_ERR_INVALID_ARG;
     if (tokens < 0 || tokens > h->max_tokens) return TP_MLP_ERR_SHAPE;
     Problem p = problem_of(h, tokens);
-    // plan choice
+    // plan choice: GEMV for 1..4 tokens, tcgen05 skinny up to 128, tcgen05 wide beyond
     int plan = h->plan;
-    if (plan == TP_MLP_PLAN_AUTO) plan = gemv_supported(p) ? TP_MLP_PLAN_GEMV : TP_MLP_PLAN_SIMT;
-    if (plan == TP_MLP_PLAN_GEMV && !gemv_supported(p) && tokens > 0) return TP_MLP_ERR_UNSUPPORTED;
-    if (plan == TP_MLP_PLAN_TC) return TP_MLP_ERR_UNSUPPORTED;
+    const bool tc_ok = tc_supported(p);
+    if (plan == TP_MLP_PLAN_AUTO) {
+        if (gemv_supported(p)) plan = TP_MLP_PLAN_GEMV;
+        else if (tc_ok) plan = tokens <= kTcSkinnyMaxTokens ? TP_MLP_PLAN_TC_SKINNY : TP_MLP_PLAN_TC_WIDE;
+        else plan = TP_MLP_PLAN_SIMT;
+    } else if (plan == TP_MLP_PLAN_TC) {
+        plan = tokens <= kTcSkinnyMaxTokens ? TP_MLP_PLAN_TC_SKINNY : TP_MLP_PLAN_TC_WIDE;
+    }
+    if (tokens > 0) {
+        if (plan == TP_MLP_PLAN_GEMV && !gemv_supported(p)) return TP_MLP_ERR_UNSUPPORTED;
+        if ((plan == TP_MLP_PLAN_TC_WIDE || plan == TP_MLP_PLAN_TC_SKINNY) && !tc_ok) return TP_MLP_ERR_UNSUPPORTED;
+        if (plan == TP_MLP_PLAN_TC_SKINNY && tokens > kTcSkinnyMaxTokens) return TP_MLP_ERR_UNSUPPORTED;
+    }
     if (tokens == 0) {
         h->last_plan = plan;
         h->last_launches = 0;
@@ -309,6 +340,9 @@ int tp_mlp_forward_packed(tp_mlp_t h, const void *x, int tokens, const void *pac
     if (plan == TP_MLP_PLAN_GEMV) {
         ce = launch_gemv(p, x, w1p, w2p, hbuf, out, part, counters, h->num_sms, st, h->marks,
                          &launches);
+    } else if (plan == TP_MLP_PLAN_TC_WIDE || plan == TP_MLP_PLAN_TC_SKINNY) {
+        ce = launch_tc(p, plan == TP_MLP_PLAN_TC_SKINNY, x, w1p, w2p, hbuf, out, part,
+                       counters + gemv_counters_n(h), status_word(h), h->num_sms, st, h->marks);
     } else {
         ShardPtrs a, b;
         memset(&a, 0, sizeof(a));
@@ -323,9 +357,20 @@ int tp_mlp_forward_packed(tp_mlp_t h, const void *x, int tokens, const void *pac
     return TP_MLP_OK;
 }
 
+int tp_mlp_get_device_status(tp_mlp_t h) {
+    if (!h) return TP_MLP_ERR_INVALID_ARG;
+    if (!h->ws) return TP_MLP_ERR_WORKSPACE;
+    int v = 0;
+    if (cudaMemcpy(&v, status_word(h), sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return TP_MLP_ERR_CUDA;
+    if (v == 0) return TP_MLP_OK;
+    const int zero = 0;
+    if (cudaMemcpy(status_word(h), &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return TP_MLP_ERR_CUDA;
+    return TP_MLP_ERR_TIMEOUT;
+}
+
 int tp_mlp_set_plan(tp_mlp_t h, int plan) {
     if (!h) return TP_MLP_ERR_INVALID_ARG;
-    if (plan < TP_MLP_PLAN_AUTO || plan > TP_MLP_PLAN_TC) return TP_MLP_ERR_INVALID_ARG;
+    if (plan < TP_MLP_PLAN_AUTO || plan > TP_MLP_PLAN_TC_SKINNY) return TP_MLP_ERR_INVALID_ARG;
     h->plan = plan;
     return TP_MLP_OK;
 }

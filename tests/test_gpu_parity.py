@@ -129,7 +129,7 @@ def _expected_packed(p, tp, esize):
 @pytest.mark.parametrize("act", ["tanh", "swiglu", "identity"])
 @pytest.mark.parametrize("tp", [1, 2, 4, 8])
 def test_pack_layout_and_roundtrip_bit_exact(dtype, act, tp):
-    p = inputs.generate(3, 40, 8 * 25 * 2, 24, act, dtype, seed=tp + 10)   # f = 400, ragged 128-blocks
+    p = inputs.generate(3, 40, 400, act, dtype, seed=tp + 10, d_out=24)   # f = 400: ragged 128-blocks
     Ad, Bd, A, Bs = _upload(p, tp, dtype)
     m = _mlp(p, tp, dtype)
     packed = m.pack(Ad, Bd)

@@ -1,0 +1,116 @@
+"""GPU parity of the tcgen05 path (both tilings) against the oracle.
+
+The skinny tiling splits the weight stream evenly over the SMs, so tiles are
+shared between CTAs and finished from fp32 partial slots; the shapes below
+cover whole and split tiles, ragged K, ragged weight rows and token counts
+on both sides of every token-tile width.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from helpers import assert_close, dev
+from tensor_sharded_mlp_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from tensor_sharded_mlp_b200 import build
+    build.build()
+
+
+def B():
+    from tensor_sharded_mlp_b200 import binding
+    return binding
+
+
+def _run(p, tp, plan, max_tokens=None):
+    A, Bs = p.shards(tp)
+    Ad = [dev(a, "bf16") for a in A]
+    Bd = [dev(b, "bf16") for b in Bs]
+    m = B().TpMlp(p.d_in, p.d_ff, tp, p.act, "bf16", max_tokens or p.tokens, d_out=p.d_out)
+    m.set_plan(plan)
+    packed = m.pack(Ad, Bd)
+    out = m.forward_packed(dev(p.x, "bf16"), packed)
+    torch.cuda.synchronize()
+    B().tp_mlp_get_device_status(m.h)
+    return m, out, A, Bs, packed
+
+
+def test_tc_first_small_case():
+    """One small skinny case and one small wide case, run first."""
+    p = inputs.generate(8, 256, 512, "swiglu", "bf16", seed=1, init="fan_in", d_out=256)
+    A, Bs = p.shards(2)
+    ref = oracle.tp_mlp_sharded(p.x, A, Bs, "swiglu")
+    for plan in ("tc_skinny", "tc_wide"):
+        m, out, _, _, _ = _run(p, 2, plan)
+        assert m.last_plan == plan
+        assert_close(out, ref, "bf16", plan)
+
+
+@pytest.mark.parametrize("plan,T", [("tc_skinny", 1), ("tc_skinny", 16), ("tc_skinny", 33),
+                                    ("tc_wide", 1), ("tc_wide", 130)])
+def test_tc_integer_exact(plan, T):
+    """Small integers: tensor-core fp32 sums are exact, so the only rounding is
+    the final bf16 one -> GPU == round_to_bf16(oracle) bit for bit."""
+    p = inputs.integer_inputs(T, 64, 256, 264, "identity", seed=T, lo=-1, hi=1)
+    A, Bs = p.shards(4)
+    ref = oracle.tp_mlp_sharded(p.x, A, Bs, "identity")
+    _, out, _, _, _ = _run(p, 4, plan)
+    assert np.array_equal(out.float().cpu().numpy(), inputs.round_to_bf16(ref.astype(np.float32)))
+
+
+SHAPES = [  # (d_in, d_ff, d_out, tp)
+    (512, 1024, 384, 4),
+    (520, 384, 264, 2),     # ragged K (not a multiple of 64) and ragged output rows
+    (4096, 1024, 256, 8),   # long K: tiles split across CTAs
+    (256, 8192, 512, 8),    # long second projection K
+]
+
+
+@pytest.mark.parametrize("act", ["swiglu", "tanh", "identity"])
+@pytest.mark.parametrize("T", [1, 5, 16, 17, 32, 33, 64, 100, 128])
+@pytest.mark.parametrize("shape", SHAPES)
+def test_tc_skinny_parity(act, T, shape):
+    d, f, dout, tp = shape
+    p = inputs.generate(T, d, f, act, "bf16", seed=T + f, init="fan_in", d_out=dout)
+    A, Bs = p.shards(tp)
+    ref = oracle.tp_mlp_sharded(p.x, A, Bs, act)
+    m, out, _, _, packed = _run(p, tp, "tc_skinny")
+    assert m.last_plan == "tc_skinny"
+    assert_close(out, ref, "bf16", f"skinny T={T}")
+    again = m.forward_packed(dev(p.x, "bf16"), packed)   # tile counters were reset
+    assert torch.equal(out, again)
+
+
+@pytest.mark.parametrize("act", ["swiglu", "tanh"])
+@pytest.mark.parametrize("T", [1, 127, 128, 129, 300, 1000])
+@pytest.mark.parametrize("shape", SHAPES[:3])
+def test_tc_wide_parity(act, T, shape):
+    d, f, dout, tp = shape
+    p = inputs.generate(T, d, f, act, "bf16", seed=T + d, init="fan_in", d_out=dout)
+    A, Bs = p.shards(tp)
+    rows = p.sample_rows(64)
+    ref = oracle.tp_mlp_sharded(p.x[rows], A, Bs, act)
+    m, out, _, _, _ = _run(p, tp, "tc_wide")
+    assert m.last_plan == "tc_wide"
+    assert_close(out[torch.from_numpy(rows).cuda()], ref, "bf16", f"wide T={T}")
+
+
+def test_auto_plan_uses_tensor_cores():
+    p = inputs.generate(300, 256, 512, "swiglu", "bf16", seed=2)
+    A, Bs = p.shards(2)
+    m = B().TpMlp(256, 512, 2, "swiglu", "bf16", max_tokens=300)
+    packed = m.pack([dev(a, "bf16") for a in A], [dev(b, "bf16") for b in Bs])
+    x = dev(p.x, "bf16")
+    m.forward_packed(x[:32], packed)
+    assert m.last_plan == "tc_skinny"
+    m.forward_packed(x, packed)
+    assert m.last_plan == "tc_wide"
+    m.forward_packed(x[:2], packed)
+    assert m.last_plan == "gemv"
