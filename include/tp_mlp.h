@@ -204,6 +204,37 @@ int tp_mlp_get_device_status(tp_mlp_t handle);
 int tp_mlp_last_plan(tp_mlp_t handle);
 int tp_mlp_last_launches(tp_mlp_t handle);
 
+/*
+ * Decode forward that allocates nothing and needs no workspace.
+ *
+ * The pages have no counterpart of this call; it exists for callers that
+ * cannot allocate device memory (code inside host callbacks or allocator
+ * hooks, plugins whose host owns every allocation, sandboxes that forbid
+ * cudaMalloc), so they cannot provide the workspace the other calls need.
+ * It computes what tp_mlp_forward_packed computes with the GEMV kernels --
+ * bf16 only, 1..4 tokens -- but keeps the intermediate activation and the
+ * split-K scratch in one fixed 8 MiB array of device memory built into the
+ * library, which every GPU that loads the library holds until the process
+ * exits.
+ *   d_model, d_ff, d_out, tp_degree, act   describe the MLP as for tp_mlp_create
+ *   x       device, tokens x d_model bf16
+ *   packed  device, the buffer tp_mlp_pack wrote for this shape (bf16)
+ *   out     device, tokens x d_out bf16
+ * The caller still owns x, packed and out.  The first call on each device
+ * looks up that device's copy of the array (with the device current); make
+ * that first call before capturing a stream.  Every call shares the array and
+ * leaves its contents behind; each call clears, on its stream, the parts that
+ * must start at zero.  Calls whose kernels overlap on the GPU race on the
+ * array: order them on one stream or with events.
+ * Errors: TP_MLP_ERR_WORKSPACE if this shape needs more scratch than the
+ * 8 MiB array holds (nothing is launched); TP_MLP_ERR_UNSUPPORTED for shapes
+ * the GEMV kernels do not take (d_model or d_ff not a multiple of 8);
+ * otherwise as tp_mlp_forward_packed.  tokens == 0 is a no-op.
+ */
+int tp_mlp_decode_forward_static(int d_model, int d_ff, int d_out, int tp_degree, int act,
+                                 const void *x, int tokens, const void *packed, void *out,
+                                 tp_mlp_stream_t stream);
+
 /* Human-readable name of a status code (static string). */
 const char *tp_mlp_status_string(int status);
 

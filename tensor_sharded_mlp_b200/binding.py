@@ -53,6 +53,7 @@ _SIGS = {
     "tp_mlp_last_plan": (_i, [_vp]),
     "tp_mlp_last_launches": (_i, [_vp]),
     "tp_mlp_status_string": (ctypes.c_char_p, [_i]),
+    "tp_mlp_decode_forward_static": (_i, [_i, _i, _i, _i, _i, _vp, _i, _vp, _vp, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -186,6 +187,16 @@ def tp_mlp_last_launches(h) -> int:
 
 def tp_mlp_status_string(status: int) -> str:
     return _lib.tp_mlp_status_string(status).decode()
+
+
+def tp_mlp_decode_forward_static(d_model: int, d_ff: int, d_out: int, tp_degree: int, act: str,
+                                 x: torch.Tensor, packed: torch.Tensor, out: torch.Tensor,
+                                 stream=None) -> None:
+    """Decode forward for callers that cannot allocate device memory: its
+    scratch is a fixed array inside the library, so no workspace is passed."""
+    _check("tp_mlp_decode_forward_static",
+           _lib.tp_mlp_decode_forward_static(d_model, d_ff, d_out, tp_degree, ACT[act], _ptr(x), x.shape[0],
+                                             _ptr(packed), _ptr(out), _stream(stream)))
 
 
 # --- convenience wrapper -----------------------------------------------------------
