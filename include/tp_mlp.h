@@ -146,15 +146,20 @@ int tp_mlp_partials(tp_mlp_t handle, const void *x, int tokens, const void *cons
 
 /*
  * Size in bytes of the packed weight buffer (the shard-layout packer's output).
- * Layout (element = the handle's dtype; each part starts 256-byte aligned):
- *   part 1, first projection, K-major: one row of d_model elements per
- *     intermediate feature (a column of A).  tanh / identity: row n holds
- *     A[:, n] for n = 0..d_ff-1 in rank order (n = i*f_s + j).  SwiGLU: the
- *     features go in blocks of 128 (the last block may be shorter, nb rows):
- *     block b holds the nb gate rows of features 128b.. then their nb up rows.
- *   part 2, second projection, K-major: row c (0..d_out-1) holds column c of
- *     B, i.e. d_ff elements B[k][c] with k running over rank 0's rows, then
- *     rank 1's, and so on -- so one K loop over a row sums the ranks.
+ * The buffer has two parts, each a matrix of R "rows" by K, one row per output
+ * of its projection (element = the handle's dtype):
+ *   part 1, first projection, K = d_model: tanh / identity: row n holds column
+ *     n of A (n = i*f_s + j over ranks i in order), R = d_ff.  SwiGLU: row
+ *     256*b + r holds the gate column of feature 128*b + r and row 256*b + 128
+ *     + r its up column (r < 128), R = 256 * ceil(d_ff / 128).
+ *   part 2, second projection, K = d_ff: row c holds column c of B, i.e.
+ *     B[k][c] with k over rank 0's rows, then rank 1's, ... (R = d_out), so one
+ *     K loop along a row sums the ranks.
+ * Each part is stored tile-blocked: rows in tiles of 256, K in blocks of 64;
+ * element (row, k) is at ((row/256 * ceil(K/64) + k/64) * 256 + row%256) * 64
+ * + k%64, so every 256 x 64 block is contiguous and the blocks of a tile follow
+ * each other.  Unused rows and k positions are zero.  Part 2 starts at the
+ * first 256-byte boundary after part 1.
  */
 size_t tp_mlp_packed_bytes(tp_mlp_t handle);
 

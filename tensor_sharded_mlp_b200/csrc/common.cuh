@@ -57,18 +57,38 @@ __device__ __forceinline__ float activate(int act, float u, float v) {
     return u;
 }
 
-// --- packed-layout index maps (shard-layout packer) ----------------------------
-// Row of the K-major first-projection part holding feature n (0 <= n < d_ff);
-// `up` selects the up row of a SwiGLU feature.
-__host__ __device__ __forceinline__ long w1p_row(int n, bool up, int d_ff, int act) {
+// --- packed layout (shard-layout packer) --------------------------------------------
+// Each part of the packed buffer is a matrix of "rows" (one per output of its
+// projection) by K, stored tile-blocked: rows in tiles of kTileRows, K in
+// blocks of kKBlock, block (tile, kb) = kTileRows x kKBlock elements stored
+// contiguously (row-major inside), blocks of one tile consecutive in kb, tiles
+// consecutive.  So a tile x k-block is one contiguous piece (32 KB in bf16)
+// and a run of consecutive (tile, kb) pairs is one contiguous range of memory.
+// Padding (rows past the end, k past the end, absent SwiGLU features) is zero.
+constexpr int kTileRows = 256;
+constexpr int kKBlock = 64;
+
+// Row of the first-projection part holding feature n (0 <= n < d_ff); `up`
+// selects the up row of a SwiGLU feature.  SwiGLU: tile b holds the gate rows
+// of features 128b..128b+127 in rows 0..127 and their up rows in rows 128..255.
+__host__ __device__ __forceinline__ long w1p_row(int n, bool up, int act) {
     if (act != TP_MLP_ACT_SWIGLU) return n;
     const int b = n / kSwigluBlock;
-    const int r = n - b * kSwigluBlock;
-    const int nb = min(kSwigluBlock, d_ff - b * kSwigluBlock);
-    return 2L * kSwigluBlock * b + (up ? nb : 0) + r;
+    return (long)kTileRows * b + (up ? kSwigluBlock : 0) + (n - b * kSwigluBlock);
 }
+// Logical rows of the first-projection part.
 __host__ __device__ __forceinline__ long w1p_rows(int d_ff, int act) {
-    return act == TP_MLP_ACT_SWIGLU ? 2L * d_ff : (long)d_ff;
+    return act == TP_MLP_ACT_SWIGLU ? (long)kTileRows * ((d_ff + kSwigluBlock - 1) / kSwigluBlock) : (long)d_ff;
+}
+__host__ __device__ __forceinline__ long blk_tiles(long rows) { return (rows + kTileRows - 1) / kTileRows; }
+__host__ __device__ __forceinline__ long blk_kblocks(long K) { return (K + kKBlock - 1) / kKBlock; }
+// Element offset of (row, k) inside a part whose K spans KB blocks.
+__host__ __device__ __forceinline__ long blk_offset(long row, long k, long KB) {
+    return (((row / kTileRows) * KB + k / kKBlock) * kTileRows + (row % kTileRows)) * kKBlock + (k % kKBlock);
+}
+// Elements of a part (padded to whole tiles and k-blocks).
+__host__ __device__ __forceinline__ size_t part_elems(long rows, long K) {
+    return (size_t)blk_tiles(rows) * blk_kblocks(K) * kTileRows * kKBlock;
 }
 __host__ __device__ __forceinline__ size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 

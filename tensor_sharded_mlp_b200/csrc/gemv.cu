@@ -1,309 +1,327 @@
 // gemv.cu -- decode path: the MLP for 1..4 tokens on packed bf16 weights.
 //
-// Decode is memory-bound: every weight is read once per step and each weight
-// feeds only T multiply-adds ("7.4 推理侧并行", §7.4.1: at batch 1 the GEMM
-// degenerates to a GEMV whose time is the weight read).  So these kernels are
-// built to stream the K-major packed weights at HBM speed:
-//   * one warp per output feature ("group"); each lane loads 16 bytes
-//     (8 bf16) of every weight row per step with a non-allocating L1 load,
-//     several steps in flight;
-//   * X (or H) for the block's K chunk is staged once in shared memory as
-//     fp32, permuted so that every lane's 2x16-byte read is conflict-free;
-//   * warp-shuffle reduction of the per-lane sums;
-//   * split-K over blockIdx.y when K is long: each split writes fp32 partial
-//     sums to the workspace and the LAST block to finish a row range (found
-//     with one atomic counter; nothing ever waits) adds the splits in a fixed
-//     order, applies the epilogue and resets the counter.
-// First projection (MODE 0): group n = feature n; rows w1p_row(n) (+ its up
-// row for SwiGLU); H[t][n] = act(.).  Second projection (MODE 1): group c =
-// output column c; one row of d_ff elements whose K loop runs over every
-// rank's rows, so the rank sum happens in the accumulator; out[t][c].
+// Decode is memory-bound: every weight is read once per step and feeds only T
+// multiply-adds ("7.4 推理侧并行", §7.4.1: at batch 1 the GEMM degenerates to a
+// GEMV whose time is the weight read).  These kernels stream the tile-blocked
+// packed weights at HBM speed with CUDA-core arithmetic:
+//   * the weight stream is split evenly over the SMs (streamk.cuh): every CTA
+//     reads one contiguous run of 32 KB blocks (256 rows x 64 k);
+//   * one producer thread moves the blocks into a ring of shared-memory
+//     stages with bulk copies (cp.async.bulk, ~190 KB in flight per SM);
+//   * eight compute warps take 32 rows each; per step a lane reads one
+//     16-byte granule (8 weights) of one row, so a warp reads 512 contiguous
+//     bytes, and multiplies it with the matching 8 activations of each token;
+//   * the 8 lanes that share a row add their sums with warp shuffles;
+//   * a tile shared with other CTAs is finished by the last CTA to arrive,
+//     adding the fp32 partial slots in slot order (no CTA waits on another).
+// First projection: rows are features (SwiGLU: gate rows 0..127 and up rows
+// 128..255 of each tile), H[t][n] = act(.).  Second projection: rows are
+// output columns c with K = d_ff running over every rank's rows, so the sum
+// over ranks happens in the accumulation; out[t][c].
 #include "common.cuh"
 #include "internal.h"
+#include "streamk.cuh"
+#include "tc_ptx.cuh"
 
 namespace tpmlp {
 namespace {
 
-constexpr int WARPS = 8;
-constexpr int NTHR = WARPS * 32;
-constexpr int KSTEP = 256;   // elements one warp covers per load step (32 lanes x 8)
+using namespace tc;
+
+constexpr int CWARPS = 8;                    // compute warps
+constexpr int NTHR = (CWARPS + 1) * 32;      // + one producer warp
+constexpr int STAGES = 6;
+constexpr uint32_t BLK_BYTES = kTileRows * kKBlock * 2;   // 32 KB
+
+enum { MODE_FIRST = 0, MODE_SECOND = 1 };
 
 struct GemvArgs {
-    const __nv_bfloat16 *w;   // packed rows
-    long ldw;                 // row length (elements) = K
-    const __nv_bfloat16 *x;   // T x K activations (row-major, row stride K)
-    int K;
-    int Kc;                   // K chunk per split, a multiple of KSTEP
-    int S;                    // splits
-    int groups;               // output features
-    int gpb;                  // groups per block
-    int act, d_ff;            // for the first projection's row map / epilogue
-    __nv_bfloat16 *out;       // T x groups
-    float *part;              // S x groups x R x T partial sums (S > 1)
-    unsigned *counters;       // one per blockIdx.x, zero between launches
+    const __nv_bfloat16 *w;   // packed part (tile-blocked)
+    const __nv_bfloat16 *x;   // T x K activations, row-major
+    int K, KB;
+    long long total;          // tiles * KB
+    int slots;
+    int mode, act;
+    int out_cols;             // d_ff (H) or d_out
+    __nv_bfloat16 *out;       // T x out_cols
+    float *part;              // [tile][slot][T][256] fp32
+    unsigned *tile_cnt;       // k-blocks done per tile, zero between launches
+    int *status;
 };
 
-// Position of element k (0 <= k < Kc) of the staged chunk: within each 256-wide
-// step, lane l owns k = 8l..8l+7; its first four go to [l*4], its last four to
-// [128 + l*4], so a warp's float4 reads are contiguous.
-__device__ __forceinline__ int xs_pos(int k) {
-    const int step = k / KSTEP, w = k % KSTEP;
-    const int lane = w >> 3, half = (w >> 2) & 1, e = w & 3;
-    return step * KSTEP + half * 128 + lane * 4 + e;
+struct GemvSmem {
+    uint8_t *ring;
+    uint64_t *full, *empty;
+    float *rowsum;            // [T][256]
+    volatile int *abort;
+    int *flag;
+};
+
+template <int T>
+__device__ __forceinline__ GemvSmem gemv_carve(uint8_t *raw) {
+    GemvSmem s;
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(raw) + 127) & ~uintptr_t(127));
+    s.ring = base;
+    s.full = reinterpret_cast<uint64_t *>(base + STAGES * BLK_BYTES);
+    s.empty = s.full + STAGES;
+    s.rowsum = reinterpret_cast<float *>(s.empty + STAGES);
+    s.abort = reinterpret_cast<volatile int *>(s.rowsum + T * kTileRows);
+    s.flag = const_cast<int *>(s.abort) + 1;
+    return s;
 }
 
-template <int T, int R>
-__device__ __forceinline__ void fma8(float (&acc)[R][T], const uint4 (&wv)[R], const float4 (&xa)[T],
-                                     const float4 (&xb)[T]) {
+template <int T>
+constexpr size_t gemv_smem_bytes() {
+    return 128 + STAGES * (size_t)BLK_BYTES + 2 * STAGES * 8 + T * kTileRows * 4 + 16;
+}
+
+// Final value of row `row` of tile `tile` for all tokens, from s.rowsum.
+template <int T>
+__device__ __forceinline__ void finish_row(const GemvArgs &a, const GemvSmem &s, int tile, int row) {
+    if (a.mode == MODE_FIRST && a.act == TP_MLP_ACT_SWIGLU) {
+        if (row >= kSwigluBlock) return;
+        const int n = tile * kSwigluBlock + row;
+        if (n >= a.out_cols) return;
 #pragma unroll
-    for (int r = 0; r < R; ++r) {
-        const float w0 = bf16lo(wv[r].x), w1 = bf16hi(wv[r].x), w2 = bf16lo(wv[r].y), w3 = bf16hi(wv[r].y);
-        const float w4 = bf16lo(wv[r].z), w5 = bf16hi(wv[r].z), w6 = bf16lo(wv[r].w), w7 = bf16hi(wv[r].w);
+        for (int t = 0; t < T; ++t)
+            a.out[(long)t * a.out_cols + n] =
+                __float2bfloat16_rn(silu_fast(s.rowsum[t * kTileRows + row]) * s.rowsum[t * kTileRows + row + 128]);
+    } else {
+        const int n = tile * kTileRows + row;
+        if (n >= a.out_cols) return;
 #pragma unroll
         for (int t = 0; t < T; ++t) {
-            float a = acc[r][t];
-            a = fmaf(w0, xa[t].x, a); a = fmaf(w1, xa[t].y, a);
-            a = fmaf(w2, xa[t].z, a); a = fmaf(w3, xa[t].w, a);
-            a = fmaf(w4, xb[t].x, a); a = fmaf(w5, xb[t].y, a);
-            a = fmaf(w6, xb[t].z, a); a = fmaf(w7, xb[t].w, a);
-            acc[r][t] = a;
+            const float v = s.rowsum[t * kTileRows + row];
+            a.out[(long)t * a.out_cols + n] =
+                __float2bfloat16_rn(a.mode == MODE_FIRST ? activate<true>(a.act, v, 0.f) : v);
         }
     }
 }
 
-template <int T, int R, int MODE>
-__device__ __forceinline__ void finish(const GemvArgs &a, int g, const float (&v)[R][T]) {
-#pragma unroll
-    for (int t = 0; t < T; ++t) {
-        float y;
-        if (MODE == 0) y = activate<true>(a.act, v[0][t], R > 1 ? v[R - 1][t] : 0.f);
-        else y = v[0][t];
-        a.out[(long)t * a.groups + g] = __float2bfloat16_rn(y);
-    }
-}
-
-template <int T, int R, int MODE>
-__global__ void __launch_bounds__(NTHR) gemv_kernel(GemvArgs a) {
-    extern __shared__ float4 smem4[];
-    float *xs = reinterpret_cast<float *>(smem4);
-    __shared__ bool s_last;
-    constexpr int U = (R == 1) ? 8 : 4;   // load steps in flight per row
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int s = blockIdx.y;
-    const long kbase = (long)s * a.Kc;
-    const int klen = (int)min((long)a.Kc, (long)a.K - kbase);
-    const int kpad = (klen + KSTEP - 1) / KSTEP * KSTEP;
-
-    const int g0 = blockIdx.x * a.gpb;
-    const int g1 = min(a.groups, g0 + a.gpb);
-    auto rows_of = [&](int g, const __nv_bfloat16 *(&row)[R]) {
-        if (MODE == 0) {
-            row[0] = a.w + w1p_row(g, false, a.d_ff, a.act) * a.ldw + kbase;
-            if (R > 1) row[R - 1] = a.w + w1p_row(g, true, a.d_ff, a.act) * a.ldw + kbase;
-        } else {
-            row[0] = a.w + (long)g * a.ldw + kbase;
+template <int T>
+__global__ void __launch_bounds__(NTHR, 1) gemv_kernel(GemvArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    const GemvSmem s = gemv_carve<T>(smem_raw);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < STAGES; ++i) {
+            mbar_init(smem_u32(&s.full[i]), 1);
+            mbar_init(smem_u32(&s.empty[i]), CWARPS);
         }
-    };
-    auto load_bundle = [&](const __nv_bfloat16 *const (&row)[R], int k0, uint4 (&wv)[U][R]) {
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int k = k0 + u * KSTEP + lane * 8;
-#pragma unroll
-            for (int r = 0; r < R; ++r)
-                wv[u][r] = (k < klen) ? ld_stream_v4(row[r] + k) : make_uint4(0, 0, 0, 0);
-        }
-    };
-
-    // Prologue, independent of the previous kernel: let the next kernel launch,
-    // pull this warp's first rows towards L2 and issue its first weight loads.
-    pdl_allow_dependents();
-    uint4 wv[U][R];
-    {
-        const int g = g0 + warp;
-        if (g < g1) {
-            const __nv_bfloat16 *row[R];
-            rows_of(g, row);
-            if (lane < R) prefetch_l2(row[lane], (uint32_t)klen * 2u);
-            load_bundle(row, 0, wv);
-        }
-    }
-    // X (or H) is produced by the previous kernel: wait for it, then stage
-    // X[:, kbase : kbase + klen] (zero-padded to a whole step) as fp32.
-    pdl_wait_previous();
-    for (int t = 0; t < T; ++t) {
-        const __nv_bfloat16 *xr = a.x + (long)t * a.K + kbase;
-        for (int k = threadIdx.x; k < kpad; k += NTHR)
-            xs[t * kpad + xs_pos(k)] = (k < klen) ? __bfloat162float(xr[k]) : 0.f;
+        *s.abort = 0;
+        fence_barrier_init();
     }
     __syncthreads();
+    pdl_allow_dependents();
 
-    bool first = true;
-    for (int g = g0 + warp; g < g1; g += WARPS) {
-        const __nv_bfloat16 *row[R];
-        rows_of(g, row);
-        float acc[R][T];
-#pragma unroll
-        for (int r = 0; r < R; ++r)
-#pragma unroll
-            for (int t = 0; t < T; ++t) acc[r][t] = 0.f;
+    const long long total = a.total, G = gridDim.x, c = blockIdx.x;
+    const long long it_b = share_begin(c, total, G), it_e = share_begin(c + 1, total, G);
+    const int KB = a.KB;
 
-        for (int k0 = 0; k0 < klen; k0 += KSTEP * U) {
-            if (!first) load_bundle(row, k0, wv);
-            first = false;
+    if (warp == CWARPS) {
+        // producer: weights do not depend on the previous kernel, so start at once
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            const uint8_t *src = reinterpret_cast<const uint8_t *>(a.w) + it_b * (long long)BLK_BYTES;
+            for (long long it = it_b; it < it_e; ++it) {
+                if (!mbar_wait(smem_u32(&s.empty[stage]), phase ^ 1, s.abort)) break;
+                const uint32_t fb = smem_u32(&s.full[stage]);
+                mbar_arrive_expect_tx(fb, BLK_BYTES);
+                bulk_load(smem_u32(s.ring + stage * BLK_BYTES), src, BLK_BYTES, fb);
+                src += BLK_BYTES;
+                if (++stage == STAGES) { stage = 0; phase ^= 1; }
+            }
+        }
+    } else {
+        pdl_wait_previous();   // X and the outputs belong to the previous kernel until it is done
+        const int g = lane & 7;                         // granule (8 k) of the row
+        const int rbase = warp * 32 + (lane >> 3);      // rows rbase + 4j, j = 0..7
+        int stage = 0;
+        uint32_t phase = 0;
+        for (long long it = it_b; it < it_e;) {
+            const int tile = (int)(it / KB);
+            const int kb0 = (int)(it - (long long)tile * KB);
+            const int kb1 = (int)min((long long)KB, it_e - (long long)tile * KB);
+            it = (long long)tile * KB + kb1;
+            float acc[8][T];
 #pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int kk = k0 + u * KSTEP;
-                if (kk >= kpad) break;
-                float4 xa[T], xb[T];
+            for (int j = 0; j < 8; ++j)
+#pragma unroll
+                for (int t = 0; t < T; ++t) acc[j][t] = 0.f;
+            bool ok = true;
+            for (int kb = kb0; kb < kb1; ++kb) {
+                // this lane's 8 activations of every token for k = kb*64 + 8g ..
+                float xv[T][8];
+                const int k = kb * kKBlock + g * 8;
 #pragma unroll
                 for (int t = 0; t < T; ++t) {
-                    const float4 *xp = reinterpret_cast<const float4 *>(xs + t * kpad + kk);
-                    xa[t] = xp[lane];
-                    xb[t] = xp[32 + lane];
+                    if (k < a.K) {   // K is a multiple of 8: a granule is all in or all out
+                        const uint4 w4 = __ldg(reinterpret_cast<const uint4 *>(a.x + (long)t * a.K + k));
+                        xv[t][0] = bf16lo(w4.x); xv[t][1] = bf16hi(w4.x);
+                        xv[t][2] = bf16lo(w4.y); xv[t][3] = bf16hi(w4.y);
+                        xv[t][4] = bf16lo(w4.z); xv[t][5] = bf16hi(w4.z);
+                        xv[t][6] = bf16lo(w4.w); xv[t][7] = bf16hi(w4.w);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) xv[t][i] = 0.f;
+                    }
                 }
-                fma8<T, R>(acc, wv[u], xa, xb);
+                if (!mbar_wait(smem_u32(&s.full[stage]), phase, s.abort)) { ok = false; break; }
+                const uint4 *blk = reinterpret_cast<const uint4 *>(s.ring + stage * BLK_BYTES);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const uint4 wv = blk[(rbase + 4 * j) * 8 + g];
+                    const float w0 = bf16lo(wv.x), w1 = bf16hi(wv.x), w2 = bf16lo(wv.y), w3 = bf16hi(wv.y);
+                    const float w4 = bf16lo(wv.z), w5 = bf16hi(wv.z), w6 = bf16lo(wv.w), w7 = bf16hi(wv.w);
+#pragma unroll
+                    for (int t = 0; t < T; ++t) {
+                        float v = acc[j][t];
+                        v = fmaf(w0, xv[t][0], v); v = fmaf(w1, xv[t][1], v);
+                        v = fmaf(w2, xv[t][2], v); v = fmaf(w3, xv[t][3], v);
+                        v = fmaf(w4, xv[t][4], v); v = fmaf(w5, xv[t][5], v);
+                        v = fmaf(w6, xv[t][6], v); v = fmaf(w7, xv[t][7], v);
+                        acc[j][t] = v;
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&s.empty[stage]));
+                if (++stage == STAGES) { stage = 0; phase ^= 1; }
             }
-        }
+            if (!ok) break;
+            // the 8 lanes of a row hold partial sums of its 8 granules
 #pragma unroll
-        for (int r = 0; r < R; ++r)
+            for (int j = 0; j < 8; ++j)
 #pragma unroll
-            for (int t = 0; t < T; ++t) {
-                float v = acc[r][t];
+                for (int t = 0; t < T; ++t) {
+                    float v = acc[j][t];
+                    v += __shfl_xor_sync(0xffffffffu, v, 1);
+                    v += __shfl_xor_sync(0xffffffffu, v, 2);
+                    v += __shfl_xor_sync(0xffffffffu, v, 4);
+                    acc[j][t] = v;
+                }
+            if (g == 0) {
 #pragma unroll
-                for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-                acc[r][t] = v;
+                for (int j = 0; j < 8; ++j)
+#pragma unroll
+                    for (int t = 0; t < T; ++t) s.rowsum[t * kTileRows + rbase + 4 * j] = acc[j][t];
             }
-        if (lane == 0) {
-            if (a.S == 1) {
-                finish<T, R, MODE>(a, g, acc);
+            named_bar(1, CWARPS * 32);
+            const int row = threadIdx.x;   // 0..255: one row per compute thread
+            if (kb0 == 0 && kb1 == KB) {
+                finish_row<T>(a, s, tile, row);
             } else {
-                float *dst = a.part + (((long)s * a.groups + g) * R) * T;
+                const int c_first = share_owner((long long)tile * KB, total, G);
+                const int c_last = share_owner((long long)tile * KB + KB - 1, total, G);
+                float *mine = a.part + ((long long)tile * a.slots + ((int)c - c_first)) * T * kTileRows;
 #pragma unroll
-                for (int r = 0; r < R; ++r)
+                for (int t = 0; t < T; ++t) mine[t * kTileRows + row] = s.rowsum[t * kTileRows + row];
+                __threadfence();
+                named_bar(1, CWARPS * 32);
+                if (threadIdx.x == 0) {
+                    const unsigned done = atomicAdd(&a.tile_cnt[tile], (unsigned)(kb1 - kb0)) + (kb1 - kb0);
+                    *s.flag = (done == (unsigned)KB);
+                }
+                named_bar(1, CWARPS * 32);
+                if (*s.flag) {
+                    __threadfence();
+                    const float *tb = a.part + (long long)tile * a.slots * T * kTileRows;
 #pragma unroll
-                    for (int t = 0; t < T; ++t) dst[r * T + t] = acc[r][t];
+                    for (int t = 0; t < T; ++t) {
+                        float v = 0.f;
+                        for (int sl = 0; sl <= c_last - c_first; ++sl)
+                            v += __ldcg(tb + ((long long)sl * T + t) * kTileRows + row);
+                        s.rowsum[t * kTileRows + row] = v;
+                    }
+                    named_bar(1, CWARPS * 32);
+                    finish_row<T>(a, s, tile, row);
+                    if (threadIdx.x == 0) a.tile_cnt[tile] = 0u;
+                }
             }
+            named_bar(1, CWARPS * 32);   // rowsum and the flag are reused by the next tile
         }
     }
-    if (a.S == 1) return;
-
-    // split-K: the last block of this row range to arrive reduces all splits
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        const unsigned prev = atomicAdd(&a.counters[blockIdx.x], 1u);
-        s_last = (prev == (unsigned)(a.S - 1));
-    }
-    __syncthreads();
-    if (!s_last) return;
-    __threadfence();
-    for (int g = g0 + threadIdx.x; g < g1; g += NTHR) {
-        float v[R][T];
-#pragma unroll
-        for (int r = 0; r < R; ++r)
-#pragma unroll
-            for (int t = 0; t < T; ++t) v[r][t] = 0.f;
-        for (int sp = 0; sp < a.S; ++sp) {
-            const float *src = a.part + (((long)sp * a.groups + g) * R) * T;
-#pragma unroll
-            for (int r = 0; r < R; ++r)
-#pragma unroll
-                for (int t = 0; t < T; ++t) v[r][t] += __ldcg(src + r * T + t);
+    if (*s.abort) {
+        // a bounded wait gave up: let bulk copies in flight land before the CTA exits
+        if (threadIdx.x == 0) {
+            const unsigned long long t0 = globaltimer();
+            while (globaltimer() - t0 < 100000ull) {
+            }
+            atomicExch(a.status, 1);
         }
-        finish<T, R, MODE>(a, g, v);
     }
-    if (threadIdx.x == 0) a.counters[blockIdx.x] = 0u;
+    __syncthreads();
 }
 
-template <int T, int R, int MODE>
-cudaError_t launch_one(const GemvArgs &a, cudaStream_t st) {
-    const size_t smem = (size_t)T * a.Kc * sizeof(float);
-    auto kern = gemv_kernel<T, R, MODE>;
+StreamKGeom gemv_geom(long long rows, int K, int num_sms) {
+    return streamk_geom(blk_tiles(rows), blk_kblocks(K), num_sms);
+}
+
+template <int T>
+cudaError_t launch_one(const GemvArgs &a, int grid, cudaStream_t st) {
+    constexpr size_t smem = gemv_smem_bytes<T>();
+    auto kern = gemv_kernel<T>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    const dim3 grid((a.groups + a.gpb - 1) / a.gpb, a.S);
-    return launch_pdl(kern, grid, dim3(NTHR), smem, st, a);
+    return launch_pdl(kern, dim3(grid), dim3(NTHR), smem, st, a);
 }
 
-template <int R, int MODE>
-cudaError_t launch_T(int T, const GemvArgs &a, cudaStream_t st) {
+cudaError_t launch_T(int T, const GemvArgs &a, int grid, cudaStream_t st) {
     switch (T) {
-        case 1: return launch_one<1, R, MODE>(a, st);
-        case 2: return launch_one<2, R, MODE>(a, st);
-        case 3: return launch_one<3, R, MODE>(a, st);
-        case 4: return launch_one<4, R, MODE>(a, st);
+        case 1: return launch_one<1>(a, grid, st);
+        case 2: return launch_one<2>(a, grid, st);
+        case 3: return launch_one<3>(a, grid, st);
+        case 4: return launch_one<4>(a, grid, st);
     }
     return cudaErrorInvalidValue;
 }
 
-// Split count: keep the staged chunk <= kSmemBudget and give the grid enough blocks.
-constexpr size_t kSmemBudget = 48 * 1024;
-constexpr int kGpb = 16;
-
-void plan_split(int T, int K, int groups, int num_sms, int &S, int &Kc) {
-    const long steps = (K + KSTEP - 1) / KSTEP;
-    int s_smem = (int)(((size_t)T * steps * KSTEP * sizeof(float) + kSmemBudget - 1) / kSmemBudget);
-    const int blocks = (groups + kGpb - 1) / kGpb;
-    int s_occ = (int)((4L * num_sms + blocks - 1) / blocks);   // >= ~4 blocks per SM
-    S = max(1, max(s_smem, s_occ));
-    S = (int)min((long)S, steps);
-    Kc = (int)(((steps + S - 1) / S) * KSTEP);
-    S = (int)((K + Kc - 1) / Kc);
+cudaError_t run_part(const void *w, long long rows, int K, const void *x, int T, int mode, int act, void *out,
+                     int out_cols, float *part, unsigned *cnt, int *status, int num_sms, cudaStream_t st) {
+    const StreamKGeom g = gemv_geom(rows, K, num_sms);
+    GemvArgs a{};
+    a.w = static_cast<const __nv_bfloat16 *>(w);
+    a.x = static_cast<const __nv_bfloat16 *>(x);
+    a.K = K;
+    a.KB = g.KB;
+    a.total = g.total;
+    a.slots = g.slots;
+    a.mode = mode;
+    a.act = act;
+    a.out_cols = out_cols;
+    a.out = static_cast<__nv_bfloat16 *>(out);
+    a.part = part;
+    a.tile_cnt = cnt;
+    a.status = status;
+    return launch_T(T, a, g.grid, st);
 }
 
 }  // namespace
 
 bool gemv_supported(const Problem &p) {
-    return p.dtype == TP_MLP_BF16 && p.T >= 1 && p.T <= kGemvMaxTokens && p.d_in % 8 == 0 &&
-           p.d_ff % 8 == 0;
+    return p.dtype == TP_MLP_BF16 && p.T >= 1 && p.T <= kGemvMaxTokens && p.d_in % 8 == 0 && p.d_ff % 8 == 0;
 }
 
 size_t gemv_workspace_bytes(const Problem &p, int num_sms) {
     if (!gemv_supported(p)) return 0;
-    int S1, K1, S2, K2;
-    plan_split(p.T, p.d_in, p.d_ff, num_sms, S1, K1);
-    plan_split(p.T, p.d_ff, p.d_out, num_sms, S2, K2);
-    const int R1 = p.act == TP_MLP_ACT_SWIGLU ? 2 : 1;
-    const size_t a = S1 > 1 ? (size_t)S1 * p.d_ff * R1 * p.T * 4 : 0;
-    const size_t b = S2 > 1 ? (size_t)S2 * p.d_out * p.T * 4 : 0;
+    const StreamKGeom g1 = gemv_geom(w1p_rows(p.d_ff, p.act), p.d_in, num_sms);
+    const StreamKGeom g2 = gemv_geom(p.d_out, p.d_ff, num_sms);
+    const size_t a = (size_t)g1.tiles * g1.slots * p.T * kTileRows * 4;
+    const size_t b = (size_t)g2.tiles * g2.slots * p.T * kTileRows * 4;
     return align256(a > b ? a : b);
 }
 
-size_t gemv_counter_slots(const Problem &p) {
-    const int m = p.d_ff > p.d_out ? p.d_ff : p.d_out;
-    return (size_t)(m + kGpb - 1) / kGpb;
-}
-
-cudaError_t launch_gemv(const Problem &p, const void *x, const void *w1p, const void *w2p, void *h,
-                        void *out, float *part, unsigned *counters, int num_sms, cudaStream_t st,
+cudaError_t launch_gemv(const Problem &p, const void *x, const void *w1p, const void *w2p, void *h, void *out,
+                        float *part, unsigned *counters, int *status, int num_sms, cudaStream_t st,
                         const Marks &marks, int *launches) {
-    GemvArgs a{};
-    a.act = p.act;
-    a.d_ff = p.d_ff;
-    a.gpb = kGpb;
-    a.counters = counters;
-    a.part = part;
-    // first projection + activation -> H
-    a.w = static_cast<const __nv_bfloat16 *>(w1p);
-    a.ldw = p.d_in;
-    a.x = static_cast<const __nv_bfloat16 *>(x);
-    a.K = p.d_in;
-    a.groups = p.d_ff;
-    a.out = static_cast<__nv_bfloat16 *>(h);
-    plan_split(p.T, a.K, a.groups, num_sms, a.S, a.Kc);
+    const long long rows1 = w1p_rows(p.d_ff, p.act);
+    unsigned *cnt1 = counters, *cnt2 = counters + blk_tiles(rows1);
     marks.mark(0, st);
-    cudaError_t e = (p.act == TP_MLP_ACT_SWIGLU) ? launch_T<2, 0>(p.T, a, st) : launch_T<1, 0>(p.T, a, st);
+    cudaError_t e = run_part(w1p, rows1, p.d_in, x, p.T, MODE_FIRST, p.act, h, p.d_ff, part, cnt1, status,
+                             num_sms, st);
     if (e != cudaSuccess) return e;
     marks.mark(1, st);
-    // second projection over all ranks' rows (rank sum in the accumulator) -> out
-    a.w = static_cast<const __nv_bfloat16 *>(w2p);
-    a.ldw = p.d_ff;
-    a.x = static_cast<const __nv_bfloat16 *>(h);
-    a.K = p.d_ff;
-    a.groups = p.d_out;
-    a.out = static_cast<__nv_bfloat16 *>(out);
-    plan_split(p.T, a.K, a.groups, num_sms, a.S, a.Kc);
-    e = launch_T<1, 1>(p.T, a, st);
+    e = run_part(w2p, p.d_out, p.d_ff, h, p.T, MODE_SECOND, p.act, out, p.d_out, part, cnt2, status, num_sms, st);
     marks.mark(2, st);
     if (launches) *launches = 2;
     return e;

@@ -30,19 +30,21 @@ size_t packed_total_bytes(const Problem &p);
 cudaError_t launch_pack(const Problem &p, const ShardPtrs &a, const ShardPtrs &b, void *packed,
                         bool unpack, cudaStream_t s);
 
+// Split-tile counters the GEMV and tcgen05 skinny kernels need (one per
+// weight tile of both parts; first part's tiles first).
+size_t tile_counter_slots(const Problem &p);
+
 // gemv.cu: decode path, packed bf16, 1..kGemvMaxTokens tokens.
 constexpr int kGemvMaxTokens = 4;
 bool gemv_supported(const Problem &p);
 size_t gemv_workspace_bytes(const Problem &p, int num_sms);
-size_t gemv_counter_slots(const Problem &p);
-cudaError_t launch_gemv(const Problem &p, const void *x, const void *w1p, const void *w2p, void *h,
-                        void *out, float *part, unsigned *counters, int num_sms, cudaStream_t st,
+cudaError_t launch_gemv(const Problem &p, const void *x, const void *w1p, const void *w2p, void *h, void *out,
+                        float *part, unsigned *counters, int *status, int num_sms, cudaStream_t st,
                         const Marks &marks, int *launches);
 
 // tc_gemm.cu: tcgen05 path, packed bf16.  skinny: tokens <= kTcSkinnyMaxTokens.
 constexpr int kTcSkinnyMaxTokens = 128;
 bool tc_supported(const Problem &p);
-size_t tc_counter_slots(const Problem &p);
 size_t tc_workspace_bytes(const Problem &p, int num_sms);
 cudaError_t launch_tc(const Problem &p, bool skinny, const void *x, const void *w1p, const void *w2p, void *h,
                       void *out, float *part, unsigned *counters, int *status, int num_sms, cudaStream_t st,

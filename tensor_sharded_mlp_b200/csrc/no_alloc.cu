@@ -108,8 +108,9 @@ extern "C" int tp_mlp_decode_forward_static(int d_model, int d_ff, int d_out, in
     int sms = 0;
     if (!device_setup(dev, &scratch, &sms)) return TP_MLP_ERR_CUDA;
 
-    // scratch layout: [split-K counters | H (tokens x d_ff bf16) | split-K partial sums]
-    const size_t cnt_bytes = align256(gemv_counter_slots(p) * sizeof(unsigned));
+    // scratch layout: [split-tile counters | status word | H (tokens x d_ff bf16) | partial sums]
+    const size_t n_cnt = tile_counter_slots(p);
+    const size_t cnt_bytes = align256((n_cnt + 1) * sizeof(unsigned));
     const size_t h_bytes = align256((size_t)tokens * d_ff * 2);
     const size_t part_bytes = gemv_workspace_bytes(p, sms);
     if (cnt_bytes + h_bytes + part_bytes > kStaticScratchBytes) return TP_MLP_ERR_WORKSPACE;
@@ -128,7 +129,8 @@ extern "C" int tp_mlp_decode_forward_static(int d_model, int d_ff, int d_out, in
     Marks none;
     none.n = 0;
     int launches = 0;
-    if (launch_gemv(p, x, packed, w2p, h, out, part, counters, sms, st, none, &launches) != cudaSuccess)
+    int *status = reinterpret_cast<int *>(counters + n_cnt);
+    if (launch_gemv(p, x, packed, w2p, h, out, part, counters, status, sms, st, none, &launches) != cudaSuccess)
         return TP_MLP_ERR_CUDA;
     return TP_MLP_OK;
 }

@@ -4,11 +4,13 @@
 // Shards as the pages define them ("大模型推理系统揭秘（07）", §1.2.2–§1.2.3):
 // rank i holds the column block A[:, i f_s:(i+1) f_s] of the first weight and
 // the row block B[i f_s:(i+1) f_s, :] of the second.  The packed buffer holds
-//   part 1: row w1p_row(n) = column n of A (gate/up interleaved in blocks of 128
-//           features for SwiGLU), d_in elements each;
-//   part 2: row c = column c of B over all ranks' rows in rank order, d_ff each.
-// Both directions are 32x32 tiled transposes through shared memory so that the
-// reads and the writes are coalesced.  Elements are moved as raw bits.
+//   part 1: row w1p_row(n) = column n of A (gate/up paired in 256-row tiles
+//           for SwiGLU), K = d_in;
+//   part 2: row c = column c of B over all ranks' rows in rank order, K = d_ff;
+// each part tile-blocked (common.cuh): 256 rows x 64 k per contiguous block.
+// Packing zeroes the buffer first (padding must read as zero), then both
+// directions are 32x32 tiled transposes through shared memory so that reads
+// and writes are coalesced.  Elements are moved as raw bits.
 #include "common.cuh"
 #include "internal.h"
 
@@ -35,8 +37,8 @@ __device__ __forceinline__ U *shard_addr(const ShardPtrs &sh, const Problem &p, 
 
 template <typename U>
 __device__ __forceinline__ U *packed_addr(U *w1p, U *w2p, const Problem &p, int part, int k, int n) {
-    if (part < 2) return w1p + w1p_row(n, part == 1, p.d_ff, p.act) * (long)p.d_in + k;
-    return w2p + (long)n * p.d_ff + k;
+    if (part < 2) return w1p + blk_offset(w1p_row(n, part == 1, p.act), k, blk_kblocks(p.d_in));
+    return w2p + blk_offset(n, k, blk_kblocks(p.d_ff));
 }
 
 // grid: (ceil(N / 32), ceil(K / 32)), block (32, 8).  K/N of the part:
@@ -78,6 +80,10 @@ cudaError_t run_parts(const Problem &p, const ShardPtrs &a, const ShardPtrs &b, 
     U *w1p = static_cast<U *>(packed);
     U *w2p = reinterpret_cast<U *>(static_cast<char *>(packed) + packed_part2_offset(p));
     const dim3 blk(TILE, ROWS);
+    if (!UNPACK) {
+        cudaError_t e = cudaMemsetAsync(packed, 0, packed_total_bytes(p), s);
+        if (e != cudaSuccess) return e;
+    }
     const int nparts1 = p.act == TP_MLP_ACT_SWIGLU ? 2 : 1;
     for (int part = 0; part < nparts1; ++part) {
         const dim3 g((p.d_ff + TILE - 1) / TILE, (p.d_in + TILE - 1) / TILE);
@@ -92,12 +98,12 @@ cudaError_t run_parts(const Problem &p, const ShardPtrs &a, const ShardPtrs &b, 
 
 size_t packed_part2_offset(const Problem &p) {
     const size_t e = p.dtype == TP_MLP_F32 ? 4 : 2;
-    return align256((size_t)w1p_rows(p.d_ff, p.act) * p.d_in * e);
+    return align256(part_elems(w1p_rows(p.d_ff, p.act), p.d_in) * e);
 }
 
 size_t packed_total_bytes(const Problem &p) {
     const size_t e = p.dtype == TP_MLP_F32 ? 4 : 2;
-    return packed_part2_offset(p) + align256((size_t)p.d_out * p.d_ff * e);
+    return packed_part2_offset(p) + align256(part_elems(p.d_out, p.d_ff) * e);
 }
 
 cudaError_t launch_pack(const Problem &p, const ShardPtrs &a, const ShardPtrs &b, void *packed,

@@ -28,7 +28,7 @@ template <typename E, bool PACKED>
 __device__ __forceinline__ float w1_at(const ShardPtrs &w, const Problem &p, int k, int n, bool up) {
     if (PACKED) {
         const E *base = static_cast<const E *>(w.p[0]);
-        return to_f32(base[w1p_row(n, up, p.d_ff, p.act) * (long)p.d_in + k]);
+        return to_f32(base[blk_offset(w1p_row(n, up, p.act), k, blk_kblocks(p.d_in))]);
     }
     const int shard = n / p.fs;
     const int j = n - shard * p.fs;
@@ -42,7 +42,7 @@ template <typename E, bool PACKED>
 __device__ __forceinline__ float w2_at(const ShardPtrs &w, const Problem &p, int k, int c) {
     if (PACKED) {
         const E *base = static_cast<const E *>(w.p[0]);
-        return to_f32(base[(long)c * p.d_ff + k]);
+        return to_f32(base[blk_offset(c, k, blk_kblocks(p.d_ff))]);
     }
     const int shard = k / p.fs;
     const E *b = static_cast<const E *>(w.p[shard]);

@@ -30,6 +30,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "streamk.cuh"
 #include "tc_ptx.cuh"
 
 namespace tpmlp {
@@ -55,7 +56,7 @@ struct TcArgs {
     // skinny tiling (stream-K)
     long long total_iters;
     int slots;           // partial slots per weight tile
-    float *part;         // [tile][slot][256][BT] fp32
+    float *part;         // [tile][slot][BT][256] fp32 (token-major: coalesced)
     unsigned *tile_cnt;  // k-blocks done per weight tile, zero between launches
     int *status;         // set to 1 if a bounded wait ran out
 };
@@ -199,7 +200,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     const uint32_t fb = smem_u32(&s.full[stage]);
                     mbar_arrive_expect_tx(fb, A_BYTES + B_BYTES);
                     tma_load_2d(smem_u32(s.a + stage * A_BYTES), &tmX, kb * BK, mt * 128, fb);
-                    tma_load_2d(smem_u32(s.b + stage * B_BYTES), &tmW, kb * BK, nt * 256, fb);
+                    tma_load_2d(smem_u32(s.b + stage * B_BYTES), &tmW, 0, (nt * a.KB + kb) * 256, fb);
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
                 }
             }
@@ -253,14 +254,21 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     tmem_ld16(taddr + 16 * j, g);
                     tmem_ld16(taddr + 128 + 16 * j, v);
                     tmem_ld_wait();
-                    if (row_ok) {
-                        uint32_t w[8];
+                    const int col = c0 + 16 * j;
+                    if (row_ok && col < a.out_cols) {
+                        if (col + 16 <= a.out_cols) {
+                            uint32_t w[8];
 #pragma unroll
-                        for (int i = 0; i < 8; ++i)
-                            w[i] = pack_bf16x2(silu_fast(g[2 * i]) * v[2 * i], silu_fast(g[2 * i + 1]) * v[2 * i + 1]);
-                        uint4 *dst = reinterpret_cast<uint4 *>(orow + c0 + 16 * j);
-                        dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-                        dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+                            for (int i = 0; i < 8; ++i)
+                                w[i] = pack_bf16x2(silu_fast(g[2 * i]) * v[2 * i],
+                                                   silu_fast(g[2 * i + 1]) * v[2 * i + 1]);
+                            uint4 *dst = reinterpret_cast<uint4 *>(orow + col);
+                            dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+                            dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+                        } else {
+                            for (int i = 0; i < 16 && col + i < a.out_cols; ++i)
+                                orow[col + i] = __float2bfloat16_rn(silu_fast(g[i]) * v[i]);
+                        }
                     }
                 }
             } else {
@@ -300,20 +308,13 @@ done:
 
 // ================== skinny tiling: 256 weight rows x BT tokens, stream-K ==================
 
-__device__ __forceinline__ long long share_begin(long long c, long long total, long long G) {
-    return c * total / G;
-}
-// CTA whose share holds iteration `it`.
-__device__ __forceinline__ int share_owner(long long it, long long total, long long G) {
-    return (int)(((it + 1) * G - 1) / total);
-}
-
 // Final epilogue of a skinny tile for 16 tokens t0..t0+15: v0 = rows r, v1 = rows 128 + r.
 __device__ __forceinline__ void skinny_final16(const TcArgs &a, int tile, int r, int t0, const float (&v0)[16],
                                                const float (&v1)[16]) {
     const int T = a.rows_x;
     if (a.epi == EPI_H_SWIGLU) {
         const int n = tile * 128 + r;
+        if (n >= a.out_cols) return;
 #pragma unroll
         for (int i = 0; i < 16; ++i)
             if (t0 + i < T) a.out[(long)(t0 + i) * a.ldo + n] = __float2bfloat16_rn(silu_fast(v0[i]) * v1[i]);
@@ -356,7 +357,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     if (!mbar_wait(smem_u32(&s.empty[stage]), phase ^ 1, s.abort)) goto done;
                     const uint32_t fb = smem_u32(&s.full[stage]);
                     mbar_arrive_expect_tx(fb, W_BYTES + X_BYTES);
-                    tma_load_2d(smem_u32(s.a + stage * W_BYTES), &tmW, kb * BK, tile * 256, fb);
+                    tma_load_2d(smem_u32(s.a + stage * W_BYTES), &tmW, 0, (tile * KB + kb) * 256, fb);
                     if (!waited) {   // weights do not depend on the previous kernel; X does
                         pdl_wait_previous();
                         waited = true;
@@ -437,12 +438,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     tmem_ld16(taddr + t0, v0);
                     tmem_ld16(taddr + BT + t0, v1);
                     tmem_ld_wait();
-                    float4 *p0 = reinterpret_cast<float4 *>(base + (long)r * BT + t0);
-                    float4 *p1 = reinterpret_cast<float4 *>(base + (long)(128 + r) * BT + t0);
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        p0[i] = make_float4(v0[4 * i], v0[4 * i + 1], v0[4 * i + 2], v0[4 * i + 3]);
-                        p1[i] = make_float4(v1[4 * i], v1[4 * i + 1], v1[4 * i + 2], v1[4 * i + 3]);
+                    for (int i = 0; i < 16; ++i) {   // token t0+i: 32 lanes store 32 consecutive rows
+                        base[(long)(t0 + i) * 256 + r] = v0[i];
+                        base[(long)(t0 + i) * 256 + 128 + r] = v1[i];
                     }
                 }
                 __threadfence();
@@ -465,8 +464,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                             const float *sb = tb + (long long)sl * 256 * BT;
 #pragma unroll
                             for (int i = 0; i < 16; ++i) {
-                                v0[i] += __ldcg(sb + (long)r * BT + t0 + i);
-                                v1[i] += __ldcg(sb + (long)(128 + r) * BT + t0 + i);
+                                v0[i] += __ldcg(sb + (long)(t0 + i) * 256 + r);
+                                v1[i] += __ldcg(sb + (long)(t0 + i) * 256 + 128 + r);
                             }
                         }
                         skinny_final16(a, tile, r, t0, v0, v1);
@@ -522,26 +521,17 @@ bool make_map(CUtensorMap *m, const void *base, int K, int rows, int box_rows) {
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Packed weight part (tile-blocked): a 2-D view of `blocks` rows of 64 bf16
+// (128 B); one box of 256 rows = one 32 KB (tile, k-block) block.
+bool make_map_blocked(CUtensorMap *m, const void *base, long long rows_w, int K) {
+    const long long rows = (long long)blk_tiles(rows_w) * blk_kblocks(K) * kTileRows;
+    return make_map(m, base, kKBlock, (int)rows, kTileRows);
+}
+
 int skinny_bt(int T) { return T <= 16 ? 16 : T <= 32 ? 32 : T <= 64 ? 64 : 128; }
 
-struct SkinnyGeom {
-    int tiles, KB, grid, slots;
-    long long total;
-};
-
-SkinnyGeom skinny_geom(int rows_w, int K, int num_sms) {
-    SkinnyGeom g;
-    g.tiles = (rows_w + 255) / 256;
-    g.KB = (K + BK - 1) / BK;
-    g.total = (long long)g.tiles * g.KB;
-    g.grid = (int)std::min<long long>(num_sms, g.total);
-    g.slots = 1;
-    for (int t = 0; t < g.tiles; ++t) {
-        const long long b = (long long)t * g.KB, e = b + g.KB - 1;
-        const int c0 = (int)(((b + 1) * g.grid - 1) / g.total), c1 = (int)(((e + 1) * g.grid - 1) / g.total);
-        g.slots = std::max(g.slots, c1 - c0 + 1);
-    }
-    return g;
+StreamKGeom skinny_geom(long long rows_w, int K, int num_sms) {
+    return streamk_geom(blk_tiles(rows_w), blk_kblocks(K), num_sms);
 }
 
 template <typename K>
@@ -564,8 +554,8 @@ cudaError_t run_skinny(const void *w, int rows_w, const void *x, int T, int K, i
                        float *part, unsigned *cnt, int *status, int num_sms, cudaStream_t st) {
     const int BT = skinny_bt(T);
     CUtensorMap mw, mx;
-    if (!make_map(&mw, w, K, rows_w, 256) || !make_map(&mx, x, K, T, BT)) return cudaErrorInvalidValue;
-    const SkinnyGeom g = skinny_geom(rows_w, K, num_sms);
+    if (!make_map_blocked(&mw, w, rows_w, K) || !make_map(&mx, x, K, T, BT)) return cudaErrorInvalidValue;
+    const StreamKGeom g = skinny_geom(rows_w, K, num_sms);
     TcArgs a{};
     a.rows_x = T;
     a.rows_w = rows_w;
@@ -591,7 +581,7 @@ cudaError_t run_skinny(const void *w, int rows_w, const void *x, int T, int K, i
 cudaError_t run_wide(const void *x, int T, const void *w, int rows_w, int K, int epi, void *out, int out_cols,
                      int *status, int num_sms, cudaStream_t st) {
     CUtensorMap mx, mw;
-    if (!make_map(&mx, x, K, T, 128) || !make_map(&mw, w, K, rows_w, 256)) return cudaErrorInvalidValue;
+    if (!make_map(&mx, x, K, T, 128) || !make_map_blocked(&mw, w, rows_w, K)) return cudaErrorInvalidValue;
     TcArgs a{};
     a.rows_x = T;
     a.rows_w = rows_w;
@@ -618,19 +608,18 @@ int first_epi(int act) {
 
 bool tc_supported(const Problem &p) {
     return p.dtype == TP_MLP_BF16 && p.d_in % 8 == 0 && p.d_ff % 8 == 0 && p.d_out % 8 == 0 &&
-           (p.act != TP_MLP_ACT_SWIGLU || p.d_ff % 128 == 0) && encode_fn() != nullptr;
+           encode_fn() != nullptr;
 }
 
-size_t tc_counter_slots(const Problem &p) {
-    const long rows1 = w1p_rows(p.d_ff, p.act);
-    return (size_t)((rows1 + 255) / 256 + (p.d_out + 255) / 256);
+size_t tile_counter_slots(const Problem &p) {
+    return (size_t)(blk_tiles(w1p_rows(p.d_ff, p.act)) + blk_tiles(p.d_out));
 }
 
 size_t tc_workspace_bytes(const Problem &p, int num_sms) {
     if (p.T < 1 || p.T > kTcSkinnyMaxTokens) return 0;
     const int BT = skinny_bt(p.T);
-    const SkinnyGeom g1 = skinny_geom((int)w1p_rows(p.d_ff, p.act), p.d_in, num_sms);
-    const SkinnyGeom g2 = skinny_geom(p.d_out, p.d_ff, num_sms);
+    const StreamKGeom g1 = skinny_geom(w1p_rows(p.d_ff, p.act), p.d_in, num_sms);
+    const StreamKGeom g2 = skinny_geom(p.d_out, p.d_ff, num_sms);
     const size_t s1 = (size_t)g1.tiles * g1.slots * 256 * BT * 4;
     const size_t s2 = (size_t)g2.tiles * g2.slots * 256 * BT * 4;
     return align256(s1 > s2 ? s1 : s2);
@@ -643,7 +632,7 @@ cudaError_t launch_tc(const Problem &p, bool skinny, const void *x, const void *
     cudaError_t e;
     marks.mark(0, st);
     if (skinny) {
-        unsigned *cnt1 = counters, *cnt2 = counters + (rows1 + 255) / 256;
+        unsigned *cnt1 = counters, *cnt2 = counters + blk_tiles(rows1);
         e = run_skinny(w1p, rows1, x, p.T, p.d_in, first_epi(p.act), h, p.d_ff, part, cnt1, status, num_sms, st);
         if (e != cudaSuccess) return e;
         marks.mark(1, st);

@@ -79,16 +79,14 @@ Problem problem_of(const tp_mlp_s *h, int tokens) {
 }
 
 // Workspace layout:
-//   [GEMV counters | tcgen05 tile counters | status word]  (zeroed by set_workspace)
+//   [split-tile counters (GEMV and tcgen05 skinny share them) | status word]
+//        (zeroed by set_workspace; the kernels leave the counters at zero)
 //   [H: tokens x d_ff]
-//   [split-K partial sums]
-size_t gemv_counters_n(const tp_mlp_s *h) { return gemv_counter_slots(problem_of(h, 1)); }
-size_t tc_counters_n(const tp_mlp_s *h) { return tc_counter_slots(problem_of(h, 1)); }
-size_t counters_bytes(const tp_mlp_s *h) {
-    return align256((gemv_counters_n(h) + tc_counters_n(h) + 1) * sizeof(unsigned));
-}
+//   [split-tile partial sums]
+size_t tile_counters_n(const tp_mlp_s *h) { return tile_counter_slots(problem_of(h, 1)); }
+size_t counters_bytes(const tp_mlp_s *h) { return align256((tile_counters_n(h) + 1) * sizeof(unsigned)); }
 int *status_word(const tp_mlp_s *h) {
-    return reinterpret_cast<int *>(static_cast<unsigned *>(h->ws) + gemv_counters_n(h) + tc_counters_n(h));
+    return reinterpret_cast<int *>(static_cast<unsigned *>(h->ws) + tile_counters_n(h));
 }
 size_t h_bytes(const tp_mlp_s *h, int tokens) {
     return align256((size_t)tokens * h->d_ff * elem_bytes(h->dtype));
@@ -338,11 +336,11 @@ int tp_mlp_forward_packed(tp_mlp_t h, const void *x, int tokens, const void *pac
     cudaError_t ce;
     int launches = 2;
     if (plan == TP_MLP_PLAN_GEMV) {
-        ce = launch_gemv(p, x, w1p, w2p, hbuf, out, part, counters, h->num_sms, st, h->marks,
+        ce = launch_gemv(p, x, w1p, w2p, hbuf, out, part, counters, status_word(h), h->num_sms, st, h->marks,
                          &launches);
     } else if (plan == TP_MLP_PLAN_TC_WIDE || plan == TP_MLP_PLAN_TC_SKINNY) {
-        ce = launch_tc(p, plan == TP_MLP_PLAN_TC_SKINNY, x, w1p, w2p, hbuf, out, part,
-                       counters + gemv_counters_n(h), status_word(h), h->num_sms, st, h->marks);
+        ce = launch_tc(p, plan == TP_MLP_PLAN_TC_SKINNY, x, w1p, w2p, hbuf, out, part, counters,
+                       status_word(h), h->num_sms, st, h->marks);
     } else {
         ShardPtrs a, b;
         memset(&a, 0, sizeof(a));

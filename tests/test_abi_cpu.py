@@ -69,7 +69,8 @@ def test_header_compiles_as_c(tmp_path, lib):
                     str(src), "-o", str(exe), lib._name, "-Wl,-rpath," + os.path.dirname(lib._name)],
                    check=True)
     out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()
-    assert out[0] == "0" and int(out[1]) == 64 * 256 * 4 + 256 * 64 * 4
+    # part 1: 256 rows x 64 k = one block; part 2: 64 rows padded to a 256-row tile x 4 k-blocks
+    assert out[0] == "0" and int(out[1]) == 256 * 64 * 4 + 256 * 256 * 4
 
 
 def test_create_argument_errors(b):
@@ -97,8 +98,11 @@ def test_sizes_follow_the_documented_layout(b):
                                        ("swiglu", "bf16", 40, 200, 24, 4), ("identity", "bf16", 8, 8, 4, 4)]:
         h = b.tp_mlp_create(d, f, dout, tp, act, dtype, 32)
         e = 4 if dtype == "f32" else 2
-        rows1 = 2 * f if act == "swiglu" else f
-        assert b.tp_mlp_packed_bytes(h) == a256(rows1 * d * e) + a256(dout * f * e)
+        rows1 = 256 * -(-f // 128) if act == "swiglu" else f
+
+        def blocked(R, K):   # whole 256-row tiles x whole 64-wide k-blocks
+            return -(-R // 256) * 256 * -(-K // 64) * 64
+        assert b.tp_mlp_packed_bytes(h) == a256(blocked(rows1, d) * e) + a256(blocked(dout, f) * e)
         w = [b.tp_mlp_workspace_bytes(h, t) for t in range(0, 33)]
         assert all(x > 0 for x in w) and all(w[i] <= w[i + 1] for i in range(32))
         assert w[32] >= 32 * f * e            # holds H

@@ -97,32 +97,39 @@ def test_integer_inputs_bf16_exact_rounding(plan, T):
 
 # --- the shard-layout packer -----------------------------------------------------------
 
+def _blocked(mat, esize):
+    """A part (rows x K) in the tile-blocked order the header documents:
+    256-row tiles, 64-wide k-blocks, each 256 x 64 block contiguous."""
+    R, K = mat.shape
+    tiles, kbs = -(-R // 256), -(-K // 64)
+    pad = np.zeros((tiles * 256, kbs * 64), np.float32)
+    pad[:R, :K] = mat
+    blk = np.ascontiguousarray(pad.reshape(tiles, 256, kbs, 64).transpose(0, 2, 1, 3))
+    raw = blk.view(np.uint32) if esize == 4 else (blk.view(np.uint32) >> 16).astype(np.uint16)
+    return np.frombuffer(raw.tobytes(), np.uint8)
+
+
 def _expected_packed(p, tp, esize):
-    """The packed layout as the header documents it, built on the host."""
+    """The packed buffer as the header documents it, built on the host."""
     def a256(v):
         return (v + 255) // 256 * 256
-    f, d, dout = p.d_ff, p.d_in, p.d_out
+    f, d = p.d_ff, p.d_in
     if p.act == "swiglu":
-        rows = []
-        for b0 in range(0, f, 128):
-            nb = min(128, f - b0)
-            rows += [p.gate[:, b0 + r] for r in range(nb)] + [p.up[:, b0 + r] for r in range(nb)]
-        part1 = np.stack(rows)
+        nb = -(-f // 128)
+        part1 = np.zeros((256 * nb, d), np.float32)
+        for n in range(f):
+            b, r = divmod(n, 128)
+            part1[256 * b + r] = p.gate[:, n]
+            part1[256 * b + 128 + r] = p.up[:, n]
     else:
         part1 = p.a.T
     part2 = p.b.T          # row c = column c of B over all ranks' rows in rank order
-    dt = np.float32 if esize == 4 else np.uint16
-    def raw(m):
-        m = np.ascontiguousarray(m, dtype=np.float32)
-        return m.view(np.uint32) if esize == 4 else (m.view(np.uint32) >> 16).astype(np.uint16)
-    buf = np.zeros(a256(part1.size * esize) + a256(part2.size * esize), dtype=np.uint8)
-    b1 = raw(part1).tobytes()
-    buf[:len(b1)] = np.frombuffer(b1, np.uint8)
-    off = a256(part1.size * esize)
-    b2 = raw(part2).tobytes()
-    buf[off:off + len(b2)] = np.frombuffer(b2, np.uint8)
-    _ = dt
-    return buf, off, len(b1), len(b2)
+    b1, b2 = _blocked(part1, esize), _blocked(part2, esize)
+    off = a256(b1.size)
+    buf = np.zeros(off + a256(b2.size), np.uint8)
+    buf[:b1.size] = b1
+    buf[off:off + b2.size] = b2
+    return buf, off, b1.size, b2.size
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
