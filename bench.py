@@ -22,7 +22,6 @@ bounded sample of the same workload; under torchrun only rank 0 runs it.
 from __future__ import annotations
 
 import argparse
-import hashlib
 import json
 import os
 import statistics
@@ -88,24 +87,16 @@ def load_peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
-def csrc_hash() -> str:
-    h = hashlib.sha256()
-    d = os.path.join(ROOT, "tensor_sharded_mlp_b200", "csrc")
-    for n in sorted(os.listdir(d)):
-        with open(os.path.join(d, n), "rb") as f:
-            h.update(n.encode() + f.read())
-    return h.hexdigest()[:16]
-
-
 def recorded_traffic(kernel: str, workload: str):
-    """DRAM bytes per launch from a committed ncu summary, if taken on this exact source."""
+    """DRAM bytes per launch from a committed ncu summary, if taken on the current kernel source."""
+    from tensor_sharded_mlp_b200.counts import kernel_source_hash
     path = os.path.join(ROOT, "profiles", "dram_traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         rec = json.load(f)
     e = rec.get(f"{kernel}|{workload}")
-    if not e or e.get("csrc_hash") != csrc_hash():
+    if not e or e.get("source_hash") != kernel_source_hash(kernel.split(":")[0]):
         return None
     return e.get("bytes_per_launch")
 

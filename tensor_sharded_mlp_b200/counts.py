@@ -14,6 +14,9 @@ FLOPs.
 """
 from __future__ import annotations
 
+import hashlib
+import os
+
 ELEM_BYTES = {"f32": 4, "bf16": 2}
 
 
@@ -71,3 +74,22 @@ def columns_per_rank(columns: int, tp: int) -> int:
 def allreduce_bytes(batch: int, seq: int, d_model: int, elem_bytes: int) -> int:
     """Bytes one tensor-parallel all-reduce carries: B * S * d_model * bytes."""
     return batch * seq * d_model * elem_bytes
+
+
+# Source files that define each kernel family (for "was this profile taken on
+# the current kernel?" checks).
+_KERNEL_SOURCES = {
+    "gemv": ["gemv.cu", "common.cuh", "streamk.cuh", "tc_ptx.cuh"],
+    "tc_skinny": ["tc_gemm.cu", "common.cuh", "streamk.cuh", "tc_ptx.cuh"],
+    "tc_wide": ["tc_gemm.cu", "common.cuh", "streamk.cuh", "tc_ptx.cuh"],
+    "simt": ["simt.cu", "common.cuh"],
+}
+
+
+def kernel_source_hash(plan: str) -> str:
+    d = os.path.join(os.path.dirname(os.path.abspath(__file__)), "csrc")
+    h = hashlib.sha256()
+    for n in _KERNEL_SOURCES.get(plan, sorted(os.listdir(d))):
+        with open(os.path.join(d, n), "rb") as f:
+            h.update(n.encode() + f.read())
+    return h.hexdigest()[:16]

@@ -56,7 +56,7 @@ struct TcArgs {
     // skinny tiling (stream-K)
     long long total_iters;
     int slots;           // partial slots per weight tile
-    float *part;         // [tile][slot][BT][256] fp32 (token-major: coalesced)
+    float *part;         // [tile][slot][BT/4][256][4] fp32 (float4 per row and 4 tokens)
     unsigned *tile_cnt;  // k-blocks done per weight tile, zero between launches
     int *status;         // set to 1 if a bounded wait ran out
 };
@@ -427,11 +427,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     skinny_final16(a, tile, r, t0, v0, v1);
                 }
             } else {
-                // this CTA's share of the tile -> its partial slot
+                // this CTA's share of the tile -> its partial slot, laid out
+                // [token/4][row][token%4]: each lane stores float4s, a warp 512 B at a time
                 const int c_first = share_owner((long long)tile * KB, total, G);
                 const int c_last = share_owner((long long)tile * KB + KB - 1, total, G);
                 const int slot = (int)c - c_first;
-                float *base = a.part + ((long long)tile * a.slots + slot) * 256 * BT;
+                float4 *base = reinterpret_cast<float4 *>(a.part + ((long long)tile * a.slots + slot) * 256 * BT);
 #pragma unroll 1
                 for (int t0 = 0; t0 < BT; t0 += 16) {
                     float v0[16], v1[16];
@@ -439,9 +440,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     tmem_ld16(taddr + BT + t0, v1);
                     tmem_ld_wait();
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {   // token t0+i: 32 lanes store 32 consecutive rows
-                        base[(long)(t0 + i) * 256 + r] = v0[i];
-                        base[(long)(t0 + i) * 256 + 128 + r] = v1[i];
+                    for (int q = 0; q < 4; ++q) {
+                        const int qd = t0 / 4 + q;
+                        base[qd * 256 + r] = make_float4(v0[4 * q], v0[4 * q + 1], v0[4 * q + 2], v0[4 * q + 3]);
+                        base[qd * 256 + 128 + r] = make_float4(v1[4 * q], v1[4 * q + 1], v1[4 * q + 2], v1[4 * q + 3]);
                     }
                 }
                 __threadfence();
@@ -453,20 +455,47 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 named_bar(1, 128);
                 if (*s.flag) {
                     __threadfence();
-                    const float *tb = a.part + (long long)tile * a.slots * 256 * BT;
+                    const float4 *tb = reinterpret_cast<const float4 *>(a.part + (long long)tile * a.slots * 256 * BT);
                     const int n = c_last - c_first + 1;
+                    constexpr long SLOT4 = 256L * BT / 4;   // float4s per slot
 #pragma unroll 1
                     for (int t0 = 0; t0 < BT; t0 += 16) {
+                        float4 s0[4], s1[4];
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) s0[q] = s1[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+                        int sl = 0;
+                        for (; sl + 1 < n; sl += 2) {   // two slots' loads in flight together
+                            float4 u0[4], u1[4], w0[4], w1[4];
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) {
+                                const long o = (long)(t0 / 4 + q) * 256 + r;
+                                u0[q] = __ldcg(tb + sl * SLOT4 + o);
+                                u1[q] = __ldcg(tb + sl * SLOT4 + o + 128);
+                                w0[q] = __ldcg(tb + (sl + 1) * SLOT4 + o);
+                                w1[q] = __ldcg(tb + (sl + 1) * SLOT4 + o + 128);
+                            }
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) {
+                                s0[q].x += u0[q].x; s0[q].y += u0[q].y; s0[q].z += u0[q].z; s0[q].w += u0[q].w;
+                                s1[q].x += u1[q].x; s1[q].y += u1[q].y; s1[q].z += u1[q].z; s1[q].w += u1[q].w;
+                                s0[q].x += w0[q].x; s0[q].y += w0[q].y; s0[q].z += w0[q].z; s0[q].w += w0[q].w;
+                                s1[q].x += w1[q].x; s1[q].y += w1[q].y; s1[q].z += w1[q].z; s1[q].w += w1[q].w;
+                            }
+                        }
+                        if (sl < n) {
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) {
+                                const long o = (long)(t0 / 4 + q) * 256 + r;
+                                const float4 u0 = __ldcg(tb + sl * SLOT4 + o), u1 = __ldcg(tb + sl * SLOT4 + o + 128);
+                                s0[q].x += u0.x; s0[q].y += u0.y; s0[q].z += u0.z; s0[q].w += u0.w;
+                                s1[q].x += u1.x; s1[q].y += u1.y; s1[q].z += u1.z; s1[q].w += u1.w;
+                            }
+                        }
                         float v0[16], v1[16];
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) v0[i] = v1[i] = 0.f;
-                        for (int sl = 0; sl < n; ++sl) {
-                            const float *sb = tb + (long long)sl * 256 * BT;
-#pragma unroll
-                            for (int i = 0; i < 16; ++i) {
-                                v0[i] += __ldcg(sb + (long)(t0 + i) * 256 + r);
-                                v1[i] += __ldcg(sb + (long)(t0 + i) * 256 + 128 + r);
-                            }
+                        for (int q = 0; q < 4; ++q) {
+                            v0[4 * q] = s0[q].x; v0[4 * q + 1] = s0[q].y; v0[4 * q + 2] = s0[q].z; v0[4 * q + 3] = s0[q].w;
+                            v1[4 * q] = s1[q].x; v1[4 * q + 1] = s1[q].y; v1[4 * q + 2] = s1[q].z; v1[4 * q + 3] = s1[q].w;
                         }
                         skinny_final16(a, tile, r, t0, v0, v1);
                     }

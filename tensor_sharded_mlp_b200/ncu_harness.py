@@ -15,7 +15,7 @@ open the report (``ncu -i``).  Three kinds of capture, all with
   by the units processed) in profiles/dram_traffic.json for bench.py:
       python -m tensor_sharded_mlp_b200.ncu_harness summarize-list launches.csv --title ... --out ...
       python -m tensor_sharded_mlp_b200.ncu_harness summarize-full prof.ncu-rep --title ... --out ... \
-          [--traffic-key plan:first|config --scale 4.0]
+          [--traffic-key plan:first|config --scale 4.0 --launch 0]
 
 Each summary records the command that produced it.
 """
@@ -24,7 +24,6 @@ from __future__ import annotations
 import argparse
 import collections
 import csv
-import hashlib
 import io
 import json
 import os
@@ -58,15 +57,6 @@ FULL_METRICS = [
     "sm__cycles_elapsed.avg.per_second",
     "dram__cycles_elapsed.avg.per_second",
 ]
-
-
-def _csrc_hash() -> str:
-    h = hashlib.sha256()
-    d = os.path.join(ROOT, "tensor_sharded_mlp_b200", "csrc")
-    for n in sorted(os.listdir(d)):
-        with open(os.path.join(d, n), "rb") as f:
-            h.update(n.encode() + f.read())
-    return h.hexdigest()[:16]
 
 
 def bench_cmd(config: str, extra: list[str]) -> str:
@@ -122,13 +112,13 @@ def _raw(report: str):
     return rows[0], rows[1], rows[2:]
 
 
-def summarize_full(report: str, title: str, cmd: str, traffic_key=None, scale=1.0, note=""):
+def summarize_full(report: str, title: str, cmd: str, traffic_key=None, scale=1.0, note="", launch=0):
     h, units, rows = _raw(report)
     idx = {n: i for i, n in enumerate(h)}
     out = [f"# {title}", "", "One `--set full` capture (clocks not locked).  " + note, "", "Command:", "", "```",
            cmd, "```", ""]
     traffic = None
-    for r in rows:
+    for li, r in enumerate(rows):
         kname = r[idx["Kernel Name"]].split("(")[0]
         out += [f"## `{kname}`", "", "| metric | value | unit |", "|---|---:|---|"]
         for m in FULL_METRICS:
@@ -140,7 +130,8 @@ def summarize_full(report: str, title: str, cmd: str, traffic_key=None, scale=1.
                 u = units[idx[m]]
                 return v * {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9}.get(u, 1)
             rd, wr = val("dram__bytes_read.sum"), val("dram__bytes_write.sum")
-            traffic = (rd + wr) * scale
+            if li == launch:
+                traffic = (rd + wr) * scale
             out += ["", f"DRAM traffic per launch: {(rd + wr) / 1e6:.1f} MB"
                     + (f"; scaled ×{scale:g} to the full workload: {traffic / 1e6:.1f} MB" if scale != 1 else "")]
         except (KeyError, ValueError):
@@ -149,8 +140,9 @@ def summarize_full(report: str, title: str, cmd: str, traffic_key=None, scale=1.
     if traffic_key and traffic is not None:
         path = os.path.join(ROOT, "profiles", "dram_traffic.json")
         rec = json.load(open(path)) if os.path.exists(path) else {}
-        rec[traffic_key] = {"bytes_per_launch": traffic, "csrc_hash": _csrc_hash(), "report": os.path.basename(report),
-                            "scale": scale}
+        from tensor_sharded_mlp_b200.counts import kernel_source_hash
+        rec[traffic_key] = {"bytes_per_launch": traffic, "report": os.path.basename(report), "scale": scale,
+                            "source_hash": kernel_source_hash(traffic_key.split(":")[0])}
         with open(path, "w") as f:
             json.dump(rec, f, indent=1, sort_keys=True)
     return "\n".join(out)
@@ -177,6 +169,7 @@ def main(argv=None):
     p.add_argument("--traffic-key", default=None)
     p.add_argument("--scale", type=float, default=1.0)
     p.add_argument("--note", default="")
+    p.add_argument("--launch", type=int, default=0, help="which captured launch the traffic key takes")
     a = ap.parse_args(argv)
     if a.cmd == "list-cmd":
         print(list_cmd(a))
@@ -185,7 +178,8 @@ def main(argv=None):
     elif a.cmd == "summarize-list":
         open(a.out, "w").write(summarize_list(a.csv, a.title, a.command))
     else:
-        open(a.out, "w").write(summarize_full(a.report, a.title, a.command, a.traffic_key, a.scale, a.note))
+        open(a.out, "w").write(summarize_full(a.report, a.title, a.command, a.traffic_key, a.scale, a.note,
+                                              a.launch))
     return 0
 
 

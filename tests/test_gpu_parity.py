@@ -205,6 +205,8 @@ def test_auto_plan_choice():
     packed = m.pack(Ad, Bd)
     m.forward_packed(dev(p.x[:1], "bf16"), packed)
     assert m.last_plan == "gemv"
+    m.forward_packed(dev(p.x[:3], "bf16"), packed)
+    assert m.last_plan == "tc_skinny"
 
 
 # --- the named workloads at full size ---------------------------------------------------

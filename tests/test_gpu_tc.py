@@ -113,4 +113,6 @@ def test_auto_plan_uses_tensor_cores():
     m.forward_packed(x, packed)
     assert m.last_plan == "tc_wide"
     m.forward_packed(x[:2], packed)
+    assert m.last_plan == "tc_skinny"
+    m.forward_packed(x[:1], packed)
     assert m.last_plan == "gemv"
