@@ -231,18 +231,12 @@ def main():
 
     import numpy as np
     import torch
-    import torch.distributed as dist
 
-    from tensor_sharded_mlp_b200 import binding, counts, inputs
+    from tensor_sharded_mlp_b200 import binding, counts, inputs, replicas
 
-    rank = int(os.environ.get("RANK", 0))
-    world = int(os.environ.get("WORLD_SIZE", 1))
-    local = int(os.environ.get("LOCAL_RANK", 0))
+    rank, world, local = replicas.rank_env()
     torch.cuda.set_device(local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                device_id=torch.device("cuda", local))
+    replicas.init("nccl", torch.device("cuda", local))
     c = resolve(args)
     T, d, f, tp, act, dt = c["tokens"], c["d_model"], c["d_ff"], c["tp"], c["act"], c["dtype"]
     p = inputs.generate(T, d, f, act, dt, c["seed"], c["init"])
@@ -262,8 +256,7 @@ def main():
     torch.cuda.synchronize()
 
     def barrier():
-        if world > 1:
-            dist.barrier()
+        replicas.barrier()
         torch.cuda.synchronize()
 
     K, W = args.steps, max(3, args.warmup)
@@ -300,10 +293,7 @@ def main():
     binding.tp_mlp_set_profile_events(m.h, None)
     barrier()
     kern_ms = [statistics.fmean(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(K)) for j in range(nk)]
-    if world > 1:
-        t = torch.tensor([elapsed_ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = replicas.max_over_ranks(elapsed_ms)
 
     # end to end through the public API with host buffers (pinned), copies inside the region
     e2e = None
@@ -326,17 +316,13 @@ def main():
             stream.synchronize()      # the caller reads the result every step
         e2.record(stream)
         barrier()
-        e2e_ms = s2.elapsed_time(e2)
-        if world > 1:
-            t = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
-        e2e = {"value": world * T * K / (e2e_ms / 1e3), "unit": "tokens/s",
+        e2e_ms = replicas.max_over_ranks(s2.elapsed_time(e2))
+        e2e = {"value": replicas.whole_job_rate(T, K, world, e2e_ms), "unit": "tokens/s",
                "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
                "d2h_bytes_per_step": out_host.numel() * out_host.element_size()}
     sampler.stop()
 
-    value = world * T * K / (elapsed_ms / 1e3)
+    value = replicas.whole_job_rate(T, K, world, elapsed_ms)
     peaks, src = load_peaks()
     # roofline of the dominant kernel (largest share of the step)
     j = int(np.argmax(kern_ms))
@@ -373,9 +359,7 @@ def main():
         line["cpu_baseline"] = oracle_baseline(p, A, Bs, act)
     if rank == 0:
         print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
+    replicas.finish()
     return 0
 
 
