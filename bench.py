@@ -327,7 +327,7 @@ def main():
     # roofline of the dominant kernel (largest share of the step)
     j = int(np.argmax(kern_ms))
     names = ["first projection + activation", "second projection + rank sum"]
-    if plan == "tc":
+    if plan in ("tc_wide", "tc_wide256"):
         bound, unit = "tensor", "TFLOP/s"
         work = counts.gemm1_flops(T, d, f, act) if j == 0 else counts.gemm2_flops(T, f, d)
         achieved = work / (kern_ms[j] / 1e3) / 1e12

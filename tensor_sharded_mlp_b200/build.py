@@ -6,6 +6,9 @@ Each ``csrc/*.cu`` is compiled to an object under ``_build/`` (in parallel) and
 linked into ``tensor_sharded_mlp_b200/libtp_mlp.so`` with the CUDA runtime
 linked statically.  The driver API is reached through the runtime's entry-point
 query, so the library loads on a machine without a GPU driver.
+
+Tuning: ``TPMLP_NVCC_DEFINES`` (e.g. ``-DTPMLP_GEMV_STAGES=4``) adds
+compile-time definitions; the build remembers them and rebuilds when they change.
 """
 from __future__ import annotations
 
@@ -44,8 +47,18 @@ def _deps():
         glob.glob(os.path.join(INCLUDE, "*.h"))
 
 
+STAMP = os.path.join(BUILD, "defines.txt")
+
+
+def _defines() -> list:
+    return os.environ.get("TPMLP_NVCC_DEFINES", "").split()
+
+
 def up_to_date() -> bool:
     if not os.path.exists(LIB):
+        return False
+    old = open(STAMP).read().split() if os.path.exists(STAMP) else []
+    if old != _defines():
         return False
     t = os.path.getmtime(LIB)
     return all(os.path.getmtime(d) <= t for d in _deps())
@@ -56,7 +69,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
         return LIB
     os.makedirs(BUILD, exist_ok=True)
     cc = nvcc()
-    extra = ["-Xptxas", "-v"] if verbose else []
+    extra = (["-Xptxas", "-v"] if verbose else []) + _defines()
 
     def compile_one(src):
         obj = os.path.join(BUILD, os.path.basename(src) + ".o")
@@ -76,6 +89,8 @@ def build(force: bool = False, verbose: bool = False) -> str:
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
     os.replace(tmp, LIB)
+    with open(STAMP, "w") as f:
+        f.write(" ".join(_defines()))
     return LIB
 
 

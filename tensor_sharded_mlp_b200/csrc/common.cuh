@@ -46,13 +46,22 @@ __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w <
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
 // --- activations ---------------------------------------------------------------
-// SiLU(g) = g * sigma(g) = g / (1 + e^{-g}).  Large negative g: e^{-g} -> inf, result -> -0.
+// Precise forms (fp32 path, 1e-5 tolerance): the library's tanhf / expf.
+// SiLU(g) = g * sigma(g) = g / (1 + e^{-g}); large negative g: e^{-g} -> inf, result -> -0.
 __device__ __forceinline__ float silu_precise(float g) { return g / (1.0f + expf(-g)); }
-__device__ __forceinline__ float silu_fast(float g) { return g / (1.0f + __expf(-g)); }
+// Fast forms (bf16 paths, whose H is rounded to bf16 anyway): the hardware
+// tanh approximation (one instruction, relative error about 2^-11, below bf16's
+// 2^-9 rounding), and SiLU through sigma(g) = (1 + tanh(g/2)) / 2.
+__device__ __forceinline__ float tanh_fast(float x) {
+    float y;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float silu_fast(float g) { return g * fmaf(0.5f, tanh_fast(0.5f * g), 0.5f); }
 
 template <bool kFast>
 __device__ __forceinline__ float activate(int act, float u, float v) {
-    if (act == TP_MLP_ACT_TANH) return tanhf(u);
+    if (act == TP_MLP_ACT_TANH) return kFast ? tanh_fast(u) : tanhf(u);
     if (act == TP_MLP_ACT_SWIGLU) return (kFast ? silu_fast(u) : silu_precise(u)) * v;
     return u;
 }

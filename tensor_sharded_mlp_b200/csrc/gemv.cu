@@ -7,7 +7,7 @@
 //   * the weight stream is split evenly over the SMs (streamk.cuh): every CTA
 //     reads one contiguous run of 32 KB blocks (256 rows x 64 k);
 //   * one producer thread moves the blocks into a ring of shared-memory
-//     stages with bulk copies (cp.async.bulk, ~190 KB in flight per SM);
+//     stages with bulk copies (cp.async.bulk, 128 KB in flight per SM);
 //   * eight compute warps take 32 rows each; per step a lane reads one
 //     16-byte granule (8 weights) of one row, so a warp reads 512 contiguous
 //     bytes, and multiplies it with the matching 8 activations of each token;
@@ -30,7 +30,10 @@ using namespace tc;
 
 constexpr int CWARPS = 8;                    // compute warps
 constexpr int NTHR = (CWARPS + 1) * 32;      // + one producer warp
-constexpr int STAGES = 6;
+#ifndef TPMLP_GEMV_STAGES
+#define TPMLP_GEMV_STAGES 4   // 4 measured best on B200: the smaller carve-out leaves L1 room for X/H
+#endif
+constexpr int STAGES = TPMLP_GEMV_STAGES;   // shared-memory ring depth (32 KB per stage)
 constexpr uint32_t BLK_BYTES = kTileRows * kKBlock * 2;   // 32 KB
 
 enum { MODE_FIRST = 0, MODE_SECOND = 1 };

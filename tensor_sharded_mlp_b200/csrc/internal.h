@@ -44,9 +44,11 @@ cudaError_t launch_gemv(const Problem &p, const void *x, const void *w1p, const 
 
 // tc_gemm.cu: tcgen05 path, packed bf16.  skinny: tokens <= kTcSkinnyMaxTokens.
 constexpr int kTcSkinnyMaxTokens = 128;
+constexpr int kTcWide256MinTokens = 2048;   // auto: 256-token tiles from here on
+enum { kTilingSkinny = 0, kTilingWide128 = 1, kTilingWide256 = 2 };
 bool tc_supported(const Problem &p);
 size_t tc_workspace_bytes(const Problem &p, int num_sms);
-cudaError_t launch_tc(const Problem &p, bool skinny, const void *x, const void *w1p, const void *w2p, void *h,
+cudaError_t launch_tc(const Problem &p, int tiling, const void *x, const void *w1p, const void *w2p, void *h,
                       void *out, float *part, unsigned *counters, int *status, int num_sms, cudaStream_t st,
                       const Marks &marks);
 

@@ -62,7 +62,7 @@ struct TcArgs {
 };
 
 __device__ __forceinline__ float act_out(int epi, float u) {
-    if (epi == EPI_H_TANH) return tanhf(u);
+    if (epi == EPI_H_TANH) return tanh_fast(u);
     return u;   // identity / plain output
 }
 
@@ -162,7 +162,12 @@ __device__ __forceinline__ void teardown(const Smem &s, uint32_t tmem_base, int 
     if (threadIdx.x == 0 && *s.abort) atomicExch(status, 1);
 }
 
-// ======================= wide tiling: 128 tokens x 256 weight rows ======================
+// ============ wide tiling: 128*MH tokens x 256 weight rows per tile ============
+// MH = 1: one M=128 MMA per 16-k step, two TMEM accumulator buffers (the
+//         epilogue of one tile overlaps the next tile's MMAs), 4 stages.
+// MH = 2: two M=128 MMAs share every weight tile (256 tokens per tile), so a
+//         FLOP costs a third less operand traffic from L2; the 2 x 256-column
+//         accumulator fills TMEM, so there is one buffer, 3 stages.
 
 __device__ __forceinline__ void wide_tile(int u, int MT, int NT, int &mt, int &nt) {
     const int per_group = kGroupM * NT;
@@ -173,18 +178,86 @@ __device__ __forceinline__ void wide_tile(int u, int MT, int NT, int &mt, int &n
     mt = g * kGroupM + r % gm;
 }
 
+template <int MH>
+struct WideCfg {
+    static constexpr int STAGES = MH == 1 ? kWideStages : 3;
+    static constexpr int NACC = MH == 1 ? 2 : 1;          // TMEM accumulator buffers
+    static constexpr uint32_t A_BYTES = 128 * MH * BK * 2;
+    static constexpr uint32_t B_BYTES = 256 * BK * 2;
+};
+
+// Epilogue of one 128-token half: TMEM lanes = tokens, columns 0..255 = weight rows.
+__device__ __forceinline__ void wide_epilogue_half(const TcArgs &a, int row, int nt, uint32_t taddr) {
+    const bool row_ok = row < a.rows_x;
+    __nv_bfloat16 *orow = a.out + (long)row * a.ldo;
+    if (a.epi == EPI_H_SWIGLU) {
+        // columns 0..127 = gate rows, 128..255 = up rows of features 128*nt ..
+        const int c0 = nt * 128;
+#pragma unroll 1
+        for (int j = 0; j < 8; ++j) {
+            float g[16], v[16];
+            tmem_ld16(taddr + 16 * j, g);
+            tmem_ld16(taddr + 128 + 16 * j, v);
+            tmem_ld_wait();
+            const int col = c0 + 16 * j;
+            if (row_ok && col < a.out_cols) {
+                if (col + 16 <= a.out_cols) {
+                    uint32_t w[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        w[i] = pack_bf16x2(silu_fast(g[2 * i]) * v[2 * i], silu_fast(g[2 * i + 1]) * v[2 * i + 1]);
+                    uint4 *dst = reinterpret_cast<uint4 *>(orow + col);
+                    dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+                    dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)   // unrolled so g and v stay in registers
+                        if (col + i < a.out_cols) orow[col + i] = __float2bfloat16_rn(silu_fast(g[i]) * v[i]);
+                }
+            }
+        }
+    } else {
+        const int c0 = nt * 256;
+#pragma unroll 1
+        for (int j = 0; j < 16; ++j) {
+            float v[16];
+            tmem_ld16(taddr + 16 * j, v);
+            tmem_ld_wait();
+            const int col = c0 + 16 * j;
+            if (row_ok && col < a.out_cols) {
+                if (col + 16 <= a.out_cols) {
+                    uint32_t w[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        w[i] = pack_bf16x2(act_out(a.epi, v[2 * i]), act_out(a.epi, v[2 * i + 1]));
+                    uint4 *dst = reinterpret_cast<uint4 *>(orow + col);
+                    dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+                    dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        if (col + i < a.out_cols) orow[col + i] = __float2bfloat16_rn(act_out(a.epi, v[i]));
+                }
+            }
+        }
+    }
+}
+
+template <int MH>
 __global__ void __launch_bounds__(NTHREADS, 1)
     tc_wide_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW, TcArgs a) {
-    constexpr int STAGES = kWideStages;
-    constexpr uint32_t A_BYTES = 128 * BK * 2;   // X tile: 128 tokens
-    constexpr uint32_t B_BYTES = 256 * BK * 2;   // W tile: 256 rows
+    using C = WideCfg<MH>;
+    constexpr int STAGES = C::STAGES;
+    constexpr int NACC = C::NACC;
+    constexpr uint32_t A_BYTES = C::A_BYTES;   // X tile: 128*MH tokens
+    constexpr uint32_t B_BYTES = C::B_BYTES;   // W tile: 256 rows
     extern __shared__ uint8_t smem_raw[];
     const Smem s = carve<STAGES>(smem_raw, A_BYTES, B_BYTES);
     const uint32_t tmem_base = setup<STAGES>(s, &tmX, &tmW);
     pdl_allow_dependents();
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int MT = (a.rows_x + 127) / 128, NT = (a.rows_w + 255) / 256;
+    const int MT = (a.rows_x + 128 * MH - 1) / (128 * MH), NT = (a.rows_w + 255) / 256;
     const int units = MT * NT;
 
     if (warp == 0) {
@@ -199,7 +272,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     if (!mbar_wait(smem_u32(&s.empty[stage]), phase ^ 1, s.abort)) goto done;
                     const uint32_t fb = smem_u32(&s.full[stage]);
                     mbar_arrive_expect_tx(fb, A_BYTES + B_BYTES);
-                    tma_load_2d(smem_u32(s.a + stage * A_BYTES), &tmX, kb * BK, mt * 128, fb);
+                    tma_load_2d(smem_u32(s.a + stage * A_BYTES), &tmX, kb * BK, mt * 128 * MH, fb);
                     tma_load_2d(smem_u32(s.b + stage * B_BYTES), &tmW, 0, (nt * a.KB + kb) * 256, fb);
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
                 }
@@ -213,25 +286,28 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             for (int u = blockIdx.x; u < units; u += gridDim.x) {
                 if (!mbar_wait(smem_u32(&s.tempty[acc]), acc_phase ^ 1, s.abort)) goto done;
                 tc_fence_after();
-                const uint32_t d = tmem_base + acc * 256;
+                const uint32_t d = tmem_base + acc * 256 * MH;
                 for (int kb = 0; kb < a.KB; ++kb) {
                     if (!mbar_wait(smem_u32(&s.full[stage]), phase, s.abort)) goto done;
                     tc_fence_after();
-                    const uint64_t da = smem_desc_kmajor_sw128(smem_u32(s.a + stage * A_BYTES));
+                    const uint32_t sa = smem_u32(s.a + stage * A_BYTES);
                     const uint64_t db = smem_desc_kmajor_sw128(smem_u32(s.b + stage * B_BYTES));
 #pragma unroll
-                    for (int k = 0; k < BK / 16; ++k)   // +32 bytes along K = +2 in the address field
-                        mma_bf16(d, da + 2 * k, db + 2 * k, idesc, (kb | k) != 0);
+                    for (int k = 0; k < BK / 16; ++k) {   // +32 bytes along K = +2 in the address field
+#pragma unroll
+                        for (int h = 0; h < MH; ++h)      // token half h: rows 128h.. of the X tile
+                            mma_bf16(d + h * 256, smem_desc_kmajor_sw128(sa + h * 128 * 128) + 2 * k, db + 2 * k,
+                                     idesc, (kb | k) != 0);
+                    }
                     mma_commit(smem_u32(&s.empty[stage]));
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
                 }
                 mma_commit(smem_u32(&s.tfull[acc]));
-                acc ^= 1;
-                if (acc == 0) acc_phase ^= 1;
+                if (++acc == NACC) { acc = 0; acc_phase ^= 1; }
             }
         }
     } else {
-        // epilogue: TMEM lane quadrant q holds tokens 32q..32q+31 of the tile
+        // epilogue: TMEM lane quadrant q holds tokens 32q..32q+31 of each 128-token half
         pdl_wait_previous();   // outputs may still be read by the previous kernel
         const int q = warp & 3;
         int acc = 0;
@@ -241,65 +317,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             wide_tile(u, MT, NT, mt, nt);
             if (!mbar_wait(smem_u32(&s.tfull[acc]), acc_phase, s.abort)) break;
             tc_fence_after();
-            const int row = mt * 128 + q * 32 + lane;
-            const bool row_ok = row < a.rows_x;
-            __nv_bfloat16 *orow = a.out + (long)row * a.ldo;
-            const uint32_t taddr = tmem_base + acc * 256 + ((uint32_t)(q * 32) << 16);
-            if (a.epi == EPI_H_SWIGLU) {
-                // columns 0..127 = gate rows, 128..255 = up rows of features 128*nt ..
-                const int c0 = nt * 128;
 #pragma unroll 1
-                for (int j = 0; j < 8; ++j) {
-                    float g[16], v[16];
-                    tmem_ld16(taddr + 16 * j, g);
-                    tmem_ld16(taddr + 128 + 16 * j, v);
-                    tmem_ld_wait();
-                    const int col = c0 + 16 * j;
-                    if (row_ok && col < a.out_cols) {
-                        if (col + 16 <= a.out_cols) {
-                            uint32_t w[8];
-#pragma unroll
-                            for (int i = 0; i < 8; ++i)
-                                w[i] = pack_bf16x2(silu_fast(g[2 * i]) * v[2 * i],
-                                                   silu_fast(g[2 * i + 1]) * v[2 * i + 1]);
-                            uint4 *dst = reinterpret_cast<uint4 *>(orow + col);
-                            dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-                            dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
-                        } else {
-                            for (int i = 0; i < 16 && col + i < a.out_cols; ++i)
-                                orow[col + i] = __float2bfloat16_rn(silu_fast(g[i]) * v[i]);
-                        }
-                    }
-                }
-            } else {
-                const int c0 = nt * 256;
-#pragma unroll 1
-                for (int j = 0; j < 16; ++j) {
-                    float v[16];
-                    tmem_ld16(taddr + 16 * j, v);
-                    tmem_ld_wait();
-                    const int col = c0 + 16 * j;
-                    if (row_ok && col < a.out_cols) {
-                        if (col + 16 <= a.out_cols) {
-                            uint32_t w[8];
-#pragma unroll
-                            for (int i = 0; i < 8; ++i)
-                                w[i] = pack_bf16x2(act_out(a.epi, v[2 * i]), act_out(a.epi, v[2 * i + 1]));
-                            uint4 *dst = reinterpret_cast<uint4 *>(orow + col);
-                            dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-                            dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
-                        } else {
-                            for (int i = 0; i < 16 && col + i < a.out_cols; ++i)
-                                orow[col + i] = __float2bfloat16_rn(act_out(a.epi, v[i]));
-                        }
-                    }
-                }
-            }
+            for (int h = 0; h < MH; ++h)
+                wide_epilogue_half(a, mt * 128 * MH + h * 128 + q * 32 + lane, nt,
+                                   tmem_base + (acc * MH + h) * 256 + ((uint32_t)(q * 32) << 16));
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&s.tempty[acc]));
-            acc ^= 1;
-            if (acc == 0) acc_phase ^= 1;
+            if (++acc == NACC) { acc = 0; acc_phase ^= 1; }
         }
     }
 done:
@@ -607,10 +632,12 @@ cudaError_t run_skinny(const void *w, int rows_w, const void *x, int T, int K, i
     }
 }
 
+template <int MH>
 cudaError_t run_wide(const void *x, int T, const void *w, int rows_w, int K, int epi, void *out, int out_cols,
                      int *status, int num_sms, cudaStream_t st) {
+    using C = WideCfg<MH>;
     CUtensorMap mx, mw;
-    if (!make_map(&mx, x, K, T, 128) || !make_map_blocked(&mw, w, rows_w, K)) return cudaErrorInvalidValue;
+    if (!make_map(&mx, x, K, T, 128 * MH) || !make_map_blocked(&mw, w, rows_w, K)) return cudaErrorInvalidValue;
     TcArgs a{};
     a.rows_x = T;
     a.rows_w = rows_w;
@@ -621,12 +648,13 @@ cudaError_t run_wide(const void *x, int T, const void *w, int rows_w, int K, int
     a.ldo = out_cols;
     a.out_cols = out_cols;
     a.status = status;
-    const int units = ((T + 127) / 128) * ((rows_w + 255) / 256);
+    const int units = ((T + 128 * MH - 1) / (128 * MH)) * ((rows_w + 255) / 256);
     const int grid = std::min(units, num_sms);
-    const size_t smem = smem_bytes<kWideStages>(128 * BK * 2, 256 * BK * 2);
-    cudaError_t e = set_smem(tc_wide_kernel, smem);
+    const size_t smem = smem_bytes<C::STAGES>(C::A_BYTES, C::B_BYTES);
+    auto kern = tc_wide_kernel<MH>;
+    cudaError_t e = set_smem(kern, smem);
     if (e != cudaSuccess) return e;
-    return launch_pdl(tc_wide_kernel, dim3(grid), dim3(NTHREADS), smem, st, mx, mw, a);
+    return launch_pdl(kern, dim3(grid), dim3(NTHREADS), smem, st, mx, mw, a);
 }
 
 int first_epi(int act) {
@@ -654,9 +682,10 @@ size_t tc_workspace_bytes(const Problem &p, int num_sms) {
     return align256(s1 > s2 ? s1 : s2);
 }
 
-cudaError_t launch_tc(const Problem &p, bool skinny, const void *x, const void *w1p, const void *w2p, void *h,
+cudaError_t launch_tc(const Problem &p, int tiling, const void *x, const void *w1p, const void *w2p, void *h,
                       void *out, float *part, unsigned *counters, int *status, int num_sms, cudaStream_t st,
                       const Marks &marks) {
+    const bool skinny = tiling == kTilingSkinny;
     const int rows1 = (int)w1p_rows(p.d_ff, p.act);
     cudaError_t e;
     marks.mark(0, st);
@@ -667,10 +696,11 @@ cudaError_t launch_tc(const Problem &p, bool skinny, const void *x, const void *
         marks.mark(1, st);
         e = run_skinny(w2p, p.d_out, h, p.T, p.d_ff, EPI_OUT, out, p.d_out, part, cnt2, status, num_sms, st);
     } else {
-        e = run_wide(x, p.T, w1p, rows1, p.d_in, first_epi(p.act), h, p.d_ff, status, num_sms, st);
+        auto wide = tiling == kTilingWide256 ? run_wide<2> : run_wide<1>;
+        e = wide(x, p.T, w1p, rows1, p.d_in, first_epi(p.act), h, p.d_ff, status, num_sms, st);
         if (e != cudaSuccess) return e;
         marks.mark(1, st);
-        e = run_wide(h, p.T, w2p, p.d_out, p.d_ff, EPI_OUT, out, p.d_out, status, num_sms, st);
+        e = wide(h, p.T, w2p, p.d_out, p.d_ff, EPI_OUT, out, p.d_out, status, num_sms, st);
     }
     marks.mark(2, st);
     return e;

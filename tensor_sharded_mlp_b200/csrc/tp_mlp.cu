@@ -305,16 +305,21 @@ int tp_mlp_forward_packed(tp_mlp_t h, const void *x, int tokens, const void *pac
     // the weights as fast and its arithmetic stays hidden; wide beyond 128.
     int plan = h->plan;
     const bool tc_ok = tc_supported(p);
+    auto tc_tiling = [&](int t) {
+        return t <= kTcSkinnyMaxTokens ? TP_MLP_PLAN_TC_SKINNY
+                                       : t < kTcWide256MinTokens ? TP_MLP_PLAN_TC_WIDE : TP_MLP_PLAN_TC_WIDE256;
+    };
     if (plan == TP_MLP_PLAN_AUTO) {
         if (gemv_supported(p) && (tokens <= 1 || !tc_ok)) plan = TP_MLP_PLAN_GEMV;
-        else if (tc_ok) plan = tokens <= kTcSkinnyMaxTokens ? TP_MLP_PLAN_TC_SKINNY : TP_MLP_PLAN_TC_WIDE;
+        else if (tc_ok) plan = tc_tiling(tokens);
         else plan = TP_MLP_PLAN_SIMT;
     } else if (plan == TP_MLP_PLAN_TC) {
-        plan = tokens <= kTcSkinnyMaxTokens ? TP_MLP_PLAN_TC_SKINNY : TP_MLP_PLAN_TC_WIDE;
+        plan = tc_tiling(tokens);
     }
+    const bool is_tc = plan == TP_MLP_PLAN_TC_WIDE || plan == TP_MLP_PLAN_TC_SKINNY || plan == TP_MLP_PLAN_TC_WIDE256;
     if (tokens > 0) {
         if (plan == TP_MLP_PLAN_GEMV && !gemv_supported(p)) return TP_MLP_ERR_UNSUPPORTED;
-        if ((plan == TP_MLP_PLAN_TC_WIDE || plan == TP_MLP_PLAN_TC_SKINNY) && !tc_ok) return TP_MLP_ERR_UNSUPPORTED;
+        if (is_tc && !tc_ok) return TP_MLP_ERR_UNSUPPORTED;
         if (plan == TP_MLP_PLAN_TC_SKINNY && tokens > kTcSkinnyMaxTokens) return TP_MLP_ERR_UNSUPPORTED;
     }
     if (tokens == 0) {
@@ -340,9 +345,11 @@ int tp_mlp_forward_packed(tp_mlp_t h, const void *x, int tokens, const void *pac
     if (plan == TP_MLP_PLAN_GEMV) {
         ce = launch_gemv(p, x, w1p, w2p, hbuf, out, part, counters, status_word(h), h->num_sms, st, h->marks,
                          &launches);
-    } else if (plan == TP_MLP_PLAN_TC_WIDE || plan == TP_MLP_PLAN_TC_SKINNY) {
-        ce = launch_tc(p, plan == TP_MLP_PLAN_TC_SKINNY, x, w1p, w2p, hbuf, out, part, counters,
-                       status_word(h), h->num_sms, st, h->marks);
+    } else if (is_tc) {
+        const int tiling = plan == TP_MLP_PLAN_TC_SKINNY ? kTilingSkinny
+                           : plan == TP_MLP_PLAN_TC_WIDE ? kTilingWide128 : kTilingWide256;
+        ce = launch_tc(p, tiling, x, w1p, w2p, hbuf, out, part, counters, status_word(h), h->num_sms, st,
+                       h->marks);
     } else {
         ShardPtrs a, b;
         memset(&a, 0, sizeof(a));
@@ -370,7 +377,7 @@ int tp_mlp_get_device_status(tp_mlp_t h) {
 
 int tp_mlp_set_plan(tp_mlp_t h, int plan) {
     if (!h) return TP_MLP_ERR_INVALID_ARG;
-    if (plan < TP_MLP_PLAN_AUTO || plan > TP_MLP_PLAN_TC_SKINNY) return TP_MLP_ERR_INVALID_ARG;
+    if (plan < TP_MLP_PLAN_AUTO || plan > TP_MLP_PLAN_TC_WIDE256) return TP_MLP_ERR_INVALID_ARG;
     h->plan = plan;
     return TP_MLP_OK;
 }

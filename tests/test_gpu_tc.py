@@ -116,3 +116,30 @@ def test_auto_plan_uses_tensor_cores():
     assert m.last_plan == "tc_skinny"
     m.forward_packed(x[:1], packed)
     assert m.last_plan == "gemv"
+
+
+@pytest.mark.parametrize("act", ["swiglu", "tanh"])
+@pytest.mark.parametrize("T", [1, 255, 256, 257, 600, 2100])
+@pytest.mark.parametrize("shape", SHAPES[:3])
+def test_tc_wide256_parity(act, T, shape):
+    """256-token tiles (two M=128 MMAs per weight tile, one TMEM buffer)."""
+    d, f, dout, tp = shape
+    p = inputs.generate(T, d, f, act, "bf16", seed=T + 7 * d, init="fan_in", d_out=dout)
+    A, Bs = p.shards(tp)
+    rows = p.sample_rows(64)
+    ref = oracle.tp_mlp_sharded(p.x[rows], A, Bs, act)
+    m, out, _, _, _ = _run(p, tp, "tc_wide256")
+    assert m.last_plan == "tc_wide256"
+    assert_close(out[torch.from_numpy(rows).cuda()], ref, "bf16", f"wide256 T={T}")
+
+
+def test_auto_plan_picks_256_token_tiles_for_long_prompts():
+    p = inputs.generate(2048, 256, 512, "swiglu", "bf16", seed=3)
+    A, Bs = p.shards(2)
+    m = B().TpMlp(256, 512, 2, "swiglu", "bf16", max_tokens=2048)
+    packed = m.pack([dev(a, "bf16") for a in A], [dev(b, "bf16") for b in Bs])
+    x = dev(p.x, "bf16")
+    m.forward_packed(x, packed)
+    assert m.last_plan == "tc_wide256"
+    m.forward_packed(x[:2047], packed)
+    assert m.last_plan == "tc_wide"
