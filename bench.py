@@ -48,6 +48,8 @@ def parse():
     ap.add_argument("--plan", default="auto")
     ap.add_argument("--d-model", type=int, default=None, help="override (small cases for profiling)")
     ap.add_argument("--d-ff", type=int, default=None, help="override (small cases for profiling)")
+    ap.add_argument("--api", choices=["packed", "shard"], default="packed",
+                    help="packed: weights packed once, tp_mlp_forward_packed; shard: tp_mlp_forward on the shards")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
@@ -250,7 +252,11 @@ def main():
     m.set_plan(args.plan)
     Ad, Bd = [up(a) for a in A], [up(b) for b in Bs]
     packed = m.pack(Ad, Bd)
-    del Ad, Bd
+    if args.api == "packed":
+        del Ad, Bd
+        fwd = lambda: m.forward_packed(x, packed, out=out)            # noqa: E731
+    else:
+        fwd = lambda: m.forward(x, Ad, Bd, out=out)                   # noqa: E731
     x = up(p.x)
     out = torch.empty(T, d, dtype=tdt, device="cuda")
     torch.cuda.synchronize()
@@ -261,7 +267,7 @@ def main():
 
     K, W = args.steps, max(3, args.warmup)
     for _ in range(W):
-        m.forward_packed(x, packed, out=out)
+        fwd()
     nk = m.last_launches
     plan = m.last_plan
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)] for _ in range(K)]
@@ -279,7 +285,7 @@ def main():
     t0 = time.perf_counter()
     start.record(stream)
     for i in range(K):
-        m.forward_packed(x, packed, out=out)
+        fwd()
     end.record(stream)
     barrier()
     t1 = time.perf_counter()
@@ -289,37 +295,38 @@ def main():
     # events on the launch stream before, between and after its kernels.
     for i in range(K):
         binding.tp_mlp_set_profile_events(m.h, ev[i])
-        m.forward_packed(x, packed, out=out)
+        fwd()
     binding.tp_mlp_set_profile_events(m.h, None)
     barrier()
     kern_ms = [statistics.fmean(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(K)) for j in range(nk)]
     elapsed_ms = replicas.max_over_ranks(elapsed_ms)
 
-    # end to end through the public API with host buffers (pinned), copies inside the region
+    # end to end through the public API with host buffers (pinned), copies inside
+    # the region: binding.GraphStep replays H2D(x) + forward + D2H(out) as one
+    # CUDA graph and waits for the result every step, as a decode loop must.
     e2e = None
-    if not args.no_e2e:
-        x_host = x.cpu().pin_memory()
-        out_host = torch.empty(out.shape, dtype=tdt).pin_memory()
-        x_dev = torch.empty_like(x)
+    if not args.no_e2e and args.api == "packed":
+        step = binding.GraphStep(m, packed, T)
+        step.x_host.copy_(x.cpu())
         for _ in range(W):
-            x_dev.copy_(x_host, non_blocking=True)
-            m.forward_packed(x_dev, packed, out=out)
-            out_host.copy_(out, non_blocking=True)
-            stream.synchronize()
+            step()
         barrier()
         s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        s2.record(stream)
+        s2.record(step.stream)
         for _ in range(K):
-            x_dev.copy_(x_host, non_blocking=True)
-            m.forward_packed(x_dev, packed, out=out)
-            out_host.copy_(out, non_blocking=True)
-            stream.synchronize()      # the caller reads the result every step
-        e2.record(stream)
-        barrier()
+            step()                    # replay + wait for the result on the host
+        e2.record(step.stream)
+        e2.synchronize()
         e2e_ms = replicas.max_over_ranks(s2.elapsed_time(e2))
+        ref_out = out.cpu()
+        e2e_ok = bool(torch.equal(step.out_host, ref_out))
         e2e = {"value": replicas.whole_job_rate(T, K, world, e2e_ms), "unit": "tokens/s",
-               "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
-               "d2h_bytes_per_step": out_host.numel() * out_host.element_size()}
+               "h2d_bytes_per_step": step.x_host.numel() * step.x_host.element_size(),
+               "d2h_bytes_per_step": step.out_host.numel() * step.out_host.element_size(),
+               "api": "binding.GraphStep (CUDA graph: H2D x, tp_mlp_forward_packed, D2H out, synchronize)",
+               "timer": "CUDA events on the step's stream around K steps, host waits included",
+               "matches_device_result": e2e_ok}
+        del step
     sampler.stop()
 
     value = replicas.whole_job_rate(T, K, world, elapsed_ms)
@@ -351,7 +358,7 @@ def main():
             "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": dt, "data": "synthetic",
             "config": {"workload": c["workload"], "tokens": T, "d_model": d, "d_ff": f, "tp": tp, "act": act,
-                       "plan": plan, "parallelism": "replicas" if world > 1 else "single GPU",
+                       "plan": plan, "api": args.api, "parallelism": "replicas" if world > 1 else "single GPU",
                        "l2": "inputs larger than L2: every step re-reads %.2f GB of weights" % (step_bytes / 1e9)},
             "step_hbm_gbs": step_bytes / (ms / 1e3) / 1e9, "step_tflops": step_flops / (ms / 1e3) / 1e12,
             "roofline": roofline, "gpu_launches": K * nk, "clocks": sampler.summary(), "e2e": e2e}

@@ -290,3 +290,51 @@ class TpMlp:
     @property
     def last_launches(self) -> int:
         return tp_mlp_last_launches(self.h)
+
+
+class GraphStep:
+    """A whole decode/prefill step replayed as one CUDA graph.
+
+    Per call: copy the step's input from a pinned host buffer to the device,
+    run tp_mlp_forward_packed, copy the result back to a pinned host buffer,
+    and wait for it.  Capturing these into a graph once removes the per-kernel
+    launch cost from every later step (the pages put it at 5-10 us per kernel
+    in a decode step, "7.4 推理侧并行" §7.4.2).  The library's calls allocate
+    nothing and take no host-side decisions that change between replays, so
+    they are safe to capture; the handle's workspace and the packed weights
+    must outlive the step.
+
+        step = GraphStep(mlp, packed, tokens)
+        step.x_host.copy_(x)          # or step(x) to copy and run
+        out = step()                  # pinned host tensor, valid until the next call
+    """
+
+    def __init__(self, mlp: "TpMlp", packed: torch.Tensor, tokens: int):
+        dt = mlp.torch_dtype
+        self.mlp, self.packed = mlp, packed
+        self.x_host = torch.zeros(tokens, mlp.d_model, dtype=dt).pin_memory()
+        self.out_host = torch.zeros(tokens, mlp.d_out, dtype=dt).pin_memory()
+        self.x_dev = torch.zeros(tokens, mlp.d_model, dtype=dt, device=mlp.device)
+        self.out_dev = torch.empty(tokens, mlp.d_out, dtype=dt, device=mlp.device)
+        self.stream = torch.cuda.Stream(device=mlp.device)
+        self.stream.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(self.stream):          # warm-up outside capture
+            self._body()
+        self.stream.synchronize()
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph, stream=self.stream):
+            self._body()
+        self.launches = mlp.last_launches
+
+    def _body(self):
+        self.x_dev.copy_(self.x_host, non_blocking=True)
+        self.mlp.forward_packed(self.x_dev, self.packed, out=self.out_dev)
+        self.out_host.copy_(self.out_dev, non_blocking=True)
+
+    def __call__(self, x: Optional[torch.Tensor] = None) -> torch.Tensor:
+        if x is not None:
+            self.x_host.copy_(x)
+        with torch.cuda.stream(self.stream):   # replay() launches on the current stream
+            self.graph.replay()
+        self.stream.synchronize()
+        return self.out_host

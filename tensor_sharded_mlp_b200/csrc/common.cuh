@@ -126,6 +126,23 @@ __device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes) {
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
 
+// cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per kernel and device
+// (a per-device property; repeating it on every launch costs host time).
+// Registry keyed by the kernel's address (host code only).
+bool smem_attr_done(const void *fn, int dev);
+void smem_attr_mark(const void *fn, int dev);
+
+template <typename K>
+cudaError_t ensure_smem_attr(K kern, size_t bytes) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+    const void *fn = reinterpret_cast<const void *>(kern);
+    if (smem_attr_done(fn, dev)) return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e == cudaSuccess) smem_attr_mark(fn, dev);
+    return e;
+}
+
 // Launch with the programmatic-stream-serialization attribute, so the kernel may
 // begin while the previous kernel in the stream drains (it must call
 // pdl_wait_previous() before touching that kernel's outputs).

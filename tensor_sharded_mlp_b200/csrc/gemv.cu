@@ -264,7 +264,7 @@ template <int T>
 cudaError_t launch_one(const GemvArgs &a, int grid, cudaStream_t st) {
     constexpr size_t smem = gemv_smem_bytes<T>();
     auto kern = gemv_kernel<T>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = ensure_smem_attr(kern, smem);
     if (e != cudaSuccess) return e;
     return launch_pdl(kern, dim3(grid), dim3(NTHR), smem, st, a);
 }

@@ -590,7 +590,7 @@ StreamKGeom skinny_geom(long long rows_w, int K, int num_sms) {
 
 template <typename K>
 cudaError_t set_smem(K kern, size_t bytes) {
-    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    return ensure_smem_attr(kern, bytes);
 }
 
 template <int BT, int STAGES>

@@ -9,10 +9,45 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <mutex>
 #include <new>
 
 #include "common.cuh"
 #include "internal.h"
+
+namespace tpmlp {
+
+// Kernels whose dynamic shared-memory limit has been raised, per device.
+namespace {
+std::mutex g_attr_mutex;
+struct AttrEntry {
+    const void *fn;
+    unsigned long long devices;   // bit d: done on device d (d < 64)
+};
+AttrEntry g_attr[64];
+int g_attr_n = 0;
+}  // namespace
+
+bool smem_attr_done(const void *fn, int dev) {
+    if (dev < 0 || dev >= 64) return false;
+    std::lock_guard<std::mutex> lock(g_attr_mutex);
+    for (int i = 0; i < g_attr_n; ++i)
+        if (g_attr[i].fn == fn) return (g_attr[i].devices >> dev) & 1ull;
+    return false;
+}
+
+void smem_attr_mark(const void *fn, int dev) {
+    if (dev < 0 || dev >= 64) return;
+    std::lock_guard<std::mutex> lock(g_attr_mutex);
+    for (int i = 0; i < g_attr_n; ++i)
+        if (g_attr[i].fn == fn) {
+            g_attr[i].devices |= 1ull << dev;
+            return;
+        }
+    if (g_attr_n < 64) g_attr[g_attr_n++] = AttrEntry{fn, 1ull << dev};   // full table: just re-set next time
+}
+
+}  // namespace tpmlp
 
 using namespace tpmlp;
 

@@ -341,3 +341,57 @@ def test_profile_events_bracket_the_kernels():
     b.tp_mlp_set_profile_events(m.h, None)
     torch.cuda.synchronize()
     assert ev[0].elapsed_time(ev[1]) > 0 and ev[1].elapsed_time(ev[2]) > 0
+
+
+def test_graph_step_replays_copies_and_forward():
+    b = B()
+    p = inputs.generate(2, 512, 1024, "swiglu", "bf16", seed=8)
+    A, Bs = p.shards(4)
+    ref = oracle.tp_mlp_sharded(p.x, A, Bs, "swiglu")
+    m = b.TpMlp(512, 1024, 4, "swiglu", "bf16", max_tokens=2)
+    packed = m.pack([dev(a, "bf16") for a in A], [dev(x, "bf16") for x in Bs])
+    step = b.GraphStep(m, packed, 2)
+    x = torch.from_numpy(p.x).to(torch.bfloat16)
+    first = step(x).clone()
+    assert_close(first, ref, "bf16", "graph step")
+    assert torch.equal(first, m.forward_packed(x.cuda(), packed).cpu())
+    # every call must wait for its own result: a new input must show up at once
+    for sign in (-1.0, 1.0, -1.0):
+        step.out_host.fill_(float("nan"))
+        got = step(sign * x)
+        assert torch.isfinite(got.float()).all()
+        want = m.forward_packed((sign * x).cuda(), packed).cpu()
+        assert torch.equal(got, want)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_page_worked_example_shapes(dtype):
+    """"大模型推理系统揭秘（07）" §1.2.3: X in R^{Bx8}, W1 8x8 split by columns into
+    four 8x2 blocks, W2 8x4 split by rows into four 2x4 blocks (d_out = 4 != d_in)."""
+    for act in ("identity", "tanh", "swiglu"):
+        p = inputs.generate(3, 8, 8, act, dtype, seed=11, init="fan_in", d_out=4)
+        A, Bs = p.shards(4)
+        ref = oracle.tp_mlp_sharded(p.x, A, Bs, act)
+        m = B().TpMlp(8, 8, 4, act, dtype, max_tokens=3, d_out=4)
+        Ad, Bd = [dev(a, dtype) for a in A], [dev(b, dtype) for b in Bs]
+        x = dev(p.x, dtype)
+        assert_close(m.forward(x, Ad, Bd), ref, dtype, f"{act} shard form")
+        parts = m.partials(x, Ad, Bd)
+        assert_close(parts.sum(0), ref, dtype, f"{act} partials")
+        packed = m.pack(Ad, Bd)
+        for T in (1, 3):
+            r = oracle.tp_mlp_sharded(p.x[:T], A, Bs, act)
+            assert_close(m.forward_packed(x[:T], packed), r, dtype, f"{act} packed T={T} ({m.last_plan})")
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_one_feature_per_rank(dtype):
+    """Degenerate split: d_ff == tp, so every rank holds a single feature."""
+    p = inputs.generate(5, 16, 8, "tanh", dtype, seed=12, init="fan_in", d_out=24)
+    A, Bs = p.shards(8)
+    assert all(a.shape == (16, 1) for a in A)
+    ref = oracle.tp_mlp_sharded(p.x, A, Bs, "tanh")
+    m = B().TpMlp(16, 8, 8, "tanh", dtype, max_tokens=5, d_out=24)
+    Ad, Bd = [dev(a, dtype) for a in A], [dev(b, dtype) for b in Bs]
+    assert_close(m.forward(dev(p.x, dtype), Ad, Bd), ref, dtype, "shard form")
+    assert_close(m.forward_packed(dev(p.x, dtype), m.pack(Ad, Bd)), ref, dtype, f"packed ({m.last_plan})")
