@@ -129,7 +129,9 @@ int tp_mlp_set_workspace(tp_mlp_t handle, void *dev_ptr, size_t bytes);
  *   act        must equal the handle's
  *   out        device, tokens x d_out
  *   stream     CUDA stream
- * tokens == 0 is a no-op.  Uses the workspace.
+ * tokens == 0 is a no-op.  Uses the workspace.  For bf16 with f_s a multiple
+ * of 64 (and d_model, d_ff, d_out multiples of 8) the tcgen05 kernels read the
+ * shards directly, as MN-major operands; otherwise CUDA-core kernels run.
  */
 int tp_mlp_forward(tp_mlp_t handle, const void *x, int tokens, const void *const *A_shards,
                    const void *const *B_shards, int tp_degree, int act, void *out,

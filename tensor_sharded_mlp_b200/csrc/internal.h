@@ -47,9 +47,11 @@ constexpr int kTcSkinnyMaxTokens = 128;
 constexpr int kTcWide256MinTokens = 2048;   // auto: 256-token tiles from here on
 enum { kTilingSkinny = 0, kTilingWide128 = 1, kTilingWide256 = 2 };
 bool tc_supported(const Problem &p);
+bool tc_raw_supported(const Problem &p);   // also needs f_s % 64 == 0
 size_t tc_workspace_bytes(const Problem &p, int num_sms);
-cudaError_t launch_tc(const Problem &p, int tiling, const void *x, const void *w1p, const void *w2p, void *h,
-                      void *out, float *part, unsigned *counters, int *status, int num_sms, cudaStream_t st,
-                      const Marks &marks);
+// Packed weights (w1p/w2p), or the per-rank shards when rawA/rawB are given.
+cudaError_t launch_tc(const Problem &p, int tiling, const void *x, const void *w1p, const void *w2p,
+                      const ShardPtrs *rawA, const ShardPtrs *rawB, void *h, void *out, float *part,
+                      unsigned *counters, int *status, int num_sms, cudaStream_t st, const Marks &marks);
 
 }  // namespace tpmlp

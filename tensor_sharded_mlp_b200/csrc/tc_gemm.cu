@@ -26,6 +26,8 @@
 // abort flag that every role checks, and the CTA records it in a status word.
 #include <cuda.h>
 
+#include <string.h>
+
 #include <algorithm>
 
 #include "common.cuh"
@@ -59,7 +61,57 @@ struct TcArgs {
     float *part;         // [tile][slot][BT/4][256][4] fp32 (float4 per row and 4 tokens)
     unsigned *tile_cnt;  // k-blocks done per weight tile, zero between launches
     int *status;         // set to 1 if a bounded wait ran out
+    // first projection read straight from the per-rank shards: tile t covers
+    // features of rank t / tps only (tps tiles per rank of fs features)
+    int raw_first, tps, fs;
 };
+
+// Weight operand of one projection, for the producer's TMA loads.
+//   packed: map[0] views the tile-blocked part; one 32 KB box per (tile, k-block).
+//   raw:    per-rank row-major shards; four 64 (columns) x 64 (k rows) boxes per
+//           (tile, k-block).  First projection: map[i] = A_i (tanh) or gate_i,
+//           map[kMaxTp + i] = up_i; a tile is 256 features (tanh) or 128 gate +
+//           the same 128 up features (SwiGLU) of one rank.  Second projection:
+//           map[i] = B_i; a tile is 256 output columns, k-block kb comes from
+//           rank kb / kbps.
+struct WeightMaps {
+    CUtensorMap map[2 * kMaxTp];
+    int first, swiglu, tps, kbps;
+};
+
+template <bool RAW>
+__device__ __forceinline__ void load_w_tile(uint32_t dst, const WeightMaps &wm, int tile, int kb, int KB,
+                                            uint32_t bar) {
+    if (!RAW) {
+        tma_load_2d(dst, &wm.map[0], 0, (tile * KB + kb) * 256, bar);
+        return;
+    }
+    if (wm.first) {
+        const int per = wm.swiglu ? 128 : 256;
+        const int i = tile / wm.tps, n0 = (tile - i * wm.tps) * per;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const CUtensorMap *m = (wm.swiglu && q >= 2) ? &wm.map[kMaxTp + i] : &wm.map[i];
+            const int x = n0 + 64 * (wm.swiglu ? (q & 1) : q);
+            tma_load_2d(dst + q * 8192, m, x, kb * BK, bar);
+        }
+    } else {
+        const int i = kb / wm.kbps, kl = kb - i * wm.kbps;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) tma_load_2d(dst + q * 8192, &wm.map[i], tile * 256 + 64 * q, kl * BK, bar);
+    }
+}
+
+// Output column of element `local` (0 .. per-1) of weight tile `tile`, or -1 when
+// it is padding.  per = 128 for the SwiGLU first projection, 256 otherwise.
+__device__ __forceinline__ int tile_col(const TcArgs &a, int tile, int local, int per) {
+    if (!a.raw_first) {
+        const int n = tile * per + local;
+        return n < a.out_cols ? n : -1;
+    }
+    const int i = tile / a.tps, l = (tile - i * a.tps) * per + local;
+    return l < a.fs ? i * a.fs + l : -1;
+}
 
 __device__ __forceinline__ float act_out(int epi, float u) {
     if (epi == EPI_H_TANH) return tanh_fast(u);
@@ -187,65 +239,42 @@ struct WideCfg {
 };
 
 // Epilogue of one 128-token half: TMEM lanes = tokens, columns 0..255 = weight rows.
+// Output columns come in runs of 16 that are all valid or all padding, except
+// at a packed part's ragged end (handled element by element).
 __device__ __forceinline__ void wide_epilogue_half(const TcArgs &a, int row, int nt, uint32_t taddr) {
     const bool row_ok = row < a.rows_x;
     __nv_bfloat16 *orow = a.out + (long)row * a.ldo;
-    if (a.epi == EPI_H_SWIGLU) {
-        // columns 0..127 = gate rows, 128..255 = up rows of features 128*nt ..
-        const int c0 = nt * 128;
+    const bool swiglu = a.epi == EPI_H_SWIGLU;
+    const int per = swiglu ? 128 : 256;
 #pragma unroll 1
-        for (int j = 0; j < 8; ++j) {
-            float g[16], v[16];
-            tmem_ld16(taddr + 16 * j, g);
-            tmem_ld16(taddr + 128 + 16 * j, v);
-            tmem_ld_wait();
-            const int col = c0 + 16 * j;
-            if (row_ok && col < a.out_cols) {
-                if (col + 16 <= a.out_cols) {
-                    uint32_t w[8];
+    for (int j = 0; j < per / 16; ++j) {
+        float g[16], v[16];
+        tmem_ld16(taddr + 16 * j, g);
+        if (swiglu) tmem_ld16(taddr + 128 + 16 * j, v);
+        tmem_ld_wait();
+        const int col = tile_col(a, nt, 16 * j, per);
+        if (!row_ok || col < 0) continue;
+        float y[16];
 #pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        w[i] = pack_bf16x2(silu_fast(g[2 * i]) * v[2 * i], silu_fast(g[2 * i + 1]) * v[2 * i + 1]);
-                    uint4 *dst = reinterpret_cast<uint4 *>(orow + col);
-                    dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-                    dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
-                } else {
+        for (int i = 0; i < 16; ++i) y[i] = swiglu ? silu_fast(g[i]) * v[i] : act_out(a.epi, g[i]);
+        if (a.raw_first || col + 16 <= a.out_cols) {
+            uint32_t w[8];
 #pragma unroll
-                    for (int i = 0; i < 16; ++i)   // unrolled so g and v stay in registers
-                        if (col + i < a.out_cols) orow[col + i] = __float2bfloat16_rn(silu_fast(g[i]) * v[i]);
-                }
-            }
-        }
-    } else {
-        const int c0 = nt * 256;
-#pragma unroll 1
-        for (int j = 0; j < 16; ++j) {
-            float v[16];
-            tmem_ld16(taddr + 16 * j, v);
-            tmem_ld_wait();
-            const int col = c0 + 16 * j;
-            if (row_ok && col < a.out_cols) {
-                if (col + 16 <= a.out_cols) {
-                    uint32_t w[8];
+            for (int i = 0; i < 8; ++i) w[i] = pack_bf16x2(y[2 * i], y[2 * i + 1]);
+            uint4 *dst = reinterpret_cast<uint4 *>(orow + col);
+            dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+            dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+        } else {
 #pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        w[i] = pack_bf16x2(act_out(a.epi, v[2 * i]), act_out(a.epi, v[2 * i + 1]));
-                    uint4 *dst = reinterpret_cast<uint4 *>(orow + col);
-                    dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-                    dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
-                } else {
-#pragma unroll
-                    for (int i = 0; i < 16; ++i)
-                        if (col + i < a.out_cols) orow[col + i] = __float2bfloat16_rn(act_out(a.epi, v[i]));
-                }
-            }
+            for (int i = 0; i < 16; ++i)   // unrolled so y stays in registers
+                if (col + i < a.out_cols) orow[col + i] = __float2bfloat16_rn(y[i]);
         }
     }
 }
 
-template <int MH>
+template <int MH, bool RAW>
 __global__ void __launch_bounds__(NTHREADS, 1)
-    tc_wide_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW, TcArgs a) {
+    tc_wide_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ WeightMaps wm, TcArgs a) {
     using C = WideCfg<MH>;
     constexpr int STAGES = C::STAGES;
     constexpr int NACC = C::NACC;
@@ -253,11 +282,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     constexpr uint32_t B_BYTES = C::B_BYTES;   // W tile: 256 rows
     extern __shared__ uint8_t smem_raw[];
     const Smem s = carve<STAGES>(smem_raw, A_BYTES, B_BYTES);
-    const uint32_t tmem_base = setup<STAGES>(s, &tmX, &tmW);
+    const uint32_t tmem_base = setup<STAGES>(s, &tmX, &wm.map[0]);
     pdl_allow_dependents();
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int MT = (a.rows_x + 128 * MH - 1) / (128 * MH), NT = (a.rows_w + 255) / 256;
+    const int MT = (a.rows_x + 128 * MH - 1) / (128 * MH), NT = a.rows_w;   // rows_w: weight tiles
     const int units = MT * NT;
 
     if (warp == 0) {
@@ -273,14 +302,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     const uint32_t fb = smem_u32(&s.full[stage]);
                     mbar_arrive_expect_tx(fb, A_BYTES + B_BYTES);
                     tma_load_2d(smem_u32(s.a + stage * A_BYTES), &tmX, kb * BK, mt * 128 * MH, fb);
-                    tma_load_2d(smem_u32(s.b + stage * B_BYTES), &tmW, 0, (nt * a.KB + kb) * 256, fb);
+                    load_w_tile<RAW>(smem_u32(s.b + stage * B_BYTES), wm, nt, kb, a.KB, fb);
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
                 }
             }
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            const uint32_t idesc = idesc_bf16_f32(128, 256);
+            const uint32_t idesc = idesc_bf16_f32(128, 256) | (RAW ? kIdescBMajorMN : 0u);
             int stage = 0, acc = 0;
             uint32_t phase = 0, acc_phase = 0;
             for (int u = blockIdx.x; u < units; u += gridDim.x) {
@@ -291,13 +320,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     if (!mbar_wait(smem_u32(&s.full[stage]), phase, s.abort)) goto done;
                     tc_fence_after();
                     const uint32_t sa = smem_u32(s.a + stage * A_BYTES);
-                    const uint64_t db = smem_desc_kmajor_sw128(smem_u32(s.b + stage * B_BYTES));
+                    const uint32_t sb = smem_u32(s.b + stage * B_BYTES);
+                    // K-major: +32 bytes per 16 k (+2 in the address field); MN-major: +2048 bytes (+128)
+                    const uint64_t db = RAW ? smem_desc_mnmajor_sw128(sb) : smem_desc_kmajor_sw128(sb);
+                    constexpr uint32_t kstep_b = RAW ? 128 : 2;
 #pragma unroll
-                    for (int k = 0; k < BK / 16; ++k) {   // +32 bytes along K = +2 in the address field
+                    for (int k = 0; k < BK / 16; ++k) {
 #pragma unroll
                         for (int h = 0; h < MH; ++h)      // token half h: rows 128h.. of the X tile
-                            mma_bf16(d + h * 256, smem_desc_kmajor_sw128(sa + h * 128 * 128) + 2 * k, db + 2 * k,
-                                     idesc, (kb | k) != 0);
+                            mma_bf16(d + h * 256, smem_desc_kmajor_sw128(sa + h * 128 * 128) + 2 * k,
+                                     db + kstep_b * k, idesc, (kb | k) != 0);
                     }
                     mma_commit(smem_u32(&s.empty[stage]));
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
@@ -338,30 +370,30 @@ __device__ __forceinline__ void skinny_final16(const TcArgs &a, int tile, int r,
                                                const float (&v1)[16]) {
     const int T = a.rows_x;
     if (a.epi == EPI_H_SWIGLU) {
-        const int n = tile * 128 + r;
-        if (n >= a.out_cols) return;
+        const int n = tile_col(a, tile, r, 128);
+        if (n < 0) return;
 #pragma unroll
         for (int i = 0; i < 16; ++i)
             if (t0 + i < T) a.out[(long)(t0 + i) * a.ldo + n] = __float2bfloat16_rn(silu_fast(v0[i]) * v1[i]);
     } else {
-        const int n0 = tile * 256 + r, n1 = n0 + 128;
+        const int n0 = tile_col(a, tile, r, 256), n1 = tile_col(a, tile, r + 128, 256);
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
             if (t0 + i >= T) break;
-            if (n0 < a.out_cols) a.out[(long)(t0 + i) * a.ldo + n0] = __float2bfloat16_rn(act_out(a.epi, v0[i]));
-            if (n1 < a.out_cols) a.out[(long)(t0 + i) * a.ldo + n1] = __float2bfloat16_rn(act_out(a.epi, v1[i]));
+            if (n0 >= 0) a.out[(long)(t0 + i) * a.ldo + n0] = __float2bfloat16_rn(act_out(a.epi, v0[i]));
+            if (n1 >= 0) a.out[(long)(t0 + i) * a.ldo + n1] = __float2bfloat16_rn(act_out(a.epi, v1[i]));
         }
     }
 }
 
-template <int BT, int STAGES>
+template <int BT, int STAGES, bool RAW>
 __global__ void __launch_bounds__(NTHREADS, 1)
-    tc_skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX, TcArgs a) {
+    tc_skinny_kernel(const __grid_constant__ WeightMaps wm, const __grid_constant__ CUtensorMap tmX, TcArgs a) {
     constexpr uint32_t W_BYTES = 256 * BK * 2;   // 256 weight rows (two M=128 halves)
     constexpr uint32_t X_BYTES = BT * BK * 2;
     extern __shared__ uint8_t smem_raw[];
     const Smem s = carve<STAGES>(smem_raw, W_BYTES, X_BYTES);
-    const uint32_t tmem_base = setup<STAGES>(s, &tmW, &tmX);
+    const uint32_t tmem_base = setup<STAGES>(s, &wm.map[0], &tmX);
     pdl_allow_dependents();
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -382,7 +414,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     if (!mbar_wait(smem_u32(&s.empty[stage]), phase ^ 1, s.abort)) goto done;
                     const uint32_t fb = smem_u32(&s.full[stage]);
                     mbar_arrive_expect_tx(fb, W_BYTES + X_BYTES);
-                    tma_load_2d(smem_u32(s.a + stage * W_BYTES), &tmW, 0, (tile * KB + kb) * 256, fb);
+                    load_w_tile<RAW>(smem_u32(s.a + stage * W_BYTES), wm, tile, kb, KB, fb);
                     if (!waited) {   // weights do not depend on the previous kernel; X does
                         pdl_wait_previous();
                         waited = true;
@@ -395,7 +427,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            const uint32_t idesc = idesc_bf16_f32(128, BT);
+            const uint32_t idesc = idesc_bf16_f32(128, BT) | (RAW ? kIdescAMajorMN : 0u);
             int stage = 0, acc = 0;
             uint32_t phase = 0, acc_phase = 0;
             for (long long it = it_b; it < it_e;) {
@@ -409,14 +441,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     if (!mbar_wait(smem_u32(&s.full[stage]), phase, s.abort)) goto done;
                     tc_fence_after();
                     const uint32_t wa = smem_u32(s.a + stage * W_BYTES);
-                    const uint64_t dw0 = smem_desc_kmajor_sw128(wa);
-                    const uint64_t dw1 = smem_desc_kmajor_sw128(wa + 128 * 128);   // rows 128..255
+                    // rows 128..255 of the tile: K-major 16 KB in; MN-major atoms 2-3, 16 KB in
+                    const uint64_t dw0 = RAW ? smem_desc_mnmajor_sw128(wa) : smem_desc_kmajor_sw128(wa);
+                    const uint64_t dw1 =
+                        RAW ? smem_desc_mnmajor_sw128(wa + 16384) : smem_desc_kmajor_sw128(wa + 128 * 128);
+                    constexpr uint32_t kstep_w = RAW ? 128 : 2;
                     const uint64_t dx = smem_desc_kmajor_sw128(smem_u32(s.b + stage * X_BYTES));
 #pragma unroll
                     for (int k = 0; k < BK / 16; ++k) {
                         const uint32_t accum = (kb != kb0 || k != 0) ? 1u : 0u;
-                        mma_bf16(d0, dw0 + 2 * k, dx + 2 * k, idesc, accum);
-                        mma_bf16(d1, dw1 + 2 * k, dx + 2 * k, idesc, accum);
+                        mma_bf16(d0, dw0 + kstep_w * k, dx + 2 * k, idesc, accum);
+                        mma_bf16(d1, dw1 + kstep_w * k, dx + 2 * k, idesc, accum);
                     }
                     mma_commit(smem_u32(&s.empty[stage]));
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
@@ -561,13 +596,14 @@ PFN_encodeTiled encode_fn() {
     return fn;
 }
 
-// K-major bf16 matrix (rows x K, row stride K), box = 64 (K) x box_rows, 128-byte swizzle,
-// out-of-range elements read as zero.
-bool make_map(CUtensorMap *m, const void *base, int K, int rows, int box_rows) {
+// 2-D bf16 tensor (inner x rows, rows `row_bytes` apart), box = 64 (inner) x box_rows,
+// 128-byte swizzle, out-of-range elements read as zero.
+bool make_map2d(CUtensorMap *m, const void *base, long long inner, long long rows, long long row_bytes,
+                int box_rows) {
     PFN_encodeTiled enc = encode_fn();
     if (!enc) return false;
-    const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
-    const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+    const cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
     const cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
     const cuuint32_t estr[2] = {1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
@@ -575,18 +611,68 @@ bool make_map(CUtensorMap *m, const void *base, int K, int rows, int box_rows) {
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Packed weight part (tile-blocked): a 2-D view of `blocks` rows of 64 bf16
-// (128 B); one box of 256 rows = one 32 KB (tile, k-block) block.
-bool make_map_blocked(CUtensorMap *m, const void *base, long long rows_w, int K) {
-    const long long rows = (long long)blk_tiles(rows_w) * blk_kblocks(K) * kTileRows;
-    return make_map(m, base, kKBlock, (int)rows, kTileRows);
+// Activations: K-major rows x K, row stride K; box = 64 (K) x box_rows.
+bool make_map(CUtensorMap *m, const void *base, int K, int rows, int box_rows) {
+    return make_map2d(m, base, K, rows, (long long)K * 2, box_rows);
+}
+
+// One projection's weight operand and its tile geometry.
+struct WeightOperand {
+    WeightMaps wm;
+    bool raw;
+    int tiles, KB;
+    int raw_first, tps, fs;
+};
+
+// Packed part (tile-blocked): a 2-D view of rows of 64 bf16 (128 B); one box of
+// 256 rows = one 32 KB (tile, k-block) block.
+bool weight_packed(WeightOperand *w, const void *base, long long rows_w, int K) {
+    memset(w, 0, sizeof(*w));
+    w->tiles = (int)blk_tiles(rows_w);
+    w->KB = (int)blk_kblocks(K);
+    const long long rows = (long long)w->tiles * w->KB * kTileRows;
+    return make_map2d(&w->wm.map[0], base, kKBlock, rows, kKBlock * 2, kTileRows);
+}
+
+// First projection straight from the shards A_i (d_in x lda row-major, lda = f_s
+// or 2 f_s for [gate_i | up_i]): maps over each rank's f_s columns, boxes of
+// 64 columns x 64 k rows.
+bool weight_raw_first(WeightOperand *w, const Problem &p, const ShardPtrs &A) {
+    memset(w, 0, sizeof(*w));
+    const bool sw = p.act == TP_MLP_ACT_SWIGLU;
+    const long long lda = sw ? 2LL * p.fs : p.fs;
+    const int per = sw ? 128 : 256;
+    w->raw = true;
+    w->tps = (p.fs + per - 1) / per;
+    w->tiles = p.tp * w->tps;
+    w->KB = (int)blk_kblocks(p.d_in);
+    w->raw_first = 1;
+    w->fs = p.fs;
+    w->wm.first = 1;
+    w->wm.swiglu = sw;
+    w->wm.tps = w->tps;
+    for (int i = 0; i < p.tp; ++i) {
+        const __nv_bfloat16 *a = static_cast<const __nv_bfloat16 *>(A.p[i]);
+        if (!make_map2d(&w->wm.map[i], a, p.fs, p.d_in, lda * 2, BK)) return false;
+        if (sw && !make_map2d(&w->wm.map[kMaxTp + i], a + p.fs, p.fs, p.d_in, lda * 2, BK)) return false;
+    }
+    return true;
+}
+
+// Second projection straight from the shards B_i (f_s x d_out row-major); the K
+// loop runs over rank 0's rows, then rank 1's, ... (needs f_s % 64 == 0).
+bool weight_raw_second(WeightOperand *w, const Problem &p, const ShardPtrs &B) {
+    memset(w, 0, sizeof(*w));
+    w->raw = true;
+    w->tiles = (int)blk_tiles(p.d_out);
+    w->KB = p.d_ff / BK;
+    w->wm.kbps = p.fs / BK;
+    for (int i = 0; i < p.tp; ++i)
+        if (!make_map2d(&w->wm.map[i], B.p[i], p.d_out, p.fs, (long long)p.d_out * 2, BK)) return false;
+    return true;
 }
 
 int skinny_bt(int T) { return T <= 16 ? 16 : T <= 32 ? 32 : T <= 64 ? 64 : 128; }
-
-StreamKGeom skinny_geom(long long rows_w, int K, int num_sms) {
-    return streamk_geom(blk_tiles(rows_w), blk_kblocks(K), num_sms);
-}
 
 template <typename K>
 cudaError_t set_smem(K kern, size_t bytes) {
@@ -594,25 +680,31 @@ cudaError_t set_smem(K kern, size_t bytes) {
 }
 
 template <int BT, int STAGES>
-cudaError_t launch_skinny_bt(const CUtensorMap &mw, const CUtensorMap &mx, const TcArgs &a, int grid,
+cudaError_t launch_skinny_bt(const WeightOperand &w, const CUtensorMap &mx, const TcArgs &a, int grid,
                              cudaStream_t st) {
-    auto kern = tc_skinny_kernel<BT, STAGES>;
     const size_t smem = smem_bytes<STAGES>(256 * BK * 2, BT * BK * 2);
+    if (w.raw) {
+        auto kern = tc_skinny_kernel<BT, STAGES, true>;
+        cudaError_t e = set_smem(kern, smem);
+        if (e != cudaSuccess) return e;
+        return launch_pdl(kern, dim3(grid), dim3(NTHREADS), smem, st, w.wm, mx, a);
+    }
+    auto kern = tc_skinny_kernel<BT, STAGES, false>;
     cudaError_t e = set_smem(kern, smem);
     if (e != cudaSuccess) return e;
-    return launch_pdl(kern, dim3(grid), dim3(NTHREADS), smem, st, mw, mx, a);
+    return launch_pdl(kern, dim3(grid), dim3(NTHREADS), smem, st, w.wm, mx, a);
 }
 
-// One projection with the skinny tiling.  w: rows_w x K packed weights; x: T x K.
-cudaError_t run_skinny(const void *w, int rows_w, const void *x, int T, int K, int epi, void *out, int out_cols,
+// One projection with the skinny tiling; x: T x K activations.
+cudaError_t run_skinny(const WeightOperand &w, const void *x, int T, int K, int epi, void *out, int out_cols,
                        float *part, unsigned *cnt, int *status, int num_sms, cudaStream_t st) {
     const int BT = skinny_bt(T);
-    CUtensorMap mw, mx;
-    if (!make_map_blocked(&mw, w, rows_w, K) || !make_map(&mx, x, K, T, BT)) return cudaErrorInvalidValue;
-    const StreamKGeom g = skinny_geom(rows_w, K, num_sms);
+    CUtensorMap mx;
+    if (!make_map(&mx, x, K, T, BT)) return cudaErrorInvalidValue;
+    const StreamKGeom g = streamk_geom(w.tiles, w.KB, num_sms);
     TcArgs a{};
     a.rows_x = T;
-    a.rows_w = rows_w;
+    a.rows_w = w.tiles;
     a.K = K;
     a.KB = g.KB;
     a.epi = epi;
@@ -624,41 +716,61 @@ cudaError_t run_skinny(const void *w, int rows_w, const void *x, int T, int K, i
     a.part = part;
     a.tile_cnt = cnt;
     a.status = status;
+    a.raw_first = w.raw_first;
+    a.tps = w.tps;
+    a.fs = w.fs;
     switch (BT) {
-        case 16: return launch_skinny_bt<16, 6>(mw, mx, a, g.grid, st);
-        case 32: return launch_skinny_bt<32, 6>(mw, mx, a, g.grid, st);
-        case 64: return launch_skinny_bt<64, 5>(mw, mx, a, g.grid, st);
-        default: return launch_skinny_bt<128, 4>(mw, mx, a, g.grid, st);
+        case 16: return launch_skinny_bt<16, 6>(w, mx, a, g.grid, st);
+        case 32: return launch_skinny_bt<32, 6>(w, mx, a, g.grid, st);
+        case 64: return launch_skinny_bt<64, 5>(w, mx, a, g.grid, st);
+        default: return launch_skinny_bt<128, 4>(w, mx, a, g.grid, st);
     }
 }
 
 template <int MH>
-cudaError_t run_wide(const void *x, int T, const void *w, int rows_w, int K, int epi, void *out, int out_cols,
+cudaError_t run_wide(const WeightOperand &w, const void *x, int T, int K, int epi, void *out, int out_cols,
                      int *status, int num_sms, cudaStream_t st) {
     using C = WideCfg<MH>;
-    CUtensorMap mx, mw;
-    if (!make_map(&mx, x, K, T, 128 * MH) || !make_map_blocked(&mw, w, rows_w, K)) return cudaErrorInvalidValue;
+    CUtensorMap mx;
+    if (!make_map(&mx, x, K, T, 128 * MH)) return cudaErrorInvalidValue;
     TcArgs a{};
     a.rows_x = T;
-    a.rows_w = rows_w;
+    a.rows_w = w.tiles;
     a.K = K;
-    a.KB = (K + BK - 1) / BK;
+    a.KB = w.KB;
     a.epi = epi;
     a.out = static_cast<__nv_bfloat16 *>(out);
     a.ldo = out_cols;
     a.out_cols = out_cols;
     a.status = status;
-    const int units = ((T + 128 * MH - 1) / (128 * MH)) * ((rows_w + 255) / 256);
+    a.raw_first = w.raw_first;
+    a.tps = w.tps;
+    a.fs = w.fs;
+    const int units = ((T + 128 * MH - 1) / (128 * MH)) * w.tiles;
     const int grid = std::min(units, num_sms);
     const size_t smem = smem_bytes<C::STAGES>(C::A_BYTES, C::B_BYTES);
-    auto kern = tc_wide_kernel<MH>;
+    if (w.raw) {
+        auto kern = tc_wide_kernel<MH, true>;
+        cudaError_t e = set_smem(kern, smem);
+        if (e != cudaSuccess) return e;
+        return launch_pdl(kern, dim3(grid), dim3(NTHREADS), smem, st, mx, w.wm, a);
+    }
+    auto kern = tc_wide_kernel<MH, false>;
     cudaError_t e = set_smem(kern, smem);
     if (e != cudaSuccess) return e;
-    return launch_pdl(kern, dim3(grid), dim3(NTHREADS), smem, st, mx, mw, a);
+    return launch_pdl(kern, dim3(grid), dim3(NTHREADS), smem, st, mx, w.wm, a);
 }
 
 int first_epi(int act) {
     return act == TP_MLP_ACT_SWIGLU ? EPI_H_SWIGLU : act == TP_MLP_ACT_TANH ? EPI_H_TANH : EPI_H_IDENT;
+}
+
+// Weight tiles of the first projection in either layout (the larger count sizes
+// the split-tile scratch).
+long long first_tiles(const Problem &p, bool raw) {
+    if (!raw) return blk_tiles(w1p_rows(p.d_ff, p.act));
+    const int per = p.act == TP_MLP_ACT_SWIGLU ? 128 : 256;
+    return (long long)p.tp * ((p.fs + per - 1) / per);
 }
 
 }  // namespace
@@ -668,39 +780,50 @@ bool tc_supported(const Problem &p) {
            encode_fn() != nullptr;
 }
 
+bool tc_raw_supported(const Problem &p) { return tc_supported(p) && p.fs % BK == 0; }
+
 size_t tile_counter_slots(const Problem &p) {
-    return (size_t)(blk_tiles(w1p_rows(p.d_ff, p.act)) + blk_tiles(p.d_out));
+    return (size_t)(std::max(first_tiles(p, false), first_tiles(p, true)) + blk_tiles(p.d_out));
 }
 
 size_t tc_workspace_bytes(const Problem &p, int num_sms) {
     if (p.T < 1 || p.T > kTcSkinnyMaxTokens) return 0;
-    const int BT = skinny_bt(p.T);
-    const StreamKGeom g1 = skinny_geom(w1p_rows(p.d_ff, p.act), p.d_in, num_sms);
-    const StreamKGeom g2 = skinny_geom(p.d_out, p.d_ff, num_sms);
-    const size_t s1 = (size_t)g1.tiles * g1.slots * 256 * BT * 4;
-    const size_t s2 = (size_t)g2.tiles * g2.slots * 256 * BT * 4;
-    return align256(s1 > s2 ? s1 : s2);
+    const size_t BT = skinny_bt(p.T);
+    size_t m = 0;
+    for (int raw = 0; raw < 2; ++raw) {
+        const StreamKGeom g1 = streamk_geom(first_tiles(p, raw), blk_kblocks(p.d_in), num_sms);
+        const StreamKGeom g2 = streamk_geom(blk_tiles(p.d_out), blk_kblocks(p.d_ff), num_sms);
+        m = std::max(m, (size_t)g1.tiles * g1.slots * 256 * BT * 4);
+        m = std::max(m, (size_t)g2.tiles * g2.slots * 256 * BT * 4);
+    }
+    return align256(m);
 }
 
-cudaError_t launch_tc(const Problem &p, int tiling, const void *x, const void *w1p, const void *w2p, void *h,
-                      void *out, float *part, unsigned *counters, int *status, int num_sms, cudaStream_t st,
-                      const Marks &marks) {
-    const bool skinny = tiling == kTilingSkinny;
-    const int rows1 = (int)w1p_rows(p.d_ff, p.act);
+cudaError_t launch_tc(const Problem &p, int tiling, const void *x, const void *w1p, const void *w2p,
+                      const ShardPtrs *rawA, const ShardPtrs *rawB, void *h, void *out, float *part,
+                      unsigned *counters, int *status, int num_sms, cudaStream_t st, const Marks &marks) {
+    WeightOperand w1, w2;
+    const bool raw = rawA != nullptr;
+    if (raw) {
+        if (!weight_raw_first(&w1, p, *rawA) || !weight_raw_second(&w2, p, *rawB)) return cudaErrorInvalidValue;
+    } else if (!weight_packed(&w1, w1p, w1p_rows(p.d_ff, p.act), p.d_in) ||
+               !weight_packed(&w2, w2p, p.d_out, p.d_ff)) {
+        return cudaErrorInvalidValue;
+    }
     cudaError_t e;
     marks.mark(0, st);
-    if (skinny) {
-        unsigned *cnt1 = counters, *cnt2 = counters + blk_tiles(rows1);
-        e = run_skinny(w1p, rows1, x, p.T, p.d_in, first_epi(p.act), h, p.d_ff, part, cnt1, status, num_sms, st);
+    if (tiling == kTilingSkinny) {
+        unsigned *cnt1 = counters, *cnt2 = counters + w1.tiles;
+        e = run_skinny(w1, x, p.T, p.d_in, first_epi(p.act), h, p.d_ff, part, cnt1, status, num_sms, st);
         if (e != cudaSuccess) return e;
         marks.mark(1, st);
-        e = run_skinny(w2p, p.d_out, h, p.T, p.d_ff, EPI_OUT, out, p.d_out, part, cnt2, status, num_sms, st);
+        e = run_skinny(w2, h, p.T, p.d_ff, EPI_OUT, out, p.d_out, part, cnt2, status, num_sms, st);
     } else {
         auto wide = tiling == kTilingWide256 ? run_wide<2> : run_wide<1>;
-        e = wide(x, p.T, w1p, rows1, p.d_in, first_epi(p.act), h, p.d_ff, status, num_sms, st);
+        e = wide(w1, x, p.T, p.d_in, first_epi(p.act), h, p.d_ff, status, num_sms, st);
         if (e != cudaSuccess) return e;
         marks.mark(1, st);
-        e = wide(h, p.T, w2p, p.d_out, p.d_ff, EPI_OUT, out, p.d_out, status, num_sms, st);
+        e = wide(w2, h, p.T, p.d_ff, EPI_OUT, out, p.d_out, status, num_sms, st);
     }
     marks.mark(2, st);
     return e;

@@ -266,9 +266,22 @@ static int run_shard_form(tp_mlp_t h, const void *x, int tokens, const void *con
                           tp_mlp_stream_t stream) {
     int s = check_common(h, x, tokens, tp_degree, act);
     if (s) return s;
-    if (h->plan != TP_MLP_PLAN_AUTO && h->plan != TP_MLP_PLAN_SIMT) return TP_MLP_ERR_UNSUPPORTED;
+    Problem p = problem_of(h, tokens);
+    // The forward reads the shards straight into the tcgen05 kernels when the
+    // shape allows (bf16, f_s % 64 == 0); the partials call and other shapes use
+    // the CUDA-core kernels.  The GEMV needs the packed layout.
+    const bool tc_ok = !partials && tc_raw_supported(p);
+    int plan = h->plan;
+    if (plan == TP_MLP_PLAN_AUTO) plan = tc_ok ? TP_MLP_PLAN_TC : TP_MLP_PLAN_SIMT;
+    if (plan == TP_MLP_PLAN_TC)
+        plan = tokens <= kTcSkinnyMaxTokens ? TP_MLP_PLAN_TC_SKINNY
+                                            : tokens < kTcWide256MinTokens ? TP_MLP_PLAN_TC_WIDE : TP_MLP_PLAN_TC_WIDE256;
+    const bool is_tc = plan == TP_MLP_PLAN_TC_WIDE || plan == TP_MLP_PLAN_TC_SKINNY || plan == TP_MLP_PLAN_TC_WIDE256;
+    if (plan != TP_MLP_PLAN_SIMT && !is_tc) return TP_MLP_ERR_UNSUPPORTED;
+    if (is_tc && tokens > 0 && (!tc_ok || (plan == TP_MLP_PLAN_TC_SKINNY && tokens > kTcSkinnyMaxTokens)))
+        return TP_MLP_ERR_UNSUPPORTED;
     if (tokens == 0) {
-        h->last_plan = TP_MLP_PLAN_SIMT;
+        h->last_plan = plan;
         h->last_launches = 0;
         return TP_MLP_OK;
     }
@@ -281,12 +294,22 @@ static int run_shard_form(tp_mlp_t h, const void *x, int tokens, const void *con
     }
     if ((s = check_shards(h, A, B))) return s;
     if ((s = check_workspace(h, tokens))) return s;
-    Problem p = problem_of(h, tokens);
-    void *hbuf = static_cast<char *>(h->ws) + counters_bytes(h);
-    cudaError_t ce = launch_simt(p, false, x, to_ptrs(A, h->tp), to_ptrs(B, h->tp), hbuf, out,
-                                 partials, reinterpret_cast<cudaStream_t>(stream), h->marks);
+    char *ws = static_cast<char *>(h->ws);
+    void *hbuf = ws + counters_bytes(h);
+    const ShardPtrs a = to_ptrs(A, h->tp), b = to_ptrs(B, h->tp);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t ce;
+    if (is_tc) {
+        const int tiling = plan == TP_MLP_PLAN_TC_SKINNY ? kTilingSkinny
+                           : plan == TP_MLP_PLAN_TC_WIDE ? kTilingWide128 : kTilingWide256;
+        float *part = reinterpret_cast<float *>(ws + counters_bytes(h) + h_bytes(h, tokens));
+        ce = launch_tc(p, tiling, x, nullptr, nullptr, &a, &b, hbuf, out, part, reinterpret_cast<unsigned *>(ws),
+                       status_word(h), h->num_sms, st, h->marks);
+    } else {
+        ce = launch_simt(p, false, x, a, b, hbuf, out, partials, st, h->marks);
+    }
     if (ce != cudaSuccess) return TP_MLP_ERR_CUDA;
-    h->last_plan = TP_MLP_PLAN_SIMT;
+    h->last_plan = plan;
     h->last_launches = 2;
     return TP_MLP_OK;
 }
@@ -383,8 +406,8 @@ int tp_mlp_forward_packed(tp_mlp_t h, const void *x, int tokens, const void *pac
     } else if (is_tc) {
         const int tiling = plan == TP_MLP_PLAN_TC_SKINNY ? kTilingSkinny
                            : plan == TP_MLP_PLAN_TC_WIDE ? kTilingWide128 : kTilingWide256;
-        ce = launch_tc(p, tiling, x, w1p, w2p, hbuf, out, part, counters, status_word(h), h->num_sms, st,
-                       h->marks);
+        ce = launch_tc(p, tiling, x, w1p, w2p, nullptr, nullptr, hbuf, out, part, counters, status_word(h),
+                       h->num_sms, st, h->marks);
     } else {
         ShardPtrs a, b;
         memset(&a, 0, sizeof(a));

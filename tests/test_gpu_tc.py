@@ -143,3 +143,52 @@ def test_auto_plan_picks_256_token_tiles_for_long_prompts():
     assert m.last_plan == "tc_wide256"
     m.forward_packed(x[:2047], packed)
     assert m.last_plan == "tc_wide"
+
+
+# --- the shard form read directly by the tensor cores (MN-major weight operand) ---
+
+RAW_SHAPES = [  # (d_in, d_ff, d_out, tp); f_s = d_ff / tp is a multiple of 64
+    (512, 1024, 384, 4),
+    (520, 384, 264, 2),     # ragged K and output width; f_s = 192: a rank's last tile is part padding
+    (4096, 1024, 256, 8),   # long K, split tiles
+    (256, 8192, 512, 8),    # long second-projection K over 8 ranks
+]
+
+
+def _run_shard_form(p, tp, plan, max_tokens=None):
+    A, Bs = p.shards(tp)
+    m = B().TpMlp(p.d_in, p.d_ff, tp, p.act, "bf16", max_tokens or p.tokens, d_out=p.d_out)
+    m.set_plan(plan)
+    out = m.forward(dev(p.x, "bf16"), [dev(a, "bf16") for a in A], [dev(b, "bf16") for b in Bs])
+    torch.cuda.synchronize()
+    B().tp_mlp_get_device_status(m.h)
+    return m, out, A, Bs
+
+
+@pytest.mark.parametrize("act", ["swiglu", "tanh", "identity"])
+@pytest.mark.parametrize("plan,T", [("tc_skinny", 1), ("tc_skinny", 5), ("tc_skinny", 33), ("tc_skinny", 128),
+                                    ("tc_wide", 129), ("tc_wide", 300), ("tc_wide256", 300), ("auto", 2)])
+@pytest.mark.parametrize("shape", RAW_SHAPES)
+def test_tc_shard_form_parity(act, plan, T, shape):
+    d, f, dout, tp = shape
+    p = inputs.generate(T, d, f, act, "bf16", seed=T + 3 * f + dout, init="fan_in", d_out=dout)
+    m, out, A, Bs = _run_shard_form(p, tp, plan)
+    assert m.last_plan == (plan if plan != "auto" else "tc_skinny")
+    rows = p.sample_rows(64)
+    ref = oracle.tp_mlp_sharded(p.x[rows], A, Bs, act)
+    assert_close(out[torch.from_numpy(rows).cuda()], ref, "bf16", f"shard form {plan} T={T}")
+
+
+@pytest.mark.parametrize("plan,T", [("tc_skinny", 3), ("tc_wide", 130), ("tc_wide256", 257)])
+def test_tc_shard_form_integer_exact(plan, T):
+    p = inputs.integer_inputs(T, 64, 512, 264, "identity", seed=T + 1, lo=-1, hi=1)
+    _, out, A, Bs = _run_shard_form(p, 4, plan)
+    ref = oracle.tp_mlp_sharded(p.x, A, Bs, "identity")
+    assert np.array_equal(out.float().cpu().numpy(), inputs.round_to_bf16(ref.astype(np.float32)))
+
+
+def test_shard_form_falls_back_when_ranks_are_not_64_aligned():
+    p = inputs.generate(4, 128, 8 * 40, "tanh", "bf16", seed=1)     # f_s = 40
+    m, out, A, Bs = _run_shard_form(p, 8, "auto")
+    assert m.last_plan == "simt"
+    assert_close(out, oracle.tp_mlp_sharded(p.x, A, Bs, "tanh"), "bf16", "simt fallback")
