@@ -207,6 +207,17 @@ int tp_mlp_set_profile_events(tp_mlp_t handle, void *const *events, int n);
  */
 int tp_mlp_get_device_status(tp_mlp_t handle);
 
+/*
+ * Self-test of failure detection (the pages describe none): launches one
+ * small kernel that waits, through the same bounded mbarrier wait every
+ * pipelined kernel here uses, on a barrier nothing will complete.  The wait
+ * gives up after wait_us microseconds (1..100000), the kernel records the
+ * timeout in the handle's status word and returns; nothing traps.  A later
+ * tp_mlp_get_device_status then returns TP_MLP_ERR_TIMEOUT (and clears it),
+ * and the context stays usable.  Needs a workspace.
+ */
+int tp_mlp_selftest_bounded_wait(tp_mlp_t handle, unsigned wait_us, tp_mlp_stream_t stream);
+
 /* Plan (tp_mlp_plan) and number of kernel launches of the last successful
  * forward / partials call on this handle; -1 before the first. */
 int tp_mlp_last_plan(tp_mlp_t handle);

@@ -50,6 +50,7 @@ _SIGS = {
     "tp_mlp_set_plan": (_i, [_vp, _i]),
     "tp_mlp_set_profile_events": (_i, [_vp, _vpp, _i]),
     "tp_mlp_get_device_status": (_i, [_vp]),
+    "tp_mlp_selftest_bounded_wait": (_i, [_vp, ctypes.c_uint, _vp]),
     "tp_mlp_last_plan": (_i, [_vp]),
     "tp_mlp_last_launches": (_i, [_vp]),
     "tp_mlp_status_string": (ctypes.c_char_p, [_i]),
@@ -175,6 +176,10 @@ def tp_mlp_set_profile_events(h, events) -> None:
 
 def tp_mlp_get_device_status(h) -> None:
     _check("tp_mlp_get_device_status", _lib.tp_mlp_get_device_status(h))
+
+
+def tp_mlp_selftest_bounded_wait(h, wait_us: int, stream=None) -> None:
+    _check("tp_mlp_selftest_bounded_wait", _lib.tp_mlp_selftest_bounded_wait(h, wait_us, _stream(stream)))
 
 
 def tp_mlp_last_plan(h) -> str:

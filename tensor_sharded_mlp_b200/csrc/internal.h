@@ -30,6 +30,9 @@ size_t packed_total_bytes(const Problem &p);
 cudaError_t launch_pack(const Problem &p, const ShardPtrs &a, const ShardPtrs &b, void *packed,
                         bool unpack, cudaStream_t s);
 
+// selftest.cu: a bounded wait that runs out, recorded in *status.
+cudaError_t launch_bounded_wait_selftest(int *status, unsigned wait_us, cudaStream_t st);
+
 // Split-tile counters the GEMV and tcgen05 skinny kernels need (one per
 // weight tile of both parts; first part's tiles first).
 size_t tile_counter_slots(const Problem &p);

@@ -433,6 +433,14 @@ int tp_mlp_get_device_status(tp_mlp_t h) {
     return TP_MLP_ERR_TIMEOUT;
 }
 
+int tp_mlp_selftest_bounded_wait(tp_mlp_t h, unsigned wait_us, tp_mlp_stream_t stream) {
+    if (!h) return TP_MLP_ERR_INVALID_ARG;
+    if (!h->ws) return TP_MLP_ERR_WORKSPACE;
+    if (wait_us == 0 || wait_us > 100000) return TP_MLP_ERR_INVALID_ARG;
+    return from_cuda(launch_bounded_wait_selftest(status_word(h), wait_us,
+                                                  reinterpret_cast<cudaStream_t>(stream)));
+}
+
 int tp_mlp_set_plan(tp_mlp_t h, int plan) {
     if (!h) return TP_MLP_ERR_INVALID_ARG;
     if (plan < TP_MLP_PLAN_AUTO || plan > TP_MLP_PLAN_TC_WIDE256) return TP_MLP_ERR_INVALID_ARG;

@@ -69,3 +69,32 @@ def test_reference_arm_under_torchrun_prints_once():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
+
+
+def _worker_one_leaves(rank, world, port, out_dir):
+    os.environ.update(RANK=str(rank), WORLD_SIZE=str(world), LOCAL_RANK=str(rank),
+                      MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.path.insert(0, ROOT)
+    import time
+    from tensor_sharded_mlp_b200 import replicas
+    replicas.init("gloo", timeout_s=5)
+    replicas.barrier()                     # both ranks are up
+    if rank == 1:
+        return                             # rank 1 leaves between steps, with nothing in flight
+    t0 = time.time()
+    outcome = "no error"
+    try:
+        replicas.max_over_ranks(1.0)       # the next collective must fail, not hang
+    except Exception as e:                 # gloo reports the lost peer or the timeout
+        outcome = type(e).__name__
+    with open(os.path.join(out_dir, "survivor.json"), "w") as f:
+        json.dump({"outcome": outcome, "seconds": time.time() - t0}, f)
+
+
+def test_a_rank_that_leaves_is_detected_by_the_next_collective(tmp_path):
+    port = _free_port()
+    mp.start_processes(_worker_one_leaves, args=(2, port, str(tmp_path)), nprocs=2, start_method="spawn",
+                       join=True)
+    r = json.load(open(tmp_path / "survivor.json"))
+    assert r["outcome"] != "no error"
+    assert r["seconds"] < 60
