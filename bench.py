@@ -46,6 +46,8 @@ def parse():
     ap.add_argument("--tokens", type=int, default=None)
     ap.add_argument("--tp", type=int, default=None)
     ap.add_argument("--plan", default="auto")
+    ap.add_argument("--splitk", choices=["auto", "in_kernel", "separate"], default="auto",
+                    help="how the skinny tensor-core tiling finishes split tiles")
     ap.add_argument("--d-model", type=int, default=None, help="override (small cases for profiling)")
     ap.add_argument("--d-ff", type=int, default=None, help="override (small cases for profiling)")
     ap.add_argument("--api", choices=["packed", "shard"], default="packed",
@@ -250,6 +252,7 @@ def main():
 
     m = binding.TpMlp(d, f, tp, act, dt, max_tokens=T)
     m.set_plan(args.plan)
+    m.set_splitk(args.splitk)
     Ad, Bd = [up(a) for a in A], [up(b) for b in Bs]
     packed = m.pack(Ad, Bd)
     if args.api == "packed":
@@ -270,7 +273,10 @@ def main():
         fwd()
     nk = m.last_launches
     plan = m.last_plan
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)] for _ in range(K)]
+    # the library marks phases: before the first projection's kernels, between
+    # the projections and after the second's (a phase may be more than one kernel)
+    nph = 2
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nph + 1)] for _ in range(K)]
     stream = torch.cuda.current_stream()
     for row in ev:
         for e in row:
@@ -298,7 +304,7 @@ def main():
         fwd()
     binding.tp_mlp_set_profile_events(m.h, None)
     barrier()
-    kern_ms = [statistics.fmean(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(K)) for j in range(nk)]
+    kern_ms = [statistics.fmean(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(K)) for j in range(nph)]
     elapsed_ms = replicas.max_over_ranks(elapsed_ms)
 
     # end to end through the public API with host buffers (pinned), copies inside
@@ -348,7 +354,7 @@ def main():
         peak_note = f"hbm_gbs ({src})"
     kname = f"{plan}:{'first' if j == 0 else 'second'}"
     roofline = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
-                "traffic": recorded_traffic(kname, args.config), "kernel": names[j] if j < 2 else str(j),
+                "traffic": recorded_traffic(kname, args.config), "kernel": names[j] + (" (GEMM + split-tile reduction kernel)" if nk > 2 and plan == "tc_skinny" else ""),
                 "kernel_ms": kern_ms[j], "algorithmic_per_launch": work, "peak_source": peak_note,
                 "kernel_ms_all": kern_ms}
     step_bytes = counts.algorithmic_bytes(T, d, f, d, act, dt)
@@ -358,7 +364,7 @@ def main():
             "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": dt, "data": "synthetic",
             "config": {"workload": c["workload"], "tokens": T, "d_model": d, "d_ff": f, "tp": tp, "act": act,
-                       "plan": plan, "api": args.api, "parallelism": "replicas" if world > 1 else "single GPU",
+                       "plan": plan, "splitk": args.splitk, "api": args.api, "parallelism": "replicas" if world > 1 else "single GPU",
                        "l2": "inputs larger than L2: every step re-reads %.2f GB of weights" % (step_bytes / 1e9)},
             "step_hbm_gbs": step_bytes / (ms / 1e3) / 1e9, "step_tflops": step_flops / (ms / 1e3) / 1e12,
             "roofline": roofline, "gpu_launches": K * nk, "clocks": sampler.summary(), "e2e": e2e}

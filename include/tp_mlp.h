@@ -190,10 +190,26 @@ int tp_mlp_forward_packed(tp_mlp_t handle, const void *x, int tokens, const void
 int tp_mlp_set_plan(tp_mlp_t handle, int plan);
 
 /*
+ * How the skinny tensor-core tiling (TP_MLP_PLAN_TC_SKINNY) finishes a weight
+ * tile whose K loop is split between CTAs.  Both add the fp32 partial slots in
+ * the same fixed order, so they give identical results; they differ in speed.
+ */
+typedef enum {
+    TP_MLP_SPLITK_AUTO = 0,      /* by the size of the partials (default)            */
+    TP_MLP_SPLITK_IN_KERNEL = 1, /* the last CTA to finish its share adds the slots   */
+    TP_MLP_SPLITK_SEPARATE = 2   /* a reduction kernel behind each GEMM adds them,
+                                    spread over the whole GPU                        */
+} tp_mlp_splitk;
+
+/* Choose the split-tile finish (tp_mlp_splitk) for later forwards.  Returns
+ * TP_MLP_ERR_INVALID_ARG for another value.  Other plans ignore it. */
+int tp_mlp_set_splitk(tp_mlp_t handle, int mode);
+
+/*
  * Timing hook: with n > 0, later forward / forward_packed / partials calls
- * record events[0] on their stream before their first kernel and events[j]
- * after their j-th kernel (j = 1 .. n-1; kernels beyond that are not
- * marked).  The events are caller-owned cudaEvent_t handles (created with
+ * record events[0] on their stream before their first kernel, events[1] after
+ * the first projection's kernels and events[2] after the second projection's
+ * (events beyond events[2] are not recorded).  The events are caller-owned cudaEvent_t handles (created with
  * timing enabled) and must stay valid while calls use them; n = 0 (or
  * events = NULL) turns the hook off.  At most 8 events.
  */

@@ -48,6 +48,7 @@ _SIGS = {
     "tp_mlp_unpack": (_i, [_vp, _vp, _vpp, _vpp, _vp]),
     "tp_mlp_forward_packed": (_i, [_vp, _vp, _i, _vp, _vp, _vp]),
     "tp_mlp_set_plan": (_i, [_vp, _i]),
+    "tp_mlp_set_splitk": (_i, [_vp, _i]),
     "tp_mlp_set_profile_events": (_i, [_vp, _vpp, _i]),
     "tp_mlp_get_device_status": (_i, [_vp]),
     "tp_mlp_selftest_bounded_wait": (_i, [_vp, ctypes.c_uint, _vp]),
@@ -161,6 +162,13 @@ def tp_mlp_forward_packed(h, x: torch.Tensor, packed: torch.Tensor, out: torch.T
 
 def tp_mlp_set_plan(h, plan: str) -> None:
     _check("tp_mlp_set_plan", _lib.tp_mlp_set_plan(h, PLAN[plan]))
+
+
+SPLITK = {"auto": 0, "in_kernel": 1, "separate": 2}
+
+
+def tp_mlp_set_splitk(h, mode: str) -> None:
+    _check("tp_mlp_set_splitk", _lib.tp_mlp_set_splitk(h, SPLITK[mode]))
 
 
 def tp_mlp_set_profile_events(h, events) -> None:
@@ -287,6 +295,9 @@ class TpMlp:
 
     def set_plan(self, plan: str):
         tp_mlp_set_plan(self.h, plan)
+
+    def set_splitk(self, mode: str):
+        tp_mlp_set_splitk(self.h, mode)
 
     @property
     def last_plan(self) -> str:

@@ -52,9 +52,14 @@ enum { kTilingSkinny = 0, kTilingWide128 = 1, kTilingWide256 = 2 };
 bool tc_supported(const Problem &p);
 bool tc_raw_supported(const Problem &p);   // also needs f_s % 64 == 0
 size_t tc_workspace_bytes(const Problem &p, int num_sms);
+// Split tiles of the skinny tiling (values of tp_mlp_splitk): finished by the
+// last CTA to arrive, inside the GEMM kernel, or by a reduction kernel behind it.
+enum { kSplitAuto = 0, kSplitInKernel = 1, kSplitSeparate = 2 };
 // Packed weights (w1p/w2p), or the per-rank shards when rawA/rawB are given.
+// *launches receives the number of kernels launched.
 cudaError_t launch_tc(const Problem &p, int tiling, const void *x, const void *w1p, const void *w2p,
                       const ShardPtrs *rawA, const ShardPtrs *rawB, void *h, void *out, float *part,
-                      unsigned *counters, int *status, int num_sms, cudaStream_t st, const Marks &marks);
+                      unsigned *counters, int *status, int num_sms, cudaStream_t st, const Marks &marks,
+                      int split_mode, int *launches);
 
 }  // namespace tpmlp

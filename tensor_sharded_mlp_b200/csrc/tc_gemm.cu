@@ -16,9 +16,10 @@
 //          describes): operands swapped -- M is 128 weight rows (two MMAs per
 //          256-row weight tile), N is the token count rounded up to BT.  The
 //          weight stream is cut into equal contiguous shares, one per CTA
-//          ("stream-K"); a tile split between CTAs is finished by the last CTA
-//          to arrive, which adds the fp32 partial slots in a fixed order.
-//          Nothing waits on another CTA.
+//          ("stream-K"); a tile split between CTAs is finished from fp32
+//          partial slots added in a fixed order, either by a reduction kernel
+//          behind the GEMM (default) or by the last CTA to arrive.  Nothing
+//          waits on another CTA.
 //
 // Roles: warp 0 lane 0 issues TMA loads, warp 1 allocates TMEM and lane 0
 // issues the MMAs, warps 2..5 run the epilogue (TMEM lanes 32*(warp%4)...).
@@ -60,6 +61,8 @@ struct TcArgs {
     int slots;           // partial slots per weight tile
     float *part;         // [tile][slot][BT/4][256][4] fp32 (float4 per row and 4 tokens)
     unsigned *tile_cnt;  // k-blocks done per weight tile, zero between launches
+    int split_mode;      // kSplitInKernel or kSplitSeparate (see internal.h)
+    int grid;            // CTAs of the skinny launch (the stream-K split)
     int *status;         // set to 1 if a bounded wait ran out
     // first projection read straight from the per-rank shards: tile t covers
     // features of rank t / tps only (tps tiles per rank of fs features)
@@ -386,6 +389,27 @@ __device__ __forceinline__ void skinny_final16(const TcArgs &a, int tile, int r,
     }
 }
 
+// Final epilogue of 4 tokens t0..t0+3: v0 = row r, v1 = row 128 + r.
+__device__ __forceinline__ void skinny_final4(const TcArgs &a, int tile, int r, int t0, float4 v0, float4 v1) {
+    const float g[4] = {v0.x, v0.y, v0.z, v0.w}, u[4] = {v1.x, v1.y, v1.z, v1.w};
+    const int T = a.rows_x;
+    if (a.epi == EPI_H_SWIGLU) {
+        const int n = tile_col(a, tile, r, 128);
+        if (n < 0) return;
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            if (t0 + i < T) a.out[(long)(t0 + i) * a.ldo + n] = __float2bfloat16_rn(silu_fast(g[i]) * u[i]);
+    } else {
+        const int n0 = tile_col(a, tile, r, 256), n1 = tile_col(a, tile, r + 128, 256);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            if (t0 + i >= T) break;
+            if (n0 >= 0) a.out[(long)(t0 + i) * a.ldo + n0] = __float2bfloat16_rn(act_out(a.epi, g[i]));
+            if (n1 >= 0) a.out[(long)(t0 + i) * a.ldo + n1] = __float2bfloat16_rn(act_out(a.epi, u[i]));
+        }
+    }
+}
+
 template <int BT, int STAGES, bool RAW>
 __global__ void __launch_bounds__(NTHREADS, 1)
     tc_skinny_kernel(const __grid_constant__ WeightMaps wm, const __grid_constant__ CUtensorMap tmX, TcArgs a) {
@@ -486,6 +510,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     tmem_ld_wait();
                     skinny_final16(a, tile, r, t0, v0, v1);
                 }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&s.tempty[acc]));
             } else {
                 // this CTA's share of the tile -> its partial slot, laid out
                 // [token/4][row][token%4]: each lane stores float4s, a warp 512 B at a time
@@ -506,6 +533,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         base[qd * 256 + 128 + r] = make_float4(v1[4 * q], v1[4 * q + 1], v1[4 * q + 2], v1[4 * q + 3]);
                     }
                 }
+                // the accumulator is copied out: hand TMEM back to the MMA before the fixup
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&s.tempty[acc]));
+                if (a.split_mode == kSplitSeparate) {   // skinny_reduce_kernel adds the slots
+                    acc ^= 1;
+                    if (acc == 0) acc_phase ^= 1;
+                    continue;
+                }
                 __threadfence();
                 named_bar(1, 128);
                 if (threadIdx.x == 64) {
@@ -514,64 +550,79 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 }
                 named_bar(1, 128);
                 if (*s.flag) {
+                    // Last to arrive: add the n slots in slot order.  Each thread walks
+                    // whole float4 positions (row r, 4 tokens) so the loads of several
+                    // positions and slots are in flight together.
                     __threadfence();
                     const float4 *tb = reinterpret_cast<const float4 *>(a.part + (long long)tile * a.slots * 256 * BT);
                     const int n = c_last - c_first + 1;
                     constexpr long SLOT4 = 256L * BT / 4;   // float4s per slot
+                    constexpr int NPOS = (BT / 4) * 128;     // (token quad, row pair) positions
+                    constexpr int U = 4;
 #pragma unroll 1
-                    for (int t0 = 0; t0 < BT; t0 += 16) {
-                        float4 s0[4], s1[4];
+                    for (int p0 = threadIdx.x - 64; p0 < NPOS; p0 += 128 * U) {
+                        float4 s0[U], s1[U];
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) s0[q] = s1[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-                        int sl = 0;
-                        for (; sl + 1 < n; sl += 2) {   // two slots' loads in flight together
-                            float4 u0[4], u1[4], w0[4], w1[4];
+                        for (int u = 0; u < U; ++u) s0[u] = s1[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 2
+                        for (int sl = 0; sl < n; ++sl) {
 #pragma unroll
-                            for (int q = 0; q < 4; ++q) {
-                                const long o = (long)(t0 / 4 + q) * 256 + r;
-                                u0[q] = __ldcg(tb + sl * SLOT4 + o);
-                                u1[q] = __ldcg(tb + sl * SLOT4 + o + 128);
-                                w0[q] = __ldcg(tb + (sl + 1) * SLOT4 + o);
-                                w1[q] = __ldcg(tb + (sl + 1) * SLOT4 + o + 128);
-                            }
-#pragma unroll
-                            for (int q = 0; q < 4; ++q) {
-                                s0[q].x += u0[q].x; s0[q].y += u0[q].y; s0[q].z += u0[q].z; s0[q].w += u0[q].w;
-                                s1[q].x += u1[q].x; s1[q].y += u1[q].y; s1[q].z += u1[q].z; s1[q].w += u1[q].w;
-                                s0[q].x += w0[q].x; s0[q].y += w0[q].y; s0[q].z += w0[q].z; s0[q].w += w0[q].w;
-                                s1[q].x += w1[q].x; s1[q].y += w1[q].y; s1[q].z += w1[q].z; s1[q].w += w1[q].w;
+                            for (int u = 0; u < U; ++u) {
+                                const int pos = p0 + u * 128;
+                                if (pos < NPOS) {
+                                    const long o = sl * SLOT4 + (long)(pos >> 7) * 256 + (pos & 127);
+                                    const float4 g = __ldcg(tb + o), h = __ldcg(tb + o + 128);
+                                    s0[u].x += g.x; s0[u].y += g.y; s0[u].z += g.z; s0[u].w += g.w;
+                                    s1[u].x += h.x; s1[u].y += h.y; s1[u].z += h.z; s1[u].w += h.w;
+                                }
                             }
                         }
-                        if (sl < n) {
 #pragma unroll
-                            for (int q = 0; q < 4; ++q) {
-                                const long o = (long)(t0 / 4 + q) * 256 + r;
-                                const float4 u0 = __ldcg(tb + sl * SLOT4 + o), u1 = __ldcg(tb + sl * SLOT4 + o + 128);
-                                s0[q].x += u0.x; s0[q].y += u0.y; s0[q].z += u0.z; s0[q].w += u0.w;
-                                s1[q].x += u1.x; s1[q].y += u1.y; s1[q].z += u1.z; s1[q].w += u1.w;
-                            }
+                        for (int u = 0; u < U; ++u) {
+                            const int pos = p0 + u * 128;
+                            if (pos < NPOS) skinny_final4(a, tile, pos & 127, (pos >> 7) * 4, s0[u], s1[u]);
                         }
-                        float v0[16], v1[16];
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            v0[4 * q] = s0[q].x; v0[4 * q + 1] = s0[q].y; v0[4 * q + 2] = s0[q].z; v0[4 * q + 3] = s0[q].w;
-                            v1[4 * q] = s1[q].x; v1[4 * q + 1] = s1[q].y; v1[4 * q + 2] = s1[q].z; v1[4 * q + 3] = s1[q].w;
-                        }
-                        skinny_final16(a, tile, r, t0, v0, v1);
                     }
                     if (threadIdx.x == 64) a.tile_cnt[tile] = 0u;
                 }
                 named_bar(1, 128);   // the flag is reused by the next split tile
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&s.tempty[acc]));
             acc ^= 1;
             if (acc == 0) acc_phase ^= 1;
         }
     }
 done:
     teardown(s, tmem_base, a.status);
+}
+
+// Split tiles of the skinny tiling finished by a kernel of their own: the
+// last-arriver fixup above leaves one CTA to read every slot of a tile, which
+// at 128 tokens is ~0.4-1.2 MB of latency-bound reads at the very end of the
+// kernel.  Here one CTA of 128 threads takes one (tile, 4-token group), thread
+// r adds rows r and 128 + r over the slots in slot order -- the fixup's order,
+// so both routes give the same bits -- and applies the same epilogue.  Launched
+// behind the skinny kernel with programmatic dependent launch; tiles one CTA
+// finished whole are skipped.
+__global__ void __launch_bounds__(128) skinny_reduce_kernel(TcArgs a, int BT) {
+    pdl_allow_dependents();
+    const int quads = BT / 4;
+    const int tile = blockIdx.x / quads, qd = blockIdx.x - tile * quads;
+    const long long it0 = (long long)tile * a.KB;
+    const int c_first = share_owner(it0, a.total_iters, a.grid);
+    const int n = share_owner(it0 + a.KB - 1, a.total_iters, a.grid) - c_first + 1;
+    if (n == 1 || qd * 4 >= a.rows_x) return;
+    pdl_wait_previous();
+    const int r = threadIdx.x;
+    const long long SLOT4 = 64LL * BT;   // float4s per slot (256 rows x BT tokens)
+    const float4 *p = reinterpret_cast<const float4 *>(a.part) + (long long)tile * a.slots * SLOT4 + qd * 256 + r;
+    float4 s0 = make_float4(0.f, 0.f, 0.f, 0.f), s1 = s0;
+#pragma unroll 4
+    for (int sl = 0; sl < n; ++sl) {
+        const float4 g = __ldcg(p + sl * SLOT4), h = __ldcg(p + sl * SLOT4 + 128);
+        s0.x += g.x; s0.y += g.y; s0.z += g.z; s0.w += g.w;
+        s1.x += h.x; s1.y += h.y; s1.z += h.z; s1.w += h.w;
+    }
+    skinny_final4(a, tile, r, qd * 4, s0, s1);
 }
 
 // ======================================= host side =======================================
@@ -695,9 +746,15 @@ cudaError_t launch_skinny_bt(const WeightOperand &w, const CUtensorMap &mx, cons
     return launch_pdl(kern, dim3(grid), dim3(NTHREADS), smem, st, w.wm, mx, a);
 }
 
+// Auto: the reduction kernel.  On B200 it measured faster at every width (16 to
+// 128 tokens: 4-42 % of the step), even where the last-arriver fixup reads only
+// two 32 KB slots, because the fixup sits at the end of the GEMM's critical path.
+int resolve_split(int mode) { return mode == kSplitAuto ? kSplitSeparate : mode; }
+
 // One projection with the skinny tiling; x: T x K activations.
 cudaError_t run_skinny(const WeightOperand &w, const void *x, int T, int K, int epi, void *out, int out_cols,
-                       float *part, unsigned *cnt, int *status, int num_sms, cudaStream_t st) {
+                       float *part, unsigned *cnt, int *status, int num_sms, cudaStream_t st, int split_mode,
+                       int *launches) {
     const int BT = skinny_bt(T);
     CUtensorMap mx;
     if (!make_map(&mx, x, K, T, BT)) return cudaErrorInvalidValue;
@@ -715,16 +772,23 @@ cudaError_t run_skinny(const WeightOperand &w, const void *x, int T, int K, int 
     a.slots = g.slots;
     a.part = part;
     a.tile_cnt = cnt;
+    a.split_mode = g.slots > 1 ? resolve_split(split_mode) : kSplitInKernel;
+    a.grid = g.grid;
     a.status = status;
     a.raw_first = w.raw_first;
     a.tps = w.tps;
     a.fs = w.fs;
+    cudaError_t e;
     switch (BT) {
-        case 16: return launch_skinny_bt<16, 6>(w, mx, a, g.grid, st);
-        case 32: return launch_skinny_bt<32, 6>(w, mx, a, g.grid, st);
-        case 64: return launch_skinny_bt<64, 5>(w, mx, a, g.grid, st);
-        default: return launch_skinny_bt<128, 4>(w, mx, a, g.grid, st);
+        case 16: e = launch_skinny_bt<16, 6>(w, mx, a, g.grid, st); break;
+        case 32: e = launch_skinny_bt<32, 6>(w, mx, a, g.grid, st); break;
+        case 64: e = launch_skinny_bt<64, 5>(w, mx, a, g.grid, st); break;
+        default: e = launch_skinny_bt<128, 4>(w, mx, a, g.grid, st); break;
     }
+    ++*launches;
+    if (e != cudaSuccess || a.split_mode != kSplitSeparate) return e;
+    ++*launches;
+    return launch_pdl(skinny_reduce_kernel, dim3(g.tiles * (BT / 4)), dim3(128), 0, st, a, BT);
 }
 
 template <int MH>
@@ -801,7 +865,9 @@ size_t tc_workspace_bytes(const Problem &p, int num_sms) {
 
 cudaError_t launch_tc(const Problem &p, int tiling, const void *x, const void *w1p, const void *w2p,
                       const ShardPtrs *rawA, const ShardPtrs *rawB, void *h, void *out, float *part,
-                      unsigned *counters, int *status, int num_sms, cudaStream_t st, const Marks &marks) {
+                      unsigned *counters, int *status, int num_sms, cudaStream_t st, const Marks &marks,
+                      int split_mode, int *launches) {
+    *launches = 0;
     WeightOperand w1, w2;
     const bool raw = rawA != nullptr;
     if (raw) {
@@ -814,16 +880,19 @@ cudaError_t launch_tc(const Problem &p, int tiling, const void *x, const void *w
     marks.mark(0, st);
     if (tiling == kTilingSkinny) {
         unsigned *cnt1 = counters, *cnt2 = counters + w1.tiles;
-        e = run_skinny(w1, x, p.T, p.d_in, first_epi(p.act), h, p.d_ff, part, cnt1, status, num_sms, st);
+        e = run_skinny(w1, x, p.T, p.d_in, first_epi(p.act), h, p.d_ff, part, cnt1, status, num_sms, st,
+                       split_mode, launches);
         if (e != cudaSuccess) return e;
         marks.mark(1, st);
-        e = run_skinny(w2, h, p.T, p.d_ff, EPI_OUT, out, p.d_out, part, cnt2, status, num_sms, st);
+        e = run_skinny(w2, h, p.T, p.d_ff, EPI_OUT, out, p.d_out, part, cnt2, status, num_sms, st, split_mode,
+                       launches);
     } else {
         auto wide = tiling == kTilingWide256 ? run_wide<2> : run_wide<1>;
         e = wide(w1, x, p.T, p.d_in, first_epi(p.act), h, p.d_ff, status, num_sms, st);
         if (e != cudaSuccess) return e;
         marks.mark(1, st);
         e = wide(w2, h, p.T, p.d_ff, EPI_OUT, out, p.d_out, status, num_sms, st);
+        *launches = 2;
     }
     marks.mark(2, st);
     return e;

@@ -57,6 +57,7 @@ struct tp_mlp_s {
     void *ws;
     size_t ws_bytes;
     int plan;            // forced tp_mlp_plan
+    int splitk;          // tp_mlp_splitk: how the skinny tiling finishes split tiles
     int last_plan, last_launches;
     Marks marks;         // timing hook
     // split-K scratch each token count needs, precomputed at creation:
@@ -212,6 +213,7 @@ int tp_mlp_create(tp_mlp_t *handle, int d_model, int d_ff, int d_out, int tp_deg
     h->ws = nullptr;
     h->ws_bytes = 0;
     h->plan = TP_MLP_PLAN_AUTO;
+    h->splitk = TP_MLP_SPLITK_AUTO;
     h->last_plan = -1;
     h->last_launches = -1;
     memset(&h->marks, 0, sizeof(h->marks));
@@ -299,18 +301,19 @@ static int run_shard_form(tp_mlp_t h, const void *x, int tokens, const void *con
     const ShardPtrs a = to_ptrs(A, h->tp), b = to_ptrs(B, h->tp);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t ce;
+    int launches = 2;
     if (is_tc) {
         const int tiling = plan == TP_MLP_PLAN_TC_SKINNY ? kTilingSkinny
                            : plan == TP_MLP_PLAN_TC_WIDE ? kTilingWide128 : kTilingWide256;
         float *part = reinterpret_cast<float *>(ws + counters_bytes(h) + h_bytes(h, tokens));
         ce = launch_tc(p, tiling, x, nullptr, nullptr, &a, &b, hbuf, out, part, reinterpret_cast<unsigned *>(ws),
-                       status_word(h), h->num_sms, st, h->marks);
+                       status_word(h), h->num_sms, st, h->marks, h->splitk, &launches);
     } else {
         ce = launch_simt(p, false, x, a, b, hbuf, out, partials, st, h->marks);
     }
     if (ce != cudaSuccess) return TP_MLP_ERR_CUDA;
     h->last_plan = plan;
-    h->last_launches = 2;
+    h->last_launches = launches;
     return TP_MLP_OK;
 }
 
@@ -407,7 +410,7 @@ int tp_mlp_forward_packed(tp_mlp_t h, const void *x, int tokens, const void *pac
         const int tiling = plan == TP_MLP_PLAN_TC_SKINNY ? kTilingSkinny
                            : plan == TP_MLP_PLAN_TC_WIDE ? kTilingWide128 : kTilingWide256;
         ce = launch_tc(p, tiling, x, w1p, w2p, nullptr, nullptr, hbuf, out, part, counters, status_word(h),
-                       h->num_sms, st, h->marks);
+                       h->num_sms, st, h->marks, h->splitk, &launches);
     } else {
         ShardPtrs a, b;
         memset(&a, 0, sizeof(a));
@@ -445,6 +448,13 @@ int tp_mlp_set_plan(tp_mlp_t h, int plan) {
     if (!h) return TP_MLP_ERR_INVALID_ARG;
     if (plan < TP_MLP_PLAN_AUTO || plan > TP_MLP_PLAN_TC_WIDE256) return TP_MLP_ERR_INVALID_ARG;
     h->plan = plan;
+    return TP_MLP_OK;
+}
+
+int tp_mlp_set_splitk(tp_mlp_t h, int mode) {
+    if (!h) return TP_MLP_ERR_INVALID_ARG;
+    if (mode < TP_MLP_SPLITK_AUTO || mode > TP_MLP_SPLITK_SEPARATE) return TP_MLP_ERR_INVALID_ARG;
+    h->splitk = mode;
     return TP_MLP_OK;
 }
 

@@ -89,6 +89,36 @@ def test_tc_skinny_parity(act, T, shape):
 
 
 @pytest.mark.parametrize("act", ["swiglu", "tanh"])
+@pytest.mark.parametrize("T", [5, 32, 100, 128])
+@pytest.mark.parametrize("shape", SHAPES)
+def test_tc_skinny_split_finish_modes_agree(act, T, shape):
+    """Split tiles finished by the last CTA inside the GEMM, or by the reduction
+    kernel behind it: both add the partial slots in slot order, so the outputs
+    are identical, and both match the oracle."""
+    d, f, dout, tp = shape
+    p = inputs.generate(T, d, f, act, "bf16", seed=7 * T + f, init="fan_in", d_out=dout)
+    A, Bs = p.shards(tp)
+    ref = oracle.tp_mlp_sharded(p.x, A, Bs, act)
+    m = B().TpMlp(d, f, tp, act, "bf16", T, d_out=dout)
+    m.set_plan("tc_skinny")
+    packed = m.pack([dev(a, "bf16") for a in A], [dev(b, "bf16") for b in Bs])
+    x = dev(p.x, "bf16")
+    outs = {}
+    for mode in ("in_kernel", "separate", "in_kernel"):
+        m.set_splitk(mode)
+        out = m.forward_packed(x, packed)
+        torch.cuda.synchronize()
+        B().tp_mlp_get_device_status(m.h)
+        assert_close(out, ref, "bf16", f"skinny {mode} T={T}")
+        # every tile of these shapes is split: one reduction kernel per projection
+        assert m.last_launches == (4 if mode == "separate" else 2)
+        if mode in outs:
+            assert torch.equal(out, outs[mode])     # counters were left at zero
+        outs[mode] = out
+    assert torch.equal(outs["in_kernel"], outs["separate"])
+
+
+@pytest.mark.parametrize("act", ["swiglu", "tanh"])
 @pytest.mark.parametrize("T", [1, 127, 128, 129, 300, 1000])
 @pytest.mark.parametrize("shape", SHAPES[:3])
 def test_tc_wide_parity(act, T, shape):
@@ -177,6 +207,25 @@ def test_tc_shard_form_parity(act, plan, T, shape):
     rows = p.sample_rows(64)
     ref = oracle.tp_mlp_sharded(p.x[rows], A, Bs, act)
     assert_close(out[torch.from_numpy(rows).cuda()], ref, "bf16", f"shard form {plan} T={T}")
+
+
+@pytest.mark.parametrize("T", [9, 64, 128])
+def test_tc_shard_form_split_finish_modes_agree(T):
+    d, f, dout, tp = RAW_SHAPES[0]
+    p = inputs.generate(T, d, f, "swiglu", "bf16", seed=T + 11, init="fan_in", d_out=dout)
+    A, Bs = p.shards(tp)
+    Ad, Bd = [dev(a, "bf16") for a in A], [dev(b, "bf16") for b in Bs]
+    ref = oracle.tp_mlp_sharded(p.x, A, Bs, "swiglu")
+    m = B().TpMlp(d, f, tp, "swiglu", "bf16", T, d_out=dout)
+    m.set_plan("tc_skinny")
+    outs = []
+    for mode in ("in_kernel", "separate"):
+        m.set_splitk(mode)
+        outs.append(m.forward(dev(p.x, "bf16"), Ad, Bd))
+        torch.cuda.synchronize()
+        B().tp_mlp_get_device_status(m.h)
+        assert_close(outs[-1], ref, "bf16", f"shard form {mode} T={T}")
+    assert torch.equal(outs[0], outs[1])
 
 
 @pytest.mark.parametrize("plan,T", [("tc_skinny", 3), ("tc_wide", 130), ("tc_wide256", 257)])
