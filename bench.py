@@ -54,6 +54,7 @@ def parse():
                     help="packed: weights packed once, tp_mlp_forward_packed; shard: tp_mlp_forward on the shards")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph replay percentiles")
     return ap.parse_args()
 
 
@@ -170,20 +171,73 @@ class ClockSampler:
                 "window": "timed region" if sel is not self.samples else "warm-up + timed region"}
 
 
-def oracle_baseline(p, A, Bs, act, budget_s=12.0, max_calls=50):
-    """Time the oracle as it stands on a bounded sample: whole calls until the budget is spent."""
+def _oracle_rate(p, A, Bs, act, budget_s, max_calls):
     import oracle
-    T = p.tokens
     calls, t_total = 0, 0.0
     while calls < max_calls and t_total < budget_s:
         t0 = time.perf_counter()
         oracle.tp_mlp_sharded(p.x, A, Bs, act)
         t_total += time.perf_counter() - t0
         calls += 1
+    return p.tokens * calls / t_total, calls, t_total
+
+
+def oracle_baseline(p, A, Bs, act, budget_s=12.0, max_calls=50):
+    """Time the oracle as it stands on a bounded sample: whole calls until the budget is spent.
+    With more than one token the oracle's OpenMP loop can use several cores, so it is
+    also timed on one core; with one token both are the same run."""
+    import oracle
+    T = p.tokens
+    nproc = os.cpu_count()
+    try:
+        affinity = len(os.sched_getaffinity(0))
+    except AttributeError:
+        affinity = nproc
     threads = min(oracle.max_threads(), T)
-    return {"value": T * calls / t_total, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-            "sample": f"{calls} full forward(s) of this workload ({T} token(s) each) on the host, "
-                      f"{t_total:.1f} s; the oracle runs OpenMP over tokens"}
+    value, calls, t_total = _oracle_rate(p, A, Bs, act, budget_s, max_calls)
+    out = {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+           "host_nproc": nproc, "host_affinity": affinity,
+           "sample": f"{calls} full forward(s) of this workload ({T} token(s) each) on the host, "
+                     f"{t_total:.1f} s; the oracle runs OpenMP over tokens"}
+    if threads > 1:
+        oracle.set_threads(1)
+        try:
+            v1, c1, t1 = _oracle_rate(p, A, Bs, act, budget_s / 2, max_calls)
+        finally:
+            oracle.set_threads(oracle.max_threads())
+        out["one_core"] = {"value": v1, "sample": f"{c1} full forward(s), {t1:.1f} s"}
+    return out
+
+
+def graph_replay_stats(fwd, K, W):
+    """Per-step device time of the forward captured once in a CUDA graph and
+    replayed K times, each replay bracketed by its own events (so a replay does
+    not overlap the previous one): median and 10th / 90th percentiles, in us."""
+    import torch
+    gs = torch.cuda.Stream()
+    gs.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(gs):
+        fwd()
+    gs.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=gs):
+        fwd()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    with torch.cuda.stream(gs):
+        for _ in range(W):
+            g.replay()
+        for a, b in ev:
+            a.record(gs)
+            g.replay()
+            b.record(gs)
+    gs.synchronize()
+    d = sorted(a.elapsed_time(b) * 1e3 for a, b in ev)
+    del g
+
+    def pct(q):
+        return d[min(len(d) - 1, int(round(q * (len(d) - 1))))]
+    return {"p10_us": pct(0.1), "p50_us": pct(0.5), "p90_us": pct(0.9), "replays": K,
+            "timer": "CUDA events around each replay of the captured forward"}
 
 
 def run_reference(args):
@@ -306,6 +360,10 @@ def main():
     barrier()
     kern_ms = [statistics.fmean(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(K)) for j in range(nph)]
     elapsed_ms = replicas.max_over_ranks(elapsed_ms)
+    graph_steps = None
+    if not args.no_graph:
+        graph_steps = graph_replay_stats(fwd, max(K, 50), W)
+        barrier()
 
     # end to end through the public API with host buffers (pinned), copies inside
     # the region: binding.GraphStep replays H2D(x) + forward + D2H(out) as one
@@ -367,7 +425,8 @@ def main():
                        "plan": plan, "splitk": args.splitk, "api": args.api, "parallelism": "replicas" if world > 1 else "single GPU",
                        "l2": "inputs larger than L2: every step re-reads %.2f GB of weights" % (step_bytes / 1e9)},
             "step_hbm_gbs": step_bytes / (ms / 1e3) / 1e9, "step_tflops": step_flops / (ms / 1e3) / 1e12,
-            "roofline": roofline, "gpu_launches": K * nk, "clocks": sampler.summary(), "e2e": e2e}
+            "roofline": roofline, "gpu_launches": K * nk, "clocks": sampler.summary(), "e2e": e2e,
+            "graph_step": graph_steps}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = oracle_baseline(p, A, Bs, act)
     if rank == 0:

@@ -10,11 +10,15 @@ arithmetic.
 The arithmetic lives in ``tp_mlp_oracle.c`` (plain C loops, fp64).  This module
 compiles it with gcc on first use and marshals numpy arrays into it.
 
+The fused all-reduce + residual add + RMSNorm lives in ``fused_norm_oracle.c``.
+
 Sources (page title and section):
   * "LLM 推理并行化：先找瓶颈，再决定怎么切", §三 2) 张量并行（TP） — the
     tensor_parallel_output function: per rank act(x @ A_i) @ B_i, summed.
   * "大模型推理系统揭秘（07）：Multi-GPU：一张卡不够时如何扩展？", §1.2.2–§1.2.4
     (column/row parallel linears, Z = sum_i Y_i W_2i) and §1.4.3 (SwiGLU).
+  * "7.4 推理侧并行", §7.4.2, optimisation 2 — the residual add and RMSNorm
+    that follow the all-reduce, fused with it.
 """
 from __future__ import annotations
 
@@ -26,7 +30,7 @@ import threading
 import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-_SRC = os.path.join(_HERE, "tp_mlp_oracle.c")
+_SRCS = [os.path.join(_HERE, n) for n in ("tp_mlp_oracle.c", "fused_norm_oracle.c")]
 _LIB = os.path.join(_HERE, "libtp_mlp_oracle.so")
 _lock = threading.Lock()
 _lib = None
@@ -36,10 +40,11 @@ ACTS = {"tanh": 0, "swiglu": 1, "identity": 2}
 
 def build(force: bool = False) -> str:
     """Compile the oracle with gcc (-O2, OpenMP, no FMA contraction)."""
-    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+    stale = not os.path.exists(_LIB) or any(os.path.getmtime(_LIB) < os.path.getmtime(s) for s in _SRCS)
+    if force or stale:
         tmp = _LIB + f".tmp{os.getpid()}"
         cmd = ["gcc", "-O2", "-std=c11", "-fopenmp", "-ffp-contract=off", "-fno-fast-math",
-               "-fPIC", "-shared", "-o", tmp, _SRC, "-lm"]
+               "-fPIC", "-shared", "-o", tmp] + _SRCS + ["-lm"]
         subprocess.run(cmd, check=True)
         os.replace(tmp, _LIB)
     return _LIB
@@ -61,6 +66,9 @@ def _load():
             lib.oracle_tp_mlp_unsharded.argtypes = [
                 fp, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                 fp, fp, fp, dp]
+            lib.oracle_allreduce_residual_rmsnorm.restype = ctypes.c_int
+            lib.oracle_allreduce_residual_rmsnorm.argtypes = [
+                fp, ctypes.c_int, ctypes.c_int, ctypes.c_int, fp, fp, ctypes.c_double, dp, dp]
             lib.oracle_max_threads.restype = ctypes.c_int
             lib.oracle_set_threads.argtypes = [ctypes.c_int]
             _lib = lib
@@ -177,3 +185,28 @@ def tp_mlp_unsharded(x, a, b, act: str = "tanh", a_up=None, *, return_macs=False
     if macs < 0:
         raise ValueError("oracle rejected the arguments")
     return (z, int(macs)) if return_macs else z
+
+
+def allreduce_residual_rmsnorm(partials, residual, gamma, eps: float):
+    """The rank sum followed by the residual add and RMSNorm, in fp64.
+
+    partials: P x T x d (every rank's Z_i); residual: T x d; gamma: d.
+    h = residual + sum_i Z_i (ranks in order); y = h / sqrt(mean(h^2) + eps) * gamma,
+    row by row.  Returns (y, h), both T x d float64.
+    """
+    p = _f32(partials)
+    r = _f32(residual)
+    g = _f32(gamma)
+    if p.ndim != 3 or r.ndim != 2 or g.ndim != 1:
+        raise ValueError("partials must be P x T x d, residual T x d, gamma d")
+    P, T, d = p.shape
+    if r.shape != (T, d) or g.shape != (d,):
+        raise ValueError(f"residual {r.shape} / gamma {g.shape} do not match partials {p.shape}")
+    y = np.full((T, d), np.nan, dtype=np.float64)
+    h = np.full((T, d), np.nan, dtype=np.float64)
+    dp = ctypes.POINTER(ctypes.c_double)
+    rc = _load().oracle_allreduce_residual_rmsnorm(_fptr(p), P, T, d, _fptr(r), _fptr(g), float(eps),
+                                                   y.ctypes.data_as(dp), h.ctypes.data_as(dp))
+    if rc != 0:
+        raise ValueError("oracle rejected the arguments")
+    return y, h
