@@ -133,7 +133,8 @@ def summarize_full(report: str, title: str, cmd: str, traffic_key=None, scale=1.
             if li == launch:
                 traffic = (rd + wr) * scale
             out += ["", f"DRAM traffic per launch: {(rd + wr) / 1e6:.1f} MB"
-                    + (f"; scaled ×{scale:g} to the full workload: {traffic / 1e6:.1f} MB" if scale != 1 else "")]
+                    + (f"; scaled ×{scale:g} to the full workload: {(rd + wr) * scale / 1e6:.1f} MB"
+                       if scale != 1 else "")]
         except (KeyError, ValueError):
             pass
         out.append("")
