@@ -270,6 +270,37 @@ int tp_mlp_decode_forward_static(int d_model, int d_ff, int d_out, int tp_degree
                                  const void *x, int tokens, const void *packed, void *out,
                                  tp_mlp_stream_t stream);
 
+/*
+ * The all-reduce of the ranks' partial outputs fused with the residual add and
+ * RMSNorm that follow it ("7.4 推理侧并行", §7.4.2, optimisation 2: fusing
+ * them saves a round trip of the summed activations through memory).  With
+ * every rank on one GPU the all-reduce is the sum of the fp32 partials that
+ * tp_mlp_partials returns.  For every token row t (ranks added in order,
+ * fp32 arithmetic):
+ *     h               = residual[t] + sum_i partials[i][t]
+ *     residual_out[t] = h
+ *     y[t]            = h / sqrt(mean_j h_j^2 + eps) * gamma
+ * The pages do not define RMSNorm; this is the textbook form (no mean
+ * subtraction, no bias).  Needs no handle and no workspace.
+ *
+ *   partials      device fp32, tp_degree x tokens x d, row-major (rank-major)
+ *   residual      device, tokens x d, element type `dtype` (tp_mlp_dtype)
+ *   gamma         device, d elements of `dtype`
+ *   y             device, tokens x d of `dtype`
+ *   residual_out  device, tokens x d of `dtype`; may be `residual` itself
+ *                 (updated in place).  Other overlaps between the buffers are
+ *                 not allowed.
+ * Requirements: 1 <= tp_degree <= 8, tokens >= 0 (0 is a no-op),
+ * 4 <= d <= 49152 with d % 4 == 0 (TP_MLP_ERR_SHAPE otherwise), eps >= 0 and
+ * finite (TP_MLP_ERR_INVALID_ARG), every pointer 16-byte aligned
+ * (TP_MLP_ERR_ALIGNMENT) and inside a device allocation of the stated size
+ * (TP_MLP_ERR_SHAPE / TP_MLP_ERR_INVALID_ARG).  Asynchronous on `stream`;
+ * the caller owns every buffer.
+ */
+int tp_mlp_allreduce_residual_rmsnorm(const float *partials, int tp_degree, int tokens, int d,
+                                      const void *residual, const void *gamma, float eps, int dtype,
+                                      void *y, void *residual_out, tp_mlp_stream_t stream);
+
 /* Human-readable name of a status code (static string). */
 const char *tp_mlp_status_string(int status);
 

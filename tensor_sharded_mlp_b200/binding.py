@@ -49,6 +49,7 @@ _SIGS = {
     "tp_mlp_forward_packed": (_i, [_vp, _vp, _i, _vp, _vp, _vp]),
     "tp_mlp_set_plan": (_i, [_vp, _i]),
     "tp_mlp_set_splitk": (_i, [_vp, _i]),
+    "tp_mlp_allreduce_residual_rmsnorm": (_i, [_vp, _i, _i, _i, _vp, _vp, ctypes.c_float, _i, _vp, _vp, _vp]),
     "tp_mlp_set_profile_events": (_i, [_vp, _vpp, _i]),
     "tp_mlp_get_device_status": (_i, [_vp]),
     "tp_mlp_selftest_bounded_wait": (_i, [_vp, ctypes.c_uint, _vp]),
@@ -210,6 +211,37 @@ def tp_mlp_decode_forward_static(d_model: int, d_ff: int, d_out: int, tp_degree:
     _check("tp_mlp_decode_forward_static",
            _lib.tp_mlp_decode_forward_static(d_model, d_ff, d_out, tp_degree, ACT[act], _ptr(x), x.shape[0],
                                              _ptr(packed), _ptr(out), _stream(stream)))
+
+
+def tp_mlp_allreduce_residual_rmsnorm(partials: torch.Tensor, residual: torch.Tensor, gamma: torch.Tensor,
+                                      eps: float, y: Optional[torch.Tensor] = None,
+                                      residual_out: Optional[torch.Tensor] = None, stream=None):
+    """The rank sum of fp32 partials (P x T x d) fused with the residual add and
+    RMSNorm: h = residual + sum_i partials[i], y = h / sqrt(mean(h^2) + eps) * gamma.
+    residual_out may be residual itself (in-place update).  Returns (y, residual_out)."""
+    if partials.dtype != torch.float32 or partials.dim() != 3 or not partials.is_contiguous():
+        raise ValueError("partials must be a contiguous float32 tensor (P, T, d)")
+    P, T, d = partials.shape
+    dt = residual.dtype
+    if dt not in (torch.float32, torch.bfloat16):
+        raise ValueError("residual must be float32 or bfloat16")
+    if residual.shape != (T, d) or gamma.shape != (d,) or gamma.dtype != dt:
+        raise ValueError("residual must be (T, d) and gamma (d,), of one dtype")
+    for t in (partials, residual, gamma):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("tensors must be contiguous CUDA tensors")
+    if y is None:
+        y = torch.empty_like(residual)
+    if residual_out is None:
+        residual_out = torch.empty_like(residual)
+    for t in (y, residual_out):
+        if t.shape != (T, d) or t.dtype != dt or not t.is_contiguous():
+            raise ValueError("y / residual_out must be contiguous (T, d) tensors of the residual's dtype")
+    _check("tp_mlp_allreduce_residual_rmsnorm",
+           _lib.tp_mlp_allreduce_residual_rmsnorm(_ptr(partials), P, T, d, _ptr(residual), _ptr(gamma),
+                                                  float(eps), DTYPE["f32" if dt == torch.float32 else "bf16"],
+                                                  _ptr(y), _ptr(residual_out), _stream(stream)))
+    return y, residual_out
 
 
 # --- convenience wrapper -----------------------------------------------------------

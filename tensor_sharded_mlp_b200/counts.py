@@ -76,9 +76,27 @@ def allreduce_bytes(batch: int, seq: int, d_model: int, elem_bytes: int) -> int:
     return batch * seq * d_model * elem_bytes
 
 
+def fused_norm_bytes(tp: int, tokens: int, d_model: int, dtype: str) -> int:
+    """Bytes the fused all-reduce + residual add + RMSNorm must move: every
+    rank's fp32 partial row read once, the residual and gamma read, y and the
+    updated residual written ("7.4 推理侧并行" §7.4.2, optimisation 2)."""
+    e = 4 if dtype == "f32" else 2
+    n = tokens * d_model
+    return tp * n * 4 + n * e + d_model * e + 2 * n * e
+
+
+def unfused_norm_bytes(tp: int, tokens: int, d_model: int, dtype: str) -> int:
+    """The same step as three kernels (all-reduce writing Z in the activation
+    dtype, residual add, RMSNorm): Z and h each make one extra round trip."""
+    e = 4 if dtype == "f32" else 2
+    n = tokens * d_model
+    return fused_norm_bytes(tp, tokens, d_model, dtype) + 2 * (2 * n * e)
+
+
 # Source files that define each kernel family (for "was this profile taken on
 # the current kernel?" checks).
 _KERNEL_SOURCES = {
+    "fused_norm": ["fused_norm.cu", "common.cuh", "tc_ptx.cuh"],
     "gemv": ["gemv.cu", "common.cuh", "streamk.cuh", "tc_ptx.cuh"],
     "tc_skinny": ["tc_gemm.cu", "common.cuh", "streamk.cuh", "tc_ptx.cuh"],
     "tc_wide": ["tc_gemm.cu", "common.cuh", "streamk.cuh", "tc_ptx.cuh"],

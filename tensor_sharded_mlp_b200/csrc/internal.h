@@ -33,6 +33,14 @@ cudaError_t launch_pack(const Problem &p, const ShardPtrs &a, const ShardPtrs &b
 // selftest.cu: a bounded wait that runs out, recorded in *status.
 cudaError_t launch_bounded_wait_selftest(int *status, unsigned wait_us, cudaStream_t st);
 
+// fused_norm.cu: the rank sum of fp32 partials (P x rows x d) + residual add +
+// RMSNorm, one kernel (clusters of up to kNormClusterMax CTAs per row).
+constexpr int kNormClusterMax = 8;
+constexpr int kNormMaxWidth = 49152;   // h of a row chunk lives in shared memory
+cudaError_t launch_allreduce_norm(const float *partials, int P, int rows, int d, const void *residual,
+                                  const void *gamma, float eps, int dtype, void *y, void *residual_out,
+                                  int num_sms, cudaStream_t st);
+
 // Split-tile counters the GEMV and tcgen05 skinny kernels need (one per
 // weight tile of both parts; first part's tiles first).
 size_t tile_counter_slots(const Problem &p);

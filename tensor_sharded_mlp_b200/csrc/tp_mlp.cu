@@ -9,6 +9,7 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <cmath>
 #include <mutex>
 #include <new>
 
@@ -449,6 +450,30 @@ int tp_mlp_set_plan(tp_mlp_t h, int plan) {
     if (plan < TP_MLP_PLAN_AUTO || plan > TP_MLP_PLAN_TC_WIDE256) return TP_MLP_ERR_INVALID_ARG;
     h->plan = plan;
     return TP_MLP_OK;
+}
+
+int tp_mlp_allreduce_residual_rmsnorm(const float *partials, int tp_degree, int tokens, int d,
+                                      const void *residual, const void *gamma, float eps, int dtype,
+                                      void *y, void *residual_out, tp_mlp_stream_t stream) {
+    if (tp_degree < 1 || tp_degree > kMaxTp || tokens < 0) return TP_MLP_ERR_SHAPE;
+    if (d < 4 || d > kNormMaxWidth || d % 4 != 0) return TP_MLP_ERR_SHAPE;
+    if (!(eps >= 0.f) || !std::isfinite(eps)) return TP_MLP_ERR_INVALID_ARG;
+    if (dtype != TP_MLP_F32 && dtype != TP_MLP_BF16) return TP_MLP_ERR_INVALID_ARG;
+    if (tokens == 0) return TP_MLP_OK;   // empty tensors may carry null pointers
+    if (!partials || !residual || !gamma || !y || !residual_out) return TP_MLP_ERR_INVALID_ARG;
+    const size_t e = elem_bytes(dtype), n = (size_t)tokens * d;
+    int s;
+    if ((s = check_dev(partials, (size_t)tp_degree * n * sizeof(float)))) return s;
+    if ((s = check_dev(residual, n * e))) return s;
+    if ((s = check_dev(gamma, (size_t)d * e))) return s;
+    if ((s = check_dev(y, n * e))) return s;
+    if ((s = check_dev(residual_out, n * e))) return s;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
+        return TP_MLP_ERR_CUDA;
+    return from_cuda(launch_allreduce_norm(partials, tp_degree, tokens, d, residual, gamma, eps, dtype, y,
+                                           residual_out, sms, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 int tp_mlp_set_splitk(tp_mlp_t h, int mode) {

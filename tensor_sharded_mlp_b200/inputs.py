@@ -48,6 +48,40 @@ CONFIGS = {
 }
 
 
+# The fused all-reduce + residual add + RMSNorm step ("7.4 推理侧并行" §7.4.2):
+# P rank partials of the second projection's output, the residual stream and
+# the norm's gain, at the decode batch-32 and prefill shapes of the MLP configs.
+FUSED_NORM_CONFIGS = {
+    "fused_norm_decode_bs32": dict(dtype="bf16", tokens=32, d_model=8192, tp=8, eps=1e-5, seed=21),
+    "fused_norm_prefill": dict(dtype="bf16", tokens=8192, d_model=8192, tp=8, eps=1e-5, seed=22),
+}
+
+
+@dataclasses.dataclass
+class FusedNormInputs:
+    partials: np.ndarray   # P x T x d, fp32
+    residual: np.ndarray   # T x d (dtype-representable values in fp32)
+    gamma: np.ndarray      # d
+    eps: float
+
+
+def generate_fused_norm(tokens: int, d_model: int, tp: int, dtype: str, seed: int, eps: float = 1e-5
+                        ) -> FusedNormInputs:
+    """Seeded inputs of the fused step: rng(seed), float64 standard normals drawn
+    in the order partials (P x T x d, N(0, 1), kept fp32), residual (T x d,
+    N(0, 1)), gamma (d, 1 + 0.1 N(0, 1)); residual and gamma rounded to bf16 for
+    a bf16 config."""
+    rng = np.random.default_rng(seed)
+    part = np.empty((tp, tokens, d_model), np.float32)
+    for i in range(tp):
+        part[i] = _draw(rng, tokens, d_model, 1.0, "f32")
+    res = _draw(rng, tokens, d_model, 1.0, dtype)
+    g = (1.0 + 0.1 * rng.standard_normal(d_model)).astype(np.float32)
+    if dtype == "bf16":
+        g = round_to_bf16(g)
+    return FusedNormInputs(part, res, g, eps)
+
+
 def round_to_bf16(a: np.ndarray) -> np.ndarray:
     """Round fp32 values to the nearest bf16 (ties to even); returns fp32 holding them."""
     a = np.ascontiguousarray(a, dtype=np.float32)

@@ -141,6 +141,16 @@ def test_call_argument_errors_before_any_launch(b):
     assert L.tp_mlp_set_profile_events(h, None, 9) == 1
     assert L.tp_mlp_set_splitk(h, 3) == 1 and L.tp_mlp_set_splitk(h, -1) == 1
     assert L.tp_mlp_set_splitk(None, 0) == 1
+    # fused all-reduce + residual + RMSNorm: argument checks come before any pointer use
+    F = L.tp_mlp_allreduce_residual_rmsnorm
+    assert F(None, 0, 1, 64, None, None, 0.0, 0, None, None, None) == 2       # tp_degree
+    assert F(None, 2, 1, 62, None, None, 0.0, 0, None, None, None) == 2       # d % 4
+    assert F(None, 2, 1, 49156, None, None, 0.0, 0, None, None, None) == 2    # too wide
+    assert F(None, 2, 1, 64, None, None, -1.0, 0, None, None, None) == 1      # eps < 0
+    assert F(None, 2, 1, 64, None, None, float("inf"), 0, None, None, None) == 1
+    assert F(None, 2, 1, 64, None, None, 0.0, 7, None, None, None) == 1       # dtype
+    assert F(None, 2, 1, 64, None, None, 0.0, 0, None, None, None) == 1       # null pointers
+    assert F(None, 2, 0, 64, None, None, 0.0, 0, None, None, None) == 0       # no tokens: no-op
     for mode in (2, 1, 0):
         assert L.tp_mlp_set_splitk(h, mode) == 0
     assert L.tp_mlp_last_plan(h) == 1 and L.tp_mlp_last_launches(h) == 0        # the 0-token no-op
