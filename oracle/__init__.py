@@ -10,7 +10,8 @@ arithmetic.
 The arithmetic lives in ``tp_mlp_oracle.c`` (plain C loops, fp64).  This module
 compiles it with gcc on first use and marshals numpy arrays into it.
 
-The fused all-reduce + residual add + RMSNorm lives in ``fused_norm_oracle.c``.
+The fused all-reduce + residual add + RMSNorm lives in ``fused_norm_oracle.c``,
+the merge of attention partials across KV shards in ``attn_merge_oracle.c``.
 
 Sources (page title and section):
   * "LLM 推理并行化：先找瓶颈，再决定怎么切", §三 2) 张量并行（TP） — the
@@ -19,6 +20,8 @@ Sources (page title and section):
     (column/row parallel linears, Z = sum_i Y_i W_2i) and §1.4.3 (SwiGLU).
   * "7.4 推理侧并行", §7.4.2, optimisation 2 — the residual add and RMSNorm
     that follow the all-reduce, fused with it.
+  * "LLM 推理并行化：先找瓶颈，再决定怎么切", §三 4) 上下文并行（CP） — decode
+    context parallelism: merging the ranks' partial attention results.
 """
 from __future__ import annotations
 
@@ -30,7 +33,7 @@ import threading
 import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-_SRCS = [os.path.join(_HERE, n) for n in ("tp_mlp_oracle.c", "fused_norm_oracle.c")]
+_SRCS = [os.path.join(_HERE, n) for n in ("tp_mlp_oracle.c", "fused_norm_oracle.c", "attn_merge_oracle.c")]
 _LIB = os.path.join(_HERE, "libtp_mlp_oracle.so")
 _lock = threading.Lock()
 _lib = None
@@ -69,6 +72,13 @@ def _load():
             lib.oracle_allreduce_residual_rmsnorm.restype = ctypes.c_int
             lib.oracle_allreduce_residual_rmsnorm.argtypes = [
                 fp, ctypes.c_int, ctypes.c_int, ctypes.c_int, fp, fp, ctypes.c_double, dp, dp]
+            for name in ("oracle_attention_partial", "oracle_merge_attention_partials", "oracle_attention_full"):
+                getattr(lib, name).restype = ctypes.c_int
+            lib.oracle_attention_partial.argtypes = [fp, fp, fp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                     ctypes.c_double, dp, dp, dp]
+            lib.oracle_merge_attention_partials.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, fp, fp, fp, dp]
+            lib.oracle_attention_full.argtypes = [fp, fp, fp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                  ctypes.c_double, dp]
             lib.oracle_max_threads.restype = ctypes.c_int
             lib.oracle_set_threads.argtypes = [ctypes.c_int]
             _lib = lib
@@ -210,3 +220,48 @@ def allreduce_residual_rmsnorm(partials, residual, gamma, eps: float):
     if rc != 0:
         raise ValueError("oracle rejected the arguments")
     return y, h
+
+
+def attention_partial(q, k, v, scale: float):
+    """One rank's partial attention over its KV shard, in fp64: per query row the
+    maximum score, the sum of exp(score - maximum) and the exp-weighted sum of
+    the values.  q: rows x D, k and v: n_keys x D (n_keys may be 0)."""
+    q, k, v = _f32(q), _f32(k), _f32(v)
+    rows, D = q.shape
+    n = k.shape[0]
+    if k.shape != (n, D) or v.shape != (n, D):
+        raise ValueError("k and v must be n_keys x D")
+    m = np.full(rows, np.nan)
+    s = np.full(rows, np.nan)
+    w = np.full((rows, D), np.nan)
+    dp = ctypes.POINTER(ctypes.c_double)
+    if _load().oracle_attention_partial(_fptr(q), _fptr(k), _fptr(v), rows, n, D, float(scale),
+                                        m.ctypes.data_as(dp), s.ctypes.data_as(dp), w.ctypes.data_as(dp)) != 0:
+        raise ValueError("oracle rejected the arguments")
+    return m, s, w
+
+
+def merge_attention_partials(maximum, exp_sum, weighted):
+    """Merge P ranks' partials (maximum, exp_sum: P x rows; weighted: P x rows x D),
+    in fp64: rescale each rank by exp(its maximum - the global maximum), add,
+    divide.  Rows with every rank empty (maximum -inf) merge to zeros."""
+    m, s, w = _f32(maximum), _f32(exp_sum), _f32(weighted)
+    if m.ndim != 2 or s.shape != m.shape or w.ndim != 3 or w.shape[:2] != m.shape:
+        raise ValueError("maximum and exp_sum must be P x rows, weighted P x rows x D")
+    P, rows, D = w.shape
+    out = np.full((rows, D), np.nan)
+    if _load().oracle_merge_attention_partials(P, rows, D, _fptr(m), _fptr(s), _fptr(w),
+                                               out.ctypes.data_as(ctypes.POINTER(ctypes.c_double))) != 0:
+        raise ValueError("oracle rejected the arguments")
+    return out
+
+
+def attention_full(q, k, v, scale: float):
+    """Softmax attention of every query row over all keys, in fp64."""
+    q, k, v = _f32(q), _f32(k), _f32(v)
+    rows, D = q.shape
+    out = np.full((rows, D), np.nan)
+    if _load().oracle_attention_full(_fptr(q), _fptr(k), _fptr(v), rows, k.shape[0], D, float(scale),
+                                     out.ctypes.data_as(ctypes.POINTER(ctypes.c_double))) != 0:
+        raise ValueError("oracle rejected the arguments")
+    return out
