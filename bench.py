@@ -240,35 +240,6 @@ def graph_replay_stats(fwd, K, W):
             "timer": "CUDA events around each replay of the captured forward"}
 
 
-def run_fused_norm_reference(args):
-    """Reference arm of the fused step: the oracle on whole rows, bounded."""
-    if int(os.environ.get("RANK", 0)) != 0:
-        return 0
-    from tensor_sharded_mlp_b200 import inputs
-    c = _fused_norm_config(args)
-    fi = inputs.generate_fused_norm(c["tokens"], c["d_model"], c["tp"], c["dtype"], c["seed"], c["eps"])
-    budget = 150.0 / max(1, args.steps + args.warmup)
-    rates = []
-    for i in range(args.warmup + args.steps):
-        v, rows, tt = fused_norm_oracle_rate(fi, budget)
-        if i >= args.warmup:
-            rates.append((rows, tt))
-    rows = sum(r for r, _ in rates)
-    tt = sum(t for _, t in rates)
-    value = rows / tt
-    sample = f"each step: the oracle on whole token rows for about {budget:.1f} s ({rows} rows in all)"
-    line = {"impl": "reference", "metric": FUSED_NORM_METRIC, "value": value, "unit": "tokens/s",
-            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": tt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": c["workload"], "tokens": c["tokens"], "d_model": c["d_model"], "tp": c["tp"],
-                       "parallelism": "host oracle"},
-            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample},
-            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
-    print(json.dumps(line), flush=True)
-    return 0
-
-
 def run_reference(args):
     rank = int(os.environ.get("RANK", 0))
     if rank != 0:
@@ -312,65 +283,159 @@ def run_reference(args):
 
 
 FUSED_NORM_METRIC = "fused TP all-reduce + residual add + RMSNorm: token rows/s; HBM GB/s vs B200 peak"
+ATTN_MERGE_METRIC = "DCP merge of KV-shard attention partials: query rows/s; HBM GB/s vs B200 peak"
 
 
-def _fused_norm_config(args):
+class FusedNormOp:
+    """The all-reduce + residual add + RMSNorm step ("7.4 推理侧并行" §7.4.2)."""
+    metric = FUSED_NORM_METRIC
+    kernel = "allreduce_norm_kernel"
+    library_ops = "torch sum over ranks, add, rms_norm"
+
+    def __init__(self, args):
+        from tensor_sharded_mlp_b200 import inputs
+        c = dict(inputs.FUSED_NORM_CONFIGS[args.config])
+        if args.tokens is not None:
+            c["tokens"] = args.tokens
+        if args.tp is not None:
+            c["tp"] = args.tp
+        self.c = c
+        self.units = c["tokens"]
+        self.dtype = c["dtype"]
+        self.workload = (f"{args.config}: all-reduce of {c['tp']} fp32 rank partials + residual add + RMSNorm "
+                         f"({c['dtype']} residual/gamma/outputs), tokens={c['tokens']}, d_model={c['d_model']}, "
+                         f"eps={c['eps']}, partials and residual ~N(0,1), gamma ~1+0.1 N(0,1), seed {c['seed']}")
+        self.config = {"tokens": c["tokens"], "d_model": c["d_model"], "tp": c["tp"], "eps": c["eps"]}
+        self.host = inputs.generate_fused_norm(c["tokens"], c["d_model"], c["tp"], c["dtype"], c["seed"], c["eps"])
+
+    def step_bytes(self):
+        from tensor_sharded_mlp_b200 import counts
+        return counts.fused_norm_bytes(self.c["tp"], self.c["tokens"], self.c["d_model"], self.dtype)
+
+    def library_bytes(self):
+        from tensor_sharded_mlp_b200 import counts
+        return counts.unfused_norm_bytes(self.c["tp"], self.c["tokens"], self.c["d_model"], self.dtype)
+
+    def device(self, torch, tdt):
+        """(inputs that differ per rotated copy, fixed inputs, outputs)."""
+        p = torch.from_numpy(self.host.partials).cuda()
+        r = torch.from_numpy(self.host.residual).cuda().to(tdt)
+        g = torch.from_numpy(self.host.gamma).cuda().to(tdt)
+        T, d = self.c["tokens"], self.c["d_model"]
+        return (p, r), (g,), (torch.empty(T, d, dtype=tdt, device="cuda"), torch.empty(T, d, dtype=tdt, device="cuda"))
+
+    def launch(self, binding, ins, fixed, outs):
+        binding.tp_mlp_allreduce_residual_rmsnorm(ins[0], ins[1], fixed[0], self.c["eps"], outs[0], outs[1])
+
+    def library(self, torch, ins, fixed):
+        p, r = ins
+        h = (p.sum(dim=0) + r.float()).to(r.dtype)
+        return torch.nn.functional.rms_norm(h.float(), (h.shape[1],), weight=fixed[0].float(),
+                                            eps=self.c["eps"]).to(r.dtype), h
+
+    def oracle_rate(self, budget_s):
+        import oracle
+        fi, T = self.host, self.c["tokens"]
+        rows, t_total, n = 0, 0.0, 1
+        while t_total < budget_s:
+            n = min(T, n)
+            t0 = time.perf_counter()
+            oracle.allreduce_residual_rmsnorm(fi.partials[:, :n], fi.residual[:n], fi.gamma, fi.eps)
+            t_total += time.perf_counter() - t0
+            rows += n
+            n *= 2
+        return rows / t_total, rows, t_total
+
+
+class AttnMergeOp:
+    """The merge of KV shards' partial attention results ("LLM 推理并行化" §三 4), DCP)."""
+    metric = ATTN_MERGE_METRIC
+    kernel = "attn_merge_kernel"
+    library_ops = "torch max, exp, weighted sums and division over ranks"
+
+    def __init__(self, args):
+        from tensor_sharded_mlp_b200 import inputs
+        c = dict(inputs.ATTN_MERGE_CONFIGS[args.config])
+        if args.tokens is not None:
+            c["tokens"] = args.tokens
+        if args.tp is not None:
+            c["tp"] = args.tp
+        self.c = c
+        self.rows = c["tokens"] * c["heads"]
+        self.units = self.rows
+        self.dtype = c["dtype"]
+        self.workload = (f"{args.config}: merge of {c['tp']} KV shards' attention partials, {c['tokens']} decode "
+                         f"queries x {c['heads']} heads of {c['head_dim']} ({c['dtype']} weighted sums, fp32 maxima "
+                         f"and sums), maxima ~N(0,4), sums ~1+U*(keys_per_rank-1) with {c['keys_per_rank']} keys "
+                         f"per rank, weighted ~N(0,1)*sqrt(sum), seed {c['seed']}")
+        self.config = {"tokens": c["tokens"], "heads": c["heads"], "head_dim": c["head_dim"], "tp": c["tp"]}
+        self.host = inputs.generate_attn_merge(c["tp"], self.rows, c["head_dim"], c["dtype"], c["seed"],
+                                               c["keys_per_rank"])
+
+    def step_bytes(self):
+        e = 4 if self.dtype == "f32" else 2
+        P, D = self.c["tp"], self.c["head_dim"]
+        return P * self.rows * (8 + D * e) + self.rows * D * e
+
+    def library_bytes(self):
+        return None
+
+    def device(self, torch, tdt):
+        m = torch.from_numpy(self.host.maximum).cuda()
+        s = torch.from_numpy(self.host.exp_sum).cuda()
+        w = torch.from_numpy(self.host.weighted).cuda().to(tdt)
+        return (m, s, w), (), (torch.empty(self.rows, self.c["head_dim"], dtype=tdt, device="cuda"),)
+
+    def launch(self, binding, ins, fixed, outs):
+        binding.tp_mlp_merge_attention_partials(ins[0], ins[1], ins[2], outs[0])
+
+    def library(self, torch, ins, fixed):
+        m, s, w = ins
+        c = torch.exp(m - m.max(dim=0, keepdim=True).values)
+        return ((c[:, :, None] * w.float()).sum(dim=0) / (c * s).sum(dim=0)[:, None]).to(w.dtype)
+
+    def oracle_rate(self, budget_s):
+        import oracle
+        a = self.host
+        rows, t_total, n = 0, 0.0, 64
+        while t_total < budget_s:
+            n = min(self.rows, n)
+            t0 = time.perf_counter()
+            oracle.merge_attention_partials(a.maximum[:, :n], a.exp_sum[:, :n], a.weighted[:, :n])
+            t_total += time.perf_counter() - t0
+            rows += n
+            n *= 2
+        return rows / t_total, rows, t_total
+
+
+def small_op(args):
     from tensor_sharded_mlp_b200 import inputs
-    c = dict(inputs.FUSED_NORM_CONFIGS[args.config])
-    if args.tokens is not None:
-        c["tokens"] = args.tokens
-    if args.tp is not None:
-        c["tp"] = args.tp
-    c["workload"] = (f"{args.config}: all-reduce of {c['tp']} fp32 rank partials + residual add + RMSNorm "
-                     f"({c['dtype']} residual/gamma/outputs), tokens={c['tokens']}, d_model={c['d_model']}, "
-                     f"eps={c['eps']}, partials and residual ~N(0,1), gamma ~1+0.1 N(0,1), seed {c['seed']}")
-    return c
+    if args.config in inputs.FUSED_NORM_CONFIGS:
+        return FusedNormOp(args)
+    if args.config in inputs.ATTN_MERGE_CONFIGS:
+        return AttnMergeOp(args)
+    return None
 
 
-def fused_norm_oracle_rate(fi, budget_s):
-    """The oracle as it stands on whole token rows, for about budget_s seconds."""
-    import oracle
-    T = fi.residual.shape[0]
-    rows, t_total, n = 0, 0.0, 1
-    while t_total < budget_s:
-        n = min(T, n)
-        t0 = time.perf_counter()
-        oracle.allreduce_residual_rmsnorm(fi.partials[:, :n], fi.residual[:n], fi.gamma, fi.eps)
-        t_total += time.perf_counter() - t0
-        rows += n
-        n *= 2
-    return rows / t_total, rows, t_total
-
-
-def run_fused_norm(args):
-    """The fused all-reduce + residual + RMSNorm step ("7.4 推理侧并行" §7.4.2):
-    one tp_mlp_allreduce_residual_rmsnorm launch per step."""
-    import numpy as np
+def run_small_op(args, op):
+    """One launch of a small memory-bound operator per step."""
     import torch
 
-    from tensor_sharded_mlp_b200 import binding, counts, inputs, replicas
+    from tensor_sharded_mlp_b200 import binding, replicas
 
     rank, world, local = replicas.rank_env()
     torch.cuda.set_device(local)
     replicas.init("nccl", torch.device("cuda", local))
-    c = _fused_norm_config(args)
-    T, d, P, dt, eps = c["tokens"], c["d_model"], c["tp"], c["dtype"], c["eps"]
-    fi = inputs.generate_fused_norm(T, d, P, dt, c["seed"], eps)
-    tdt = torch.bfloat16 if dt == "bf16" else torch.float32
-    step_bytes = counts.fused_norm_bytes(P, T, d, dt)
+    tdt = torch.bfloat16 if op.dtype == "bf16" else torch.float32
+    step_bytes = op.step_bytes()
     # inputs smaller than L2 are rotated through enough copies to exceed it
     copies = max(1, -(-2 * 126 * 2 ** 20 // step_bytes))
-    p0 = torch.from_numpy(fi.partials).cuda()
-    r0 = torch.from_numpy(fi.residual).cuda().to(tdt)
-    g = torch.from_numpy(fi.gamma).cuda().to(tdt)
-    sets = [(p0, r0)] + [(p0.clone(), r0.clone()) for _ in range(copies - 1)]
-    y = torch.empty(T, d, dtype=tdt, device="cuda")
-    ro = torch.empty(T, d, dtype=tdt, device="cuda")
+    ins0, fixed, outs = op.device(torch, tdt)
+    sets = [ins0] + [tuple(t.clone() for t in ins0) for _ in range(copies - 1)]
     K, W = args.steps, max(3, args.warmup)
 
     def step(i):
-        pi, ri = sets[i % copies]
-        binding.tp_mlp_allreduce_residual_rmsnorm(pi, ri, g, eps, y, ro)
+        op.launch(binding, sets[i % copies], fixed, outs)
 
     for i in range(W):
         step(i)
@@ -404,6 +469,7 @@ def run_fused_norm(args):
     sampler.mark(t0, time.perf_counter())
     elapsed_ms = replicas.max_over_ranks(start.elapsed_time(end))
     launch_ms = start.elapsed_time(end) / K    # back-to-back launches inside the graph
+    del graph
     # the same K launches issued from Python one by one (host-bound when small)
     h0, h1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     h0.record(stream)
@@ -412,85 +478,98 @@ def run_fused_norm(args):
     h1.record(stream)
     torch.cuda.synchronize()
     api_ms = h0.elapsed_time(h1) / K
-    del graph
-    # the same step unfused, with library ops: sum over ranks, residual add, RMSNorm
-    def unfused(i):
-        pi, ri = sets[i % copies]
-        h = (pi.sum(dim=0) + ri.float()).to(tdt)
-        return torch.nn.functional.rms_norm(h.float(), (d,), weight=g.float(), eps=eps).to(tdt), h
+    # the same step with library ops (several kernels), for comparison
     for i in range(W):
-        unfused(i)
-    ue = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-    for i, (a, b) in enumerate(ue):
-        a.record(stream)
-        unfused(i)
-        b.record(stream)
+        op.library(torch, sets[i % copies], fixed)
+    u0, u1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    u0.record(stream)
+    for i in range(K):
+        op.library(torch, sets[i % copies], fixed)
+    u1.record(stream)
     torch.cuda.synchronize()
-    unfused_ms = statistics.fmean(a.elapsed_time(b) for a, b in ue)
-    # end to end: pinned host inputs in, both outputs back, every step
+    library_ms = u0.elapsed_time(u1) / K
+    # end to end: pinned host inputs in, outputs back, every step
     e2e = None
     if not args.no_e2e:
-        hp = torch.from_numpy(fi.partials).pin_memory()
-        hr = r0.cpu().pin_memory()
-        hy = torch.empty(T, d, dtype=tdt).pin_memory()
-        hro = torch.empty(T, d, dtype=tdt).pin_memory()
-        dp, dr = sets[0]
-        for _ in range(W):
-            dp.copy_(hp, non_blocking=True)
+        host_in = [t.cpu().pin_memory() for t in sets[0]]
+        host_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in outs]
         s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        s2.record(stream)
-        for _ in range(K):
-            dp.copy_(hp, non_blocking=True)
-            dr.copy_(hr, non_blocking=True)
-            binding.tp_mlp_allreduce_residual_rmsnorm(dp, dr, g, eps, y, ro)
-            hy.copy_(y, non_blocking=True)
-            hro.copy_(ro, non_blocking=True)
+        for it in range(W + K):
+            if it == W:
+                s2.record(stream)
+            for dst, src in zip(sets[0], host_in):
+                dst.copy_(src, non_blocking=True)
+            op.launch(binding, sets[0], fixed, outs)
+            for dst, src in zip(host_out, outs):
+                dst.copy_(src, non_blocking=True)
             stream.synchronize()
         e2.record(stream)
         e2.synchronize()
         e2e_ms = replicas.max_over_ranks(s2.elapsed_time(e2))
-        e2e = {"value": replicas.whole_job_rate(T, K, world, e2e_ms), "unit": "tokens/s",
-               "h2d_bytes_per_step": hp.numel() * 4 + hr.numel() * hr.element_size(),
-               "d2h_bytes_per_step": 2 * hy.numel() * hy.element_size(),
-               "api": "binding.tp_mlp_allreduce_residual_rmsnorm with pinned host buffers, synchronize per step"}
+        e2e = {"value": replicas.whole_job_rate(op.units, K, world, e2e_ms), "unit": "rows/s",
+               "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in host_in),
+               "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in host_out),
+               "api": "the binding call with pinned host buffers copied in and out, synchronize per step"}
     sampler.stop()
     peaks, src = load_peaks()
     achieved = step_bytes / (launch_ms / 1e3) / 1e9
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm_gbs"], "traffic": recorded_traffic("fused_norm:norm", args.config),
-                "kernel": "allreduce_norm_kernel", "kernel_ms": launch_ms, "algorithmic_per_launch": step_bytes,
+                "frac": achieved / peaks["hbm_gbs"], "traffic": recorded_traffic(f"{op.kernel}:op", args.config),
+                "kernel": op.kernel, "kernel_ms": launch_ms, "algorithmic_per_launch": step_bytes,
                 "peak_source": f"hbm_gbs ({src})"}
     ms = elapsed_ms / K
-    line = {"metric": FUSED_NORM_METRIC, "value": replicas.whole_job_rate(T, K, world, elapsed_ms),
-            "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W, "ms_per_step": ms,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": dt, "data": "synthetic",
-            "config": {"workload": c["workload"], "tokens": T, "d_model": d, "tp": P, "eps": eps,
-                       "parallelism": "replicas" if world > 1 else "single GPU",
-                       "l2": (f"{copies} input copies rotated ({copies * step_bytes / 2 ** 20:.0f} MiB > L2)"
-                              if copies > 1 else "inputs larger than L2")},
+    line = {"metric": op.metric, "value": replicas.whole_job_rate(op.units, K, world, elapsed_ms),
+            "unit": "rows/s", "n_gpus": world, "steps": K, "warmup": W, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": op.dtype,
+            "data": "synthetic",
+            "config": dict({"workload": op.workload, "parallelism": "replicas" if world > 1 else "single GPU",
+                            "l2": (f"{copies} input copies rotated ({copies * step_bytes / 2 ** 20:.0f} MiB > L2)"
+                                   if copies > 1 else "inputs larger than L2")}, **op.config),
             "step_hbm_gbs": step_bytes / (ms / 1e3) / 1e9, "roofline": roofline, "gpu_launches": K,
             "clocks": sampler.summary(), "e2e": e2e,
             "timer": "CUDA events around one replay of a CUDA graph holding the K launches",
             "python_call_us": api_ms * 1e3,
-            "unfused_library_ops": {"ms": unfused_ms, "ops": "torch sum over ranks, add, rms_norm",
-                                    "algorithmic_bytes": counts.unfused_norm_bytes(P, T, d, dt)}}
+            "library_ops": {"ms": library_ms, "ops": op.library_ops, "algorithmic_bytes": op.library_bytes()}}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, rows, tt = fused_norm_oracle_rate(fi, 10.0)
-        line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                                "sample": f"{rows} token rows of this workload on one host core, {tt:.1f} s"}
+        v, rows, tt = op.oracle_rate(10.0)
+        line["cpu_baseline"] = {"value": v, "unit": "rows/s", "cores": 1, "kind": "oracle",
+                                "sample": f"{rows} rows of this workload on one host core, {tt:.1f} s"}
     if rank == 0:
         print(json.dumps(line), flush=True)
     replicas.finish()
     return 0
 
 
+def run_small_op_reference(args, op):
+    """Reference arm of a small operator: its oracle on whole rows, bounded."""
+    if int(os.environ.get("RANK", 0)) != 0:
+        return 0
+    budget = 150.0 / max(1, args.steps + args.warmup)
+    done = []
+    for i in range(args.warmup + args.steps):
+        _, rows, tt = op.oracle_rate(budget)
+        if i >= args.warmup:
+            done.append((rows, tt))
+    rows = sum(r for r, _ in done)
+    tt = sum(t for _, t in done)
+    value = rows / tt
+    sample = f"each step: the oracle on whole rows for about {budget:.1f} s ({rows} rows in all)"
+    line = {"impl": "reference", "metric": op.metric, "value": value, "unit": "rows/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": tt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": dict({"workload": op.workload, "parallelism": "host oracle"}, **op.config),
+            "cpu_baseline": {"value": value, "unit": "rows/s", "cores": 1, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "rows/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse()
-    from tensor_sharded_mlp_b200 import inputs as _inputs
-    if args.config in _inputs.FUSED_NORM_CONFIGS:
-        if args.impl == "reference":
-            return run_fused_norm_reference(args)
-        return run_fused_norm(args)
+    op = small_op(args)
+    if op is not None:
+        return run_small_op_reference(args, op) if args.impl == "reference" else run_small_op(args, op)
     if args.impl == "reference":
         return run_reference(args)
 

@@ -301,6 +301,33 @@ int tp_mlp_allreduce_residual_rmsnorm(const float *partials, int tp_degree, int 
                                       const void *residual, const void *gamma, float eps, int dtype,
                                       void *y, void *residual_out, tp_mlp_stream_t stream);
 
+/*
+ * Merge of partial attention results across KV shards (decode context
+ * parallelism; "LLM 推理并行化：先找瓶颈，再决定怎么切", §三 4) 上下文并行（CP））.
+ * Each of the tp_degree ranks attended over its own part of the KV history
+ * and reports, for every query row (one token and head): its maximum score,
+ * the sum of exp(score - maximum) and the exp-weighted sum of the values.
+ * The merge takes the global maximum M of a row, rescales every rank by
+ * exp(maximum_i - M), adds, and divides the merged weighted sum by the merged
+ * exponential sum -- attention over the whole history.  A rank with no keys
+ * for a row reports maximum -inf (and 0, 0) and contributes nothing; a row
+ * with every rank empty is written as zeros.  Needs no handle and no workspace.
+ *
+ *   maximum, exp_sum  device fp32, tp_degree x rows (rank-major)
+ *   weighted          device, tp_degree x rows x head_dim, element type `dtype`
+ *   out               device, rows x head_dim of `dtype`; must not overlap
+ *                     the inputs
+ * Requirements: 1 <= tp_degree <= 8, rows >= 0 (0 is a no-op), 4 <= head_dim
+ * <= 4096 with head_dim % 4 == 0 (TP_MLP_ERR_SHAPE otherwise), a valid dtype
+ * (TP_MLP_ERR_INVALID_ARG), every pointer 16-byte aligned
+ * (TP_MLP_ERR_ALIGNMENT) and inside a device allocation of the stated size
+ * (TP_MLP_ERR_SHAPE / TP_MLP_ERR_INVALID_ARG).  fp32 arithmetic; asynchronous
+ * on `stream`; the caller owns every buffer.
+ */
+int tp_mlp_merge_attention_partials(int tp_degree, int rows, int head_dim, const float *maximum,
+                                    const float *exp_sum, const void *weighted, int dtype, void *out,
+                                    tp_mlp_stream_t stream);
+
 /* Human-readable name of a status code (static string). */
 const char *tp_mlp_status_string(int status);
 

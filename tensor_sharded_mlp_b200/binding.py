@@ -50,6 +50,7 @@ _SIGS = {
     "tp_mlp_set_plan": (_i, [_vp, _i]),
     "tp_mlp_set_splitk": (_i, [_vp, _i]),
     "tp_mlp_allreduce_residual_rmsnorm": (_i, [_vp, _i, _i, _i, _vp, _vp, ctypes.c_float, _i, _vp, _vp, _vp]),
+    "tp_mlp_merge_attention_partials": (_i, [_i, _i, _i, _vp, _vp, _vp, _i, _vp, _vp]),
     "tp_mlp_set_profile_events": (_i, [_vp, _vpp, _i]),
     "tp_mlp_get_device_status": (_i, [_vp]),
     "tp_mlp_selftest_bounded_wait": (_i, [_vp, ctypes.c_uint, _vp]),
@@ -242,6 +243,30 @@ def tp_mlp_allreduce_residual_rmsnorm(partials: torch.Tensor, residual: torch.Te
                                                   float(eps), DTYPE["f32" if dt == torch.float32 else "bf16"],
                                                   _ptr(y), _ptr(residual_out), _stream(stream)))
     return y, residual_out
+
+
+def tp_mlp_merge_attention_partials(maximum: torch.Tensor, exp_sum: torch.Tensor, weighted: torch.Tensor,
+                                    out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Merge P ranks' partial attention results: maximum, exp_sum (P, rows) float32,
+    weighted (P, rows, head_dim) float32 or bfloat16 -> out (rows, head_dim)."""
+    if weighted.dim() != 3 or weighted.dtype not in (torch.float32, torch.bfloat16):
+        raise ValueError("weighted must be a float32 or bfloat16 tensor (P, rows, head_dim)")
+    P, rows, D = weighted.shape
+    for t in (maximum, exp_sum):
+        if t.dtype != torch.float32 or t.shape != (P, rows):
+            raise ValueError("maximum and exp_sum must be float32 (P, rows)")
+    for t in (maximum, exp_sum, weighted):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("inputs must be contiguous CUDA tensors")
+    if out is None:
+        out = torch.empty(rows, D, dtype=weighted.dtype, device=weighted.device)
+    if out.shape != (rows, D) or out.dtype != weighted.dtype or not out.is_contiguous():
+        raise ValueError("out must be a contiguous (rows, head_dim) tensor of weighted's dtype")
+    _check("tp_mlp_merge_attention_partials",
+           _lib.tp_mlp_merge_attention_partials(P, rows, D, _ptr(maximum), _ptr(exp_sum), _ptr(weighted),
+                                                DTYPE["f32" if weighted.dtype == torch.float32 else "bf16"],
+                                                _ptr(out), _stream(stream)))
+    return out
 
 
 # --- convenience wrapper -----------------------------------------------------------

@@ -96,7 +96,8 @@ def unfused_norm_bytes(tp: int, tokens: int, d_model: int, dtype: str) -> int:
 # Source files that define each kernel family (for "was this profile taken on
 # the current kernel?" checks).
 _KERNEL_SOURCES = {
-    "fused_norm": ["fused_norm.cu", "common.cuh", "tc_ptx.cuh"],
+    "fused_norm": ["fused_norm.cu", "vec_io.cuh", "common.cuh", "tc_ptx.cuh"],
+    "attn_merge": ["attn_merge.cu", "vec_io.cuh", "common.cuh"],
     "gemv": ["gemv.cu", "common.cuh", "streamk.cuh", "tc_ptx.cuh"],
     "tc_skinny": ["tc_gemm.cu", "common.cuh", "streamk.cuh", "tc_ptx.cuh"],
     "tc_wide": ["tc_gemm.cu", "common.cuh", "streamk.cuh", "tc_ptx.cuh"],

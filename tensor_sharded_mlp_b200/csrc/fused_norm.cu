@@ -21,6 +21,7 @@
 #include "common.cuh"
 #include "internal.h"
 #include "tc_ptx.cuh"
+#include "vec_io.cuh"
 
 namespace tpmlp {
 namespace {
@@ -28,25 +29,6 @@ namespace {
 using tc::smem_u32;
 
 constexpr int kNormThreads = 256;
-
-__device__ __forceinline__ float4 load4(const float *p) { return *reinterpret_cast<const float4 *>(p); }
-__device__ __forceinline__ float4 load4(const __nv_bfloat16 *p) {
-    const uint2 u = *reinterpret_cast<const uint2 *>(p);
-    return make_float4(bf16lo(u.x), bf16hi(u.x), bf16lo(u.y), bf16hi(u.y));
-}
-__device__ __forceinline__ void store4(float *p, float4 v) { *reinterpret_cast<float4 *>(p) = v; }
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-    return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(lo)) |
-           ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hi)) << 16);
-}
-__device__ __forceinline__ void store4(__nv_bfloat16 *p, float4 v) {
-    *reinterpret_cast<uint2 *>(p) = make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
-}
-// fp32 rank partials are read once: streaming loads that do not allocate in L1
-__device__ __forceinline__ float4 ld_partial(const float *p) {
-    const uint4 u = ld_stream_v4(p);
-    return make_float4(__uint_as_float(u.x), __uint_as_float(u.y), __uint_as_float(u.z), __uint_as_float(u.w));
-}
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {
     uint32_t r;
@@ -91,7 +73,7 @@ __global__ void __launch_bounds__(kNormThreads)
         const float *pz = part + row + 4LL * q;
         float4 w[P];
 #pragma unroll
-        for (int i = 0; i < P; ++i) w[i] = ld_partial(pz + i * rank_stride);
+        for (int i = 0; i < P; ++i) w[i] = load4_stream(pz + i * rank_stride);
         const float4 r = load4(res + row + 4LL * q);
         float4 z = w[0];
 #pragma unroll

@@ -41,6 +41,12 @@ cudaError_t launch_allreduce_norm(const float *partials, int P, int rows, int d,
                                   const void *gamma, float eps, int dtype, void *y, void *residual_out,
                                   int num_sms, cudaStream_t st);
 
+// attn_merge.cu: merge of P ranks' partial attention results (maximum,
+// exp_sum: P x rows fp32; weighted: P x rows x D of dtype) into rows x D.
+constexpr int kMergeMaxHeadDim = 4096;
+cudaError_t launch_attn_merge(int P, int rows, int D, const float *maximum, const float *exp_sum,
+                              const void *weighted, int dtype, void *out, cudaStream_t st);
+
 // Split-tile counters the GEMV and tcgen05 skinny kernels need (one per
 // weight tile of both parts; first part's tiles first).
 size_t tile_counter_slots(const Problem &p);

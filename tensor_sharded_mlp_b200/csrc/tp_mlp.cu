@@ -476,6 +476,24 @@ int tp_mlp_allreduce_residual_rmsnorm(const float *partials, int tp_degree, int 
                                            residual_out, sms, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+int tp_mlp_merge_attention_partials(int tp_degree, int rows, int head_dim, const float *maximum,
+                                    const float *exp_sum, const void *weighted, int dtype, void *out,
+                                    tp_mlp_stream_t stream) {
+    if (tp_degree < 1 || tp_degree > kMaxTp || rows < 0) return TP_MLP_ERR_SHAPE;
+    if (head_dim < 4 || head_dim > kMergeMaxHeadDim || head_dim % 4 != 0) return TP_MLP_ERR_SHAPE;
+    if (dtype != TP_MLP_F32 && dtype != TP_MLP_BF16) return TP_MLP_ERR_INVALID_ARG;
+    if (rows == 0) return TP_MLP_OK;   // empty tensors may carry null pointers
+    if (!maximum || !exp_sum || !weighted || !out) return TP_MLP_ERR_INVALID_ARG;
+    const size_t e = elem_bytes(dtype), pr = (size_t)tp_degree * rows;
+    int s;
+    if ((s = check_dev(maximum, pr * sizeof(float)))) return s;
+    if ((s = check_dev(exp_sum, pr * sizeof(float)))) return s;
+    if ((s = check_dev(weighted, pr * head_dim * e))) return s;
+    if ((s = check_dev(out, (size_t)rows * head_dim * e))) return s;
+    return from_cuda(launch_attn_merge(tp_degree, rows, head_dim, maximum, exp_sum, weighted, dtype, out,
+                                       reinterpret_cast<cudaStream_t>(stream)));
+}
+
 int tp_mlp_set_splitk(tp_mlp_t h, int mode) {
     if (!h) return TP_MLP_ERR_INVALID_ARG;
     if (mode < TP_MLP_SPLITK_AUTO || mode > TP_MLP_SPLITK_SEPARATE) return TP_MLP_ERR_INVALID_ARG;

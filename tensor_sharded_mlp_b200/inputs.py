@@ -82,6 +82,44 @@ def generate_fused_norm(tokens: int, d_model: int, tp: int, dtype: str, seed: in
     return FusedNormInputs(part, res, g, eps)
 
 
+# Merging partial attention results across KV shards (decode context
+# parallelism, "LLM 推理并行化" §三 4)): P ranks' per-row statistics for a
+# decode batch of `tokens` queries over `heads` heads of `head_dim`, the head
+# layout of the d_model 8192 configs (64 heads of 128).
+ATTN_MERGE_CONFIGS = {
+    "attn_merge_decode_bs32": dict(dtype="f32", tokens=32, heads=64, head_dim=128, tp=8, keys_per_rank=512,
+                                   seed=31),
+    "attn_merge_decode_bs256": dict(dtype="bf16", tokens=256, heads=64, head_dim=128, tp=8, keys_per_rank=512,
+                                    seed=32),
+}
+
+
+@dataclasses.dataclass
+class AttnMergeInputs:
+    maximum: np.ndarray    # P x rows, fp32
+    exp_sum: np.ndarray    # P x rows, fp32
+    weighted: np.ndarray   # P x rows x head_dim (dtype-representable values in fp32)
+
+
+def generate_attn_merge(tp: int, rows: int, head_dim: int, dtype: str, seed: int, keys_per_rank: int = 512
+                        ) -> AttnMergeInputs:
+    """Seeded per-rank statistics: rng(seed) draws, in order, the maxima
+    (P x rows, N(0, 2^2)), the exponential sums (P x rows, 1 + U(0,1) *
+    (keys_per_rank - 1): at least the maximum's own term, at most one per key)
+    and the weighted sums (P x rows x head_dim, N(0, 1) * sqrt(exp_sum), a sum
+    of that many unit-scale values); the weighted sums are rounded to bf16 for a
+    bf16 config."""
+    rng = np.random.default_rng(seed)
+    m = (rng.standard_normal((tp, rows)) * 2.0).astype(np.float32)
+    s = (1.0 + rng.random((tp, rows)) * (keys_per_rank - 1)).astype(np.float32)
+    w = np.empty((tp, rows, head_dim), np.float32)
+    for i in range(tp):
+        w[i] = _draw(rng, rows, head_dim, 1.0, "f32") * np.sqrt(s[i])[:, None].astype(np.float32)
+    if dtype == "bf16":
+        w = round_to_bf16(w)
+    return AttnMergeInputs(m, s, w)
+
+
 def round_to_bf16(a: np.ndarray) -> np.ndarray:
     """Round fp32 values to the nearest bf16 (ties to even); returns fp32 holding them."""
     a = np.ascontiguousarray(a, dtype=np.float32)

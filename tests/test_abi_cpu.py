@@ -151,6 +151,14 @@ def test_call_argument_errors_before_any_launch(b):
     assert F(None, 2, 1, 64, None, None, 0.0, 7, None, None, None) == 1       # dtype
     assert F(None, 2, 1, 64, None, None, 0.0, 0, None, None, None) == 1       # null pointers
     assert F(None, 2, 0, 64, None, None, 0.0, 0, None, None, None) == 0       # no tokens: no-op
+    # merge of attention partials
+    M = L.tp_mlp_merge_attention_partials
+    assert M(0, 4, 128, None, None, None, 0, None, None) == 2                  # tp_degree
+    assert M(2, 4, 130, None, None, None, 0, None, None) == 2                  # head_dim % 4
+    assert M(2, 4, 4100, None, None, None, 0, None, None) == 2                 # head_dim too large
+    assert M(2, 4, 128, None, None, None, 3, None, None) == 1                  # dtype
+    assert M(2, 4, 128, None, None, None, 1, None, None) == 1                  # null pointers
+    assert M(2, 0, 128, None, None, None, 1, None, None) == 0                  # no rows: no-op
     for mode in (2, 1, 0):
         assert L.tp_mlp_set_splitk(h, mode) == 0
     assert L.tp_mlp_last_plan(h) == 1 and L.tp_mlp_last_launches(h) == 0        # the 0-token no-op
