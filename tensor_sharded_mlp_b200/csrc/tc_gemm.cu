@@ -82,11 +82,28 @@ struct WeightMaps {
     int first, swiglu, tps, kbps;
 };
 
-template <bool RAW>
+// HALF: 128-row tiles (tile t = rows [128 (t % 2), +128) of 256-row block t / 2
+// in the packed layout; two 64-column boxes in the shard form).
+template <bool RAW, bool HALF = false>
 __device__ __forceinline__ void load_w_tile(uint32_t dst, const WeightMaps &wm, int tile, int kb, int KB,
                                             uint32_t bar) {
     if (!RAW) {
-        tma_load_2d(dst, &wm.map[0], 0, (tile * KB + kb) * 256, bar);
+        if (HALF)
+            tma_load_2d(dst, &wm.map[0], 0, ((tile >> 1) * KB + kb) * 256 + (tile & 1) * 128, bar);
+        else
+            tma_load_2d(dst, &wm.map[0], 0, (tile * KB + kb) * 256, bar);
+        return;
+    }
+    if (HALF) {   // tanh / identity first projection or the second projection: 128 columns
+        if (wm.first) {
+            const int i = tile / wm.tps, n0 = (tile - i * wm.tps) * 128;
+#pragma unroll
+            for (int q = 0; q < 2; ++q) tma_load_2d(dst + q * 8192, &wm.map[i], n0 + 64 * q, kb * BK, bar);
+        } else {
+            const int i = kb / wm.kbps, kl = kb - i * wm.kbps;
+#pragma unroll
+            for (int q = 0; q < 2; ++q) tma_load_2d(dst + q * 8192, &wm.map[i], tile * 128 + 64 * q, kl * BK, bar);
+        }
         return;
     }
     if (wm.first) {
@@ -410,10 +427,23 @@ __device__ __forceinline__ void skinny_final4(const TcArgs &a, int tile, int r, 
     }
 }
 
-template <int BT, int STAGES, bool RAW>
+// Final epilogue of a 128-row tile (tanh / identity / output): 4 tokens of row r.
+__device__ __forceinline__ void skinny_final_half4(const TcArgs &a, int tile, int r, int t0, float4 v) {
+    const int n = tile_col(a, tile, r, 128);
+    if (n < 0) return;
+    const float g[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        if (t0 + i < a.rows_x) a.out[(long)(t0 + i) * a.ldo + n] = __float2bfloat16_rn(act_out(a.epi, g[i]));
+}
+
+// HALF: 128-row weight tiles, one M=128 MMA per 16-k step (never SwiGLU's first
+// projection, whose gate and up rows must share a tile); split tiles always go
+// to skinny_reduce_kernel.
+template <int BT, int STAGES, bool RAW, bool HALF>
 __global__ void __launch_bounds__(NTHREADS, 1)
     tc_skinny_kernel(const __grid_constant__ WeightMaps wm, const __grid_constant__ CUtensorMap tmX, TcArgs a) {
-    constexpr uint32_t W_BYTES = 256 * BK * 2;   // 256 weight rows (two M=128 halves)
+    constexpr uint32_t W_BYTES = (HALF ? 128 : 256) * BK * 2;   // 256 weight rows: two M=128 halves
     constexpr uint32_t X_BYTES = BT * BK * 2;
     extern __shared__ uint8_t smem_raw[];
     const Smem s = carve<STAGES>(smem_raw, W_BYTES, X_BYTES);
@@ -438,7 +468,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 const int tile = (int)(it / KB), kb = (int)(it - (long long)tile * KB);
                 const uint32_t fb = smem_u32(&s.full[i]);
                 mbar_arrive_expect_tx(fb, W_BYTES + X_BYTES);   // first use of stage i: it is empty
-                load_w_tile<RAW>(smem_u32(s.a + i * W_BYTES), wm, tile, kb, KB, fb);
+                load_w_tile<RAW, HALF>(smem_u32(s.a + i * W_BYTES), wm, tile, kb, KB, fb);
             }
             pdl_wait_previous();
             for (int i = 0; i < npre; ++i)
@@ -451,7 +481,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 if (!mbar_wait(smem_u32(&s.empty[stage]), phase ^ 1, s.abort)) goto done;
                 const uint32_t fb = smem_u32(&s.full[stage]);
                 mbar_arrive_expect_tx(fb, W_BYTES + X_BYTES);
-                load_w_tile<RAW>(smem_u32(s.a + stage * W_BYTES), wm, tile, kb, KB, fb);
+                load_w_tile<RAW, HALF>(smem_u32(s.a + stage * W_BYTES), wm, tile, kb, KB, fb);
                 tma_load_2d(smem_u32(s.b + stage * X_BYTES), &tmX, kb * BK, 0, fb);
                 if (++stage == STAGES) { stage = 0; phase ^= 1; }
             }
@@ -482,7 +512,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     for (int k = 0; k < BK / 16; ++k) {
                         const uint32_t accum = (kb != kb0 || k != 0) ? 1u : 0u;
                         mma_bf16(d0, dw0 + kstep_w * k, dx + 2 * k, idesc, accum);
-                        mma_bf16(d1, dw1 + kstep_w * k, dx + 2 * k, idesc, accum);
+                        if (!HALF) mma_bf16(d1, dw1 + kstep_w * k, dx + 2 * k, idesc, accum);
                     }
                     mma_commit(smem_u32(&s.empty[stage]));
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
@@ -513,9 +543,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 for (int t0 = 0; t0 < BT; t0 += 16) {
                     float v0[16], v1[16];
                     tmem_ld16(taddr + t0, v0);
-                    tmem_ld16(taddr + BT + t0, v1);
+                    if (!HALF) tmem_ld16(taddr + BT + t0, v1);
                     tmem_ld_wait();
-                    skinny_final16(a, tile, r, t0, v0, v1);
+                    if (HALF) {
+#pragma unroll
+                        for (int q4 = 0; q4 < 4; ++q4)
+                            skinny_final_half4(a, tile, r, t0 + 4 * q4,
+                                               make_float4(v0[4 * q4], v0[4 * q4 + 1], v0[4 * q4 + 2], v0[4 * q4 + 3]));
+                    } else {
+                        skinny_final16(a, tile, r, t0, v0, v1);
+                    }
                 }
                 tc_fence_before();
                 __syncwarp();
@@ -526,25 +563,28 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 const int c_first = share_owner((long long)tile * KB, total, G);
                 const int c_last = share_owner((long long)tile * KB + KB - 1, total, G);
                 const int slot = (int)c - c_first;
-                float4 *base = reinterpret_cast<float4 *>(a.part + ((long long)tile * a.slots + slot) * 256 * BT);
+                constexpr int ROWS = HALF ? 128 : 256;   // slot: [token/4][ROWS][4]
+                float4 *base = reinterpret_cast<float4 *>(a.part + ((long long)tile * a.slots + slot) * ROWS * BT);
 #pragma unroll 1
                 for (int t0 = 0; t0 < BT; t0 += 16) {
                     float v0[16], v1[16];
                     tmem_ld16(taddr + t0, v0);
-                    tmem_ld16(taddr + BT + t0, v1);
+                    if (!HALF) tmem_ld16(taddr + BT + t0, v1);
                     tmem_ld_wait();
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
                         const int qd = t0 / 4 + q;
-                        base[qd * 256 + r] = make_float4(v0[4 * q], v0[4 * q + 1], v0[4 * q + 2], v0[4 * q + 3]);
-                        base[qd * 256 + 128 + r] = make_float4(v1[4 * q], v1[4 * q + 1], v1[4 * q + 2], v1[4 * q + 3]);
+                        base[qd * ROWS + r] = make_float4(v0[4 * q], v0[4 * q + 1], v0[4 * q + 2], v0[4 * q + 3]);
+                        if (!HALF)
+                            base[qd * ROWS + 128 + r] =
+                                make_float4(v1[4 * q], v1[4 * q + 1], v1[4 * q + 2], v1[4 * q + 3]);
                     }
                 }
                 // the accumulator is copied out: hand TMEM back to the MMA before the fixup
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_u32(&s.tempty[acc]));
-                if (a.split_mode == kSplitSeparate) {   // skinny_reduce_kernel adds the slots
+                if (HALF || a.split_mode == kSplitSeparate) {   // skinny_reduce_kernel adds the slots
                     acc ^= 1;
                     if (acc == 0) acc_phase ^= 1;
                     continue;
@@ -610,12 +650,15 @@ done:
 // so both routes give the same bits -- and applies the same epilogue.  Launched
 // behind the skinny kernel with programmatic dependent launch; tiles one CTA
 // finished whole are skipped.
+// HALF: 128-row tiles, slots [token/4][128][4], one row per thread.
+template <bool HALF>
 __global__ void __launch_bounds__(128) skinny_reduce_kernel(TcArgs a, int BT) {
     pdl_allow_dependents();
+    constexpr int ROWS = HALF ? 128 : 256;
     const int quads = BT / 4;
     const int units = a.rows_w * quads;   // rows_w: weight tiles
     const int r = threadIdx.x;
-    const long long SLOT4 = 64LL * BT;   // float4s per slot (256 rows x BT tokens)
+    const long long SLOT4 = (long long)ROWS / 4 * BT;   // float4s per slot (ROWS rows x BT tokens)
     bool waited = false;
     for (int u = blockIdx.x; u < units; u += gridDim.x) {
         const int tile = u / quads, qd = u - tile * quads;
@@ -628,15 +671,21 @@ __global__ void __launch_bounds__(128) skinny_reduce_kernel(TcArgs a, int BT) {
             waited = true;
         }
         const float4 *p =
-            reinterpret_cast<const float4 *>(a.part) + (long long)tile * a.slots * SLOT4 + qd * 256 + r;
+            reinterpret_cast<const float4 *>(a.part) + (long long)tile * a.slots * SLOT4 + qd * ROWS + r;
         float4 s0 = make_float4(0.f, 0.f, 0.f, 0.f), s1 = s0;
 #pragma unroll 4
         for (int sl = 0; sl < n; ++sl) {
-            const float4 g = __ldcg(p + sl * SLOT4), h = __ldcg(p + sl * SLOT4 + 128);
+            const float4 g = __ldcg(p + sl * SLOT4);
             s0.x += g.x; s0.y += g.y; s0.z += g.z; s0.w += g.w;
-            s1.x += h.x; s1.y += h.y; s1.z += h.z; s1.w += h.w;
+            if (!HALF) {
+                const float4 h = __ldcg(p + sl * SLOT4 + 128);
+                s1.x += h.x; s1.y += h.y; s1.z += h.z; s1.w += h.w;
+            }
         }
-        skinny_final4(a, tile, r, qd * 4, s0, s1);
+        if (HALF)
+            skinny_final_half4(a, tile, r, qd * 4, s0);
+        else
+            skinny_final4(a, tile, r, qd * 4, s0, s1);
     }
 }
 
@@ -685,32 +734,59 @@ bool make_map(CUtensorMap *m, const void *base, int K, int rows, int box_rows) {
 // One projection's weight operand and its tile geometry.
 struct WeightOperand {
     WeightMaps wm;
-    bool raw;
+    bool raw, half;
     int tiles, KB;
     int raw_first, tps, fs;
 };
 
+// Token-tile widths from which the skinny tiling uses 128-row weight tiles
+// (packed layout) and whole CTAs per tile (below); both measured best from the
+// narrowest width on (sweep at 16 / 64 / 128 tokens: 54.4 -> 49.9, 63.6 ->
+// 52.9, 68.4 -> 58.0 us; decode batch 32: 226 -> 222.5 us).
+#ifndef TPMLP_SKINNY_HALF_MIN_BT
+#define TPMLP_SKINNY_HALF_MIN_BT 16
+#endif
+#ifndef TPMLP_SKINNY_ALIGN_MIN_BT
+#define TPMLP_SKINNY_ALIGN_MIN_BT 16
+#endif
+
+// Weight tiles of projection `proj` (0 first, 1 second) in the packed layout or
+// the shard form, of 256 rows or (half) 128 rows.
+long long skinny_tiles(const Problem &p, int proj, bool raw, bool half) {
+    if (proj == 1) return half ? (p.d_out + 127) / 128 : blk_tiles(p.d_out);
+    if (!raw) {
+        const long long rows = w1p_rows(p.d_ff, p.act);
+        return half ? (rows + 127) / 128 : blk_tiles(rows);
+    }
+    const int per = (p.act == TP_MLP_ACT_SWIGLU || half) ? 128 : 256;
+    return (long long)p.tp * ((p.fs + per - 1) / per);
+}
+
 // Packed part (tile-blocked): a 2-D view of rows of 64 bf16 (128 B); one box of
-// 256 rows = one 32 KB (tile, k-block) block.
-bool weight_packed(WeightOperand *w, const void *base, long long rows_w, int K) {
+// 256 rows = one 32 KB (tile, k-block) block, or of 128 rows = half of one.
+bool weight_packed(WeightOperand *w, const Problem &p, int proj, const void *base, bool half) {
     memset(w, 0, sizeof(*w));
-    w->tiles = (int)blk_tiles(rows_w);
+    const long long rows_w = proj == 0 ? w1p_rows(p.d_ff, p.act) : p.d_out;
+    const int K = proj == 0 ? p.d_in : p.d_ff;
+    w->half = half;
+    w->tiles = (int)skinny_tiles(p, proj, false, half);
     w->KB = (int)blk_kblocks(K);
-    const long long rows = (long long)w->tiles * w->KB * kTileRows;
-    return make_map2d(&w->wm.map[0], base, kKBlock, rows, kKBlock * 2, kTileRows);
+    const long long rows = blk_tiles(rows_w) * w->KB * kTileRows;
+    return make_map2d(&w->wm.map[0], base, kKBlock, rows, kKBlock * 2, half ? kTileRows / 2 : kTileRows);
 }
 
 // First projection straight from the shards A_i (d_in x lda row-major, lda = f_s
 // or 2 f_s for [gate_i | up_i]): maps over each rank's f_s columns, boxes of
 // 64 columns x 64 k rows.
-bool weight_raw_first(WeightOperand *w, const Problem &p, const ShardPtrs &A) {
+bool weight_raw_first(WeightOperand *w, const Problem &p, const ShardPtrs &A, bool half) {
     memset(w, 0, sizeof(*w));
     const bool sw = p.act == TP_MLP_ACT_SWIGLU;
     const long long lda = sw ? 2LL * p.fs : p.fs;
-    const int per = sw ? 128 : 256;
+    const int per = (sw || half) ? 128 : 256;
     w->raw = true;
+    w->half = half;
     w->tps = (p.fs + per - 1) / per;
-    w->tiles = p.tp * w->tps;
+    w->tiles = (int)skinny_tiles(p, 0, true, half);
     w->KB = (int)blk_kblocks(p.d_in);
     w->raw_first = 1;
     w->fs = p.fs;
@@ -727,10 +803,11 @@ bool weight_raw_first(WeightOperand *w, const Problem &p, const ShardPtrs &A) {
 
 // Second projection straight from the shards B_i (f_s x d_out row-major); the K
 // loop runs over rank 0's rows, then rank 1's, ... (needs f_s % 64 == 0).
-bool weight_raw_second(WeightOperand *w, const Problem &p, const ShardPtrs &B) {
+bool weight_raw_second(WeightOperand *w, const Problem &p, const ShardPtrs &B, bool half) {
     memset(w, 0, sizeof(*w));
     w->raw = true;
-    w->tiles = (int)blk_tiles(p.d_out);
+    w->half = half;
+    w->tiles = (int)skinny_tiles(p, 1, true, half);
     w->KB = p.d_ff / BK;
     w->wm.kbps = p.fs / BK;
     for (int i = 0; i < p.tp; ++i)
@@ -745,17 +822,17 @@ cudaError_t set_smem(K kern, size_t bytes) {
     return ensure_smem_attr(kern, bytes);
 }
 
-template <int BT, int STAGES>
+template <int BT, int STAGES, bool HALF>
 cudaError_t launch_skinny_bt(const WeightOperand &w, const CUtensorMap &mx, const TcArgs &a, int grid,
                              cudaStream_t st) {
-    const size_t smem = smem_bytes<STAGES>(256 * BK * 2, BT * BK * 2);
+    const size_t smem = smem_bytes<STAGES>((HALF ? 128 : 256) * BK * 2, BT * BK * 2);
     if (w.raw) {
-        auto kern = tc_skinny_kernel<BT, STAGES, true>;
+        auto kern = tc_skinny_kernel<BT, STAGES, true, HALF>;
         cudaError_t e = set_smem(kern, smem);
         if (e != cudaSuccess) return e;
         return launch_pdl(kern, dim3(grid), dim3(NTHREADS), smem, st, w.wm, mx, a);
     }
-    auto kern = tc_skinny_kernel<BT, STAGES, false>;
+    auto kern = tc_skinny_kernel<BT, STAGES, false, HALF>;
     cudaError_t e = set_smem(kern, smem);
     if (e != cudaSuccess) return e;
     return launch_pdl(kern, dim3(grid), dim3(NTHREADS), smem, st, w.wm, mx, a);
@@ -766,6 +843,34 @@ cudaError_t launch_skinny_bt(const WeightOperand &w, const CUtensorMap &mx, cons
 // two 32 KB slots, because the fixup sits at the end of the GEMM's critical path.
 int resolve_split(int mode) { return mode == kSplitAuto ? kSplitSeparate : mode; }
 
+// 128-row tiles: never for SwiGLU's first projection (gate and up share a
+// tile), the in-kernel fixup (256-row slots only) or the shard form, whose
+// 64-column boxes of row-major shards then fetch 256-byte row pieces (T = 128:
+// 66.6 us with 256-row tiles, 74.1 with 128).
+bool skinny_half(int proj, int act, int BT, int split_mode, bool raw) {
+    if (raw || resolve_split(split_mode) == kSplitInKernel) return false;
+    if (proj == 0 && act == TP_MLP_ACT_SWIGLU) return false;
+    return BT >= TPMLP_SKINNY_HALF_MIN_BT;
+}
+
+// Grid of a skinny projection.  Normally every SM, the weight stream cut into
+// equal shares (stream-K).  With fewer tiles than SMs and wide token tiles,
+// whose split-tile slots are large, a whole number s of CTAs per tile instead:
+// every CTA then stays inside one tile, each tile has exactly s slots, and with
+// as many tiles as SMs (s = 1) nothing is split at all -- provided that keeps
+// at least 80 % of the SMs busy.
+int skinny_grid(int tiles, int KB, int BT, int num_sms) {
+    if (BT >= TPMLP_SKINNY_ALIGN_MIN_BT && tiles <= num_sms) {
+        const int s = std::min(num_sms / tiles, KB);
+        if (s >= 1 && 5LL * tiles * s >= 4LL * num_sms) return tiles * s;
+    }
+    return num_sms;
+}
+
+StreamKGeom skinny_geom(int tiles, int KB, int BT, int num_sms) {
+    return streamk_geom(tiles, KB, skinny_grid(tiles, KB, BT, num_sms));
+}
+
 // One projection with the skinny tiling; x: T x K activations.
 cudaError_t run_skinny(const WeightOperand &w, const void *x, int T, int K, int epi, void *out, int out_cols,
                        float *part, unsigned *cnt, int *status, int num_sms, cudaStream_t st, int split_mode,
@@ -773,7 +878,7 @@ cudaError_t run_skinny(const WeightOperand &w, const void *x, int T, int K, int 
     const int BT = skinny_bt(T);
     CUtensorMap mx;
     if (!make_map(&mx, x, K, T, BT)) return cudaErrorInvalidValue;
-    const StreamKGeom g = streamk_geom(w.tiles, w.KB, num_sms);
+    const StreamKGeom g = skinny_geom(w.tiles, w.KB, BT, num_sms);
     TcArgs a{};
     a.rows_x = T;
     a.rows_w = w.tiles;
@@ -787,25 +892,37 @@ cudaError_t run_skinny(const WeightOperand &w, const void *x, int T, int K, int 
     a.slots = g.slots;
     a.part = part;
     a.tile_cnt = cnt;
-    a.split_mode = g.slots > 1 ? resolve_split(split_mode) : kSplitInKernel;
+    a.split_mode = g.slots > 1 ? (w.half ? kSplitSeparate : resolve_split(split_mode)) : kSplitInKernel;
     a.grid = g.grid;
     a.status = status;
     a.raw_first = w.raw_first;
     a.tps = w.tps;
     a.fs = w.fs;
     cudaError_t e;
-    switch (BT) {
-        case 16: e = launch_skinny_bt<16, 6>(w, mx, a, g.grid, st); break;
-        case 32: e = launch_skinny_bt<32, 6>(w, mx, a, g.grid, st); break;
-        case 64: e = launch_skinny_bt<64, 5>(w, mx, a, g.grid, st); break;
-        default: e = launch_skinny_bt<128, 4>(w, mx, a, g.grid, st); break;
+    // a 128-row tile stage holds half the weights, so the ring gets more stages
+    if (w.half) {
+        switch (BT) {
+            case 16: e = launch_skinny_bt<16, 8, true>(w, mx, a, g.grid, st); break;
+            case 32: e = launch_skinny_bt<32, 8, true>(w, mx, a, g.grid, st); break;
+            case 64: e = launch_skinny_bt<64, 8, true>(w, mx, a, g.grid, st); break;
+            default: e = launch_skinny_bt<128, 6, true>(w, mx, a, g.grid, st); break;
+        }
+    } else {
+        switch (BT) {
+            case 16: e = launch_skinny_bt<16, 6, false>(w, mx, a, g.grid, st); break;
+            case 32: e = launch_skinny_bt<32, 6, false>(w, mx, a, g.grid, st); break;
+            case 64: e = launch_skinny_bt<64, 5, false>(w, mx, a, g.grid, st); break;
+            default: e = launch_skinny_bt<128, 4, false>(w, mx, a, g.grid, st); break;
+        }
     }
     ++*launches;
     if (e != cudaSuccess || a.split_mode != kSplitSeparate) return e;
     ++*launches;
     // one CTA per unit: a grid capped at 2 CTAs per SM (so the next GEMM's CTAs
     // fit beside the waiting ones) measured 20-30 % slower at 32-128 tokens
-    return launch_pdl(skinny_reduce_kernel, dim3(g.tiles * (BT / 4)), dim3(128), 0, st, a, BT);
+    const dim3 rgrid(g.tiles * (BT / 4));
+    return w.half ? launch_pdl(skinny_reduce_kernel<true>, rgrid, dim3(128), 0, st, a, BT)
+                  : launch_pdl(skinny_reduce_kernel<false>, rgrid, dim3(128), 0, st, a, BT);
 }
 
 template <int MH>
@@ -846,14 +963,6 @@ int first_epi(int act) {
     return act == TP_MLP_ACT_SWIGLU ? EPI_H_SWIGLU : act == TP_MLP_ACT_TANH ? EPI_H_TANH : EPI_H_IDENT;
 }
 
-// Weight tiles of the first projection in either layout (the larger count sizes
-// the split-tile scratch).
-long long first_tiles(const Problem &p, bool raw) {
-    if (!raw) return blk_tiles(w1p_rows(p.d_ff, p.act));
-    const int per = p.act == TP_MLP_ACT_SWIGLU ? 128 : 256;
-    return (long long)p.tp * ((p.fs + per - 1) / per);
-}
-
 }  // namespace
 
 bool tc_supported(const Problem &p) {
@@ -863,20 +972,27 @@ bool tc_supported(const Problem &p) {
 
 bool tc_raw_supported(const Problem &p) { return tc_supported(p) && p.fs % BK == 0; }
 
+// Counters serve the in-kernel fixup, which only runs 256-row tiles: the first
+// projection's tiles (either layout) then the second's.
 size_t tile_counter_slots(const Problem &p) {
-    return (size_t)(std::max(first_tiles(p, false), first_tiles(p, true)) + blk_tiles(p.d_out));
+    return (size_t)(std::max(skinny_tiles(p, 0, false, false), skinny_tiles(p, 0, true, false)) +
+                    blk_tiles(p.d_out));
 }
 
+// Split-tile scratch: the largest over both layouts, both projections and both
+// tile heights, since the split mode may change after the workspace is sized.
 size_t tc_workspace_bytes(const Problem &p, int num_sms) {
     if (p.T < 1 || p.T > kTcSkinnyMaxTokens) return 0;
-    const size_t BT = skinny_bt(p.T);
+    const int BT = skinny_bt(p.T);
     size_t m = 0;
-    for (int raw = 0; raw < 2; ++raw) {
-        const StreamKGeom g1 = streamk_geom(first_tiles(p, raw), blk_kblocks(p.d_in), num_sms);
-        const StreamKGeom g2 = streamk_geom(blk_tiles(p.d_out), blk_kblocks(p.d_ff), num_sms);
-        m = std::max(m, (size_t)g1.tiles * g1.slots * 256 * BT * 4);
-        m = std::max(m, (size_t)g2.tiles * g2.slots * 256 * BT * 4);
-    }
+    for (int raw = 0; raw < 2; ++raw)
+        for (int proj = 0; proj < 2; ++proj)
+            for (int half = 0; half < 2; ++half) {
+                if (half && proj == 0 && p.act == TP_MLP_ACT_SWIGLU) continue;
+                const long long tiles = skinny_tiles(p, proj, raw, half);
+                const StreamKGeom g = skinny_geom((int)tiles, (int)blk_kblocks(proj ? p.d_ff : p.d_in), BT, num_sms);
+                m = std::max(m, (size_t)g.tiles * g.slots * (half ? 128 : 256) * BT * 4);
+            }
     return align256(m);
 }
 
@@ -887,16 +1003,21 @@ cudaError_t launch_tc(const Problem &p, int tiling, const void *x, const void *w
     *launches = 0;
     WeightOperand w1, w2;
     const bool raw = rawA != nullptr;
+    const bool skinny = tiling == kTilingSkinny;
+    const int BT = skinny_bt(p.T);
+    const bool half1 = skinny && skinny_half(0, p.act, BT, split_mode, raw);
+    const bool half2 = skinny && skinny_half(1, p.act, BT, split_mode, raw);
     if (raw) {
-        if (!weight_raw_first(&w1, p, *rawA) || !weight_raw_second(&w2, p, *rawB)) return cudaErrorInvalidValue;
-    } else if (!weight_packed(&w1, w1p, w1p_rows(p.d_ff, p.act), p.d_in) ||
-               !weight_packed(&w2, w2p, p.d_out, p.d_ff)) {
+        if (!weight_raw_first(&w1, p, *rawA, half1) || !weight_raw_second(&w2, p, *rawB, half2))
+            return cudaErrorInvalidValue;
+    } else if (!weight_packed(&w1, p, 0, w1p, half1) || !weight_packed(&w2, p, 1, w2p, half2)) {
         return cudaErrorInvalidValue;
     }
     cudaError_t e;
     marks.mark(0, st);
-    if (tiling == kTilingSkinny) {
-        unsigned *cnt1 = counters, *cnt2 = counters + w1.tiles;
+    if (skinny) {
+        unsigned *cnt1 = counters;
+        unsigned *cnt2 = counters + std::max(skinny_tiles(p, 0, false, false), skinny_tiles(p, 0, true, false));
         e = run_skinny(w1, x, p.T, p.d_in, first_epi(p.act), h, p.d_ff, part, cnt1, status, num_sms, st,
                        split_mode, launches);
         if (e != cudaSuccess) return e;

@@ -93,8 +93,10 @@ def test_tc_skinny_parity(act, T, shape):
 @pytest.mark.parametrize("shape", SHAPES)
 def test_tc_skinny_split_finish_modes_agree(act, T, shape):
     """Split tiles finished by the last CTA inside the GEMM, or by the reduction
-    kernel behind it: both add the partial slots in slot order, so the outputs
-    are identical, and both match the oracle."""
+    kernel behind it.  On packed weights the reduction route also uses 128-row
+    tiles where it can (the in-kernel fixup keeps 256), so the split points
+    differ and the oracle decides; the shard-form test below, where both
+    routes tile alike, checks that they agree bit for bit."""
     d, f, dout, tp = shape
     p = inputs.generate(T, d, f, act, "bf16", seed=7 * T + f, init="fan_in", d_out=dout)
     A, Bs = p.shards(tp)
@@ -115,7 +117,34 @@ def test_tc_skinny_split_finish_modes_agree(act, T, shape):
         if mode in outs:
             assert torch.equal(out, outs[mode])     # counters were left at zero
         outs[mode] = out
-    assert torch.equal(outs["in_kernel"], outs["separate"])
+    assert set(outs) == {"in_kernel", "separate"}
+
+
+
+@pytest.mark.parametrize("api", ["packed", "shard"])
+@pytest.mark.parametrize("T", [40, 100])
+def test_tc_skinny_whole_128_row_tiles(api, T):
+    """About as many 128-row tiles as SMs (packed weights): each CTA takes one
+    whole first-projection tile (no partial slots, no reduction kernel); the
+    second projection's few tiles are split evenly, every CTA inside one tile.
+    The shard form keeps 256-row tiles, split evenly in two."""
+    d, f, dout, tp = 256, 16384, 512, 8
+    p = inputs.generate(T, d, f, "tanh", "bf16", seed=T + 5, init="fan_in", d_out=dout)
+    A, Bs = p.shards(tp)
+    ref = oracle.tp_mlp_sharded(p.x, A, Bs, "tanh")
+    m = B().TpMlp(d, f, tp, "tanh", "bf16", T, d_out=dout)
+    m.set_plan("tc_skinny")
+    Ad, Bd = [dev(a, "bf16") for a in A], [dev(b, "bf16") for b in Bs]
+    if api == "packed":
+        out = m.forward_packed(dev(p.x, "bf16"), m.pack(Ad, Bd))
+    else:
+        out = m.forward(dev(p.x, "bf16"), Ad, Bd)
+    torch.cuda.synchronize()
+    B().tp_mlp_get_device_status(m.h)
+    assert_close(out, ref, "bf16", f"whole 128-row tiles {api} T={T}")
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    if api == "packed" and 5 * 128 >= 4 * sms and 128 <= sms:   # 128 first-projection tiles fit the rule
+        assert m.last_launches == 3                 # GEMM, GEMM + reduction
 
 
 @pytest.mark.parametrize("act", ["swiglu", "tanh"])
@@ -225,6 +254,7 @@ def test_tc_shard_form_split_finish_modes_agree(T):
         torch.cuda.synchronize()
         B().tp_mlp_get_device_status(m.h)
         assert_close(outs[-1], ref, "bf16", f"shard form {mode} T={T}")
+    # the shard form keeps 256-row tiles on both routes: same split, same order
     assert torch.equal(outs[0], outs[1])
 
 
