@@ -290,6 +290,7 @@ class FusedNormOp:
     """The all-reduce + residual add + RMSNorm step ("7.4 推理侧并行" §7.4.2)."""
     metric = FUSED_NORM_METRIC
     kernel = "allreduce_norm_kernel"
+    family = "fused_norm"
     library_ops = "torch sum over ranks, add, rms_norm"
 
     def __init__(self, args):
@@ -351,6 +352,7 @@ class AttnMergeOp:
     """The merge of KV shards' partial attention results ("LLM 推理并行化" §三 4), DCP)."""
     metric = ATTN_MERGE_METRIC
     kernel = "attn_merge_kernel"
+    family = "attn_merge"
     library_ops = "torch max, exp, weighted sums and division over ranks"
 
     def __init__(self, args):
@@ -514,7 +516,7 @@ def run_small_op(args, op):
     peaks, src = load_peaks()
     achieved = step_bytes / (launch_ms / 1e3) / 1e9
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm_gbs"], "traffic": recorded_traffic(f"{op.kernel}:op", args.config),
+                "frac": achieved / peaks["hbm_gbs"], "traffic": recorded_traffic(f"{op.family}:op", args.config),
                 "kernel": op.kernel, "kernel_ms": launch_ms, "algorithmic_per_launch": step_bytes,
                 "peak_source": f"hbm_gbs ({src})"}
     ms = elapsed_ms / K

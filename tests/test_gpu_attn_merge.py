@@ -103,3 +103,13 @@ def test_merge_rejects_bad_arguments_before_launch():
     assert L.tp_mlp_merge_attention_partials(2, 100000, 64, ptr(m), ptr(s), ptr(w), 0, ptr(out), None) == 2
     misaligned = B().ctypes.c_void_p(w.data_ptr() + 8)
     assert L.tp_mlp_merge_attention_partials(2, 4, 64, ptr(m), ptr(s), misaligned, 0, ptr(out), None) == 3
+
+
+@pytest.mark.parametrize("name", ["attn_merge_decode_bs32", "attn_merge_decode_bs256"])
+def test_merge_bench_configs_full_size(name):
+    """The workloads bench.py times, at their full sizes, every row checked."""
+    c = inputs.ATTN_MERGE_CONFIGS[name]
+    a = inputs.generate_attn_merge(c["tp"], c["tokens"] * c["heads"], c["head_dim"], c["dtype"], c["seed"],
+                                   c["keys_per_rank"])
+    got = _merge(a.maximum, a.exp_sum, a.weighted, c["dtype"])
+    assert_close(got, oracle.merge_attention_partials(a.maximum, a.exp_sum, a.weighted), c["dtype"], name)

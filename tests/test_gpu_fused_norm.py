@@ -143,3 +143,19 @@ def test_fused_norm_rejects_bad_arguments_before_launch():
     misaligned = B().ctypes.c_void_p(p.data_ptr() + 4)
     assert L.tp_mlp_allreduce_residual_rmsnorm(misaligned, 2, 1, 64, ptr(r), ptr(g), 0.0, 0, ptr(y), ptr(y),
                                                None) == 3
+
+
+@pytest.mark.parametrize("name", ["fused_norm_decode_bs32", "fused_norm_prefill"])
+def test_fused_norm_bench_configs_full_size(name):
+    """The workloads bench.py times, at their full sizes; the prefill shape is
+    checked on 256 seeded rows (the oracle handles rows independently)."""
+    c = inputs.FUSED_NORM_CONFIGS[name]
+    fi = inputs.generate_fused_norm(c["tokens"], c["d_model"], c["tp"], c["dtype"], c["seed"], c["eps"])
+    y, ro = _run(fi.partials, fi.residual, fi.gamma, c["eps"], c["dtype"])
+    rows = np.arange(c["tokens"])
+    if c["tokens"] > 256:
+        rows = np.sort(np.random.default_rng(c["seed"]).choice(c["tokens"], 256, replace=False))
+    y_ref, h_ref = oracle.allreduce_residual_rmsnorm(fi.partials[:, rows], fi.residual[rows], fi.gamma, c["eps"])
+    idx = torch.from_numpy(rows).cuda()
+    assert_close(y[idx], y_ref, c["dtype"], f"{name} y")
+    assert_close(ro[idx], h_ref, c["dtype"], f"{name} residual")

@@ -238,8 +238,11 @@ def test_sweep_config(T):
         if ref is None:
             ref = oracle.tp_mlp_sharded(p.x[rows], A, Bs, "tanh")
         m = _mlp(p, tp, "bf16", max_tokens=T)
-        out = m.forward_packed(dev(p.x, "bf16"), m.pack(Ad, Bd))
+        x = dev(p.x, "bf16")
+        out = m.forward_packed(x, m.pack(Ad, Bd))
         assert_close(out[torch.from_numpy(rows).cuda()], ref, "bf16", f"sweep T={T} tp={tp}")
+        out = m.forward(x, Ad, Bd)          # the shard form (its own tiling and grid)
+        assert_close(out[torch.from_numpy(rows).cuda()], ref, "bf16", f"sweep T={T} tp={tp} shard form")
         del Ad, Bd, m
 
 
