@@ -16,6 +16,7 @@ from __future__ import annotations
 
 import hashlib
 import os
+import re
 
 ELEM_BYTES = {"f32": 4, "bf16": 2}
 
@@ -106,10 +107,18 @@ _KERNEL_SOURCES = {
 }
 
 
+def _code_only(text: str) -> str:
+    """C/CUDA source without comments or layout: what the compiler sees of it."""
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
 def kernel_source_hash(plan: str) -> str:
+    """Hash of the code (comments and whitespace ignored) of a kernel family's sources."""
     d = os.path.join(os.path.dirname(os.path.abspath(__file__)), "csrc")
     h = hashlib.sha256()
     for n in _KERNEL_SOURCES.get(plan, sorted(os.listdir(d))):
-        with open(os.path.join(d, n), "rb") as f:
-            h.update(n.encode() + f.read())
+        with open(os.path.join(d, n), encoding="utf-8") as f:
+            h.update(n.encode() + _code_only(f.read()).encode())
     return h.hexdigest()[:16]

@@ -14,12 +14,13 @@
 //          kGroupM token tiles so a weight tile is reused from L2;
 //   skinny (few tokens, memory-bound, the decode case "7.4 推理侧并行" §7.4.1
 //          describes): operands swapped -- M is 128 weight rows (two MMAs per
-//          256-row weight tile), N is the token count rounded up to BT.  The
-//          weight stream is cut into equal contiguous shares, one per CTA
-//          ("stream-K"); a tile split between CTAs is finished from fp32
-//          partial slots added in a fixed order, either by a reduction kernel
-//          behind the GEMM (default) or by the last CTA to arrive.  Nothing
-//          waits on another CTA.
+//          256-row weight tile, or one per 128-row tile), N is the token count
+//          rounded up to BT.  The weight stream is cut into equal contiguous
+//          shares, one per CTA ("stream-K"), or -- with few tiles -- a whole
+//          number of CTAs per tile; a tile split between CTAs is finished from
+//          fp32 partial slots added in a fixed order, either by a reduction
+//          kernel behind the GEMM (default) or by the last CTA to arrive.
+//          Nothing waits on another CTA.
 //
 // Roles: warp 0 lane 0 issues TMA loads, warp 1 allocates TMEM and lane 0
 // issues the MMAs, warps 2..5 run the epilogue (TMEM lanes 32*(warp%4)...).
