@@ -438,6 +438,28 @@ __device__ __forceinline__ void skinny_final_half4(const TcArgs &a, int tile, in
         if (t0 + i < a.rows_x) a.out[(long)(t0 + i) * a.ldo + n] = __float2bfloat16_rn(act_out(a.epi, g[i]));
 }
 
+// Whole 128-row tile, 16 tokens t0.. of row r (TMEM lane r): the activation,
+// then the columns of two neighbouring rows go out together as one 4-byte
+// bf16 pair.  Lanes 2k and 2k+1 hold columns n, n+1; per pair of tokens they
+// swap one value with a shuffle, the even lane stores both columns of the even
+// token and the odd lane those of the odd one -- half the stores of one column
+// per lane.  (Output widths are multiples of 8, so n and n+1 are both real
+// columns or both padding, and a pair is 4-byte aligned.)
+__device__ __forceinline__ void skinny_store_pairs16(const TcArgs &a, int tile, int r, int t0, const float (&v)[16]) {
+    const bool odd = threadIdx.x & 1;
+    const int n = tile_col(a, tile, r & ~1, 128);
+#pragma unroll
+    for (int j = 0; j < 16; j += 2) {
+        const float e = act_out(a.epi, v[j]), o = act_out(a.epi, v[j + 1]);
+        const float recv = __shfl_xor_sync(0xffffffffu, odd ? e : o, 1);
+        const int t = t0 + j + (odd ? 1 : 0);
+        if (n >= 0 && t < a.rows_x) {
+            const __nv_bfloat162 pr = odd ? __floats2bfloat162_rn(recv, o) : __floats2bfloat162_rn(e, recv);
+            *reinterpret_cast<__nv_bfloat162 *>(a.out + (long)t * a.ldo + n) = pr;
+        }
+    }
+}
+
 // HALF: 128-row weight tiles, one M=128 MMA per 16-k step (never SwiGLU's first
 // projection, whose gate and up rows must share a tile); split tiles always go
 // to skinny_reduce_kernel.
@@ -547,10 +569,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     if (!HALF) tmem_ld16(taddr + BT + t0, v1);
                     tmem_ld_wait();
                     if (HALF) {
-#pragma unroll
-                        for (int q4 = 0; q4 < 4; ++q4)
-                            skinny_final_half4(a, tile, r, t0 + 4 * q4,
-                                               make_float4(v0[4 * q4], v0[4 * q4 + 1], v0[4 * q4 + 2], v0[4 * q4 + 3]));
+                        skinny_store_pairs16(a, tile, r, t0, v0);
                     } else {
                         skinny_final16(a, tile, r, t0, v0, v1);
                     }
