@@ -66,12 +66,12 @@ def bench_cmd(config: str, extra: list[str]) -> str:
 
 def list_cmd(a) -> str:
     return (f"ncu --metrics gpu__time_duration.sum --clock-control none --csv "
-            f"--log-file gpurun_out/launches_{a.config}.csv {bench_cmd(a.config, a.extra)}")
+            f"--log-file {a.out_dir}/launches_{a.config}.csv {bench_cmd(a.config, a.extra)}")
 
 
 def full_cmd(a) -> str:
     return (f"ncu --set full --clock-control none -k regex:{a.kernel} -s 3 -c 1 "
-            f"-o gpurun_out/prof_{a.kernel}_{a.config} {bench_cmd(a.config, a.extra)}")
+            f"-o {a.out_dir}/prof_{a.kernel}_{a.config} {bench_cmd(a.config, a.extra)}")
 
 
 def _read_csv_rows(text: str):
@@ -156,6 +156,7 @@ def main(argv=None):
         p = sub.add_parser(n)
         p.add_argument("--config", default="decode_bs1")
         p.add_argument("--kernel", default="gemv_kernel")
+        p.add_argument("--out-dir", default="ncu_out", help="where ncu writes the CSV or report")
         p.add_argument("extra", nargs=argparse.REMAINDER)
     p = sub.add_parser("summarize-list")
     p.add_argument("csv")
