@@ -74,8 +74,10 @@ typedef enum {
     TP_MLP_PLAN_TC = 3,     /* packed bf16: tcgen05 tensor-core GEMMs (TMA + TMEM);
                                the library picks the tiling from the token count      */
     TP_MLP_PLAN_TC_WIDE = 4,   /* tcgen05, tiles of 128 tokens x 256 weight rows      */
-    TP_MLP_PLAN_TC_SKINNY = 5, /* tcgen05, weights as the MMA's M, 1..128 tokens as N,
-                                  weight stream split evenly over the SMs             */
+    TP_MLP_PLAN_TC_SKINNY = 5, /* tcgen05, weights as the MMA's M (tiles of 128 or 256
+                                  rows), 1..128 tokens as N; the weight stream split
+                                  evenly over the SMs, or whole CTAs per tile when
+                                  tiles are few                                       */
     TP_MLP_PLAN_TC_WIDE256 = 6 /* tcgen05, tiles of 256 tokens x 256 weight rows      */
 } tp_mlp_plan;
 

@@ -96,3 +96,38 @@ def test_counts_for_decode_config():
     tot = counts.algorithmic_bytes(32, 8192, 28672, 8192, "swiglu", "bf16")
     assert tot == counts.gemm1_bytes(32, 8192, 28672, "swiglu", "bf16") + \
         counts.gemm2_bytes(32, 28672, 8192, "bf16")
+
+
+def test_fused_norm_inputs_are_seeded_and_dtype_exact():
+    a = inputs.generate_fused_norm(3, 16, 2, "bf16", seed=4)
+    b = inputs.generate_fused_norm(3, 16, 2, "bf16", seed=4)
+    assert a.partials.shape == (2, 3, 16) and a.residual.shape == (3, 16) and a.gamma.shape == (16,)
+    for x, y in ((a.partials, b.partials), (a.residual, b.residual), (a.gamma, b.gamma)):
+        assert x.dtype == np.float32 and np.array_equal(x, y)
+    # residual and gamma hold bf16 values; the fp32 partials are not rounded
+    assert np.array_equal(a.residual, inputs.round_to_bf16(a.residual))
+    assert np.array_equal(a.gamma, inputs.round_to_bf16(a.gamma))
+    assert not np.array_equal(a.partials, inputs.round_to_bf16(a.partials))
+    assert not np.array_equal(a.partials, inputs.generate_fused_norm(3, 16, 2, "bf16", seed=5).partials)
+
+
+def test_attn_merge_inputs_are_seeded_and_in_range():
+    a = inputs.generate_attn_merge(4, 10, 8, "bf16", seed=7, keys_per_rank=64)
+    assert a.maximum.shape == (4, 10) and a.exp_sum.shape == (4, 10) and a.weighted.shape == (4, 10, 8)
+    assert np.all(a.exp_sum >= 1.0) and np.all(a.exp_sum <= 64.0)   # at least the maximum's own term
+    assert np.array_equal(a.weighted, inputs.round_to_bf16(a.weighted))
+    b = inputs.generate_attn_merge(4, 10, 8, "bf16", seed=7, keys_per_rank=64)
+    assert np.array_equal(a.weighted, b.weighted) and np.array_equal(a.maximum, b.maximum)
+
+
+def test_fused_norm_byte_counts():
+    # 2 ranks, 3 tokens, width 4, bf16: partials 2*3*4*4, residual 3*4*2, gamma 4*2, outputs 2*3*4*2
+    assert counts.fused_norm_bytes(2, 3, 4, "bf16") == 96 + 24 + 8 + 48
+    # unfused: Z and h each written and read once more (2 * 2 * n * e)
+    assert counts.unfused_norm_bytes(2, 3, 4, "bf16") - counts.fused_norm_bytes(2, 3, 4, "bf16") == 2 * 2 * 12 * 2
+
+
+def test_kernel_source_hash_ignores_comments_only():
+    code = "int f(int a) { return a + 1; }"
+    assert counts._code_only("// lead\nint f(int a) {  /* note */ return a + 1; }  // tail") == code
+    assert counts._code_only(code) != counts._code_only(code.replace("+ 1", "+ 2"))
