@@ -15,6 +15,12 @@
  * Here every rank's shards live in the memory of ONE GPU, so the all-reduce
  * is a sum on the device, fused into the second projection's accumulation.
  *
+ * Two more operators from the same pages take no handle but follow the same
+ * conventions: tp_mlp_allreduce_residual_rmsnorm (the all-reduce of the
+ * ranks' partials fused with the residual add and RMSNorm that follow it) and
+ * tp_mlp_merge_attention_partials (decode context parallelism's merge of the
+ * KV shards' partial attention results).  Their declarations are at the end.
+ *
  * Conventions for every entry point
  *   - Matrices are row-major and densely packed (row stride = row length).
  *   - "device pointer" = memory of the current CUDA device; "host" = CPU memory.
