@@ -66,7 +66,7 @@ typedef enum {
     TP_MLP_ERR_INVALID_ARG = 1,  /* NULL handle/pointer, unknown enum value            */
     TP_MLP_ERR_SHAPE = 2,        /* sizes, shard count, d_ff % tp, tokens > max_tokens */
     TP_MLP_ERR_ALIGNMENT = 3,    /* a pointer is not 16-byte aligned                   */
-    TP_MLP_ERR_UNSUPPORTED = 4,  /* valid request this build cannot serve              */
+    TP_MLP_ERR_UNSUPPORTED = 4,  /* valid request the library cannot serve            */
     TP_MLP_ERR_CUDA = 5,         /* a CUDA runtime call failed (launch or earlier work) */
     TP_MLP_ERR_TIMEOUT = 6,      /* reserved: a bounded device-side wait ran out       */
     TP_MLP_ERR_WORKSPACE = 7     /* no workspace set, or smaller than required         */

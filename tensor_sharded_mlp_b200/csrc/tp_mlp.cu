@@ -519,7 +519,7 @@ const char *tp_mlp_status_string(int status) {
         case TP_MLP_ERR_INVALID_ARG: return "invalid argument";
         case TP_MLP_ERR_SHAPE: return "shape mismatch";
         case TP_MLP_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
-        case TP_MLP_ERR_UNSUPPORTED: return "unsupported by this build";
+        case TP_MLP_ERR_UNSUPPORTED: return "unsupported by the library";
         case TP_MLP_ERR_CUDA: return "CUDA error";
         case TP_MLP_ERR_TIMEOUT: return "device wait timed out";
         case TP_MLP_ERR_WORKSPACE: return "workspace missing or too small";
