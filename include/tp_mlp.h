@@ -280,8 +280,8 @@ int tp_mlp_decode_forward_static(int d_model, int d_ff, int d_out, int tp_degree
 
 /*
  * The all-reduce of the ranks' partial outputs fused with the residual add and
- * RMSNorm that follow it ("7.4 推理侧并行", §7.4.2, optimisation 2: fusing
- * them saves a round trip of the summed activations through memory).  With
+ * RMSNorm that follow it ("7.4 推理侧并行", §7.4.2, optimisation 2: done in
+ * one kernel, the summed activations are not stored and reloaded).  With
  * every rank on one GPU the all-reduce is the sum of the fp32 partials that
  * tp_mlp_partials returns.  For every token row t (ranks added in order,
  * fp32 arithmetic):

@@ -8,8 +8,9 @@
  * What it computes, and where the pages say so:
  *
  *  - "7.4 推理侧并行", §7.4.2, optimisation 2 (custom all-reduce), its last
- *    point: the residual add and the RMSNorm that follow the all-reduce are
- *    fused into one kernel, which saves one round trip through device memory.
+ *    point: the kernel that sums the ranks' outputs also does the residual
+ *    add and the RMSNorm that come next, so the summed activations are not
+ *    written to device memory and read back by a separate kernel.
  *  - The all-reduce sums the ranks' partial outputs Z_i of the row-parallel
  *    second projection ("大模型推理系统揭秘（07）", §1.2.3: Z = sum_i Y_i W_2i),
  *    in rank order as in tp_mlp_oracle.c.
