@@ -3,7 +3,10 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--config decode_bs1|decode_bs32|prefill|sweep|tiny] [--tokens T] [--tp P]
-                    [--plan auto|gemv|simt|tc]
+                    [--plan auto|simt|gemv|tc|tc_skinny|tc_wide|tc_wide256] [--api packed|shard]
+                    [--splitk auto|in_kernel|separate] [--no-e2e] [--no-cpu-baseline] [--no-graph]
+    python bench.py --config fused_norm_decode_bs32|fused_norm_prefill|
+                             attn_merge_decode_bs32|attn_merge_decode_bs256 [...]
 
 One step = one forward of the whole hot path (first projection + activation,
 second projection with the ranks' partial sums reduced on the device) over one
@@ -18,6 +21,11 @@ the data path); the reported time is the max over ranks.
 
 --impl reference times the oracle (plain fp64 C loops on the host cores) on a
 bounded sample of the same workload; under torchrun only rank 0 runs it.
+
+The fused_norm_* and attn_merge_* configs time the two other operators (the
+all-reduce fused with residual add and RMSNorm; the merge of attention
+partials across KV shards): one launch per step, the K steps captured in a
+CUDA graph, inputs smaller than L2 rotated through enough copies to exceed it.
 """
 from __future__ import annotations
 
@@ -42,7 +50,10 @@ def parse():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", default="decode_bs1")
+    ap.add_argument("--config", default="decode_bs1",
+                    help="MLP: tiny, decode_bs1, decode_bs32, sweep, prefill; other operators: "
+                         "fused_norm_decode_bs32, fused_norm_prefill, attn_merge_decode_bs32, "
+                         "attn_merge_decode_bs256")
     ap.add_argument("--tokens", type=int, default=None)
     ap.add_argument("--tp", type=int, default=None)
     ap.add_argument("--plan", default="auto")
@@ -52,8 +63,8 @@ def parse():
     ap.add_argument("--d-ff", type=int, default=None, help="override (small cases for profiling)")
     ap.add_argument("--api", choices=["packed", "shard"], default="packed",
                     help="packed: weights packed once, tp_mlp_forward_packed; shard: tp_mlp_forward on the shards")
-    ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) measurement")
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip timing the oracle on the host")
     ap.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph replay percentiles")
     return ap.parse_args()
 
