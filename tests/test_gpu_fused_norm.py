@@ -11,7 +11,7 @@ import pytest
 import torch
 
 import oracle
-from helpers import TOL, assert_close, dev
+from helpers import assert_close, dev
 from tensor_sharded_mlp_b200 import inputs
 
 pytestmark = pytest.mark.gpu

@@ -10,7 +10,7 @@ import pytest
 import torch
 
 import oracle
-from helpers import TOL, assert_close, dev, rel_err
+from helpers import assert_close, dev
 from tensor_sharded_mlp_b200 import inputs
 
 pytestmark = pytest.mark.gpu
