@@ -438,25 +438,20 @@ __device__ __forceinline__ void skinny_final_half4(const TcArgs &a, int tile, in
         if (t0 + i < a.rows_x) a.out[(long)(t0 + i) * a.ldo + n] = __float2bfloat16_rn(act_out(a.epi, g[i]));
 }
 
-// Whole 128-row tile, 16 tokens t0.. of row r (TMEM lane r): the activation,
-// then the columns of two neighbouring rows go out together as one 4-byte
-// bf16 pair.  Lanes 2k and 2k+1 hold columns n, n+1; per pair of tokens they
-// swap one value with a shuffle, the even lane stores both columns of the even
-// token and the odd lane those of the odd one -- half the stores of one column
-// per lane.  (Output widths are multiples of 8, so n and n+1 are both real
-// columns or both padding, and a pair is 4-byte aligned.)
-__device__ __forceinline__ void skinny_store_pairs16(const TcArgs &a, int tile, int r, int t0, const float (&v)[16]) {
-    const bool odd = threadIdx.x & 1;
-    const int n = tile_col(a, tile, r & ~1, 128);
-#pragma unroll
-    for (int j = 0; j < 16; j += 2) {
-        const float e = act_out(a.epi, v[j]), o = act_out(a.epi, v[j + 1]);
-        const float recv = __shfl_xor_sync(0xffffffffu, odd ? e : o, 1);
-        const int t = t0 + j + (odd ? 1 : 0);
-        if (n >= 0 && t < a.rows_x) {
-            const __nv_bfloat162 pr = odd ? __floats2bfloat162_rn(recv, o) : __floats2bfloat162_rn(e, recv);
-            *reinterpret_cast<__nv_bfloat162 *>(a.out + (long)t * a.ldo + n) = pr;
-        }
+// Whole 128-row tile: the epilogue warps stage the BT x 128 bf16 outputs (after
+// the activation) in shared memory, one column per thread, then write them out
+// as 16-byte pieces of 8 columns of one token -- a sixteenth of the stores of
+// one 2-byte column per thread.  `so` holds BT rows of 128 columns.  Output
+// widths are multiples of 8, so a piece is all real columns or all padding and
+// is 16-byte aligned.  Runs on the 128 epilogue threads (named barrier 1).
+__device__ __forceinline__ void skinny_store_staged(const TcArgs &a, int tile, int BT, const __nv_bfloat16 *so) {
+    const int et = threadIdx.x - 64;                 // 0..127
+    for (int c = et; c < BT * 16; c += 128) {
+        const int t = c >> 4, j = c & 15;
+        const int col = tile_col(a, tile, 8 * j, 128);
+        if (t < a.rows_x && col >= 0)
+            *reinterpret_cast<uint4 *>(a.out + (long)t * a.ldo + col) =
+                *reinterpret_cast<const uint4 *>(so + t * 128 + 8 * j);
     }
 }
 
@@ -470,6 +465,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     constexpr uint32_t X_BYTES = BT * BK * 2;
     extern __shared__ uint8_t smem_raw[];
     const Smem s = carve<STAGES>(smem_raw, W_BYTES, X_BYTES);
+    // HALF: BT x 128 bf16 output staging after the barrier block (16-byte aligned)
+    __nv_bfloat16 *stage_out = reinterpret_cast<__nv_bfloat16 *>(
+        (reinterpret_cast<uintptr_t>(s.tmem_slot) + 16 + 15) & ~uintptr_t(15));
     const uint32_t tmem_base = setup<STAGES>(s, &wm.map[0], &tmX);
     pdl_allow_dependents();
 
@@ -569,7 +567,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     if (!HALF) tmem_ld16(taddr + BT + t0, v1);
                     tmem_ld_wait();
                     if (HALF) {
-                        skinny_store_pairs16(a, tile, r, t0, v0);
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            stage_out[(t0 + i) * 128 + r] = __float2bfloat16_rn(act_out(a.epi, v0[i]));
                     } else {
                         skinny_final16(a, tile, r, t0, v0, v1);
                     }
@@ -577,6 +577,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_u32(&s.tempty[acc]));
+                if (HALF) {
+                    named_bar(1, 128);   // the whole tile is staged
+                    skinny_store_staged(a, tile, BT, stage_out);
+                    named_bar(1, 128);   // staging is free for the next tile
+                }
             } else {
                 // this CTA's share of the tile -> its partial slot, laid out
                 // [token/4][row][token%4]: each lane stores float4s, a warp 512 B at a time
@@ -845,7 +850,8 @@ cudaError_t set_smem(K kern, size_t bytes) {
 template <int BT, int STAGES, bool HALF>
 cudaError_t launch_skinny_bt(const WeightOperand &w, const CUtensorMap &mx, const TcArgs &a, int grid,
                              cudaStream_t st) {
-    const size_t smem = smem_bytes<STAGES>((HALF ? 128 : 256) * BK * 2, BT * BK * 2);
+    // HALF adds the epilogue's BT x 128 bf16 staging (+16 for its alignment)
+    const size_t smem = smem_bytes<STAGES>((HALF ? 128 : 256) * BK * 2, BT * BK * 2) + (HALF ? BT * 256 + 16 : 0);
     if (w.raw) {
         auto kern = tc_skinny_kernel<BT, STAGES, true, HALF>;
         cudaError_t e = set_smem(kern, smem);
