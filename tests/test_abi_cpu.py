@@ -175,3 +175,49 @@ def test_binding_pairs_shards_strictly(b):
     with pytest.raises(ValueError):
         b.tp_mlp_forward(h, torch.zeros(1, 8), [t, t], [t], 2, "tanh", torch.zeros(1, 4))
     b.tp_mlp_destroy(h)
+
+
+def _model_slots(tiles, KB, BT, sms=148):
+    """Split pieces per tile under the documented grid rule: floor(sms / tiles)
+    CTAs per tile when that keeps 80 % of the SMs busy, else equal contiguous
+    shares of the (tile, k-block) stream over every SM."""
+    G = sms
+    if tiles <= sms:
+        s = min(sms // tiles, KB)
+        if s >= 1 and 5 * tiles * s >= 4 * sms:
+            G = tiles * s
+    total = tiles * KB
+    G = min(G, total)
+
+    def owner(it):
+        return ((it + 1) * G - 1) // total
+    return max(owner(t * KB + KB - 1) - owner(t * KB) + 1 for t in range(tiles))
+
+
+@pytest.mark.parametrize("act,d,f,dout,tp", [("tanh", 4096, 16384, 4096, 8), ("swiglu", 8192, 28672, 8192, 8),
+                                             ("tanh", 512, 1024, 384, 4)])
+def test_workspace_covers_every_skinny_tiling(b, act, d, f, dout, tp):
+    """The split-tile scratch must hold the largest of every tiling the skinny
+    path may pick (packed or shard form, 256- or 128-row tiles, either
+    projection), since the split mode can change after the workspace is sized."""
+    h = b.tp_mlp_create(d, f, dout, tp, act, "bf16", 128)
+    fs = f // tp
+    for T, BT in ((16, 16), (32, 32), (64, 64), (128, 128)):
+        need = 0
+        for proj in (0, 1):
+            KB = -(-(d if proj == 0 else f) // 64)
+            for raw in (False, True):
+                for half in (False, True):
+                    if half and proj == 0 and act == "swiglu":
+                        continue
+                    rows = 128 if half else 256
+                    if proj == 1:
+                        tiles = -(-dout // rows)
+                    elif not raw:
+                        tiles = -(-((2 * f) if act == "swiglu" else f) // rows)
+                    else:
+                        per = 128 if (act == "swiglu" or half) else 256
+                        tiles = tp * -(-fs // per)
+                    need = max(need, tiles * _model_slots(tiles, KB, BT) * rows * BT * 4)
+        assert b.tp_mlp_workspace_bytes(h, T) >= T * f * 2 + need, (T, need)
+    b.tp_mlp_destroy(h)
