@@ -607,7 +607,14 @@ def main():
     m.set_plan(args.plan)
     m.set_splitk(args.splitk)
     Ad, Bd = [up(a) for a in A], [up(b) for b in Bs]
+    # the one-off shard-layout pack, timed on its own (not part of a step)
+    torch.cuda.synchronize()
+    p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    p0.record()
     packed = m.pack(Ad, Bd)
+    p1.record()
+    p1.synchronize()
+    pack_ms = p0.elapsed_time(p1)
     if args.api == "packed":
         del Ad, Bd
         fwd = lambda: m.forward_packed(x, packed, out=out)            # noqa: E731
@@ -725,7 +732,10 @@ def main():
                        "l2": "inputs larger than L2: every step re-reads %.2f GB of weights" % (step_bytes / 1e9)},
             "step_hbm_gbs": step_bytes / (ms / 1e3) / 1e9, "step_tflops": step_flops / (ms / 1e3) / 1e12,
             "roofline": roofline, "gpu_launches": K * nk, "clocks": sampler.summary(), "e2e": e2e,
-            "graph_step": graph_steps}
+            "graph_step": graph_steps,
+            "pack": {"ms": pack_ms, "note": "one-off shard-layout pack before timing (first call, includes "
+                                           "the packer's launch set-up); reads and writes every weight once",
+                     "GBs": 2 * counts.weight_bytes(d, f, d, act, dt) / (pack_ms / 1e3) / 1e9}}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = oracle_baseline(p, A, Bs, act)
     if rank == 0:
