@@ -5,6 +5,7 @@
                     [--config decode_bs1|decode_bs32|prefill|sweep|tiny] [--tokens T] [--tp P]
                     [--plan auto|simt|gemv|tc|tc_skinny|tc_wide|tc_wide256] [--api packed|shard]
                     [--splitk auto|in_kernel|separate] [--no-e2e] [--no-cpu-baseline] [--no-graph]
+                    [--configs auto|all|none]
     python bench.py --config fused_norm_decode_bs32|fused_norm_prefill|
                              attn_merge_decode_bs32|attn_merge_decode_bs256 [...]
 
@@ -14,6 +15,12 @@ batch of seeded synthetic input, on weights packed once before timing.  The
 default workload is decode at batch 1 (bf16 SwiGLU, d_model 8192, d_ff 28672,
 8 ranks' shards on one GPU).  The weights (1.41 GB) are far larger than L2, so
 every step re-reads them from HBM; no L2 flush is needed.
+
+The default invocation also times the rest of the metric in the same run and
+adds it to the line as "configs": decode at batch 32, prefill (8192 tokens,
+tp 8; TFLOP/s against the bf16 peak) and the TP x token sweep at 16, 128 and
+1024 tokens (tp 8), each with its own inputs, steps, per-kernel roofline,
+clock record and CPU baseline (--configs none skips them).
 
 Rank 0 prints one JSON line.  With N > 1 (torchrun) each GPU runs an
 independent replica on its own batch (data-parallel replicas: no collective on
@@ -36,6 +43,8 @@ import statistics
 import sys
 import threading
 import time
+
+import numpy as np
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
@@ -66,6 +75,10 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip timing the oracle on the host")
     ap.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph replay percentiles")
+    ap.add_argument("--configs", choices=["auto", "all", "none"], default="auto",
+                    help="also time decode_bs32, prefill (tp 8) and the sweep at T=16/128/1024 (tp 8) in the same "
+                         "run, each in the 'configs' block of the JSON line; auto: only for the default "
+                         "invocation (decode_bs1, nothing overridden), on one GPU")
     return ap.parse_args()
 
 
@@ -182,21 +195,22 @@ class ClockSampler:
                 "window": "timed region" if sel is not self.samples else "warm-up + timed region"}
 
 
-def _oracle_rate(p, A, Bs, act, budget_s, max_calls):
+def _oracle_rate(x, A, Bs, act, budget_s, max_calls):
     import oracle
     calls, t_total = 0, 0.0
     while calls < max_calls and t_total < budget_s:
         t0 = time.perf_counter()
-        oracle.tp_mlp_sharded(p.x, A, Bs, act)
+        oracle.tp_mlp_sharded(x, A, Bs, act)
         t_total += time.perf_counter() - t0
         calls += 1
-    return p.tokens * calls / t_total, calls, t_total
+    return x.shape[0] * calls / t_total, calls, t_total
 
 
-def oracle_baseline(p, A, Bs, act, budget_s=12.0, max_calls=50):
-    """Time the oracle as it stands on a bounded sample: whole calls until the budget is spent.
-    With more than one token the oracle's OpenMP loop can use several cores, so it is
-    also timed on one core; with one token both are the same run."""
+def oracle_baseline(p, A, Bs, act, budget_s=12.0, max_calls=50, sample_rows=None, one_core=True):
+    """Time the oracle as it stands on a bounded sample: whole calls until the budget is spent
+    (at least one).  With sample_rows, each call takes that many seeded-sampled token rows
+    instead of the whole batch.  With more than one token the oracle's OpenMP loop can use
+    several cores, so it is also timed on one core; with one token both are the same run."""
     import oracle
     T = p.tokens
     nproc = os.cpu_count()
@@ -204,19 +218,26 @@ def oracle_baseline(p, A, Bs, act, budget_s=12.0, max_calls=50):
         affinity = len(os.sched_getaffinity(0))
     except AttributeError:
         affinity = nproc
-    threads = min(oracle.max_threads(), T)
-    value, calls, t_total = _oracle_rate(p, A, Bs, act, budget_s, max_calls)
+    x = p.x
+    what = f"full forward(s) of this workload ({T} token(s) each)"
+    if sample_rows is not None and sample_rows < T:
+        rows = p.sample_rows(sample_rows)
+        x = np.ascontiguousarray(p.x[rows])
+        what = f"forward(s) of {len(rows)} seeded-sampled of the {T} token rows"
+    n = x.shape[0]
+    threads = min(oracle.max_threads(), n)
+    value, calls, t_total = _oracle_rate(x, A, Bs, act, budget_s, max_calls)
     out = {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
            "host_nproc": nproc, "host_affinity": affinity,
-           "sample": f"{calls} full forward(s) of this workload ({T} token(s) each) on the host, "
-                     f"{t_total:.1f} s; the oracle runs OpenMP over tokens"}
-    if threads > 1:
+           "sample": f"{calls} {what} on the host, {t_total:.1f} s; the oracle runs OpenMP over tokens"}
+    if threads > 1 and one_core:
         oracle.set_threads(1)
         try:
-            v1, c1, t1 = _oracle_rate(p, A, Bs, act, budget_s / 2, max_calls)
+            x1 = x[:max(1, n // threads)]
+            v1, c1, t1 = _oracle_rate(x1, A, Bs, act, budget_s / 2, max_calls)
         finally:
             oracle.set_threads(oracle.max_threads())
-        out["one_core"] = {"value": v1, "sample": f"{c1} full forward(s), {t1:.1f} s"}
+        out["one_core"] = {"value": v1, "sample": f"{c1} forward(s) of {x1.shape[0]} of those rows, {t1:.1f} s"}
     return out
 
 
@@ -578,6 +599,193 @@ def run_small_op_reference(args, op):
     return 0
 
 
+# Workloads the default run times beside the headline, each on its own seeded
+# inputs (name, tokens, tp): the rest of the metric -- decode at batch 32,
+# prefill (TFLOP/s against the bf16 peak) and the TP x token sweep's
+# memory-bound middle and compute-bound end.
+EXTRA_CONFIGS = (("decode_bs32", None, None), ("prefill", None, 8), ("sweep", 16, 8), ("sweep", 128, 8),
+                 ("sweep", 1024, 8))
+EXTRA_MIN_TIMED_S = 0.25     # timed window of each extra workload (room for clock samples)
+EXTRA_ORACLE_BUDGET_S = 4.0  # CPU-baseline budget of each extra workload (at least one call)
+PHASE_NAMES = ["first projection + activation", "second projection + rank sum"]
+
+
+def config_of(name, tokens=None, tp=None):
+    ns = argparse.Namespace(config=name, tokens=tokens, tp=tp, d_model=None, d_ff=None)
+    return resolve(ns)
+
+
+class MlpRun:
+    """One MLP workload on this GPU: seeded inputs, handle, weights packed once
+    (or kept as shards), and the timing passes."""
+
+    def __init__(self, c, plan="auto", splitk="auto", api="packed"):
+        import torch
+
+        from tensor_sharded_mlp_b200 import binding, inputs
+        self.torch, self.binding, self.c, self.api = torch, binding, c, api
+        T, d, f, tp, act, dt = c["tokens"], c["d_model"], c["d_ff"], c["tp"], c["act"], c["dtype"]
+        self.p = inputs.generate(T, d, f, act, dt, c["seed"], c["init"])
+        self.A, self.Bs = self.p.shards(tp)
+        tdt = torch.bfloat16 if dt == "bf16" else torch.float32
+
+        def up(a):
+            return torch.from_numpy(a).cuda().to(tdt).contiguous()
+
+        self.m = binding.TpMlp(d, f, tp, act, dt, max_tokens=T)
+        self.m.set_plan(plan)
+        self.m.set_splitk(splitk)
+        Ad, Bd = [up(a) for a in self.A], [up(b) for b in self.Bs]
+        # the one-off shard-layout pack, timed on its own (not part of a step)
+        torch.cuda.synchronize()
+        p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        p0.record()
+        self.packed = self.m.pack(Ad, Bd)
+        p1.record()
+        p1.synchronize()
+        self.pack_ms = p0.elapsed_time(p1)
+        self.x = up(self.p.x)
+        self.out = torch.empty(T, d, dtype=tdt, device="cuda")
+        if api == "packed":
+            del Ad, Bd
+            self.fwd = lambda: self.m.forward_packed(self.x, self.packed, out=self.out)   # noqa: E731
+        else:
+            self.fwd = lambda: self.m.forward(self.x, Ad, Bd, out=self.out)              # noqa: E731
+        torch.cuda.synchronize()
+
+    def warm(self, W):
+        for _ in range(W):
+            self.fwd()
+        self.torch.cuda.synchronize()
+        self.nk = self.m.last_launches
+        self.plan = self.m.last_plan
+
+    def estimate_ms(self, n=5):
+        torch = self.torch
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(n):
+            self.fwd()
+        b.record()
+        b.synchronize()
+        return a.elapsed_time(b) / n
+
+    def timed(self, K, barrier):
+        """K clean steps back to back (each may overlap the previous one's tail
+        through programmatic dependent launch), CUDA events on the launch stream,
+        NVML clocks sampled over the window.  Returns (ms, clock summary)."""
+        torch = self.torch
+        stream = torch.cuda.current_stream()
+        sampler = ClockSampler(torch.cuda.current_device())
+        sampler.start()
+        time.sleep(0.1)
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        t0 = time.perf_counter()
+        start.record(stream)
+        for _ in range(K):
+            self.fwd()
+        end.record(stream)
+        barrier()
+        sampler.mark(t0, time.perf_counter())
+        sampler.stop()
+        return start.elapsed_time(end), sampler.summary()
+
+    def phases(self, K, barrier):
+        """The same K steps again with the library recording events before, between
+        and after its kernels (kept apart from the timed pass: an event between two
+        kernels disables their programmatic overlap).  Mean ms per phase."""
+        torch = self.torch
+        stream = torch.cuda.current_stream()
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+        for row in ev:
+            for e in row:
+                e.record(stream)
+        for i in range(K):
+            self.binding.tp_mlp_set_profile_events(self.m.h, ev[i])
+            self.fwd()
+        self.binding.tp_mlp_set_profile_events(self.m.h, None)
+        barrier()
+        return [statistics.fmean(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(K)) for j in range(2)]
+
+    def roofline(self, kern_ms, peaks, src, workload_key):
+        """Roofline of the dominant kernel (largest share of the step): HBM bytes for
+        the memory-bound tilings, FLOPs against the bf16 peak for the wide ones."""
+        from tensor_sharded_mlp_b200 import counts
+        c = self.c
+        T, d, f, act, dt = c["tokens"], c["d_model"], c["d_ff"], c["act"], c["dtype"]
+        j = int(np.argmax(kern_ms))
+        extra = {}
+        if self.plan in ("tc_wide", "tc_wide256"):
+            bound, unit = "tensor", "TFLOP/s"
+            work = counts.gemm1_flops(T, d, f, act) if j == 0 else counts.gemm2_flops(T, f, d)
+            achieved = work / (kern_ms[j] / 1e3) / 1e12
+            peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+            peak_note = f"bf16_tflops, burst ({src})"
+            sus = peaks.get("bf16_tflops_sustained")
+            if sus:
+                extra = {"peak_sustained": sus, "frac_sustained": achieved / sus}
+        else:
+            bound, unit = "hbm", "GB/s"
+            work = counts.gemm1_bytes(T, d, f, act, dt) if j == 0 else counts.gemm2_bytes(T, f, d, dt)
+            achieved = work / (kern_ms[j] / 1e3) / 1e9
+            peak = peaks["hbm_gbs"]
+            peak_note = f"hbm_gbs ({src})"
+        kname = f"{self.plan}:{'first' if j == 0 else 'second'}"
+        split = " (GEMM + split-tile reduction kernel)" if self.nk > 2 and self.plan == "tc_skinny" else ""
+        r = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
+             "traffic": recorded_traffic(kname, workload_key), "kernel": PHASE_NAMES[j] + split,
+             "kernel_ms": kern_ms[j], "algorithmic_per_launch": work, "peak_source": peak_note,
+             "kernel_ms_all": kern_ms}
+        r.update(extra)
+        return r
+
+    def step_rates(self, ms):
+        from tensor_sharded_mlp_b200 import counts
+        c = self.c
+        T, d, f, act, dt = c["tokens"], c["d_model"], c["d_ff"], c["act"], c["dtype"]
+        step_bytes = counts.algorithmic_bytes(T, d, f, d, act, dt)
+        return {"step_hbm_gbs": step_bytes / (ms / 1e3) / 1e9,
+                "step_tflops": counts.forward_flops(T, d, f, d, act) / (ms / 1e3) / 1e12}, step_bytes
+
+
+def measure_extra(name, tokens, tp, args, peaks, src, barrier, cpu):
+    """One extra workload of the metric: its own inputs, warm-up, a timed window of
+    at least EXTRA_MIN_TIMED_S, per-phase kernel times, roofline, clocks, and a
+    bounded CPU baseline of the oracle."""
+    import torch
+
+    from tensor_sharded_mlp_b200 import counts
+    c = config_of(name, tokens, tp)
+    t_gen = time.perf_counter()
+    run = MlpRun(c)
+    t_gen = time.perf_counter() - t_gen
+    W = max(3, args.warmup)
+    run.warm(W)
+    est = run.estimate_ms()
+    K = max(args.steps, int(np.ceil(EXTRA_MIN_TIMED_S * 1e3 / max(est, 1e-3))))
+    ms_total, clocks = run.timed(K, barrier)
+    kern_ms = run.phases(min(K, 200), barrier)
+    ms = ms_total / K
+    rates, step_bytes = run.step_rates(ms)
+    key = name if tokens is None else f"{name}_T{tokens}"
+    e = {"workload": c["workload"], "tokens": c["tokens"], "tp": c["tp"], "plan": run.plan, "steps": K,
+         "warmup": W, "ms_per_step": ms, "value": c["tokens"] * K / (ms_total / 1e3), "unit": "tokens/s",
+         "roofline": run.roofline(kern_ms, peaks, src, key), "clocks": clocks, "gpu_launches": K * run.nk,
+         "timer": "CUDA events on the launch stream around the K steps",
+         "l2": "inputs larger than L2: every step re-reads %.2f GB of weights" % (
+             counts.weight_bytes(c["d_model"], c["d_ff"], c["d_model"], c["act"], c["dtype"]) / 1e9),
+         "pack_ms": run.pack_ms, "host_setup_s": t_gen}
+    e.update(rates)
+    if cpu:
+        sample = c.get("sample_rows", 256) if c["tokens"] > 256 else None
+        e["cpu_baseline"] = oracle_baseline(run.p, run.A, run.Bs, c["act"], budget_s=EXTRA_ORACLE_BUDGET_S,
+                                            max_calls=20, sample_rows=sample, one_core=False)
+    del run
+    torch.cuda.empty_cache()
+    return key, e
+
+
 def main():
     args = parse()
     op = small_op(args)
@@ -586,85 +794,27 @@ def main():
     if args.impl == "reference":
         return run_reference(args)
 
-    import numpy as np
     import torch
 
-    from tensor_sharded_mlp_b200 import binding, counts, inputs, replicas
+    from tensor_sharded_mlp_b200 import binding, counts, replicas
 
     rank, world, local = replicas.rank_env()
     torch.cuda.set_device(local)
     replicas.init("nccl", torch.device("cuda", local))
     c = resolve(args)
     T, d, f, tp, act, dt = c["tokens"], c["d_model"], c["d_ff"], c["tp"], c["act"], c["dtype"]
-    p = inputs.generate(T, d, f, act, dt, c["seed"], c["init"])
-    A, Bs = p.shards(tp)
-    tdt = torch.bfloat16 if dt == "bf16" else torch.float32
-
-    def up(a):
-        return torch.from_numpy(a).cuda().to(tdt).contiguous()
-
-    m = binding.TpMlp(d, f, tp, act, dt, max_tokens=T)
-    m.set_plan(args.plan)
-    m.set_splitk(args.splitk)
-    Ad, Bd = [up(a) for a in A], [up(b) for b in Bs]
-    # the one-off shard-layout pack, timed on its own (not part of a step)
-    torch.cuda.synchronize()
-    p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    p0.record()
-    packed = m.pack(Ad, Bd)
-    p1.record()
-    p1.synchronize()
-    pack_ms = p0.elapsed_time(p1)
-    if args.api == "packed":
-        del Ad, Bd
-        fwd = lambda: m.forward_packed(x, packed, out=out)            # noqa: E731
-    else:
-        fwd = lambda: m.forward(x, Ad, Bd, out=out)                   # noqa: E731
-    x = up(p.x)
-    out = torch.empty(T, d, dtype=tdt, device="cuda")
-    torch.cuda.synchronize()
+    run = MlpRun(c, args.plan, args.splitk, args.api)
+    m, packed, x, out, fwd = run.m, run.packed, run.x, run.out, run.fwd
 
     def barrier():
         replicas.barrier()
         torch.cuda.synchronize()
 
     K, W = args.steps, max(3, args.warmup)
-    for _ in range(W):
-        fwd()
-    nk = m.last_launches
-    plan = m.last_plan
-    # the library marks phases: before the first projection's kernels, between
-    # the projections and after the second's (a phase may be more than one kernel)
-    nph = 2
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nph + 1)] for _ in range(K)]
-    stream = torch.cuda.current_stream()
-    for row in ev:
-        for e in row:
-            e.record(stream)
-    sampler = ClockSampler(torch.cuda.current_device())
-    sampler.start()
-    time.sleep(0.1)
-    # Timed region: K clean steps (kernels back to back, so each may overlap the
-    # previous one's tail through programmatic dependent launch).
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier()
-    t0 = time.perf_counter()
-    start.record(stream)
-    for i in range(K):
-        fwd()
-    end.record(stream)
-    barrier()
-    t1 = time.perf_counter()
-    sampler.mark(t0, t1)
-    elapsed_ms = start.elapsed_time(end)
-    # Per-kernel durations: the same K steps again with the library recording
-    # events on the launch stream before, between and after its kernels.
-    for i in range(K):
-        binding.tp_mlp_set_profile_events(m.h, ev[i])
-        fwd()
-    binding.tp_mlp_set_profile_events(m.h, None)
-    barrier()
-    kern_ms = [statistics.fmean(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(K)) for j in range(nph)]
+    run.warm(W)
+    nk, plan = run.nk, run.plan
+    elapsed_ms, clocks = run.timed(K, barrier)
+    kern_ms = run.phases(K, barrier)
     elapsed_ms = replicas.max_over_ranks(elapsed_ms)
     graph_steps = None
     if not args.no_graph:
@@ -697,51 +847,50 @@ def main():
                "timer": "CUDA events on the step's stream around K steps, host waits included",
                "matches_device_result": e2e_ok}
         del step
-    sampler.stop()
 
     value = replicas.whole_job_rate(T, K, world, elapsed_ms)
     peaks, src = load_peaks()
-    # roofline of the dominant kernel (largest share of the step)
-    j = int(np.argmax(kern_ms))
-    names = ["first projection + activation", "second projection + rank sum"]
-    if plan in ("tc_wide", "tc_wide256"):
-        bound, unit = "tensor", "TFLOP/s"
-        work = counts.gemm1_flops(T, d, f, act) if j == 0 else counts.gemm2_flops(T, f, d)
-        achieved = work / (kern_ms[j] / 1e3) / 1e12
-        peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
-        peak_note = f"bf16_tflops_sustained ({src})"
-    else:
-        bound, unit = "hbm", "GB/s"
-        work = counts.gemm1_bytes(T, d, f, act, dt) if j == 0 else counts.gemm2_bytes(T, f, d, dt)
-        achieved = work / (kern_ms[j] / 1e3) / 1e9
-        peak = peaks["hbm_gbs"]
-        peak_note = f"hbm_gbs ({src})"
-    kname = f"{plan}:{'first' if j == 0 else 'second'}"
-    roofline = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
-                "traffic": recorded_traffic(kname, args.config), "kernel": names[j] + (" (GEMM + split-tile reduction kernel)" if nk > 2 and plan == "tc_skinny" else ""),
-                "kernel_ms": kern_ms[j], "algorithmic_per_launch": work, "peak_source": peak_note,
-                "kernel_ms_all": kern_ms}
-    step_bytes = counts.algorithmic_bytes(T, d, f, d, act, dt)
-    step_flops = counts.forward_flops(T, d, f, d, act)
     ms = elapsed_ms / K
+    rates, step_bytes = run.step_rates(ms)
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W,
             "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": dt, "data": "synthetic",
             "config": {"workload": c["workload"], "tokens": T, "d_model": d, "d_ff": f, "tp": tp, "act": act,
-                       "plan": plan, "splitk": args.splitk, "api": args.api, "parallelism": "replicas" if world > 1 else "single GPU",
+                       "plan": plan, "splitk": args.splitk, "api": args.api,
+                       "parallelism": "replicas" if world > 1 else "single GPU",
                        "l2": "inputs larger than L2: every step re-reads %.2f GB of weights" % (step_bytes / 1e9)},
-            "step_hbm_gbs": step_bytes / (ms / 1e3) / 1e9, "step_tflops": step_flops / (ms / 1e3) / 1e12,
-            "roofline": roofline, "gpu_launches": K * nk, "clocks": sampler.summary(), "e2e": e2e,
-            "graph_step": graph_steps,
-            "pack": {"ms": pack_ms, "note": "one-off shard-layout pack before timing (first call, includes "
-                                           "the packer's launch set-up); reads and writes every weight once",
-                     "GBs": 2 * counts.weight_bytes(d, f, d, act, dt) / (pack_ms / 1e3) / 1e9}}
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = oracle_baseline(p, A, Bs, act)
+            "roofline": run.roofline(kern_ms, peaks, src, args.config), "gpu_launches": K * nk,
+            "clocks": clocks, "e2e": e2e, "graph_step": graph_steps,
+            "pack": {"ms": run.pack_ms, "note": "one-off shard-layout pack before timing (first call, includes "
+                                               "the packer's launch set-up); reads and writes every weight once",
+                     "GBs": 2 * counts.weight_bytes(d, f, d, act, dt) / (run.pack_ms / 1e3) / 1e9}}
+    line.update(rates)
+    cpu = rank == 0 and world == 1 and not args.no_cpu_baseline
+    if cpu:
+        line["cpu_baseline"] = oracle_baseline(run.p, run.A, run.Bs, act)
+    del run, m, packed, x, out, fwd
+    torch.cuda.empty_cache()
+    # the rest of the metric, in the same run (one GPU only: each workload is
+    # generated on the host, and a replica per rank would multiply that)
+    if extra_configs_wanted(args) and world == 1:
+        line["configs"] = {}
+        for name, tk, tpx in EXTRA_CONFIGS:
+            key, e = measure_extra(name, tk, tpx, args, peaks, src, barrier, cpu)
+            line["configs"][key] = e
     if rank == 0:
         print(json.dumps(line), flush=True)
     replicas.finish()
     return 0
+
+
+def extra_configs_wanted(args):
+    if args.configs == "none":
+        return False
+    if args.configs == "all":
+        return True
+    # auto: the default invocation (the headline workload, nothing overridden)
+    return (args.config == "decode_bs1" and args.tokens is None and args.tp is None and args.plan == "auto"
+            and args.api == "packed" and args.splitk == "auto" and args.d_model is None and args.d_ff is None)
 
 
 if __name__ == "__main__":

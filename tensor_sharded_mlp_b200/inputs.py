@@ -26,6 +26,7 @@ Recipe (fixed, so every user of a config sees the same numbers):
 """
 from __future__ import annotations
 
+import concurrent.futures
 import dataclasses
 from typing import Optional
 
@@ -121,12 +122,16 @@ def generate_attn_merge(tp: int, rows: int, head_dim: int, dtype: str, seed: int
 
 
 def round_to_bf16(a: np.ndarray) -> np.ndarray:
-    """Round fp32 values to the nearest bf16 (ties to even); returns fp32 holding them."""
+    """Round fp32 values to the nearest bf16 (ties to even); returns fp32 holding them.
+
+    Works on the 32-bit patterns: adding 0x7FFF plus the lowest kept bit and
+    clearing the low 16 bits rounds to nearest, ties to even.  For every finite
+    input the sum stays below 2**32 (the largest finite pattern is 0xFF7FFFFF).
+    """
     a = np.ascontiguousarray(a, dtype=np.float32)
-    bits = a.view(np.uint32).astype(np.uint64)
-    lsb = (bits >> 16) & 1
-    rounded = ((bits + 0x7FFF + lsb) >> 16) << 16
-    out = (rounded & 0xFFFFFFFF).astype(np.uint32).view(np.float32)
+    bits = a.view(np.uint32)
+    lsb = (bits >> 16) & np.uint32(1)
+    out = ((bits + np.uint32(0x7FFF) + lsb) & np.uint32(0xFFFF0000)).view(np.float32)
     # NaN/Inf never occur for finite normal draws; keep them untouched anyway.
     special = ~np.isfinite(a)
     if special.any():
@@ -142,13 +147,25 @@ def _std(init, fan_in: int) -> float:
 
 
 def _draw(rng: np.random.Generator, rows: int, cols: int, std: float, dtype: str) -> np.ndarray:
+    # The draws stay in one sequential stream; scaling, the fp32 cast and the
+    # bf16 rounding of a chunk run on a worker thread while the next chunk is
+    # drawn (numpy releases the GIL in both), which leaves the values unchanged.
     out = np.empty((rows, cols), dtype=np.float32)
     step = max(1, _CHUNK_ELEMS // max(cols, 1))
-    for r0 in range(0, rows, step):
-        r1 = min(rows, r0 + step)
-        out[r0:r1] = (rng.standard_normal((r1 - r0, cols)) * std).astype(np.float32)
-    if dtype == "bf16":
-        out = round_to_bf16(out)
+
+    def finish(r0, r1, chunk):
+        v = (chunk * std).astype(np.float32)
+        out[r0:r1] = round_to_bf16(v) if dtype == "bf16" else v
+
+    with concurrent.futures.ThreadPoolExecutor(max_workers=2) as ex:
+        pending = []
+        for r0 in range(0, rows, step):
+            r1 = min(rows, r0 + step)
+            pending.append(ex.submit(finish, r0, r1, rng.standard_normal((r1 - r0, cols))))
+            if len(pending) > 2:
+                pending.pop(0).result()
+        for f in pending:
+            f.result()
     return out
 
 
