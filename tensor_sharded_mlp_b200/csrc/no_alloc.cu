@@ -14,6 +14,11 @@
 // the GPU therefore race and corrupt each other's results; callers must order
 // them (one stream, or events).  The split-K counters that must start at zero
 // are cleared by each call, on its stream, before its kernels run.
+//
+// Layout of the array: [status word, 256 bytes | split-tile counters | H |
+// split-K partial sums].  The status word sits at a fixed place that no call
+// clears; a kernel that gives up a bounded wait sets it, and
+// tp_mlp_decode_static_status reads and clears it.
 #include <cuda.h>
 
 #include <mutex>
@@ -25,6 +30,7 @@ namespace tpmlp {
 namespace {
 
 constexpr size_t kStaticScratchBytes = 8u << 20;   // 8 MiB
+constexpr size_t kStatusBytes = 256;                // the status word's slot at the front
 
 // The scratch itself.  Host code may not use this name as an address (on the
 // host it is only a stand-in); it asks the runtime for the device address.
@@ -50,29 +56,6 @@ bool device_setup(int dev, void **ptr, int *sms) {
     *ptr = g_scratch_ptr[dev];
     *sms = g_num_sms[dev];
     return true;
-}
-
-typedef CUresult (*PFN_range)(CUdeviceptr *, size_t *, CUdeviceptr);
-
-// A device pointer inside one allocation that holds `bytes` from it (a wrong
-// pointer becomes an error code rather than an out-of-bounds access).
-int check_range(const void *p, size_t bytes) {
-    static PFN_range fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void *q = nullptr;
-        cudaDriverEntryPointQueryResult r;
-        if (cudaGetDriverEntryPointByVersion("cuMemGetAddressRange", &q, 12000, cudaEnableDefault, &r) ==
-                cudaSuccess &&
-            r == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_range>(q);
-    });
-    if (!fn) return TP_MLP_ERR_CUDA;
-    CUdeviceptr base = 0;
-    size_t size = 0;
-    if (fn(&base, &size, reinterpret_cast<CUdeviceptr>(p)) != CUDA_SUCCESS) return TP_MLP_ERR_INVALID_ARG;
-    if (reinterpret_cast<uintptr_t>(p) + bytes > base + size) return TP_MLP_ERR_SHAPE;
-    return TP_MLP_OK;
 }
 
 }  // namespace
@@ -108,29 +91,47 @@ extern "C" int tp_mlp_decode_forward_static(int d_model, int d_ff, int d_out, in
     int sms = 0;
     if (!device_setup(dev, &scratch, &sms)) return TP_MLP_ERR_CUDA;
 
-    // scratch layout: [split-tile counters | status word | H (tokens x d_ff bf16) | partial sums]
+    // scratch layout: [status word | split-tile counters | H (tokens x d_ff bf16) | partial sums]
     const size_t n_cnt = tile_counter_slots(p);
-    const size_t cnt_bytes = align256((n_cnt + 1) * sizeof(unsigned));
+    const size_t cnt_bytes = align256(n_cnt * sizeof(unsigned));
     const size_t h_bytes = align256((size_t)tokens * d_ff * 2);
     const size_t part_bytes = gemv_workspace_bytes(p, sms);
-    if (cnt_bytes + h_bytes + part_bytes > kStaticScratchBytes) return TP_MLP_ERR_WORKSPACE;
+    if (kStatusBytes + cnt_bytes + h_bytes + part_bytes > kStaticScratchBytes) return TP_MLP_ERR_WORKSPACE;
     int s;
-    if ((s = check_range(x, (size_t)tokens * d_model * 2))) return s;
-    if ((s = check_range(out, (size_t)tokens * d_out * 2))) return s;
-    if ((s = check_range(packed, packed_total_bytes(p)))) return s;
+    if ((s = check_dev(x, (size_t)tokens * d_model * 2))) return s;
+    if ((s = check_dev(out, (size_t)tokens * d_out * 2))) return s;
+    if ((s = check_dev(packed, packed_total_bytes(p)))) return s;
 
     char *base = static_cast<char *>(scratch);
-    unsigned *counters = reinterpret_cast<unsigned *>(base);
-    void *h = base + cnt_bytes;
-    float *part = reinterpret_cast<float *>(base + cnt_bytes + h_bytes);
+    int *status = reinterpret_cast<int *>(base);
+    unsigned *counters = reinterpret_cast<unsigned *>(base + kStatusBytes);
+    void *h = base + kStatusBytes + cnt_bytes;
+    float *part = reinterpret_cast<float *>(base + kStatusBytes + cnt_bytes + h_bytes);
     const void *w2p = static_cast<const char *>(packed) + packed_part2_offset(p);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    if (cudaMemsetAsync(counters, 0, cnt_bytes, st) != cudaSuccess) return TP_MLP_ERR_CUDA;
+    if (cudaMemsetAsync(counters, 0, n_cnt * sizeof(unsigned), st) != cudaSuccess) return TP_MLP_ERR_CUDA;
     Marks none;
     none.n = 0;
     int launches = 0;
-    int *status = reinterpret_cast<int *>(counters + n_cnt);
     if (launch_gemv(p, x, packed, w2p, h, out, part, counters, status, sms, st, none, &launches) != cudaSuccess)
         return TP_MLP_ERR_CUDA;
     return TP_MLP_OK;
+}
+
+extern "C" int tp_mlp_decode_static_status(void) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return TP_MLP_ERR_CUDA;
+    void *scratch = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(g_mutex);
+        scratch = g_scratch_ptr[dev];
+    }
+    if (!scratch) return TP_MLP_OK;   // no call has run on this device
+    if (cudaDeviceSynchronize() != cudaSuccess) return TP_MLP_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpy(&v, scratch, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return TP_MLP_ERR_CUDA;
+    if (v == 0) return TP_MLP_OK;
+    const int zero = 0;
+    if (cudaMemcpy(scratch, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return TP_MLP_ERR_CUDA;
+    return TP_MLP_ERR_TIMEOUT;
 }
