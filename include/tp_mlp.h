@@ -68,7 +68,7 @@ typedef enum {
     TP_MLP_ERR_ALIGNMENT = 3,    /* a pointer is not 16-byte aligned                   */
     TP_MLP_ERR_UNSUPPORTED = 4,  /* valid request the library cannot serve            */
     TP_MLP_ERR_CUDA = 5,         /* a CUDA runtime call failed (launch or earlier work) */
-    TP_MLP_ERR_TIMEOUT = 6,      /* reserved: a bounded device-side wait ran out       */
+    TP_MLP_ERR_TIMEOUT = 6,      /* a bounded device-side wait ran out (status calls)  */
     TP_MLP_ERR_WORKSPACE = 7     /* no workspace set, or smaller than required         */
 } tp_mlp_status;
 
@@ -88,7 +88,9 @@ typedef enum {
 } tp_mlp_plan;
 
 /*
- * Create a handle for one MLP shape.
+ * Create a handle for one MLP shape: the shapes of the pages' call
+ * tensor_parallel_output(x, a_shards, b_shards, activation) ("LLM 推理并行化"
+ * §三 2)), fixed once.
  *   d_model    input width (columns of x, rows of every A_i), >= 1
  *   d_ff       intermediate width summed over ranks; d_ff % tp_degree == 0
  *   d_out      output width (columns of every B_i); pass d_model for the usual
@@ -102,21 +104,26 @@ typedef enum {
 int tp_mlp_create(tp_mlp_t *handle, int d_model, int d_ff, int d_out, int tp_degree,
                   int act, int dtype, int max_tokens);
 
-/* Free the handle (host memory).  NULL is accepted. */
+/* Free the handle (host memory).  NULL is accepted.  The pages' function holds
+ * no state; the handle only caches the shape of one tensor_parallel_output. */
 int tp_mlp_destroy(tp_mlp_t handle);
 
 /*
  * Device workspace (bytes) the forward / partials / packed calls need for
  * `tokens` tokens (0 <= tokens <= max_tokens).  It holds the intermediate
- * activation H (tokens x d_ff, dtype) and split-K scratch.  Returns 0 for an
- * invalid handle or token count.
+ * activation H (tokens x d_ff, dtype) -- the per-rank hidden_i = act(x @ A_i)
+ * of "LLM 推理并行化" §三 2), stored for all ranks side by side -- and split-K
+ * scratch.  The first tp_mlp_workspace_bytes(handle, 0) bytes are the split-
+ * tile counters and the device status word.  Returns 0 for an invalid handle
+ * or token count.
  */
 size_t tp_mlp_workspace_bytes(tp_mlp_t handle, int tokens);
 
 /*
  * Give the handle a device workspace of `bytes` bytes (owned by the caller,
- * kept until replaced or the handle is destroyed).  Zeroes the split-K
- * counters inside it synchronously (cudaMemset).  bytes must be at least
+ * kept until replaced or the handle is destroyed; the pages leave memory to
+ * the caller, who here is PyTorch).  Zeroes the split-K counters inside it and
+ * waits for that to finish.  bytes must be at least
  * tp_mlp_workspace_bytes(handle, max_tokens) -- or pass the size for the
  * largest token count you will use: each call checks its own need.
  */
@@ -146,10 +153,14 @@ int tp_mlp_forward(tp_mlp_t handle, const void *x, int tokens, const void *const
                    tp_mlp_stream_t stream);
 
 /*
- * Per-rank partials without the final sum: partials[i] = act(x @ A_i) @ B_i,
- * fp32, laid out tp_degree x tokens x d_out (device).  Other arguments as
- * tp_mlp_forward.  Summing them over i gives the forward's result (before
- * rounding to the output dtype).
+ * Per-rank partials without the final sum ("大模型推理系统揭秘（07）" §1.2.2,
+ * row-parallel linear: each rank's Z_i = Y_i W_2i, still to be all-reduced;
+ * "LLM 推理并行化" §三 2): partial_i = hidden_i @ B_i):
+ *   partials[i] = act(x @ A_i) @ B_i, fp32, laid out tp_degree x tokens x d_out
+ * (device).  Other arguments as tp_mlp_forward.  Summing them over i gives the
+ * forward's result (before rounding to the output dtype).  For bf16 with f_s
+ * a multiple of 64 the tcgen05 kernels run, with each rank's K loop kept
+ * apart; otherwise CUDA-core kernels.
  */
 int tp_mlp_partials(tp_mlp_t handle, const void *x, int tokens, const void *const *A_shards,
                     const void *const *B_shards, int tp_degree, int act, float *partials,
@@ -157,6 +168,9 @@ int tp_mlp_partials(tp_mlp_t handle, const void *x, int tokens, const void *cons
 
 /*
  * Size in bytes of the packed weight buffer (the shard-layout packer's output).
+ * The packer holds the column shards A_i and row shards B_i of
+ * "大模型推理系统揭秘（07）" §1.2.2-§1.2.3 (A split along columns, B along
+ * rows, each rank taking f_s = d_ff / tp of them, "LLM 推理并行化" §三 2)).
  * The buffer has two parts, each a matrix of R "rows" by K, one row per output
  * of its projection (element = the handle's dtype):
  *   part 1, first projection, K = d_model: tanh / identity: row n holds column
@@ -175,17 +189,23 @@ int tp_mlp_partials(tp_mlp_t handle, const void *x, int tokens, const void *cons
 size_t tp_mlp_packed_bytes(tp_mlp_t handle);
 
 /* Pack the shards (same arrays as tp_mlp_forward) into `packed` (device,
- * tp_mlp_packed_bytes bytes).  A bit-exact copy in a new order.  The handle's
- * tp_degree fixes how many pointers each array holds. */
+ * tp_mlp_packed_bytes bytes).  A bit-exact copy in a new order: concatenating
+ * the column shards gives A and stacking the row shards gives B
+ * ("大模型推理系统揭秘（07）" §1.2.3), and that is the order stored.  The
+ * handle's tp_degree fixes how many pointers each array holds. */
 int tp_mlp_pack(tp_mlp_t handle, const void *const *A_shards, const void *const *B_shards,
                 void *packed, tp_mlp_stream_t stream);
 
-/* Inverse of tp_mlp_pack: write the shards back from `packed` (bit-exact). */
+/* Inverse of tp_mlp_pack: cut A and B back into the per-rank shards of
+ * "大模型推理系统揭秘（07）" §1.2.2 and write them from `packed` (bit-exact). */
 int tp_mlp_unpack(tp_mlp_t handle, const void *packed, void *const *A_shards,
                   void *const *B_shards, tp_mlp_stream_t stream);
 
 /*
- * Forward pass on packed weights (the fast path; weights are packed once).
+ * Forward pass on packed weights (the fast path; weights are packed once):
+ * the same out = sum_i act(x @ A_i) @ B_i as tp_mlp_forward ("LLM 推理并行化"
+ * §三 2); "大模型推理系统揭秘（07）" §1.2.3), with the sum over ranks done
+ * inside the second projection's accumulation.
  *   x device tokens x d_model, out device tokens x d_out, packed from
  *   tp_mlp_pack.  Same result as tp_mlp_forward up to fp32 summation order.
  */
@@ -193,7 +213,8 @@ int tp_mlp_forward_packed(tp_mlp_t handle, const void *x, int tokens, const void
                           void *out, tp_mlp_stream_t stream);
 
 /* Force a kernel family (tp_mlp_plan) for later forwards; AUTO restores the
- * library's choice.  A forced plan that cannot serve a call returns
+ * library's choice (decode is weight-read-bound, prefill compute-bound,
+ * "7.4 推理侧并行" §7.4.1, so the choice follows the token count).  A forced plan that cannot serve a call returns
  * TP_MLP_ERR_UNSUPPORTED from that call. */
 int tp_mlp_set_plan(tp_mlp_t handle, int plan);
 
@@ -203,18 +224,22 @@ int tp_mlp_set_plan(tp_mlp_t handle, int plan);
  * the same fixed order, so they give identical results; they differ in speed.
  */
 typedef enum {
-    TP_MLP_SPLITK_AUTO = 0,      /* by the size of the partials (default)            */
+    TP_MLP_SPLITK_AUTO = 0,      /* default: where a whole number (2..8) of CTAs share
+                                    each tile and all fit at once, those CTAs form a
+                                    thread-block cluster and add their slots through
+                                    distributed shared memory; otherwise as SEPARATE */
     TP_MLP_SPLITK_IN_KERNEL = 1, /* the last CTA to finish its share adds the slots   */
     TP_MLP_SPLITK_SEPARATE = 2   /* a reduction kernel behind each GEMM adds them,
                                     spread over the whole GPU                        */
 } tp_mlp_splitk;
 
 /* Choose the split-tile finish (tp_mlp_splitk) for later forwards.  Returns
- * TP_MLP_ERR_INVALID_ARG for another value.  Other plans ignore it. */
+ * TP_MLP_ERR_INVALID_ARG for another value.  Other plans ignore it.  (No
+ * counterpart in the pages: how one GPU adds the pieces of one tile.) */
 int tp_mlp_set_splitk(tp_mlp_t handle, int mode);
 
 /*
- * Timing hook: with n > 0, later forward / forward_packed / partials calls
+ * Timing hook (measurement only; no counterpart in the pages): with n > 0, later forward / forward_packed / partials calls
  * record events[0] on their stream before their first kernel, events[1] after
  * the first projection's kernels and events[2] after the second projection's
  * (events beyond events[2] are not recorded).  The events are caller-owned cudaEvent_t handles (created with
@@ -224,10 +249,13 @@ int tp_mlp_set_splitk(tp_mlp_t handle, int mode);
 int tp_mlp_set_profile_events(tp_mlp_t handle, void *const *events, int n);
 
 /*
- * Device-side status of the work issued so far on this handle's workspace:
+ * Device-side status of the work issued so far on this handle's workspace
+ * (the pages describe no failure detection; this is the library's own):
  * synchronises the device, returns TP_MLP_ERR_TIMEOUT if a kernel gave up a
- * bounded internal wait (its results are then invalid) and clears the flag,
- * TP_MLP_OK otherwise.  Needs a workspace.
+ * bounded internal wait (its results are then invalid), TP_MLP_OK otherwise.
+ * On a timeout it also zeroes the split-tile counters, which the CTAs that
+ * left early may have left part-way, and the flag: calls made after a timeout
+ * and before this call may give wrong results.  Needs a workspace.
  */
 int tp_mlp_get_device_status(tp_mlp_t handle);
 
@@ -243,7 +271,9 @@ int tp_mlp_get_device_status(tp_mlp_t handle);
 int tp_mlp_selftest_bounded_wait(tp_mlp_t handle, unsigned wait_us, tp_mlp_stream_t stream);
 
 /* Plan (tp_mlp_plan) and number of kernel launches of the last successful
- * forward / partials call on this handle; -1 before the first. */
+ * forward / partials call on this handle; -1 before the first.  (Measurement
+ * hooks; the pages put each launch at 5-10 us of a decode step, "7.4 推理侧并行"
+ * §7.4.2.) */
 int tp_mlp_last_plan(tp_mlp_t handle);
 int tp_mlp_last_launches(tp_mlp_t handle);
 
@@ -268,7 +298,9 @@ int tp_mlp_last_launches(tp_mlp_t handle);
  * that first call before capturing a stream.  Every call shares the array and
  * leaves its contents behind; each call clears, on its stream, the parts that
  * must start at zero.  Calls whose kernels overlap on the GPU race on the
- * array: order them on one stream or with events.
+ * array: order them on one stream or with events.  A kernel that gives up a
+ * bounded internal wait records it in the array's status word, which no call
+ * clears; tp_mlp_decode_static_status reports it.
  * Errors: TP_MLP_ERR_WORKSPACE if this shape needs more scratch than the
  * 8 MiB array holds (nothing is launched); TP_MLP_ERR_UNSUPPORTED for shapes
  * the GEMV kernels do not take (d_model or d_ff not a multiple of 8);
@@ -277,6 +309,16 @@ int tp_mlp_last_launches(tp_mlp_t handle);
 int tp_mlp_decode_forward_static(int d_model, int d_ff, int d_out, int tp_degree, int act,
                                  const void *x, int tokens, const void *packed, void *out,
                                  tp_mlp_stream_t stream);
+
+/*
+ * Status of the tp_mlp_decode_forward_static calls issued so far on the
+ * current device (no counterpart in the pages): synchronises the device and
+ * returns TP_MLP_ERR_TIMEOUT if one of their kernels gave up a bounded
+ * internal wait -- the results of that call are invalid -- and clears the
+ * record; TP_MLP_OK otherwise (also when no call has run on this device).
+ * Allocates nothing.
+ */
+int tp_mlp_decode_static_status(void);
 
 /*
  * The all-reduce of the ranks' partial outputs fused with the residual add and
@@ -336,7 +378,91 @@ int tp_mlp_merge_attention_partials(int tp_degree, int rows, int head_dim, const
                                     const float *exp_sum, const void *weighted, int dtype, void *out,
                                     tp_mlp_stream_t stream);
 
-/* Human-readable name of a status code (static string). */
+/*
+ * Tensor parallelism across GPUs: rank i holds only A_i and B_i, and the sum of
+ * the partials is an all-reduce between GPUs ("大模型推理系统揭秘（07）" §1.2.3:
+ * Z = sum_i Y_i W_2i takes one all-reduce per MLP).  Here that all-reduce is
+ * the one-shot kind of "7.4 推理侧并行" §7.4.2, optimisation 2 -- every rank
+ * sends its whole partial to every other rank, and every rank adds them up
+ * itself -- and it is fused into the second projection: as soon as the CTAs
+ * of an output tile have added their split-K pieces (a thread-block cluster,
+ * through distributed shared memory), they store the tile's bf16 partial
+ * straight into every rank's exchange buffer (plain stores; over NVLink for a
+ * peer), publish it with a flag, wait for the same tile from every rank and
+ * add the ranks in rank order.  No library collective runs.
+ *
+ * Size of one rank's exchange buffer, for the handle's tp_degree, max_tokens
+ * and d_out.  Each rank allocates one on its own GPU, zeroes it once before
+ * the first call, and makes it reachable from every other rank (for example
+ * with tp_mlp_ipc_get_handle / tp_mlp_ipc_open_handle).
+ */
+size_t tp_mlp_xgpu_comm_bytes(tp_mlp_t handle);
+
+/*
+ * One forward of ranks rank0 .. rank0 + nranks - 1 of the handle's tp_degree:
+ *   outs[i] = sum_{r < tp_degree} act(x @ A_r) @ B_r        (for every local i)
+ *   handle     the whole MLP (d_model, d_ff, d_out, tp_degree, act; bf16),
+ *              with a workspace; f_s = d_ff / tp_degree must be a multiple of 64
+ *   rank0, nranks  the ranks this call runs: one per process and GPU
+ *              (nranks = 1), or every rank at once on one GPU (rank0 = 0,
+ *              nranks = tp_degree; a single launch then runs all ranks, which
+ *              is how one GPU checks the exchange)
+ *   x          device, tokens x d_model (the same on every rank)
+ *   A_local, B_local  host arrays of nranks device pointers: the local ranks'
+ *              shards, laid out as for tp_mlp_forward
+ *   comm       host array of tp_degree pointers: comm[r] is rank r's exchange
+ *              buffer as this process sees it (its own, or a peer's mapping)
+ *   outs       host array of nranks device pointers, tokens x d_out each
+ * Every rank must make the same calls with the same token counts, in the same
+ * order, on one stream each.  The call count is kept in the exchange buffers
+ * (zeroed once before the first call), so the calls may be captured in a CUDA
+ * graph and replayed -- the pages ask this of a custom all-reduce ("7.4 推理侧
+ * 并行" §7.4.2).  1 <= tokens <= min(max_tokens, 128) (TP_MLP_ERR_SHAPE);
+ * tokens == 0 launches nothing.  TP_MLP_ERR_UNSUPPORTED if
+ * the GPU cannot hold every CTA of the exchange at once.  A rank that waits
+ * too long for another gives up (bounded wait), and tp_mlp_get_device_status
+ * then reports TP_MLP_ERR_TIMEOUT.
+ */
+int tp_mlp_xgpu_forward(tp_mlp_t handle, int rank0, int nranks, const void *x, int tokens,
+                        const void *const *A_local, const void *const *B_local, void *const *comm,
+                        void *const *outs, tp_mlp_stream_t stream);
+
+/*
+ * The sequence-parallel form of the same step ("7.4 推理侧并行" §7.4.2,
+ * optimisation 3): outside the MLP the activations are split by token rows,
+ * so the all-reduce becomes an all-gather before the first projection and a
+ * reduce-scatter after the second, and each is overlapped with its GEMM.
+ *   x_local  host array of nranks device pointers: local rank i's own token
+ *            rows, tokens / tp_degree of them (rank r owns rows
+ *            [r * tokens / tp_degree, (r + 1) * tokens / tp_degree))
+ *   tokens   the total number of token rows, a multiple of tp_degree
+ *   outs     host array of nranks device pointers: local rank i's rows of the
+ *            output, tokens / tp_degree x d_out each
+ * A small kernel first stores each rank's rows into every rank's exchange
+ * buffer and counts itself in there; the first projection streams its
+ * weights at once and reads X only when every rank's rows have arrived.  The
+ * second projection's exchange sends each output row only to the rank that
+ * owns it, which adds the ranks' rows (in rank order) and writes its own.
+ * Other arguments, requirements and errors as tp_mlp_xgpu_forward; the two
+ * calls may be mixed on the same exchange buffers.
+ */
+int tp_mlp_xgpu_sp_forward(tp_mlp_t handle, int rank0, int nranks, const void *const *x_local, int tokens,
+                           const void *const *A_local, const void *const *B_local, void *const *comm,
+                           void *const *outs, tp_mlp_stream_t stream);
+
+/*
+ * CUDA IPC helpers for the exchange buffers (no counterpart in the pages).
+ * get_handle: a 64-byte handle for the device allocation holding dev_ptr, and
+ * dev_ptr's offset inside it.  open_handle (in another process): map that
+ * allocation and return the same address there.  close_handle: unmap it.
+ * TP_MLP_ERR_CUDA if the runtime refuses (for example memory not from
+ * cudaMalloc, or a handle opened in the process that made it).
+ */
+int tp_mlp_ipc_get_handle(const void *dev_ptr, void *handle, size_t *offset);
+int tp_mlp_ipc_open_handle(const void *handle, size_t offset, void **dev_ptr);
+int tp_mlp_ipc_close_handle(void *dev_ptr, size_t offset);
+
+/* Human-readable name of a status code (static string; no counterpart in the pages). */
 const char *tp_mlp_status_string(int status);
 
 #ifdef __cplusplus

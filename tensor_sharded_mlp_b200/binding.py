@@ -58,6 +58,13 @@ _SIGS = {
     "tp_mlp_last_launches": (_i, [_vp]),
     "tp_mlp_status_string": (ctypes.c_char_p, [_i]),
     "tp_mlp_decode_forward_static": (_i, [_i, _i, _i, _i, _i, _vp, _i, _vp, _vp, _vp]),
+    "tp_mlp_decode_static_status": (_i, []),
+    "tp_mlp_xgpu_comm_bytes": (_sz, [_vp]),
+    "tp_mlp_xgpu_forward": (_i, [_vp, _i, _i, _vp, _i, _vpp, _vpp, _vpp, _vpp, _vp]),
+    "tp_mlp_xgpu_sp_forward": (_i, [_vp, _i, _i, _vpp, _i, _vpp, _vpp, _vpp, _vpp, _vp]),
+    "tp_mlp_ipc_get_handle": (_i, [_vp, _vp, ctypes.POINTER(_sz)]),
+    "tp_mlp_ipc_open_handle": (_i, [_vp, _sz, ctypes.POINTER(_vp)]),
+    "tp_mlp_ipc_close_handle": (_i, [_vp, _sz]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -208,10 +215,98 @@ def tp_mlp_decode_forward_static(d_model: int, d_ff: int, d_out: int, tp_degree:
                                  x: torch.Tensor, packed: torch.Tensor, out: torch.Tensor,
                                  stream=None) -> None:
     """Decode forward for callers that cannot allocate device memory: its
-    scratch is a fixed array inside the library, so no workspace is passed."""
+    scratch is a fixed array inside the library, so no workspace is passed.
+    x (T, d_model) and out (T, d_out): contiguous CUDA bfloat16; packed: the
+    contiguous CUDA buffer tp_mlp_pack wrote for this shape."""
+    for t, what in ((x, "x"), (out, "out")):
+        if t.dtype != torch.bfloat16 or t.dim() != 2 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{what} must be a contiguous 2-D CUDA bfloat16 tensor")
+    if x.shape[1] != d_model or out.shape != (x.shape[0], d_out):
+        raise ValueError(f"x must be (T, {d_model}) and out (T, {d_out}); got {tuple(x.shape)}, {tuple(out.shape)}")
+    if not packed.is_cuda or not packed.is_contiguous():
+        raise ValueError("packed must be a contiguous CUDA tensor")
     _check("tp_mlp_decode_forward_static",
            _lib.tp_mlp_decode_forward_static(d_model, d_ff, d_out, tp_degree, ACT[act], _ptr(x), x.shape[0],
                                              _ptr(packed), _ptr(out), _stream(stream)))
+
+
+def tp_mlp_decode_static_status() -> None:
+    """Raise TpMlpError(ERR_TIMEOUT) if a kernel of an earlier
+    tp_mlp_decode_forward_static call on the current device gave up a bounded
+    wait (and clear that record); synchronises the device."""
+    _check("tp_mlp_decode_static_status", _lib.tp_mlp_decode_static_status())
+
+
+def tp_mlp_xgpu_comm_bytes(h) -> int:
+    return int(_lib.tp_mlp_xgpu_comm_bytes(h))
+
+
+def _raw_ptr_array(ptrs: Sequence[int]):
+    arr = (ctypes.c_void_p * max(1, len(ptrs)))(*[int(p) for p in ptrs])
+    return ctypes.cast(arr, _vpp), arr
+
+
+def tp_mlp_xgpu_forward(h, rank0: int, x: torch.Tensor, A_local, B_local, comm_ptrs: Sequence[int],
+                        outs, stream=None) -> None:
+    """Ranks rank0 .. rank0 + len(A_local) - 1 of a tensor-parallel MLP whose
+    all-reduce crosses GPUs (one-shot, fused into the second projection).
+    comm_ptrs: every rank's exchange buffer address as seen by this process."""
+    n = len(A_local)
+    if len(B_local) != n or len(outs) != n:
+        raise ValueError("A_local, B_local and outs need one entry per local rank")
+    for t in list(A_local) + list(B_local) + list(outs) + [x]:
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError("x, shards and outputs must be contiguous CUDA bfloat16 tensors")
+    a, _ka = _ptr_array(A_local, n)
+    b, _kb = _ptr_array(B_local, n)
+    o, _ko = _ptr_array(outs, n)
+    c, _kc = _raw_ptr_array(comm_ptrs)
+    _check("tp_mlp_xgpu_forward", _lib.tp_mlp_xgpu_forward(h, rank0, n, _ptr(x), x.shape[0], a, b, c, o,
+                                                           _stream(stream)))
+
+
+def tp_mlp_xgpu_sp_forward(h, rank0: int, x_local, A_local, B_local, comm_ptrs: Sequence[int], outs,
+                           stream=None) -> None:
+    """Sequence-parallel form: x_local[i] holds local rank i's tokens / tp rows;
+    the rows are gathered before the first projection and the second
+    projection's exchange is a reduce-scatter (outs[i]: rank i's own rows)."""
+    n = len(A_local)
+    if len(B_local) != n or len(outs) != n or len(x_local) != n:
+        raise ValueError("x_local, A_local, B_local and outs need one entry per local rank")
+    for t in list(x_local) + list(A_local) + list(B_local) + list(outs):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError("rows, shards and outputs must be contiguous CUDA bfloat16 tensors")
+    tp = len(comm_ptrs)
+    tokens = x_local[0].shape[0] * tp
+    xs, _kx = _ptr_array(x_local, n)
+    a, _ka = _ptr_array(A_local, n)
+    b, _kb = _ptr_array(B_local, n)
+    o, _ko = _ptr_array(outs, n)
+    c, _kc = _raw_ptr_array(comm_ptrs)
+    _check("tp_mlp_xgpu_sp_forward", _lib.tp_mlp_xgpu_sp_forward(h, rank0, n, xs, tokens, a, b, c, o,
+                                                                 _stream(stream)))
+
+
+def tp_mlp_ipc_get_handle(t: torch.Tensor):
+    """(64-byte handle, offset) of the device allocation holding tensor t."""
+    buf = ctypes.create_string_buffer(64)
+    off = ctypes.c_size_t()
+    _check("tp_mlp_ipc_get_handle", _lib.tp_mlp_ipc_get_handle(_ptr(t), buf, ctypes.byref(off)))
+    return bytes(buf.raw), int(off.value)
+
+
+def tp_mlp_ipc_open_handle(handle: bytes, offset: int) -> int:
+    """Map another process's allocation; returns the device address of handle + offset."""
+    if len(handle) != 64:
+        raise ValueError("an IPC handle is 64 bytes")
+    buf = ctypes.create_string_buffer(handle, 64)
+    p = ctypes.c_void_p()
+    _check("tp_mlp_ipc_open_handle", _lib.tp_mlp_ipc_open_handle(buf, offset, ctypes.byref(p)))
+    return int(p.value)
+
+
+def tp_mlp_ipc_close_handle(ptr: int, offset: int) -> None:
+    _check("tp_mlp_ipc_close_handle", _lib.tp_mlp_ipc_close_handle(ctypes.c_void_p(ptr), offset))
 
 
 def tp_mlp_allreduce_residual_rmsnorm(partials: torch.Tensor, residual: torch.Tensor, gamma: torch.Tensor,

@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stddef.h>
 
+#include "common.cuh"
+
 namespace tpmlp {
 
 struct Problem;
@@ -17,6 +19,10 @@ struct Marks {
         if (i < n && ev[i]) cudaEventRecord(ev[i], s);
     }
 };
+
+// tp_mlp.cu: a device pointer, 16-byte aligned, inside one device allocation
+// that holds `bytes` from it (a tp_mlp_status code; TP_MLP_OK when it does).
+int check_dev(const void *p, size_t bytes);
 
 // simt.cu: tiled CUDA-core path, any shape, both dtypes, shard or packed layout.
 // h: T x d_ff scratch (dtype).  partials != nullptr selects the per-rank output.
@@ -48,7 +54,8 @@ cudaError_t launch_attn_merge(int P, int rows, int D, const float *maximum, cons
                               const void *weighted, int dtype, void *out, cudaStream_t st);
 
 // Split-tile counters the GEMV and tcgen05 skinny kernels need (one per
-// weight tile of both parts; first part's tiles first).
+// weight tile of both parts; first part's tiles first; then the GEMV's two
+// chunk counters).
 size_t tile_counter_slots(const Problem &p);
 
 // gemv.cu: decode path, packed bf16, 1..kGemvMaxTokens tokens.
@@ -70,10 +77,39 @@ size_t tc_workspace_bytes(const Problem &p, int num_sms);
 // last CTA to arrive, inside the GEMM kernel, or by a reduction kernel behind it.
 enum { kSplitAuto = 0, kSplitInKernel = 1, kSplitSeparate = 2 };
 // Packed weights (w1p/w2p), or the per-rank shards when rawA/rawB are given.
-// *launches receives the number of kernels launched.
+// *launches receives the number of kernels launched.  partials != nullptr
+// (shard form only): the second projection writes each rank's fp32 partial
+// output to partials[rank][token][column] instead of the sum to out.
 cudaError_t launch_tc(const Problem &p, int tiling, const void *x, const void *w1p, const void *w2p,
                       const ShardPtrs *rawA, const ShardPtrs *rawB, void *h, void *out, float *part,
                       unsigned *counters, int *status, int num_sms, cudaStream_t st, const Marks &marks,
-                      int split_mode, int *launches);
+                      int split_mode, int *launches, float *partials = nullptr);
+
+// tc_gemm.cu: tensor parallelism across GPUs with the one-shot all-reduce
+// fused into the second projection (bf16, f_s % 64 == 0, 1..128 tokens).
+// Ranks rank0 .. rank0 + nranks - 1 of p.tp run here (one per GPU, or every
+// rank on one GPU); comm[r] is rank r's exchange buffer as this process sees
+// it: [control + flags (xgpu_header_bytes) | receive rows: 2 x tp x rows x
+// d_out bf16], zeroed before its first use.  The call count (epoch) lives in
+// the control words, so launches can be captured in a CUDA graph.
+struct XgpuArgs {
+    void *comm[kMaxTp];
+    void *outs[kMaxTp];     // output of local rank i (tokens x d_out bf16)
+    size_t recv_off;        // = xgpu_header_bytes(p)
+    int rows;               // receive rows per (half, rank): the handle's max tokens
+};
+size_t xgpu_header_bytes(const Problem &p);
+// Sequence-parallel variant: x_local[i] holds local rank i's T / tp token
+// rows; they are gathered into every rank's buffer at gather_off (T x d_in
+// bf16) before the first projection, and the second projection's exchange is
+// a reduce-scatter: outs[i] gets rank i's own T / tp rows.  T % tp == 0.
+cudaError_t launch_xgpu_sp(const Problem &p, int rank0, int nranks, const void *const *x_local, const ShardPtrs &A,
+                           const ShardPtrs &B, void *h, float *part, unsigned *counters, int *status, int num_sms,
+                           cudaStream_t st, const XgpuArgs &xa, size_t gather_off, int *launches);
+// h: tokens x (nranks * f_s) scratch; part / counters: split-tile scratch of
+// the first projection.  cudaErrorNotSupported: the clusters do not all fit.
+cudaError_t launch_xgpu(const Problem &p, int rank0, int nranks, const void *x, const ShardPtrs &A,
+                        const ShardPtrs &B, void *h, float *part, unsigned *counters, int *status, int num_sms,
+                        cudaStream_t st, const XgpuArgs &xa, int *launches);
 
 }  // namespace tpmlp

@@ -31,6 +31,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <mutex>
 
 #include "common.cuh"
 #include "internal.h"
@@ -47,7 +48,11 @@ constexpr int NTHREADS = 192;
 constexpr int kGroupM = 8;          // wide tiling: token tiles per raster group
 constexpr int kWideStages = 4;
 
-enum { EPI_H_TANH = 0, EPI_H_SWIGLU = 1, EPI_H_IDENT = 2, EPI_OUT = 3 };
+// EPI_PART: the second projection of one rank at a time, fp32 outputs
+// (tp_mlp_partials: Z_i = H_i B_i without the sum over ranks).
+// EPI_AR: the same per-rank second projection, then the one-shot all-reduce
+// across ranks (cross-GPU tensor parallelism; see the cluster exit below).
+enum { EPI_H_TANH = 0, EPI_H_SWIGLU = 1, EPI_H_IDENT = 2, EPI_OUT = 3, EPI_PART = 4, EPI_AR = 5 };
 
 struct TcArgs {
     int rows_x;          // X rows (tokens)
@@ -68,7 +73,95 @@ struct TcArgs {
     // first projection read straight from the per-rank shards: tile t covers
     // features of rank t / tps only (tps tiles per rank of fs features)
     int raw_first, tps, fs;
+    // per-rank partials (EPI_PART): weight tile t is output tile t % otiles of
+    // rank t / otiles, whose K loop is that rank's KB k-blocks of the full K
+    // (k-block offset rank * KB); results go to pout[rank][token][column]
+    int prank, otiles;
+    float *pout;
+    // skinny whole-CTA grids: the n CTAs sharing a tile form one thread-block
+    // cluster and add their partials through distributed shared memory (0: off)
+    int cluster_red;
+    // one-shot all-reduce (EPI_AR): this launch computes ranks ar_rank0 ..
+    // ar_rank0 + prank - 1 of ar_ranks; comm[p] is rank p's buffer as this
+    // process sees it: [control: epoch, finished-CTA count (256 B) | flags:
+    // ar_ranks x otiles x 8 u32 | recv: 2 (epoch parity) x ar_ranks x ar_rows
+    // x ldo bf16].  outs[i]: the output of local rank i (tokens x ldo bf16).
+    int ar_rank0, ar_ranks, ar_rows;
+    size_t recv_off;
+    uint8_t *comm[kMaxTp];
+    __nv_bfloat16 *outs[kMaxTp];
+    // sequence parallelism: rank o owns token rows [o sp_rows, (o + 1) sp_rows).
+    // EPI_AR with sp_rows > 0 is a reduce-scatter: a row goes only to its
+    // owner, which writes its own rows (outs[i]: sp_rows x ldo).  A first
+    // projection with sp_wait != nullptr reads X gathered from every rank and
+    // first waits until all ar_ranks arrival counts sp_wait[src] reach
+    // calls * sp_per_src (calls = *sp_epoch + 1: this is the next
+    // sequence-parallel call).
+    int sp_rows;
+    const unsigned *sp_wait;
+    const unsigned *sp_epoch;
+    unsigned sp_per_src;
 };
+
+// Weight tile and k-block of the full weight / activation that iteration
+// (tile, kb) of a launch reads.  Only the per-rank partials remap them.
+__device__ __forceinline__ int w_tile(const TcArgs &a, int tile) { return a.prank ? tile % a.otiles : tile; }
+__device__ __forceinline__ int k_block(const TcArgs &a, int tile, int kb) {
+    return a.prank ? (tile / a.otiles) * a.KB + kb : kb;
+}
+// Row t of rank (tile / otiles)'s fp32 partial output.
+__device__ __forceinline__ float *part_row(const TcArgs &a, int tile, int t) {
+    return a.pout + ((long)(tile / a.otiles) * a.rows_x + t) * a.ldo;
+}
+
+// --- thread-block clusters (split tiles added through distributed shared memory) ---
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// Hardware cluster barrier (no spinning; not the .aligned form, so a warp whose
+// lanes arrive apart is fine).  Every thread of every CTA of the cluster must
+// arrive, on every path, or the others wait for ever: the skinny kernel calls
+// it only from its common exit.
+__device__ __forceinline__ void cluster_barrier() {
+    asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+// 16 bytes at the same shared-memory address in CTA `rank` of the cluster.
+__device__ __forceinline__ float4 ld_cluster_f4(const void *local, uint32_t rank) {
+    uint32_t remote;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(rank));
+    float4 v;
+    asm volatile("ld.shared::cluster.v4.f32 {%0,%1,%2,%3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(remote)
+                 : "memory");
+    return v;
+}
+
+// --- the one-shot all-reduce across ranks (EPI_AR) ---------------------------------
+__device__ __forceinline__ void st_release_sys(unsigned *p, unsigned v) {
+    asm volatile("st.release.sys.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ unsigned ld_acquire_sys(const unsigned *p) {
+    unsigned v;
+    asm volatile("ld.acquire.sys.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+// Per rank: [0] last finished epoch, [1] finished-CTA count, [2] sequence-
+// parallel calls finished, [8 + src] rows of rank src gathered here by
+// sequence-parallel calls (in CTAs of the gather; counts only grow).
+constexpr int kArControlBytes = 256;
+__device__ __forceinline__ unsigned *ar_control(const TcArgs &a, int p) {
+    return reinterpret_cast<unsigned *>(a.comm[p]);
+}
+__device__ __forceinline__ unsigned *ar_flag(const TcArgs &a, int p, int src, int otile, int j) {
+    return reinterpret_cast<unsigned *>(a.comm[p] + kArControlBytes) + ((size_t)src * a.otiles + otile) * 8 + j;
+}
+__device__ __forceinline__ __nv_bfloat16 *ar_recv_row(const TcArgs &a, unsigned epoch, int p, int src, int t) {
+    return reinterpret_cast<__nv_bfloat16 *>(a.comm[p] + a.recv_off) +
+           (((size_t)(epoch & 1u) * a.ar_ranks + src) * a.ar_rows + t) * a.ldo;
+}
 
 // Weight operand of one projection, for the producer's TMA loads.
 //   packed: map[0] views the tile-blocked part; one 32 KB box per (tile, k-block).
@@ -262,7 +355,34 @@ struct WideCfg {
 // Epilogue of one 128-token half: TMEM lanes = tokens, columns 0..255 = weight rows.
 // Output columns come in runs of 16 that are all valid or all padding, except
 // at a packed part's ragged end (handled element by element).
+__device__ __forceinline__ void wide_epilogue_part(const TcArgs &a, int row, int nt, uint32_t taddr) {
+    const bool row_ok = row < a.rows_x;
+    float *orow = row_ok ? part_row(a, nt, row) : nullptr;
+    const int ot = w_tile(a, nt);
+#pragma unroll 1
+    for (int j = 0; j < 16; ++j) {
+        float g[16];
+        tmem_ld16(taddr + 16 * j, g);
+        tmem_ld_wait();
+        const int col = tile_col(a, ot, 16 * j, 256);
+        if (!row_ok || col < 0) continue;
+        if (col + 16 <= a.out_cols) {
+            float4 *dst = reinterpret_cast<float4 *>(orow + col);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dst[i] = make_float4(g[4 * i], g[4 * i + 1], g[4 * i + 2], g[4 * i + 3]);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                if (col + i < a.out_cols) orow[col + i] = g[i];
+        }
+    }
+}
+
 __device__ __forceinline__ void wide_epilogue_half(const TcArgs &a, int row, int nt, uint32_t taddr) {
+    if (a.epi == EPI_PART) {
+        wide_epilogue_part(a, row, nt, taddr);
+        return;
+    }
     const bool row_ok = row < a.rows_x;
     __nv_bfloat16 *orow = a.out + (long)row * a.ldo;
     const bool swiglu = a.epi == EPI_H_SWIGLU;
@@ -322,8 +442,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     if (!mbar_wait(smem_u32(&s.empty[stage]), phase ^ 1, s.abort)) goto done;
                     const uint32_t fb = smem_u32(&s.full[stage]);
                     mbar_arrive_expect_tx(fb, A_BYTES + B_BYTES);
-                    tma_load_2d(smem_u32(s.a + stage * A_BYTES), &tmX, kb * BK, mt * 128 * MH, fb);
-                    load_w_tile<RAW>(smem_u32(s.b + stage * B_BYTES), wm, nt, kb, a.KB, fb);
+                    const int gkb = k_block(a, nt, kb);
+                    tma_load_2d(smem_u32(s.a + stage * A_BYTES), &tmX, gkb * BK, mt * 128 * MH, fb);
+                    load_w_tile<RAW>(smem_u32(s.b + stage * B_BYTES), wm, w_tile(a, nt), gkb, a.KB, fb);
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
                 }
             }
@@ -390,6 +511,18 @@ done:
 __device__ __forceinline__ void skinny_final16(const TcArgs &a, int tile, int r, int t0, const float (&v0)[16],
                                                const float (&v1)[16]) {
     const int T = a.rows_x;
+    if (a.epi == EPI_PART) {
+        const int ot = w_tile(a, tile);
+        const int n0 = tile_col(a, ot, r, 256), n1 = tile_col(a, ot, r + 128, 256);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            if (t0 + i >= T) break;
+            float *row = part_row(a, tile, t0 + i);
+            if (n0 >= 0) row[n0] = v0[i];
+            if (n1 >= 0) row[n1] = v1[i];
+        }
+        return;
+    }
     if (a.epi == EPI_H_SWIGLU) {
         const int n = tile_col(a, tile, r, 128);
         if (n < 0) return;
@@ -411,6 +544,18 @@ __device__ __forceinline__ void skinny_final16(const TcArgs &a, int tile, int r,
 __device__ __forceinline__ void skinny_final4(const TcArgs &a, int tile, int r, int t0, float4 v0, float4 v1) {
     const float g[4] = {v0.x, v0.y, v0.z, v0.w}, u[4] = {v1.x, v1.y, v1.z, v1.w};
     const int T = a.rows_x;
+    if (a.epi == EPI_PART) {
+        const int ot = w_tile(a, tile);
+        const int n0 = tile_col(a, ot, r, 256), n1 = tile_col(a, ot, r + 128, 256);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            if (t0 + i >= T) break;
+            float *row = part_row(a, tile, t0 + i);
+            if (n0 >= 0) row[n0] = g[i];
+            if (n1 >= 0) row[n1] = u[i];
+        }
+        return;
+    }
     if (a.epi == EPI_H_SWIGLU) {
         const int n = tile_col(a, tile, r, 128);
         if (n < 0) return;
@@ -455,6 +600,109 @@ __device__ __forceinline__ void skinny_store_staged(const TcArgs &a, int tile, i
     }
 }
 
+// One-shot all-reduce of a 256-row tile across ranks (EPI_AR), run by the 128
+// epilogue threads of CTA j of the tile's cluster once every CTA of the
+// cluster has staged its partial sums ("7.4 推理侧并行" §7.4.2, optimisation
+// 2: each rank sends its whole partial to every other rank and every rank
+// adds them up itself, in one step).
+//   1. For the token quads j, j + n, ... of the tile: add the cluster's slots
+//      (this rank's Z_i for those tokens), round to bf16 and store them into
+//      every rank's receive buffer (plain stores; over NVLink for a peer),
+//      row block `me` of the buffer half chosen by the epoch's parity.
+//   2. Fence at system scope, then publish: flag (me, tile, j) = epoch in
+//      every rank's buffer.
+//   3. Wait (bounded) until the same unit's flag from every rank has this
+//      epoch in our own buffer, then add the ranks' rows in rank order (fp32)
+//      and write the output.
+// The epoch is kept on the device (graph replays need no new arguments): each
+// rank's buffer holds the last finished epoch, every CTA reads it at its start
+// and works on the next one, and the last CTA of the rank to finish stores it.
+// Flags only grow (the epoch goes up by one per call), so nothing is reset;
+// the two buffer halves keep a fast rank from overwriting rows a slow rank is
+// still reading: a rank reaches epoch e + 2 only after seeing every rank's
+// epoch e + 1 flags, which those ranks set after finishing epoch e.
+template <int BT>
+__device__ __forceinline__ void ar_exchange(const TcArgs &a, const Smem &s, int tile, unsigned epoch) {
+    const int r = threadIdx.x - 64;
+    const uint32_t n = (uint32_t)a.cluster_red, j = cluster_rank();
+    const int li = tile / a.otiles, otile = tile - li * a.otiles, me = a.ar_rank0 + li;
+    const int col0 = tile_col(a, otile, r, 256), col1 = tile_col(a, otile, r + 128, 256);
+    const float4 *st4 = reinterpret_cast<const float4 *>(s.a);
+    const int T = a.rows_x;
+    for (int qd = (int)j; qd < BT / 4 && qd * 4 < T; qd += (int)n) {
+        float4 s0 = make_float4(0.f, 0.f, 0.f, 0.f), s1 = s0;
+        for (uint32_t src = 0; src < n; ++src) {
+            const float4 g = ld_cluster_f4(st4 + qd * 256 + r, src);
+            const float4 h = ld_cluster_f4(st4 + qd * 256 + 128 + r, src);
+            s0.x += g.x; s0.y += g.y; s0.z += g.z; s0.w += g.w;
+            s1.x += h.x; s1.y += h.y; s1.z += h.z; s1.w += h.w;
+        }
+        const float v0[4] = {s0.x, s0.y, s0.z, s0.w}, v1[4] = {s1.x, s1.y, s1.z, s1.w};
+        if (a.sp_rows) {   // reduce-scatter: row t goes to its owner only, as the owner's row t - owner * sp_rows
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int t = qd * 4 + i;
+                if (t >= T) break;
+                const int owner = t / a.sp_rows;
+                __nv_bfloat16 *row = ar_recv_row(a, epoch, owner, me, t - owner * a.sp_rows);
+                if (col0 >= 0) row[col0] = __float2bfloat16_rn(v0[i]);
+                if (col1 >= 0) row[col1] = __float2bfloat16_rn(v1[i]);
+            }
+            continue;
+        }
+        for (int p = 0; p < a.ar_ranks; ++p)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int t = qd * 4 + i;
+                if (t >= T) break;
+                __nv_bfloat16 *row = ar_recv_row(a, epoch, p, me, t);
+                if (col0 >= 0) row[col0] = __float2bfloat16_rn(v0[i]);
+                if (col1 >= 0) row[col1] = __float2bfloat16_rn(v1[i]);
+            }
+    }
+    __threadfence_system();
+    named_bar(1, 128);
+    if (threadIdx.x == 64) {
+        for (int p = 0; p < a.ar_ranks; ++p) st_release_sys(ar_flag(a, p, me, otile, (int)j), epoch);
+        bool ok = true;
+        const unsigned long long t0 = globaltimer();
+        for (int src = 0; src < a.ar_ranks && ok; ++src) {
+            const unsigned *f = ar_flag(a, me, src, otile, (int)j);
+            while (ld_acquire_sys(f) != epoch) {
+                if (globaltimer() - t0 > kWaitLimitNs) {
+                    ok = false;
+                    *s.abort = 1;
+                    break;
+                }
+            }
+        }
+        *s.flag = ok ? 1 : 0;
+    }
+    named_bar(1, 128);
+    if (!*s.flag) return;
+    __threadfence();
+    __nv_bfloat16 *out = a.outs[li];
+    for (int qd = (int)j; qd < BT / 4 && qd * 4 < T; qd += (int)n)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            int t = qd * 4 + i;
+            if (t >= T) break;
+            if (a.sp_rows) {   // reduce-scatter: only the rows this rank owns, as its local rows
+                if (t / a.sp_rows != me) continue;
+                t -= me * a.sp_rows;
+            }
+            float z0 = 0.f, z1 = 0.f;
+            for (int src = 0; src < a.ar_ranks; ++src) {
+                const unsigned short *row =
+                    reinterpret_cast<const unsigned short *>(ar_recv_row(a, epoch, me, src, t));
+                if (col0 >= 0) z0 += __bfloat162float(__ushort_as_bfloat16(__ldcg(row + col0)));
+                if (col1 >= 0) z1 += __bfloat162float(__ushort_as_bfloat16(__ldcg(row + col1)));
+            }
+            if (col0 >= 0) out[(long)t * a.ldo + col0] = __float2bfloat16_rn(z0);
+            if (col1 >= 0) out[(long)t * a.ldo + col1] = __float2bfloat16_rn(z1);
+        }
+}
+
 // HALF: 128-row weight tiles, one M=128 MMA per 16-k step (never SwiGLU's first
 // projection, whose gate and up rows must share a tile); split tiles always go
 // to skinny_reduce_kernel.
@@ -475,7 +723,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const long long total = a.total_iters, G = gridDim.x, c = blockIdx.x;
     const long long it_b = share_begin(c, total, G), it_e = share_begin(c + 1, total, G);
     const int KB = a.KB;
+    constexpr int ROWS = HALF ? 128 : 256;   // rows of a weight tile; a partial slot is [token/4][ROWS][4]
+    int cl_tile = -1;                         // cluster route: the tile this CTA staged in shared memory
 
+    if (a.epi == EPI_AR && threadIdx.x == 0) {   // this call's epoch, read before any CTA of it finishes
+        const int li = (int)(blockIdx.x / ((unsigned)a.cluster_red * a.otiles));
+        s.tmem_slot[3] = *reinterpret_cast<volatile unsigned *>(ar_control(a, a.ar_rank0 + li)) + 1u;
+    }
     if (warp == 0) {
         if (lane == 0) {
             // The weights do not depend on the previous kernel; X does.  Every
@@ -489,12 +743,30 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 const int tile = (int)(it / KB), kb = (int)(it - (long long)tile * KB);
                 const uint32_t fb = smem_u32(&s.full[i]);
                 mbar_arrive_expect_tx(fb, W_BYTES + X_BYTES);   // first use of stage i: it is empty
-                load_w_tile<RAW, HALF>(smem_u32(s.a + i * W_BYTES), wm, tile, kb, KB, fb);
+                load_w_tile<RAW, HALF>(smem_u32(s.a + i * W_BYTES), wm, w_tile(a, tile), k_block(a, tile, kb), KB,
+                                       fb);
             }
             pdl_wait_previous();
-            for (int i = 0; i < npre; ++i)
-                tma_load_2d(smem_u32(s.b + i * X_BYTES), &tmX, (int)((it_b + i) % KB) * BK, 0,
-                            smem_u32(&s.full[i]));
+            if (a.sp_wait) {
+                // X is gathered from every rank: wait until every rank's rows have
+                // arrived (bounded), then order those generic-proxy stores before
+                // this thread's TMA reads of them.
+                const unsigned need = (*reinterpret_cast<const volatile unsigned *>(a.sp_epoch) + 1u) * a.sp_per_src;
+                const unsigned long long t0 = globaltimer();
+                for (int src = 0; src < a.ar_ranks; ++src)
+                    while (ld_acquire_sys(a.sp_wait + src) < need) {
+                        if (globaltimer() - t0 > kWaitLimitNs) {
+                            *s.abort = 1;
+                            goto done;
+                        }
+                    }
+                asm volatile("fence.proxy.async.global;" ::: "memory");
+            }
+            for (int i = 0; i < npre; ++i) {
+                const long long it = it_b + i;
+                const int tile = (int)(it / KB), kb = (int)(it - (long long)tile * KB);
+                tma_load_2d(smem_u32(s.b + i * X_BYTES), &tmX, k_block(a, tile, kb) * BK, 0, smem_u32(&s.full[i]));
+            }
             int stage = npre % STAGES;
             uint32_t phase = npre == STAGES ? 1u : 0u;
             for (long long it = it_b + npre; it < it_e; ++it) {
@@ -502,8 +774,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 if (!mbar_wait(smem_u32(&s.empty[stage]), phase ^ 1, s.abort)) goto done;
                 const uint32_t fb = smem_u32(&s.full[stage]);
                 mbar_arrive_expect_tx(fb, W_BYTES + X_BYTES);
-                load_w_tile<RAW, HALF>(smem_u32(s.a + stage * W_BYTES), wm, tile, kb, KB, fb);
-                tma_load_2d(smem_u32(s.b + stage * X_BYTES), &tmX, kb * BK, 0, fb);
+                const int gkb = k_block(a, tile, kb);
+                load_w_tile<RAW, HALF>(smem_u32(s.a + stage * W_BYTES), wm, w_tile(a, tile), gkb, KB, fb);
+                tma_load_2d(smem_u32(s.b + stage * X_BYTES), &tmX, gkb * BK, 0, fb);
                 if (++stage == STAGES) { stage = 0; phase ^= 1; }
             }
         }
@@ -558,7 +831,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             if (!mbar_wait(smem_u32(&s.tfull[acc]), acc_phase, s.abort)) break;
             tc_fence_after();
             const uint32_t taddr = tmem_base + acc * (2 * BT) + ((uint32_t)(q * 32) << 16);
-            const bool whole = (kb0 == 0 && kb1 == KB);
+            // (the cluster route stages even a whole tile: the all-reduce needs it there)
+            const bool whole = (kb0 == 0 && kb1 == KB) && !a.cluster_red;
             if (whole) {
 #pragma unroll 1
                 for (int t0 = 0; t0 < BT; t0 += 16) {
@@ -588,8 +862,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 const int c_first = share_owner((long long)tile * KB, total, G);
                 const int c_last = share_owner((long long)tile * KB + KB - 1, total, G);
                 const int slot = (int)c - c_first;
-                constexpr int ROWS = HALF ? 128 : 256;   // slot: [token/4][ROWS][4]
-                float4 *base = reinterpret_cast<float4 *>(a.part + ((long long)tile * a.slots + slot) * ROWS * BT);
+                // cluster route: the slot is this CTA's own ring (every MMA that read it is done)
+                float4 *base = a.cluster_red
+                                   ? reinterpret_cast<float4 *>(s.a)
+                                   : reinterpret_cast<float4 *>(a.part + ((long long)tile * a.slots + slot) * ROWS * BT);
 #pragma unroll 1
                 for (int t0 = 0; t0 < BT; t0 += 16) {
                     float v0[16], v1[16];
@@ -609,6 +885,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_u32(&s.tempty[acc]));
+                if (a.cluster_red) {   // added across the cluster at the exit
+                    cl_tile = tile;
+                    acc ^= 1;
+                    if (acc == 0) acc_phase ^= 1;
+                    continue;
+                }
                 if (HALF || a.split_mode == kSplitSeparate) {   // skinny_reduce_kernel adds the slots
                     acc ^= 1;
                     if (acc == 0) acc_phase ^= 1;
@@ -664,6 +946,62 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
     }
 done:
+    if (a.cluster_red) {
+        // The n CTAs of a tile (one cluster; cluster rank = slot) have staged
+        // their partial sums in their rings.  Every thread of every CTA passes
+        // both barriers, whatever happened before.  CTA j then adds, for token
+        // quads j, j + n, ..., the n slots in slot order -- the order of
+        // skinny_reduce_kernel, so both routes give the same bits -- and
+        // applies the epilogue; the second barrier keeps each ring alive until
+        // the cluster has read it.
+        __syncwarp();
+        cluster_barrier();
+        if constexpr (!HALF) {
+            if (a.epi == EPI_AR) {
+                // After the barrier nobody sets the abort flag any more, so `go`
+                // is the same in every thread of the CTA (the named barriers
+                // below need all 128 epilogue threads or none).
+                const unsigned epoch = s.tmem_slot[3];
+                const bool go = cl_tile >= 0 && !*s.abort;
+                if (go && threadIdx.x >= 64) ar_exchange<BT>(a, s, cl_tile, epoch);
+                cluster_barrier();
+                if (threadIdx.x == 0) {   // the rank's last CTA to finish records the epoch as done
+                    const int li = (int)(blockIdx.x / ((unsigned)a.cluster_red * a.otiles));
+                    unsigned *ctl = ar_control(a, a.ar_rank0 + li);
+                    __threadfence();
+                    if (atomicAdd(ctl + 1, 1u) + 1u == (unsigned)a.cluster_red * a.otiles) {
+                        ctl[1] = 0u;
+                        if (a.sp_rows) ctl[2] += 1u;
+                        __threadfence();
+                        atomicExch(ctl, epoch);
+                    }
+                }
+                goto exit;
+            }
+        }
+        if (cl_tile >= 0 && threadIdx.x >= 64) {
+            const int r = threadIdx.x - 64;
+            const uint32_t n = (uint32_t)a.cluster_red, j = cluster_rank();
+            const float4 *st4 = reinterpret_cast<const float4 *>(s.a);
+            for (int qd = (int)j; qd < BT / 4 && qd * 4 < a.rows_x; qd += (int)n) {
+                float4 s0 = make_float4(0.f, 0.f, 0.f, 0.f), s1 = s0;
+                for (uint32_t src = 0; src < n; ++src) {
+                    const float4 g = ld_cluster_f4(st4 + qd * ROWS + r, src);
+                    s0.x += g.x; s0.y += g.y; s0.z += g.z; s0.w += g.w;
+                    if (!HALF) {
+                        const float4 h = ld_cluster_f4(st4 + qd * ROWS + 128 + r, src);
+                        s1.x += h.x; s1.y += h.y; s1.z += h.z; s1.w += h.w;
+                    }
+                }
+                if (HALF)
+                    skinny_final_half4(a, cl_tile, r, qd * 4, s0);
+                else
+                    skinny_final4(a, cl_tile, r, qd * 4, s0, s1);
+            }
+        }
+        cluster_barrier();
+    }
+exit:
     teardown(s, tmem_base, a.status);
 }
 
@@ -762,6 +1100,7 @@ struct WeightOperand {
     bool raw, half;
     int tiles, KB;
     int raw_first, tps, fs;
+    int prank, otiles;   // per-rank partials: tiles = prank * otiles, KB = one rank's k-blocks
 };
 
 // Token-tile widths from which the skinny tiling uses 128-row weight tiles
@@ -828,12 +1167,20 @@ bool weight_raw_first(WeightOperand *w, const Problem &p, const ShardPtrs &A, bo
 
 // Second projection straight from the shards B_i (f_s x d_out row-major); the K
 // loop runs over rank 0's rows, then rank 1's, ... (needs f_s % 64 == 0).
-bool weight_raw_second(WeightOperand *w, const Problem &p, const ShardPtrs &B, bool half) {
+// per_rank: one weight tile per (rank, output tile), each with its rank's
+// k-blocks only (the per-rank partials), tiles rank-major.
+bool weight_raw_second(WeightOperand *w, const Problem &p, const ShardPtrs &B, bool half, bool per_rank = false) {
     memset(w, 0, sizeof(*w));
     w->raw = true;
     w->half = half;
     w->tiles = (int)skinny_tiles(p, 1, true, half);
     w->KB = p.d_ff / BK;
+    if (per_rank) {
+        w->prank = p.tp;
+        w->otiles = w->tiles;
+        w->tiles *= p.tp;
+        w->KB = p.fs / BK;
+    }
     w->wm.kbps = p.fs / BK;
     for (int i = 0; i < p.tp; ++i)
         if (!make_map2d(&w->wm.map[i], B.p[i], p.d_out, p.fs, (long long)p.d_out * 2, BK)) return false;
@@ -842,26 +1189,112 @@ bool weight_raw_second(WeightOperand *w, const Problem &p, const ShardPtrs &B, b
 
 int skinny_bt(int T) { return T <= 16 ? 16 : T <= 32 ? 32 : T <= 64 ? 64 : 128; }
 
+// Split tiles of whole-CTA grids added across a thread-block cluster (1) or by
+// skinny_reduce_kernel (0).
+#ifndef TPMLP_SKINNY_CLUSTER
+#define TPMLP_SKINNY_CLUSTER 1
+#endif
+
+// Ring depth of the skinny kernel per token width: 128-row tiles (SKH) and
+// 256-row tiles (SK).  Each stage holds one weight block and one X box, so the
+// wider the token tile, the fewer stages fit in shared memory.
+#ifndef TPMLP_SKH_S16
+#define TPMLP_SKH_S16 8
+#endif
+#ifndef TPMLP_SKH_S32
+#define TPMLP_SKH_S32 8
+#endif
+#ifndef TPMLP_SKH_S64
+#define TPMLP_SKH_S64 8
+#endif
+#ifndef TPMLP_SKH_S128
+#define TPMLP_SKH_S128 6
+#endif
+#ifndef TPMLP_SK_S16
+#define TPMLP_SK_S16 6
+#endif
+#ifndef TPMLP_SK_S32
+#define TPMLP_SK_S32 6
+#endif
+#ifndef TPMLP_SK_S64
+#define TPMLP_SK_S64 5
+#endif
+#ifndef TPMLP_SK_S128
+#define TPMLP_SK_S128 4
+#endif
+
 template <typename K>
 cudaError_t set_smem(K kern, size_t bytes) {
     return ensure_smem_attr(kern, bytes);
 }
 
-template <int BT, int STAGES, bool HALF>
-cudaError_t launch_skinny_bt(const WeightOperand &w, const CUtensorMap &mx, const TcArgs &a, int grid,
-                             cudaStream_t st) {
+// Whether `clusters` clusters of `n` CTAs of this kernel (smem bytes each) can
+// all be resident at once (the cluster route needs them in one wave).  The
+// answer is cached per kernel, cluster size and device.
+template <typename K>
+bool clusters_fit(K kern, size_t smem, int n, int clusters) {
+    struct Entry {
+        const void *fn;
+        int n, dev, max_active;
+    };
+    static Entry cache[64];
+    static int cached = 0;
+    static std::mutex mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    const void *fn = reinterpret_cast<const void *>(kern);
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        for (int i = 0; i < cached; ++i)
+            if (cache[i].fn == fn && cache[i].n == n && cache[i].dev == dev) return cache[i].max_active >= clusters;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(n * clusters);
+    cfg.blockDim = dim3(NTHREADS);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)n;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int max_active = 0;
+    if (cudaOccupancyMaxActiveClusters(&max_active, kern, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        max_active = 0;
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    if (cached < 64) cache[cached++] = Entry{fn, n, dev, max_active};
+    return max_active >= clusters;
+}
+
+template <int BT, int STAGES, bool RAW, bool HALF>
+cudaError_t launch_skinny_kern(const WeightOperand &w, const CUtensorMap &mx, TcArgs a, int grid, cudaStream_t st,
+                               int *cluster_used) {
     // HALF adds the epilogue's BT x 128 bf16 staging (+16 for its alignment)
     const size_t smem = smem_bytes<STAGES>((HALF ? 128 : 256) * BK * 2, BT * BK * 2) + (HALF ? BT * 256 + 16 : 0);
-    if (w.raw) {
-        auto kern = tc_skinny_kernel<BT, STAGES, true, HALF>;
-        cudaError_t e = set_smem(kern, smem);
-        if (e != cudaSuccess) return e;
-        return launch_pdl(kern, dim3(grid), dim3(NTHREADS), smem, st, w.wm, mx, a);
-    }
-    auto kern = tc_skinny_kernel<BT, STAGES, false, HALF>;
+    auto kern = tc_skinny_kernel<BT, STAGES, RAW, HALF>;
     cudaError_t e = set_smem(kern, smem);
     if (e != cudaSuccess) return e;
+    // the cluster route stages a (HALF ? 128 : 256) x BT fp32 slot in the ring
+    static_assert((size_t)(HALF ? 128 : 256) * BT * 4 <= (size_t)STAGES * ((HALF ? 128 : 256) + BT) * BK * 2,
+                  "ring too small to stage a split tile");
+    const int n = a.cluster_red;
+    if (n >= 2 && clusters_fit(kern, smem, n, grid / n)) {
+        *cluster_used = n;
+        return launch_pdl_cluster(kern, dim3(grid), dim3(NTHREADS), smem, st, (unsigned)n, w.wm, mx, a);
+    }
+    a.cluster_red = 0;
+    *cluster_used = 0;
     return launch_pdl(kern, dim3(grid), dim3(NTHREADS), smem, st, w.wm, mx, a);
+}
+
+template <int BT, int STAGES, bool HALF>
+cudaError_t launch_skinny_bt(const WeightOperand &w, const CUtensorMap &mx, const TcArgs &a, int grid,
+                             cudaStream_t st, int *cluster_used) {
+    if (w.raw) return launch_skinny_kern<BT, STAGES, true, HALF>(w, mx, a, grid, st, cluster_used);
+    return launch_skinny_kern<BT, STAGES, false, HALF>(w, mx, a, grid, st, cluster_used);
 }
 
 // Auto: the reduction kernel.  On B200 it measured faster at every width (16 to
@@ -898,9 +1331,16 @@ StreamKGeom skinny_geom(int tiles, int KB, int BT, int num_sms) {
 }
 
 // One projection with the skinny tiling; x: T x K activations.
+// Gather wait of a sequence-parallel first projection (see TcArgs::sp_wait).
+struct SpWait {
+    const unsigned *counts, *epoch;
+    unsigned per_src;
+    int ranks;
+};
+
 cudaError_t run_skinny(const WeightOperand &w, const void *x, int T, int K, int epi, void *out, int out_cols,
                        float *part, unsigned *cnt, int *status, int num_sms, cudaStream_t st, int split_mode,
-                       int *launches) {
+                       int *launches, int ldo = 0, const SpWait *spw = nullptr) {
     const int BT = skinny_bt(T);
     CUtensorMap mx;
     if (!make_map(&mx, x, K, T, BT)) return cudaErrorInvalidValue;
@@ -912,7 +1352,7 @@ cudaError_t run_skinny(const WeightOperand &w, const void *x, int T, int K, int 
     a.KB = g.KB;
     a.epi = epi;
     a.out = static_cast<__nv_bfloat16 *>(out);
-    a.ldo = out_cols;
+    a.ldo = ldo ? ldo : out_cols;
     a.out_cols = out_cols;
     a.total_iters = g.total;
     a.slots = g.slots;
@@ -924,25 +1364,46 @@ cudaError_t run_skinny(const WeightOperand &w, const void *x, int T, int K, int 
     a.raw_first = w.raw_first;
     a.tps = w.tps;
     a.fs = w.fs;
+    a.prank = w.prank;
+    a.otiles = w.otiles;
+    if (spw) {
+        a.sp_wait = spw->counts;
+        a.sp_epoch = spw->epoch;
+        a.sp_per_src = spw->per_src;
+        a.ar_ranks = spw->ranks;
+    }
+    if (epi == EPI_PART) {
+        a.pout = static_cast<float *>(out);
+        a.out = nullptr;
+        if (g.slots > 1) a.split_mode = kSplitSeparate;   // the counters cover whole-K tiles only
+    }
+    // A whole number n of CTAs per tile (2..8), each inside one tile: the n
+    // CTAs of a tile become one cluster and add their partials through
+    // distributed shared memory, if all the clusters fit on the GPU at once.
+    const int per_tile = g.grid / g.tiles;
+    if (TPMLP_SKINNY_CLUSTER && split_mode == kSplitAuto && g.slots > 1 && g.grid % g.tiles == 0 &&
+        per_tile >= 2 && per_tile <= 8)
+        a.cluster_red = per_tile;
+    int cl = 0;
     cudaError_t e;
     // a 128-row tile stage holds half the weights, so the ring gets more stages
     if (w.half) {
         switch (BT) {
-            case 16: e = launch_skinny_bt<16, 8, true>(w, mx, a, g.grid, st); break;
-            case 32: e = launch_skinny_bt<32, 8, true>(w, mx, a, g.grid, st); break;
-            case 64: e = launch_skinny_bt<64, 8, true>(w, mx, a, g.grid, st); break;
-            default: e = launch_skinny_bt<128, 6, true>(w, mx, a, g.grid, st); break;
+            case 16: e = launch_skinny_bt<16, TPMLP_SKH_S16, true>(w, mx, a, g.grid, st, &cl); break;
+            case 32: e = launch_skinny_bt<32, TPMLP_SKH_S32, true>(w, mx, a, g.grid, st, &cl); break;
+            case 64: e = launch_skinny_bt<64, TPMLP_SKH_S64, true>(w, mx, a, g.grid, st, &cl); break;
+            default: e = launch_skinny_bt<128, TPMLP_SKH_S128, true>(w, mx, a, g.grid, st, &cl); break;
         }
     } else {
         switch (BT) {
-            case 16: e = launch_skinny_bt<16, 6, false>(w, mx, a, g.grid, st); break;
-            case 32: e = launch_skinny_bt<32, 6, false>(w, mx, a, g.grid, st); break;
-            case 64: e = launch_skinny_bt<64, 5, false>(w, mx, a, g.grid, st); break;
-            default: e = launch_skinny_bt<128, 4, false>(w, mx, a, g.grid, st); break;
+            case 16: e = launch_skinny_bt<16, TPMLP_SK_S16, false>(w, mx, a, g.grid, st, &cl); break;
+            case 32: e = launch_skinny_bt<32, TPMLP_SK_S32, false>(w, mx, a, g.grid, st, &cl); break;
+            case 64: e = launch_skinny_bt<64, TPMLP_SK_S64, false>(w, mx, a, g.grid, st, &cl); break;
+            default: e = launch_skinny_bt<128, TPMLP_SK_S128, false>(w, mx, a, g.grid, st, &cl); break;
         }
     }
     ++*launches;
-    if (e != cudaSuccess || a.split_mode != kSplitSeparate) return e;
+    if (e != cudaSuccess || cl || a.split_mode != kSplitSeparate) return e;
     ++*launches;
     // one CTA per unit: a grid capped at 2 CTAs per SM (so the next GEMM's CTAs
     // fit beside the waiting ones) measured 20-30 % slower at 32-128 tokens
@@ -970,6 +1431,12 @@ cudaError_t run_wide(const WeightOperand &w, const void *x, int T, int K, int ep
     a.raw_first = w.raw_first;
     a.tps = w.tps;
     a.fs = w.fs;
+    a.prank = w.prank;
+    a.otiles = w.otiles;
+    if (epi == EPI_PART) {
+        a.pout = static_cast<float *>(out);
+        a.out = nullptr;
+    }
     const int units = ((T + 128 * MH - 1) / (128 * MH)) * w.tiles;
     const int grid = std::min(units, num_sms);
     const size_t smem = smem_bytes<C::STAGES>(C::A_BYTES, C::B_BYTES);
@@ -989,7 +1456,211 @@ int first_epi(int act) {
     return act == TP_MLP_ACT_SWIGLU ? EPI_H_SWIGLU : act == TP_MLP_ACT_TANH ? EPI_H_TANH : EPI_H_IDENT;
 }
 
+// Launch with thread-block clusters and without programmatic overlap.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_cluster(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                           unsigned cluster, Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = cluster;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
+// The second projection of the local ranks fused with the one-shot all-reduce:
+// n CTAs per tile (the largest n <= 8 whose clusters all fit on the GPU at
+// once -- every CTA must be resident, since units wait on other ranks).
+template <int BT, int STAGES>
+cudaError_t launch_ar_bt(const WeightOperand &w, const CUtensorMap &mx, TcArgs a, int num_sms, cudaStream_t st) {
+    const size_t smem = smem_bytes<STAGES>(256 * BK * 2, BT * BK * 2);
+    auto kern = tc_skinny_kernel<BT, STAGES, true, false>;
+    cudaError_t e = set_smem(kern, smem);
+    if (e != cudaSuccess) return e;
+    for (int n = std::min({8, num_sms / std::max(1, w.tiles), w.KB}); n >= 1; --n) {
+        if (!clusters_fit(kern, smem, n, w.tiles)) continue;
+        const int grid = w.tiles * n;
+        a.grid = grid;
+        a.slots = n;
+        a.cluster_red = n;
+        return launch_cluster(kern, dim3(grid), dim3(NTHREADS), smem, st, (unsigned)n, w.wm, mx, a);
+    }
+    return cudaErrorNotSupported;
+}
+
+// All-gather of the ranks' token rows (sequence parallelism): CTA (c, i) of
+// local rank src = rank0 + i copies its share of x_i (rows x d bf16) into
+// every rank's gather buffer at rows [src * rows, (src + 1) * rows), then
+// counts itself in at every rank (release at system scope: a rank that sees
+// the count also sees the rows).  Nothing here waits.
+struct GatherArgs {
+    const uint4 *x[kMaxTp];
+    uint8_t *comm[kMaxTp];
+    size_t gather_off;
+    int rank0, ranks, rows, d;
+};
+
+__global__ void __launch_bounds__(256) sp_gather_kernel(GatherArgs g) {
+    const int li = blockIdx.y, src = g.rank0 + li;
+    const long long n16 = (long long)g.rows * g.d / 8;   // 16-byte pieces of one rank's rows
+    const long long per = (n16 + gridDim.x - 1) / gridDim.x;
+    const long long b = (long long)blockIdx.x * per, e = min(n16, b + per);
+    const uint4 *x = g.x[li];
+    for (int p = 0; p < g.ranks; ++p) {
+        uint4 *dst = reinterpret_cast<uint4 *>(g.comm[p] + g.gather_off) + (long long)src * n16;
+        for (long long k = b + threadIdx.x; k < e; k += blockDim.x) dst[k] = x[k];
+    }
+    __threadfence_system();
+    __syncthreads();
+    if (threadIdx.x == 0)
+        for (int p = 0; p < g.ranks; ++p)
+            asm volatile("red.release.sys.global.add.u32 [%0], 1;" ::"l"(reinterpret_cast<unsigned *>(g.comm[p]) + 8 + src)
+                         : "memory");
+}
+
+constexpr int kGatherCtas = 16;   // per local rank
+
 }  // namespace
+
+cudaError_t launch_xgpu_sp(const Problem &p, int rank0, int nranks, const void *const *x_local, const ShardPtrs &A,
+                           const ShardPtrs &B, void *h, float *part, unsigned *counters, int *status, int num_sms,
+                           cudaStream_t st, const XgpuArgs &xa, size_t gather_off, int *launches) {
+    *launches = 0;
+    if (p.T < 1 || p.T > kTcSkinnyMaxTokens || p.T % p.tp || nranks < 1 || rank0 < 0 || rank0 + nranks > p.tp)
+        return cudaErrorInvalidValue;
+    const int rows = p.T / p.tp;
+    // 1. all-gather of the token rows (no programmatic overlap: it must start
+    //    after the previous call's exchange has finished and counted its epoch)
+    GatherArgs g{};
+    for (int i = 0; i < nranks; ++i) g.x[i] = static_cast<const uint4 *>(x_local[i]);
+    for (int r = 0; r < p.tp; ++r) g.comm[r] = static_cast<uint8_t *>(xa.comm[r]);
+    g.gather_off = gather_off;
+    g.rank0 = rank0;
+    g.ranks = p.tp;
+    g.rows = rows;
+    g.d = p.d_in;
+    sp_gather_kernel<<<dim3(kGatherCtas, nranks), 256, 0, st>>>(g);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    ++*launches;
+    // 2. each local rank's first projection on its gathered X, into its columns of H
+    Problem p1 = p;
+    p1.tp = 1;
+    p1.d_ff = p.fs;
+    const int ldh = nranks * p.fs;
+    for (int i = 0; i < nranks; ++i) {
+        ShardPtrs a1;
+        memset(&a1, 0, sizeof(a1));
+        a1.p[0] = A.p[i];
+        WeightOperand w1;
+        if (!weight_raw_first(&w1, p1, a1, false)) return cudaErrorInvalidValue;
+        const unsigned *ctl = static_cast<const unsigned *>(xa.comm[rank0 + i]);
+        const SpWait spw{ctl + 8, ctl + 2, (unsigned)kGatherCtas, p.tp};
+        int n = 0;
+        e = run_skinny(w1, static_cast<const uint8_t *>(xa.comm[rank0 + i]) + gather_off, p.T, p.d_in,
+                       first_epi(p.act), static_cast<__nv_bfloat16 *>(h) + (size_t)i * p.fs, p.fs, part, counters,
+                       status, num_sms, st, kSplitAuto, &n, ldh, &spw);
+        *launches += n;
+        if (e != cudaSuccess) return e;
+    }
+    // 3. second projection + reduce-scatter
+    Problem pl = p;
+    pl.tp = nranks;
+    pl.d_ff = ldh;
+    WeightOperand w2;
+    if (!weight_raw_second(&w2, pl, B, false, true)) return cudaErrorInvalidValue;
+    const int BT = skinny_bt(p.T);
+    CUtensorMap mx;
+    if (!make_map(&mx, h, ldh, p.T, BT)) return cudaErrorInvalidValue;
+    TcArgs a{};
+    a.rows_x = p.T;
+    a.rows_w = w2.tiles;
+    a.K = ldh;
+    a.KB = w2.KB;
+    a.epi = EPI_AR;
+    a.ldo = p.d_out;
+    a.out_cols = p.d_out;
+    a.total_iters = (long long)w2.tiles * w2.KB;
+    a.split_mode = kSplitSeparate;
+    a.status = status;
+    a.prank = w2.prank;
+    a.otiles = w2.otiles;
+    a.ar_rank0 = rank0;
+    a.ar_ranks = p.tp;
+    a.ar_rows = xa.rows;
+    a.recv_off = xa.recv_off;
+    a.sp_rows = rows;
+    for (int r = 0; r < p.tp; ++r) a.comm[r] = static_cast<uint8_t *>(xa.comm[r]);
+    for (int i = 0; i < nranks; ++i) a.outs[i] = static_cast<__nv_bfloat16 *>(xa.outs[i]);
+    switch (BT) {
+        case 16: e = launch_ar_bt<16, TPMLP_SK_S16>(w2, mx, a, num_sms, st); break;
+        case 32: e = launch_ar_bt<32, TPMLP_SK_S32>(w2, mx, a, num_sms, st); break;
+        case 64: e = launch_ar_bt<64, TPMLP_SK_S64>(w2, mx, a, num_sms, st); break;
+        default: e = launch_ar_bt<128, TPMLP_SK_S128>(w2, mx, a, num_sms, st); break;
+    }
+    if (e == cudaSuccess) ++*launches;
+    return e;
+}
+
+cudaError_t launch_xgpu(const Problem &p, int rank0, int nranks, const void *x, const ShardPtrs &A,
+                        const ShardPtrs &B, void *h, float *part, unsigned *counters, int *status, int num_sms,
+                        cudaStream_t st, const XgpuArgs &xa, int *launches) {
+    *launches = 0;
+    if (p.T < 1 || p.T > kTcSkinnyMaxTokens || nranks < 1 || rank0 < 0 || rank0 + nranks > p.tp)
+        return cudaErrorInvalidValue;
+    // the local ranks side by side: H = [act(x A_rank0) | ... ], K of the second
+    // projection = nranks * f_s, tile t of it = output tile t % otiles of rank t / otiles
+    Problem pl = p;
+    pl.tp = nranks;
+    pl.d_ff = nranks * p.fs;
+    WeightOperand w1, w2;
+    if (!weight_raw_first(&w1, pl, A, false) || !weight_raw_second(&w2, pl, B, false, true))
+        return cudaErrorInvalidValue;
+    cudaError_t e = run_skinny(w1, x, p.T, p.d_in, first_epi(p.act), h, pl.d_ff, part, counters, status, num_sms,
+                               st, kSplitAuto, launches);
+    if (e != cudaSuccess) return e;
+    const int BT = skinny_bt(p.T);
+    CUtensorMap mx;
+    if (!make_map(&mx, h, pl.d_ff, p.T, BT)) return cudaErrorInvalidValue;
+    TcArgs a{};
+    a.rows_x = p.T;
+    a.rows_w = w2.tiles;
+    a.K = pl.d_ff;
+    a.KB = w2.KB;
+    a.epi = EPI_AR;
+    a.ldo = p.d_out;
+    a.out_cols = p.d_out;
+    a.total_iters = (long long)w2.tiles * w2.KB;
+    a.split_mode = kSplitSeparate;
+    a.status = status;
+    a.prank = w2.prank;
+    a.otiles = w2.otiles;
+    a.ar_rank0 = rank0;
+    a.ar_ranks = p.tp;
+    a.ar_rows = xa.rows;
+    a.recv_off = xa.recv_off;
+    for (int i = 0; i < p.tp; ++i) a.comm[i] = static_cast<uint8_t *>(xa.comm[i]);
+    for (int i = 0; i < nranks; ++i) a.outs[i] = static_cast<__nv_bfloat16 *>(xa.outs[i]);
+    switch (BT) {
+        case 16: e = launch_ar_bt<16, TPMLP_SK_S16>(w2, mx, a, num_sms, st); break;
+        case 32: e = launch_ar_bt<32, TPMLP_SK_S32>(w2, mx, a, num_sms, st); break;
+        case 64: e = launch_ar_bt<64, TPMLP_SK_S64>(w2, mx, a, num_sms, st); break;
+        default: e = launch_ar_bt<128, TPMLP_SK_S128>(w2, mx, a, num_sms, st); break;
+    }
+    if (e == cudaSuccess) ++*launches;
+    return e;
+}
+
+size_t xgpu_header_bytes(const Problem &p) {
+    return kArControlBytes + align256((size_t)p.tp * blk_tiles(p.d_out) * 8 * 4);
+}
 
 bool tc_supported(const Problem &p) {
     return p.dtype == TP_MLP_BF16 && p.d_in % 8 == 0 && p.d_ff % 8 == 0 && p.d_out % 8 == 0 &&
@@ -999,10 +1670,11 @@ bool tc_supported(const Problem &p) {
 bool tc_raw_supported(const Problem &p) { return tc_supported(p) && p.fs % BK == 0; }
 
 // Counters serve the in-kernel fixup, which only runs 256-row tiles: the first
-// projection's tiles (either layout) then the second's.
+// projection's tiles (either layout) then the second's, then the two chunk
+// counters of the dynamically scheduled GEMV (one per projection).
 size_t tile_counter_slots(const Problem &p) {
     return (size_t)(std::max(skinny_tiles(p, 0, false, false), skinny_tiles(p, 0, true, false)) +
-                    blk_tiles(p.d_out));
+                    blk_tiles(p.d_out)) + 2;
 }
 
 // Split-tile scratch: the largest over both layouts, both projections and both
@@ -1019,22 +1691,30 @@ size_t tc_workspace_bytes(const Problem &p, int num_sms) {
                 const StreamKGeom g = skinny_geom((int)tiles, (int)blk_kblocks(proj ? p.d_ff : p.d_in), BT, num_sms);
                 m = std::max(m, (size_t)g.tiles * g.slots * (half ? 128 : 256) * BT * 4);
             }
+    if (p.fs % BK == 0) {   // per-rank partials: tp x the output tiles, one rank's k-blocks each
+        const long long tiles = p.tp * skinny_tiles(p, 1, true, false);
+        const StreamKGeom g = skinny_geom((int)tiles, p.fs / BK, BT, num_sms);
+        m = std::max(m, (size_t)g.tiles * g.slots * 256 * BT * 4);
+    }
     return align256(m);
 }
 
 cudaError_t launch_tc(const Problem &p, int tiling, const void *x, const void *w1p, const void *w2p,
                       const ShardPtrs *rawA, const ShardPtrs *rawB, void *h, void *out, float *part,
                       unsigned *counters, int *status, int num_sms, cudaStream_t st, const Marks &marks,
-                      int split_mode, int *launches) {
+                      int split_mode, int *launches, float *partials) {
     *launches = 0;
     WeightOperand w1, w2;
     const bool raw = rawA != nullptr;
+    if (partials && !raw) return cudaErrorInvalidValue;   // per-rank partials come from the shard form
     const bool skinny = tiling == kTilingSkinny;
     const int BT = skinny_bt(p.T);
     const bool half1 = skinny && skinny_half(0, p.act, BT, split_mode, raw);
     const bool half2 = skinny && skinny_half(1, p.act, BT, split_mode, raw);
+    const int epi2 = partials ? EPI_PART : EPI_OUT;
+    void *out2 = partials ? static_cast<void *>(partials) : out;
     if (raw) {
-        if (!weight_raw_first(&w1, p, *rawA, half1) || !weight_raw_second(&w2, p, *rawB, half2))
+        if (!weight_raw_first(&w1, p, *rawA, half1) || !weight_raw_second(&w2, p, *rawB, half2, partials != nullptr))
             return cudaErrorInvalidValue;
     } else if (!weight_packed(&w1, p, 0, w1p, half1) || !weight_packed(&w2, p, 1, w2p, half2)) {
         return cudaErrorInvalidValue;
@@ -1048,14 +1728,14 @@ cudaError_t launch_tc(const Problem &p, int tiling, const void *x, const void *w
                        split_mode, launches);
         if (e != cudaSuccess) return e;
         marks.mark(1, st);
-        e = run_skinny(w2, h, p.T, p.d_ff, EPI_OUT, out, p.d_out, part, cnt2, status, num_sms, st, split_mode,
+        e = run_skinny(w2, h, p.T, p.d_ff, epi2, out2, p.d_out, part, cnt2, status, num_sms, st, split_mode,
                        launches);
     } else {
         auto wide = tiling == kTilingWide256 ? run_wide<2> : run_wide<1>;
         e = wide(w1, x, p.T, p.d_in, first_epi(p.act), h, p.d_ff, status, num_sms, st);
         if (e != cudaSuccess) return e;
         marks.mark(1, st);
-        e = wide(w2, h, p.T, p.d_ff, EPI_OUT, out, p.d_out, status, num_sms, st);
+        e = wide(w2, h, p.T, p.d_ff, epi2, out2, p.d_out, status, num_sms, st);
         *launches = 2;
     }
     marks.mark(2, st);

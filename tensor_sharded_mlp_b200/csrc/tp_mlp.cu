@@ -67,28 +67,24 @@ struct tp_mlp_s {
     size_t tc_part[4];
 };
 
-namespace {
+namespace tpmlp {
 
 typedef CUresult (*PFN_getAddressRange)(CUdeviceptr *, size_t *, CUdeviceptr);
 
-PFN_getAddressRange address_range_fn() {
+static PFN_getAddressRange address_range_fn() {
     static PFN_getAddressRange fn = nullptr;
-    static bool tried = false;
-    if (!tried) {
-        tried = true;
+    static std::once_flag once;
+    std::call_once(once, [] {
         void *p = nullptr;
         cudaDriverEntryPointQueryResult q;
         if (cudaGetDriverEntryPointByVersion("cuMemGetAddressRange", &p, 12000, cudaEnableDefault, &q) ==
                 cudaSuccess &&
             q == cudaDriverEntryPointSuccess)
             fn = reinterpret_cast<PFN_getAddressRange>(p);
-    }
+    });
     return fn;
 }
 
-size_t elem_bytes(int dtype) { return dtype == TP_MLP_F32 ? 4 : 2; }
-
-// A device pointer, 16-byte aligned, inside an allocation holding `bytes` from it.
 int check_dev(const void *p, size_t bytes) {
     if (!p) return TP_MLP_ERR_INVALID_ARG;
     if (reinterpret_cast<uintptr_t>(p) & 15u) return TP_MLP_ERR_ALIGNMENT;
@@ -101,6 +97,12 @@ int check_dev(const void *p, size_t bytes) {
     if (reinterpret_cast<uintptr_t>(p) + bytes > base + size) return TP_MLP_ERR_SHAPE;
     return TP_MLP_OK;
 }
+
+}  // namespace tpmlp
+
+namespace {
+
+size_t elem_bytes(int dtype) { return dtype == TP_MLP_F32 ? 4 : 2; }
 
 Problem problem_of(const tp_mlp_s *h, int tokens) {
     Problem p;
@@ -258,7 +260,10 @@ int tp_mlp_set_workspace(tp_mlp_t h, void *dev_ptr, size_t bytes) {
     if (bytes < need_bytes(h, 0)) return TP_MLP_ERR_WORKSPACE;
     int s = check_dev(dev_ptr, bytes);
     if (s) return s;
-    if (cudaMemset(dev_ptr, 0, counters_bytes(h)) != cudaSuccess) return TP_MLP_ERR_CUDA;
+    // the memset runs on the legacy stream: wait for it, so that a forward on
+    // any stream sees zeroed counters
+    if (cudaMemset(dev_ptr, 0, counters_bytes(h)) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess)
+        return TP_MLP_ERR_CUDA;
     h->ws = dev_ptr;
     h->ws_bytes = bytes;
     return TP_MLP_OK;
@@ -270,10 +275,10 @@ static int run_shard_form(tp_mlp_t h, const void *x, int tokens, const void *con
     int s = check_common(h, x, tokens, tp_degree, act);
     if (s) return s;
     Problem p = problem_of(h, tokens);
-    // The forward reads the shards straight into the tcgen05 kernels when the
-    // shape allows (bf16, f_s % 64 == 0); the partials call and other shapes use
-    // the CUDA-core kernels.  The GEMV needs the packed layout.
-    const bool tc_ok = !partials && tc_raw_supported(p);
+    // The forward and the partials read the shards straight into the tcgen05
+    // kernels when the shape allows (bf16, f_s % 64 == 0); other shapes use the
+    // CUDA-core kernels.  The GEMV needs the packed layout.
+    const bool tc_ok = tc_raw_supported(p);
     int plan = h->plan;
     if (plan == TP_MLP_PLAN_AUTO) plan = tc_ok ? TP_MLP_PLAN_TC : TP_MLP_PLAN_SIMT;
     if (plan == TP_MLP_PLAN_TC)
@@ -308,7 +313,7 @@ static int run_shard_form(tp_mlp_t h, const void *x, int tokens, const void *con
                            : plan == TP_MLP_PLAN_TC_WIDE ? kTilingWide128 : kTilingWide256;
         float *part = reinterpret_cast<float *>(ws + counters_bytes(h) + h_bytes(h, tokens));
         ce = launch_tc(p, tiling, x, nullptr, nullptr, &a, &b, hbuf, out, part, reinterpret_cast<unsigned *>(ws),
-                       status_word(h), h->num_sms, st, h->marks, h->splitk, &launches);
+                       status_word(h), h->num_sms, st, h->marks, h->splitk, &launches, partials);
     } else {
         ce = launch_simt(p, false, x, a, b, hbuf, out, partials, st, h->marks);
     }
@@ -432,8 +437,11 @@ int tp_mlp_get_device_status(tp_mlp_t h) {
     int v = 0;
     if (cudaMemcpy(&v, status_word(h), sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return TP_MLP_ERR_CUDA;
     if (v == 0) return TP_MLP_OK;
-    const int zero = 0;
-    if (cudaMemcpy(status_word(h), &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return TP_MLP_ERR_CUDA;
+    // A kernel gave up a bounded wait: its CTAs left early, so split-tile
+    // counters may be left part-way.  Zero them with the status word, so the
+    // next call starts from the state set_workspace leaves.
+    if (cudaMemset(h->ws, 0, counters_bytes(h)) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess)
+        return TP_MLP_ERR_CUDA;
     return TP_MLP_ERR_TIMEOUT;
 }
 
@@ -492,6 +500,130 @@ int tp_mlp_merge_attention_partials(int tp_degree, int rows, int head_dim, const
     if ((s = check_dev(out, (size_t)rows * head_dim * e))) return s;
     return from_cuda(launch_attn_merge(tp_degree, rows, head_dim, maximum, exp_sum, weighted, dtype, out,
                                        reinterpret_cast<cudaStream_t>(stream)));
+}
+
+// Exchange buffer: [control + flags | receive rows | gathered rows (sequence parallelism)].
+static size_t xgpu_recv_bytes(const tp_mlp_s *h) { return align256(2 * (size_t)h->tp * h->max_tokens * h->d_out * 2); }
+
+size_t tp_mlp_xgpu_comm_bytes(tp_mlp_t h) {
+    if (!h) return 0;
+    const Problem p = problem_of(h, 0);
+    return xgpu_header_bytes(p) + xgpu_recv_bytes(h) + align256((size_t)h->max_tokens * h->d_model * 2);
+}
+
+static int xgpu_common(tp_mlp_t h, bool sp, int rank0, int nranks, const void *const *x, int tokens,
+                       const void *const *A_local, const void *const *B_local, void *const *comm,
+                       void *const *outs, tp_mlp_stream_t stream) {
+    if (!h) return TP_MLP_ERR_INVALID_ARG;
+    Problem p = problem_of(h, tokens);
+    if (h->dtype != TP_MLP_BF16 || !tc_raw_supported(p) || h->d_model % 8) return TP_MLP_ERR_UNSUPPORTED;
+    if (tokens < 0 || tokens > h->max_tokens || tokens > kTcSkinnyMaxTokens) return TP_MLP_ERR_SHAPE;
+    if (sp && tokens % h->tp) return TP_MLP_ERR_SHAPE;
+    if (nranks < 1 || rank0 < 0 || rank0 + nranks > h->tp) return TP_MLP_ERR_SHAPE;
+    if (!x || !A_local || !B_local || !comm || !outs) return TP_MLP_ERR_INVALID_ARG;
+    if (tokens == 0) return TP_MLP_OK;   // launches nothing
+    const size_t fs = (size_t)h->d_ff / h->tp;
+    const size_t lda = h->act == TP_MLP_ACT_SWIGLU ? 2 * fs : fs;
+    const size_t rows_in = sp ? tokens / h->tp : tokens, rows_out = rows_in;
+    int s;
+    for (int i = 0; i < (sp ? nranks : 1); ++i)
+        if ((s = check_dev(x[i], rows_in * h->d_model * 2))) return s;
+    for (int i = 0; i < nranks; ++i) {
+        if ((s = check_dev(A_local[i], (size_t)h->d_model * lda * 2))) return s;
+        if ((s = check_dev(B_local[i], fs * h->d_out * 2))) return s;
+        if ((s = check_dev(outs[i], rows_out * h->d_out * 2))) return s;
+    }
+    const size_t cb = tp_mlp_xgpu_comm_bytes(h);
+    for (int r = 0; r < h->tp; ++r) {
+        if (!comm[r]) return TP_MLP_ERR_INVALID_ARG;
+        if (reinterpret_cast<uintptr_t>(comm[r]) & 15u) return TP_MLP_ERR_ALIGNMENT;
+        // local buffers are checked in full; a peer's may be a mapping of another GPU's memory
+        if (r >= rank0 && r < rank0 + nranks && (s = check_dev(comm[r], cb))) return s;
+    }
+    Problem pl = p;
+    pl.tp = nranks;
+    pl.d_ff = nranks * p.fs;
+    const size_t hb = align256((size_t)tokens * pl.d_ff * 2);
+    const size_t need = counters_bytes(h) + hb + tc_workspace_bytes(pl, h->num_sms);
+    if (!h->ws || h->ws_bytes < need) return TP_MLP_ERR_WORKSPACE;
+    char *ws = static_cast<char *>(h->ws);
+    XgpuArgs xa;
+    memset(&xa, 0, sizeof(xa));
+    for (int r = 0; r < h->tp; ++r) xa.comm[r] = comm[r];
+    for (int i = 0; i < nranks; ++i) xa.outs[i] = outs[i];
+    xa.recv_off = xgpu_header_bytes(p);
+    xa.rows = h->max_tokens;
+    const ShardPtrs a = to_ptrs(A_local, nranks), b = to_ptrs(B_local, nranks);
+    void *hbuf = ws + counters_bytes(h);
+    float *part = reinterpret_cast<float *>(ws + counters_bytes(h) + hb);
+    unsigned *cnt = reinterpret_cast<unsigned *>(ws);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    int launches = 0;
+    const cudaError_t ce =
+        sp ? launch_xgpu_sp(p, rank0, nranks, x, a, b, hbuf, part, cnt, status_word(h), h->num_sms, st, xa,
+                            xa.recv_off + xgpu_recv_bytes(h), &launches)
+           : launch_xgpu(p, rank0, nranks, x[0], a, b, hbuf, part, cnt, status_word(h), h->num_sms, st, xa,
+                         &launches);
+    if (ce == cudaErrorNotSupported) {
+        cudaGetLastError();
+        return TP_MLP_ERR_UNSUPPORTED;
+    }
+    if (ce != cudaSuccess) return TP_MLP_ERR_CUDA;
+    h->last_plan = TP_MLP_PLAN_TC_SKINNY;
+    h->last_launches = launches;
+    return TP_MLP_OK;
+}
+
+int tp_mlp_xgpu_forward(tp_mlp_t h, int rank0, int nranks, const void *x, int tokens,
+                        const void *const *A_local, const void *const *B_local, void *const *comm,
+                        void *const *outs, tp_mlp_stream_t stream) {
+    const void *xs[1] = {x};
+    return xgpu_common(h, false, rank0, nranks, x ? xs : nullptr, tokens, A_local, B_local, comm, outs, stream);
+}
+
+int tp_mlp_xgpu_sp_forward(tp_mlp_t h, int rank0, int nranks, const void *const *x_local, int tokens,
+                           const void *const *A_local, const void *const *B_local, void *const *comm,
+                           void *const *outs, tp_mlp_stream_t stream) {
+    return xgpu_common(h, true, rank0, nranks, x_local, tokens, A_local, B_local, comm, outs, stream);
+}
+
+int tp_mlp_ipc_get_handle(const void *dev_ptr, void *handle, size_t *offset) {
+    if (!dev_ptr || !handle || !offset) return TP_MLP_ERR_INVALID_ARG;
+    PFN_getAddressRange fn = address_range_fn();
+    if (!fn) return TP_MLP_ERR_CUDA;
+    CUdeviceptr base = 0;
+    size_t size = 0;
+    if (fn(&base, &size, reinterpret_cast<CUdeviceptr>(dev_ptr)) != CUDA_SUCCESS) return TP_MLP_ERR_INVALID_ARG;
+    cudaIpcMemHandle_t hd;
+    if (cudaIpcGetMemHandle(&hd, reinterpret_cast<void *>(base)) != cudaSuccess) {
+        cudaGetLastError();
+        return TP_MLP_ERR_CUDA;
+    }
+    memcpy(handle, &hd, sizeof(hd));
+    *offset = reinterpret_cast<uintptr_t>(dev_ptr) - (uintptr_t)base;
+    return TP_MLP_OK;
+}
+
+int tp_mlp_ipc_open_handle(const void *handle, size_t offset, void **dev_ptr) {
+    if (!handle || !dev_ptr) return TP_MLP_ERR_INVALID_ARG;
+    cudaIpcMemHandle_t hd;
+    memcpy(&hd, handle, sizeof(hd));
+    void *base = nullptr;
+    if (cudaIpcOpenMemHandle(&base, hd, cudaIpcMemLazyEnablePeerAccess) != cudaSuccess) {
+        cudaGetLastError();
+        return TP_MLP_ERR_CUDA;
+    }
+    *dev_ptr = static_cast<char *>(base) + offset;
+    return TP_MLP_OK;
+}
+
+int tp_mlp_ipc_close_handle(void *dev_ptr, size_t offset) {
+    if (!dev_ptr) return TP_MLP_ERR_INVALID_ARG;
+    if (cudaIpcCloseMemHandle(static_cast<char *>(dev_ptr) - offset) != cudaSuccess) {
+        cudaGetLastError();
+        return TP_MLP_ERR_CUDA;
+    }
+    return TP_MLP_OK;
 }
 
 int tp_mlp_set_splitk(tp_mlp_t h, int mode) {

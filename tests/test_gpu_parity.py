@@ -217,13 +217,21 @@ def test_decode_configs_full_size(name):
     c = inputs.CONFIGS[name]
     p = inputs.generate_config(name)
     Ad, Bd, A, Bs = _upload(p, c["tp"], "bf16")
-    ref = oracle.tp_mlp_sharded(p.x, A, Bs, "swiglu")
+    ref, parts = oracle.tp_mlp_sharded(p.x, A, Bs, "swiglu", return_partials=True)
     m = _mlp(p, c["tp"], "bf16", max_tokens=32)
     x = dev(p.x, "bf16")
     packed = m.pack(Ad, Bd)
     del A, Bs
     assert_close(m.forward_packed(x, packed), ref, "bf16", f"{name} packed/{m.last_plan}")
-    assert_close(m.forward(x, Ad, Bd), ref, "bf16", f"{name} shard form")
+    out = m.forward(x, Ad, Bd)
+    assert_close(out, ref, "bf16", f"{name} shard form")
+    # the per-rank partials (tensor cores, each rank's K loop apart) and their sum
+    gp = m.partials(x, Ad, Bd)
+    assert m.last_plan == "tc_skinny"
+    for i in range(c["tp"]):
+        assert_close(gp[i], parts[i], "bf16", f"{name} partial {i}")
+    assert_close(gp.sum(0), ref, "bf16", f"{name} sum of partials")
+    assert_close(out, gp.sum(0).cpu().numpy(), "bf16", f"{name} forward vs sum of partials")
 
 
 @pytest.mark.slow
@@ -257,8 +265,19 @@ def test_prefill_config_sampled_rows():
         if ref is None:
             ref = oracle.tp_mlp_sharded(p.x[rows], A, Bs, "swiglu")
         m = _mlp(p, tp, "bf16", max_tokens=p.tokens)
-        out = m.forward_packed(dev(p.x, "bf16"), m.pack(Ad, Bd))
-        assert_close(out[torch.from_numpy(rows).cuda()], ref, "bf16", f"prefill tp={tp}/{m.last_plan}")
+        x = dev(p.x, "bf16")
+        out = m.forward_packed(x, m.pack(Ad, Bd))
+        r = torch.from_numpy(rows).cuda()
+        assert_close(out[r], ref, "bf16", f"prefill tp={tp}/{m.last_plan}")
+        if tp == 8:
+            # per-rank partials of all 8192 rows (fp32, 2 GiB), checked on the sample
+            _, parts = oracle.tp_mlp_sharded(p.x[rows], A, Bs, "swiglu", return_partials=True)
+            gp = m.partials(x, Ad, Bd)
+            assert m.last_plan == "tc_wide256"
+            for i in range(tp):
+                assert_close(gp[i][r], parts[i], "bf16", f"prefill partial {i}")
+            assert_close(gp.sum(0)[r], ref, "bf16", "prefill sum of partials")
+            del gp
         del Ad, Bd, m, out
         torch.cuda.empty_cache()
 

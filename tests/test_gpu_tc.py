@@ -266,6 +266,112 @@ def test_tc_shard_form_integer_exact(plan, T):
     assert np.array_equal(out.float().cpu().numpy(), inputs.round_to_bf16(ref.astype(np.float32)))
 
 
+# --- per-rank partials on the tensor cores (each rank's K loop kept apart) ---
+
+@pytest.mark.parametrize("act", ["swiglu", "tanh"])
+@pytest.mark.parametrize("plan,T", [("tc_skinny", 1), ("tc_skinny", 5), ("tc_skinny", 33), ("tc_skinny", 128),
+                                    ("tc_wide", 129), ("tc_wide", 300), ("tc_wide256", 300), ("auto", 7)])
+@pytest.mark.parametrize("shape", RAW_SHAPES)
+def test_tc_partials_parity(act, plan, T, shape):
+    """Each rank's fp32 partial Z_i = act(X A_i) B_i against the oracle's, and
+    their sum against the oracle's output and the forward on the same plan."""
+    d, f, dout, tp = shape
+    p = inputs.generate(T, d, f, act, "bf16", seed=T + 5 * f + dout, init="fan_in", d_out=dout)
+    A, Bs = p.shards(tp)
+    Ad, Bd = [dev(a, "bf16") for a in A], [dev(b, "bf16") for b in Bs]
+    m = B().TpMlp(d, f, tp, act, "bf16", T, d_out=dout)
+    m.set_plan(plan)
+    x = dev(p.x, "bf16")
+    gp = m.partials(x, Ad, Bd)
+    torch.cuda.synchronize()
+    B().tp_mlp_get_device_status(m.h)
+    assert m.last_plan == (plan if plan != "auto" else "tc_skinny")
+    assert gp.dtype == torch.float32 and gp.shape == (tp, T, dout)
+    rows = p.sample_rows(64)
+    ref, parts = oracle.tp_mlp_sharded(p.x[rows], A, Bs, act, return_partials=True)
+    r = torch.from_numpy(rows).cuda()
+    for i in range(tp):
+        assert_close(gp[i][r], parts[i], "bf16", f"partial {i} {plan} T={T}")
+    total = gp.sum(0)
+    assert_close(total[r], ref, "bf16", f"sum of partials {plan} T={T}")
+    out = m.forward(x, Ad, Bd)
+    assert_close(out, total.cpu().numpy(), "bf16", f"forward vs sum of partials {plan} T={T}")
+
+
+@pytest.mark.parametrize("plan,T", [("tc_skinny", 3), ("tc_skinny", 100), ("tc_wide", 130), ("tc_wide256", 257)])
+def test_tc_partials_integer_exact(plan, T):
+    """Small integers: every partial is exact in fp32, so each equals the
+    oracle's partial bit for bit (split tiles included: the sums stay exact)."""
+    p = inputs.integer_inputs(T, 64, 4 * 256, 264, "identity", seed=T + 2, lo=-1, hi=1)
+    A, Bs = p.shards(4)
+    m = B().TpMlp(64, 4 * 256, 4, "identity", "bf16", T, d_out=264)
+    m.set_plan(plan)
+    gp = m.partials(dev(p.x, "bf16"), [dev(a, "bf16") for a in A], [dev(b, "bf16") for b in Bs])
+    torch.cuda.synchronize()
+    assert m.last_plan == plan
+    _, parts = oracle.tp_mlp_sharded(p.x, A, Bs, "identity", return_partials=True)
+    assert np.array_equal(gp.cpu().numpy().astype(np.float64), np.asarray(parts))
+
+
+# --- split tiles added across a thread-block cluster (distributed shared memory) ---
+
+@pytest.mark.parametrize("act", ["tanh", "swiglu"])
+@pytest.mark.parametrize("T", [5, 16, 33, 100, 128])
+def test_tc_skinny_cluster_route_matches_reduction_kernel(act, T):
+    """32 weight tiles per projection on 148 SMs: 4 CTAs share each tile.  The
+    default route adds their slots across a cluster of 4 (two launches, no
+    reduction kernel); it must give the reduction kernel's bits."""
+    d, f, dout, tp = 512, 4096, 4096, 4
+    p = inputs.generate(T, d, f, act, "bf16", seed=T + 17, init="fan_in", d_out=dout)
+    A, Bs = p.shards(tp)
+    Ad, Bd = [dev(a, "bf16") for a in A], [dev(b, "bf16") for b in Bs]
+    m = B().TpMlp(d, f, tp, act, "bf16", T, d_out=dout)
+    m.set_plan("tc_skinny")
+    packed = m.pack(Ad, Bd)
+    x = dev(p.x, "bf16")
+    outs, launches = {}, {}
+    for mode in ("auto", "separate"):
+        m.set_splitk(mode)
+        outs[mode] = m.forward_packed(x, packed)
+        torch.cuda.synchronize()
+        B().tp_mlp_get_device_status(m.h)
+        launches[mode] = m.last_launches
+    assert launches["auto"] < launches["separate"], launches
+    assert torch.equal(outs["auto"], outs["separate"])
+    rows = p.sample_rows(32)
+    assert_close(outs["auto"][torch.from_numpy(rows).cuda()], oracle.tp_mlp_sharded(p.x[rows], A, Bs, act),
+                 "bf16", f"cluster route T={T}")
+
+
+@pytest.mark.parametrize("T", [3, 64])
+def test_tc_cluster_route_shard_form_and_partials(T):
+    """The shard form (256-row tiles) and the per-rank partials take the cluster
+    route too: 32 tiles on 148 SMs.  Same bits as the reduction kernel."""
+    d, f, dout, tp = 256, 2048, 8192, 2
+    p = inputs.generate(T, d, f, "swiglu", "bf16", seed=T + 29, init="fan_in", d_out=dout)
+    A, Bs = p.shards(tp)
+    Ad, Bd = [dev(a, "bf16") for a in A], [dev(b, "bf16") for b in Bs]
+    m = B().TpMlp(d, f, tp, "swiglu", "bf16", T, d_out=dout)
+    m.set_plan("tc_skinny")
+    x = dev(p.x, "bf16")
+    res = {}
+    for mode in ("auto", "separate"):
+        m.set_splitk(mode)
+        out = m.forward(x, Ad, Bd)
+        n_fwd = m.last_launches
+        parts = m.partials(x, Ad, Bd)
+        torch.cuda.synchronize()
+        B().tp_mlp_get_device_status(m.h)
+        res[mode] = (out, parts, n_fwd, m.last_launches)
+    assert torch.equal(res["auto"][0], res["separate"][0])
+    assert torch.equal(res["auto"][1], res["separate"][1])
+    assert res["auto"][2] < res["separate"][2] and res["auto"][3] < res["separate"][3]
+    ref, parts = oracle.tp_mlp_sharded(p.x, A, Bs, "swiglu", return_partials=True)
+    assert_close(res["auto"][0], ref, "bf16", "cluster route, shard form")
+    for i in range(tp):
+        assert_close(res["auto"][1][i], parts[i], "bf16", f"cluster route, partial {i}")
+
+
 def test_shard_form_falls_back_when_ranks_are_not_64_aligned():
     p = inputs.generate(4, 128, 8 * 40, "tanh", "bf16", seed=1)     # f_s = 40
     m, out, A, Bs = _run_shard_form(p, 8, "auto")
