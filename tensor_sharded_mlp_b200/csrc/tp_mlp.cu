@@ -520,8 +520,8 @@ static int xgpu_common(tp_mlp_t h, bool sp, int rank0, int nranks, const void *c
     if (tokens < 0 || tokens > h->max_tokens || tokens > kTcSkinnyMaxTokens) return TP_MLP_ERR_SHAPE;
     if (sp && tokens % h->tp) return TP_MLP_ERR_SHAPE;
     if (nranks < 1 || rank0 < 0 || rank0 + nranks > h->tp) return TP_MLP_ERR_SHAPE;
+    if (tokens == 0) return TP_MLP_OK;   // launches nothing (empty tensors may carry null pointers)
     if (!x || !A_local || !B_local || !comm || !outs) return TP_MLP_ERR_INVALID_ARG;
-    if (tokens == 0) return TP_MLP_OK;   // launches nothing
     const size_t fs = (size_t)h->d_ff / h->tp;
     const size_t lda = h->act == TP_MLP_ACT_SWIGLU ? 2 * fs : fs;
     const size_t rows_in = sp ? tokens / h->tp : tokens, rows_out = rows_in;
@@ -578,7 +578,7 @@ int tp_mlp_xgpu_forward(tp_mlp_t h, int rank0, int nranks, const void *x, int to
                         const void *const *A_local, const void *const *B_local, void *const *comm,
                         void *const *outs, tp_mlp_stream_t stream) {
     const void *xs[1] = {x};
-    return xgpu_common(h, false, rank0, nranks, x ? xs : nullptr, tokens, A_local, B_local, comm, outs, stream);
+    return xgpu_common(h, false, rank0, nranks, xs, tokens, A_local, B_local, comm, outs, stream);
 }
 
 int tp_mlp_xgpu_sp_forward(tp_mlp_t h, int rank0, int nranks, const void *const *x_local, int tokens,
