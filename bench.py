@@ -4,7 +4,7 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--config decode_bs1|decode_bs32|prefill|sweep|tiny] [--tokens T] [--tp P]
                     [--plan auto|simt|gemv|tc|tc_skinny|tc_wide|tc_wide256] [--api packed|shard]
-                    [--splitk auto|in_kernel|separate] [--no-e2e] [--no-cpu-baseline] [--no-graph]
+                    [--splitk auto|in_kernel|separate|cluster] [--no-e2e] [--no-cpu-baseline] [--no-graph]
                     [--configs auto|all|none]
     python bench.py --config fused_norm_decode_bs32|fused_norm_prefill|
                              attn_merge_decode_bs32|attn_merge_decode_bs256 [...]
@@ -66,7 +66,7 @@ def parse():
     ap.add_argument("--tokens", type=int, default=None)
     ap.add_argument("--tp", type=int, default=None)
     ap.add_argument("--plan", default="auto")
-    ap.add_argument("--splitk", choices=["auto", "in_kernel", "separate"], default="auto",
+    ap.add_argument("--splitk", choices=["auto", "in_kernel", "separate", "cluster"], default="auto",
                     help="how the skinny tensor-core tiling finishes split tiles")
     ap.add_argument("--d-model", type=int, default=None, help="override (small cases for profiling)")
     ap.add_argument("--d-ff", type=int, default=None, help="override (small cases for profiling)")

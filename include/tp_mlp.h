@@ -224,13 +224,15 @@ int tp_mlp_set_plan(tp_mlp_t handle, int plan);
  * the same fixed order, so they give identical results; they differ in speed.
  */
 typedef enum {
-    TP_MLP_SPLITK_AUTO = 0,      /* default: where a whole number (2..8) of CTAs share
-                                    each tile and all fit at once, those CTAs form a
-                                    thread-block cluster and add their slots through
-                                    distributed shared memory; otherwise as SEPARATE */
+    TP_MLP_SPLITK_AUTO = 0,      /* default: SEPARATE (measured fastest on B200)       */
     TP_MLP_SPLITK_IN_KERNEL = 1, /* the last CTA to finish its share adds the slots   */
-    TP_MLP_SPLITK_SEPARATE = 2   /* a reduction kernel behind each GEMM adds them,
+    TP_MLP_SPLITK_SEPARATE = 2,  /* a reduction kernel behind each GEMM adds them,
                                     spread over the whole GPU                        */
+    TP_MLP_SPLITK_CLUSTER = 3    /* where a whole number (2..8) of CTAs share each
+                                    tile and all fit at once, those CTAs form a
+                                    thread-block cluster and add their slots through
+                                    distributed shared memory at the end of the GEMM;
+                                    otherwise as SEPARATE                            */
 } tp_mlp_splitk;
 
 /* Choose the split-tile finish (tp_mlp_splitk) for later forwards.  Returns

@@ -173,7 +173,7 @@ def tp_mlp_set_plan(h, plan: str) -> None:
     _check("tp_mlp_set_plan", _lib.tp_mlp_set_plan(h, PLAN[plan]))
 
 
-SPLITK = {"auto": 0, "in_kernel": 1, "separate": 2}
+SPLITK = {"auto": 0, "in_kernel": 1, "separate": 2, "cluster": 3}
 
 
 def tp_mlp_set_splitk(h, mode: str) -> None:

@@ -48,14 +48,8 @@ struct GemvArgs {
     int out_cols;             // d_ff (H) or d_out
     __nv_bfloat16 *out;       // T x out_cols
     float *part;              // [tile][slot][T][256] fp32
-    unsigned *tile_cnt;       // k-blocks (static) or chunks (dynamic) done per tile, zero between launches
+    unsigned *tile_cnt;       // k-blocks done per tile, zero between launches
     int *status;
-    // dynamic assignment: the weight stream is cut into chunks of `chunk`
-    // k-blocks of one tile (cpt chunks per tile, the last one may be shorter),
-    // handed out in order from *chunk_ctr; n_chunks = tiles * cpt
-    unsigned *chunk_ctr;
-    int chunk, cpt;
-    unsigned n_chunks;
 };
 
 struct GemvSmem {
@@ -64,7 +58,6 @@ struct GemvSmem {
     float *rowsum;            // [T][256]
     volatile int *abort;
     int *flag;
-    int *info;                // dynamic assignment: what each stage holds (see gemv_dyn_kernel)
 };
 
 template <int T>
@@ -77,13 +70,12 @@ __device__ __forceinline__ GemvSmem gemv_carve(uint8_t *raw) {
     s.rowsum = reinterpret_cast<float *>(s.empty + STAGES);
     s.abort = reinterpret_cast<volatile int *>(s.rowsum + T * kTileRows);
     s.flag = const_cast<int *>(s.abort) + 1;
-    s.info = s.flag + 1;
     return s;
 }
 
 template <int T>
 constexpr size_t gemv_smem_bytes() {
-    return 128 + STAGES * (size_t)BLK_BYTES + 2 * STAGES * 8 + T * kTileRows * 4 + 16 + STAGES * 4;
+    return 128 + STAGES * (size_t)BLK_BYTES + 2 * STAGES * 8 + T * kTileRows * 4 + 16;
 }
 
 // Final value of row `row` of tile `tile` for all tokens, from s.rowsum.
@@ -264,275 +256,31 @@ __global__ void __launch_bounds__(NTHR, 1) gemv_kernel(GemvArgs a) {
     __syncthreads();
 }
 
-// The same GEMV with the weight stream handed out dynamically.  Equal static
-// shares finish far apart on B200 (some SMs draw more bandwidth than others),
-// and the step waits for the slowest; here every CTA takes the next chunk of
-// `chunk` k-blocks of one tile from a global counter until none is left, so
-// faster SMs simply take more chunks.  Each chunk's fp32 row sums go to its
-// own slot [tile][chunk of tile][T][256]; the CTA that completes a tile's last
-// chunk (one counter per tile) adds the tile's slots in chunk order -- a fixed
-// order, so results do not depend on which CTA took what -- and applies the
-// epilogue.  Nobody waits on another CTA.
-//
-// The producer tells the consumers what a stage holds in info[stage]:
-// (chunk << 8) | (block within chunk << 1) | (last block of chunk), or -1 once
-// the counter is exhausted.  The counter reaches n_chunks + gridDim.x (every CTA
-// ends with one failed grab); the CTA whose failed grab is the very last puts
-// it back to zero for the next launch.
-template <int T>
-__global__ void __launch_bounds__(NTHR, 1) gemv_dyn_kernel(GemvArgs a) {
-    extern __shared__ uint8_t smem_raw[];
-    const GemvSmem s = gemv_carve<T>(smem_raw);
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (threadIdx.x == 0) {
-        for (int i = 0; i < STAGES; ++i) {
-            mbar_init(smem_u32(&s.full[i]), 1);
-            mbar_init(smem_u32(&s.empty[i]), CWARPS);
-        }
-        *s.abort = 0;
-        fence_barrier_init();
-    }
-    __syncthreads();
-    pdl_allow_dependents();
-    const int KB = a.KB;
-
-    if (warp == CWARPS) {
-        // producer: weights do not depend on the previous kernel, so start at once
-        if (lane == 0) {
-            int stage = 0;
-            uint32_t phase = 0;
-            unsigned cur = atomicAdd(a.chunk_ctr, 1u);
-            while (true) {
-                if (cur >= a.n_chunks) {
-                    if (mbar_wait(smem_u32(&s.empty[stage]), phase ^ 1, s.abort)) {
-                        s.info[stage] = -1;
-                        mbar_arrive(smem_u32(&s.full[stage]));   // completes the phase with no bytes
-                    }
-                    if (cur == a.n_chunks + gridDim.x - 1) atomicExch(a.chunk_ctr, 0u);
-                    break;
-                }
-                const unsigned nxt = atomicAdd(a.chunk_ctr, 1u);   // in flight while this chunk streams
-                const int tile = (int)(cur / (unsigned)a.cpt), ci = (int)(cur - (unsigned)tile * a.cpt);
-                const int kb0 = ci * a.chunk, nb = min(a.chunk, KB - kb0);
-                const uint8_t *src = reinterpret_cast<const uint8_t *>(a.w) +
-                                     ((long long)tile * KB + kb0) * (long long)BLK_BYTES;
-                bool ok = true;
-                for (int b = 0; b < nb; ++b) {
-                    if (!mbar_wait(smem_u32(&s.empty[stage]), phase ^ 1, s.abort)) { ok = false; break; }
-                    s.info[stage] = (int)((cur << 8) | ((unsigned)b << 1) | (b == nb - 1 ? 1u : 0u));
-                    const uint32_t fb = smem_u32(&s.full[stage]);
-                    mbar_arrive_expect_tx(fb, BLK_BYTES);
-                    bulk_load(smem_u32(s.ring + stage * BLK_BYTES), src, BLK_BYTES, fb);
-                    src += BLK_BYTES;
-                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
-                }
-                if (!ok) break;
-                cur = nxt;
-            }
-        }
-    } else {
-        pdl_wait_previous();   // X and the outputs belong to the previous kernel until it is done
-        const int g = lane & 7;                         // granule (8 k) of the row
-        const int rbase = warp * 32 + (lane >> 3);      // rows rbase + 4j, j = 0..7
-        int stage = 0;
-        uint32_t phase = 0;
-        float acc[8][T];
-        while (true) {
-            if (!mbar_wait(smem_u32(&s.full[stage]), phase, s.abort)) break;
-            const int info = s.info[stage];
-            if (info < 0) break;
-            const unsigned chunk = (unsigned)info >> 8;
-            const int b = (info >> 1) & 127, last = info & 1;
-            const int tile = (int)(chunk / (unsigned)a.cpt), ci = (int)(chunk - (unsigned)tile * a.cpt);
-            const int kb = ci * a.chunk + b;
-            if (b == 0) {
-#pragma unroll
-                for (int j = 0; j < 8; ++j)
-#pragma unroll
-                    for (int t = 0; t < T; ++t) acc[j][t] = 0.f;
-            }
-            float xv[T][8];
-            const int k = kb * kKBlock + g * 8;
-#pragma unroll
-            for (int t = 0; t < T; ++t) {
-                if (k < a.K) {   // K is a multiple of 8: a granule is all in or all out
-                    const uint4 w4 = __ldg(reinterpret_cast<const uint4 *>(a.x + (long)t * a.K + k));
-                    xv[t][0] = bf16lo(w4.x); xv[t][1] = bf16hi(w4.x);
-                    xv[t][2] = bf16lo(w4.y); xv[t][3] = bf16hi(w4.y);
-                    xv[t][4] = bf16lo(w4.z); xv[t][5] = bf16hi(w4.z);
-                    xv[t][6] = bf16lo(w4.w); xv[t][7] = bf16hi(w4.w);
-                } else {
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) xv[t][i] = 0.f;
-                }
-            }
-            const uint4 *blk = reinterpret_cast<const uint4 *>(s.ring + stage * BLK_BYTES);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const uint4 wv = blk[(rbase + 4 * j) * 8 + g];
-                const float w0 = bf16lo(wv.x), w1 = bf16hi(wv.x), w2 = bf16lo(wv.y), w3 = bf16hi(wv.y);
-                const float w4 = bf16lo(wv.z), w5 = bf16hi(wv.z), w6 = bf16lo(wv.w), w7 = bf16hi(wv.w);
-#pragma unroll
-                for (int t = 0; t < T; ++t) {
-                    float v = acc[j][t];
-                    v = fmaf(w0, xv[t][0], v); v = fmaf(w1, xv[t][1], v);
-                    v = fmaf(w2, xv[t][2], v); v = fmaf(w3, xv[t][3], v);
-                    v = fmaf(w4, xv[t][4], v); v = fmaf(w5, xv[t][5], v);
-                    v = fmaf(w6, xv[t][6], v); v = fmaf(w7, xv[t][7], v);
-                    acc[j][t] = v;
-                }
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&s.empty[stage]));
-            if (++stage == STAGES) { stage = 0; phase ^= 1; }
-            if (!last) continue;
-            // End of a chunk, warp by warp (no CTA barrier: a warp never waits for
-            // another).  The 8 lanes of a row hold partial sums of its 8 granules.
-#pragma unroll
-            for (int j = 0; j < 8; ++j)
-#pragma unroll
-                for (int t = 0; t < T; ++t) {
-                    float v = acc[j][t];
-                    v += __shfl_xor_sync(0xffffffffu, v, 1);
-                    v += __shfl_xor_sync(0xffffffffu, v, 2);
-                    v += __shfl_xor_sync(0xffffffffu, v, 4);
-                    acc[j][t] = v;
-                }
-            float *mine = a.part + ((long long)tile * a.cpt + ci) * T * kTileRows;
-            if (g == 0) {
-#pragma unroll
-                for (int j = 0; j < 8; ++j)
-#pragma unroll
-                    for (int t = 0; t < T; ++t) mine[t * kTileRows + rbase + 4 * j] = acc[j][t];
-                __threadfence();
-            }
-            __syncwarp();
-            unsigned done = 0;
-            if (lane == 0) done = atomicAdd(&a.tile_cnt[tile], 1u) + 1u;
-            done = __shfl_sync(0xffffffffu, done, 0);
-            if (done == (unsigned)a.cpt * CWARPS) {
-                // this warp completed the tile: add its cpt slots in chunk order
-                // (lane l takes rows l + 32 i) and apply the epilogue
-                __threadfence();
-                const float *tb = a.part + (long long)tile * a.cpt * T * kTileRows;
-                float v[8][T];
-#pragma unroll
-                for (int i = 0; i < 8; ++i)
-#pragma unroll
-                    for (int t = 0; t < T; ++t) v[i][t] = 0.f;
-                for (int c = 0; c < a.cpt; ++c)
-#pragma unroll
-                    for (int i = 0; i < 8; ++i)
-#pragma unroll
-                        for (int t = 0; t < T; ++t)
-                            v[i][t] += __ldcg(tb + ((long long)c * T + t) * kTileRows + lane + 32 * i);
-                if (a.mode == MODE_FIRST && a.act == TP_MLP_ACT_SWIGLU) {
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {   // gate row r = lane + 32 i, its up row r + 128
-                        const int n = tile * kSwigluBlock + lane + 32 * i;
-                        if (n < a.out_cols)
-#pragma unroll
-                            for (int t = 0; t < T; ++t)
-                                a.out[(long)t * a.out_cols + n] = __float2bfloat16_rn(silu_fast(v[i][t]) * v[i + 4][t]);
-                    }
-                } else {
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const int n = tile * kTileRows + lane + 32 * i;
-                        if (n < a.out_cols)
-#pragma unroll
-                            for (int t = 0; t < T; ++t)
-                                a.out[(long)t * a.out_cols + n] = __float2bfloat16_rn(
-                                    a.mode == MODE_FIRST ? activate<true>(a.act, v[i][t], 0.f) : v[i][t]);
-                    }
-                }
-                if (lane == 0) atomicExch(&a.tile_cnt[tile], 0u);
-            }
-        }
-    }
-    if (*s.abort) {
-        // a bounded wait gave up: let bulk copies in flight land before the CTA exits
-        if (threadIdx.x == 0) {
-            const unsigned long long t0 = globaltimer();
-            while (globaltimer() - t0 < 100000ull) {
-            }
-            atomicExch(a.status, 1);
-        }
-    }
-    __syncthreads();
-}
-
 StreamKGeom gemv_geom(long long rows, int K, int num_sms) {
     return streamk_geom(blk_tiles(rows), blk_kblocks(K), num_sms);
 }
 
-// Weight stream handed out dynamically (gemv_dyn_kernel) or in equal static
-// shares (gemv_kernel); chunk = k-blocks per dynamic chunk.
-#ifndef TPMLP_GEMV_DYNAMIC
-#define TPMLP_GEMV_DYNAMIC 0
-#endif
-#ifndef TPMLP_GEMV_CHUNK
-#define TPMLP_GEMV_CHUNK 16
-#endif
-
-struct DynGeom {
-    int tiles, KB, chunk, cpt, grid;
-    unsigned n_chunks;
-};
-
-DynGeom gemv_dyn_geom(long long rows, int K, int num_sms) {
-    DynGeom d;
-    d.tiles = (int)blk_tiles(rows);
-    d.KB = (int)blk_kblocks(K);
-    d.chunk = std::min(TPMLP_GEMV_CHUNK, d.KB);
-    d.cpt = (d.KB + d.chunk - 1) / d.chunk;
-    d.n_chunks = (unsigned)d.tiles * (unsigned)d.cpt;
-    d.grid = (int)std::min<long long>(num_sms, d.n_chunks);
-    return d;
-}
-
 template <int T>
-cudaError_t launch_one(const GemvArgs &a, int grid, cudaStream_t st, bool dyn) {
+cudaError_t launch_one(const GemvArgs &a, int grid, cudaStream_t st) {
     constexpr size_t smem = gemv_smem_bytes<T>();
-    auto kern = dyn ? gemv_dyn_kernel<T> : gemv_kernel<T>;
+    auto kern = gemv_kernel<T>;
     cudaError_t e = ensure_smem_attr(kern, smem);
     if (e != cudaSuccess) return e;
     return launch_pdl(kern, dim3(grid), dim3(NTHR), smem, st, a);
 }
 
-cudaError_t launch_T(int T, const GemvArgs &a, int grid, cudaStream_t st, bool dyn) {
+cudaError_t launch_T(int T, const GemvArgs &a, int grid, cudaStream_t st) {
     switch (T) {
-        case 1: return launch_one<1>(a, grid, st, dyn);
-        case 2: return launch_one<2>(a, grid, st, dyn);
-        case 3: return launch_one<3>(a, grid, st, dyn);
-        case 4: return launch_one<4>(a, grid, st, dyn);
+        case 1: return launch_one<1>(a, grid, st);
+        case 2: return launch_one<2>(a, grid, st);
+        case 3: return launch_one<3>(a, grid, st);
+        case 4: return launch_one<4>(a, grid, st);
     }
     return cudaErrorInvalidValue;
 }
 
 cudaError_t run_part(const void *w, long long rows, int K, const void *x, int T, int mode, int act, void *out,
-                     int out_cols, float *part, unsigned *cnt, unsigned *chunk_ctr, int *status, int num_sms,
-                     cudaStream_t st) {
-    if (TPMLP_GEMV_DYNAMIC) {
-        const DynGeom d = gemv_dyn_geom(rows, K, num_sms);
-        GemvArgs a{};
-        a.w = static_cast<const __nv_bfloat16 *>(w);
-        a.x = static_cast<const __nv_bfloat16 *>(x);
-        a.K = K;
-        a.KB = d.KB;
-        a.mode = mode;
-        a.act = act;
-        a.out_cols = out_cols;
-        a.out = static_cast<__nv_bfloat16 *>(out);
-        a.part = part;
-        a.tile_cnt = cnt;
-        a.status = status;
-        a.chunk_ctr = chunk_ctr;
-        a.chunk = d.chunk;
-        a.cpt = d.cpt;
-        a.n_chunks = d.n_chunks;
-        return launch_T(T, a, d.grid, st, true);
-    }
+                     int out_cols, float *part, unsigned *cnt, int *status, int num_sms, cudaStream_t st) {
     const StreamKGeom g = gemv_geom(rows, K, num_sms);
     GemvArgs a{};
     a.w = static_cast<const __nv_bfloat16 *>(w);
@@ -548,7 +296,7 @@ cudaError_t run_part(const void *w, long long rows, int K, const void *x, int T,
     a.part = part;
     a.tile_cnt = cnt;
     a.status = status;
-    return launch_T(T, a, g.grid, st, false);
+    return launch_T(T, a, g.grid, st);
 }
 
 }  // namespace
@@ -561,12 +309,7 @@ size_t gemv_workspace_bytes(const Problem &p, int num_sms) {
     if (!gemv_supported(p)) return 0;
     const StreamKGeom g1 = gemv_geom(w1p_rows(p.d_ff, p.act), p.d_in, num_sms);
     const StreamKGeom g2 = gemv_geom(p.d_out, p.d_ff, num_sms);
-    size_t m = std::max((size_t)g1.tiles * g1.slots, (size_t)g2.tiles * g2.slots);
-    if (TPMLP_GEMV_DYNAMIC) {   // one slot per chunk
-        const DynGeom d1 = gemv_dyn_geom(w1p_rows(p.d_ff, p.act), p.d_in, num_sms);
-        const DynGeom d2 = gemv_dyn_geom(p.d_out, p.d_ff, num_sms);
-        m = std::max(m, std::max((size_t)d1.tiles * d1.cpt, (size_t)d2.tiles * d2.cpt));
-    }
+    const size_t m = std::max((size_t)g1.tiles * g1.slots, (size_t)g2.tiles * g2.slots);
     return align256(m * p.T * kTileRows * 4);
 }
 
@@ -575,14 +318,12 @@ cudaError_t launch_gemv(const Problem &p, const void *x, const void *w1p, const 
                         const Marks &marks, int *launches) {
     const long long rows1 = w1p_rows(p.d_ff, p.act);
     unsigned *cnt1 = counters, *cnt2 = counters + blk_tiles(rows1);
-    unsigned *chunk_ctr = counters + tile_counter_slots(p) - 2;   // one per projection
     marks.mark(0, st);
-    cudaError_t e = run_part(w1p, rows1, p.d_in, x, p.T, MODE_FIRST, p.act, h, p.d_ff, part, cnt1, chunk_ctr,
-                             status, num_sms, st);
+    cudaError_t e = run_part(w1p, rows1, p.d_in, x, p.T, MODE_FIRST, p.act, h, p.d_ff, part, cnt1, status,
+                             num_sms, st);
     if (e != cudaSuccess) return e;
     marks.mark(1, st);
-    e = run_part(w2p, p.d_out, p.d_ff, h, p.T, MODE_SECOND, p.act, out, p.d_out, part, cnt2, chunk_ctr + 1,
-                 status, num_sms, st);
+    e = run_part(w2p, p.d_out, p.d_ff, h, p.T, MODE_SECOND, p.act, out, p.d_out, part, cnt2, status, num_sms, st);
     marks.mark(2, st);
     if (launches) *launches = 2;
     return e;

@@ -54,8 +54,7 @@ cudaError_t launch_attn_merge(int P, int rows, int D, const float *maximum, cons
                               const void *weighted, int dtype, void *out, cudaStream_t st);
 
 // Split-tile counters the GEMV and tcgen05 skinny kernels need (one per
-// weight tile of both parts; first part's tiles first; then the GEMV's two
-// chunk counters).
+// weight tile of both parts; first part's tiles first).
 size_t tile_counter_slots(const Problem &p);
 
 // gemv.cu: decode path, packed bf16, 1..kGemvMaxTokens tokens.
@@ -75,7 +74,7 @@ bool tc_raw_supported(const Problem &p);   // also needs f_s % 64 == 0
 size_t tc_workspace_bytes(const Problem &p, int num_sms);
 // Split tiles of the skinny tiling (values of tp_mlp_splitk): finished by the
 // last CTA to arrive, inside the GEMM kernel, or by a reduction kernel behind it.
-enum { kSplitAuto = 0, kSplitInKernel = 1, kSplitSeparate = 2 };
+enum { kSplitAuto = 0, kSplitInKernel = 1, kSplitSeparate = 2, kSplitCluster = 3 };
 // Packed weights (w1p/w2p), or the per-rank shards when rawA/rawB are given.
 // *launches receives the number of kernels launched.  partials != nullptr
 // (shard form only): the second projection writes each rank's fp32 partial

@@ -1189,11 +1189,11 @@ bool weight_raw_second(WeightOperand *w, const Problem &p, const ShardPtrs &B, b
 
 int skinny_bt(int T) { return T <= 16 ? 16 : T <= 32 ? 32 : T <= 64 ? 64 : 128; }
 
-// Split tiles of whole-CTA grids added across a thread-block cluster (1) or by
-// skinny_reduce_kernel (0).
-#ifndef TPMLP_SKINNY_CLUSTER
-#define TPMLP_SKINNY_CLUSTER 1
-#endif
+// Split tiles of whole-CTA grids can be added across a thread-block cluster
+// (tp_mlp_splitk CLUSTER).  Measured on B200 it is 0.6-2 us slower per step
+// than skinny_reduce_kernel for the forward (sweep 16-128 tokens, decode batch
+// 32), so AUTO keeps the reduction kernel; the cross-GPU exchange needs the
+// cluster (its units finish inside the kernel).
 
 // Ring depth of the skinny kernel per token width: 128-row tiles (SKH) and
 // 256-row tiles (SK).  Each stage holds one weight block and one X box, so the
@@ -1300,7 +1300,7 @@ cudaError_t launch_skinny_bt(const WeightOperand &w, const CUtensorMap &mx, cons
 // Auto: the reduction kernel.  On B200 it measured faster at every width (16 to
 // 128 tokens: 4-42 % of the step), even where the last-arriver fixup reads only
 // two 32 KB slots, because the fixup sits at the end of the GEMM's critical path.
-int resolve_split(int mode) { return mode == kSplitAuto ? kSplitSeparate : mode; }
+int resolve_split(int mode) { return mode == kSplitAuto || mode == kSplitCluster ? kSplitSeparate : mode; }
 
 // 128-row tiles: never for SwiGLU's first projection (gate and up share a
 // tile), the in-kernel fixup (256-row slots only) or the shard form, whose
@@ -1381,8 +1381,7 @@ cudaError_t run_skinny(const WeightOperand &w, const void *x, int T, int K, int 
     // CTAs of a tile become one cluster and add their partials through
     // distributed shared memory, if all the clusters fit on the GPU at once.
     const int per_tile = g.grid / g.tiles;
-    if (TPMLP_SKINNY_CLUSTER && split_mode == kSplitAuto && g.slots > 1 && g.grid % g.tiles == 0 &&
-        per_tile >= 2 && per_tile <= 8)
+    if (split_mode == kSplitCluster && g.slots > 1 && g.grid % g.tiles == 0 && per_tile >= 2 && per_tile <= 8)
         a.cluster_red = per_tile;
     int cl = 0;
     cudaError_t e;
@@ -1670,11 +1669,10 @@ bool tc_supported(const Problem &p) {
 bool tc_raw_supported(const Problem &p) { return tc_supported(p) && p.fs % BK == 0; }
 
 // Counters serve the in-kernel fixup, which only runs 256-row tiles: the first
-// projection's tiles (either layout) then the second's, then the two chunk
-// counters of the dynamically scheduled GEMV (one per projection).
+// projection's tiles (either layout) then the second's.
 size_t tile_counter_slots(const Problem &p) {
     return (size_t)(std::max(skinny_tiles(p, 0, false, false), skinny_tiles(p, 0, true, false)) +
-                    blk_tiles(p.d_out)) + 2;
+                    blk_tiles(p.d_out));
 }
 
 // Split-tile scratch: the largest over both layouts, both projections and both

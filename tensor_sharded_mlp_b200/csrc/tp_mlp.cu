@@ -628,7 +628,7 @@ int tp_mlp_ipc_close_handle(void *dev_ptr, size_t offset) {
 
 int tp_mlp_set_splitk(tp_mlp_t h, int mode) {
     if (!h) return TP_MLP_ERR_INVALID_ARG;
-    if (mode < TP_MLP_SPLITK_AUTO || mode > TP_MLP_SPLITK_SEPARATE) return TP_MLP_ERR_INVALID_ARG;
+    if (mode < TP_MLP_SPLITK_AUTO || mode > TP_MLP_SPLITK_CLUSTER) return TP_MLP_ERR_INVALID_ARG;
     h->splitk = mode;
     return TP_MLP_OK;
 }

@@ -139,7 +139,7 @@ def test_call_argument_errors_before_any_launch(b):
     assert L.tp_mlp_set_plan(h, 0) == 0
     assert L.tp_mlp_set_workspace(h, ok_ptr, 16) == 7                           # too small
     assert L.tp_mlp_set_profile_events(h, None, 9) == 1
-    assert L.tp_mlp_set_splitk(h, 3) == 1 and L.tp_mlp_set_splitk(h, -1) == 1
+    assert L.tp_mlp_set_splitk(h, 4) == 1 and L.tp_mlp_set_splitk(h, -1) == 1
     assert L.tp_mlp_set_splitk(None, 0) == 1
     # fused all-reduce + residual + RMSNorm: argument checks come before any pointer use
     F = L.tp_mlp_allreduce_residual_rmsnorm
@@ -159,7 +159,7 @@ def test_call_argument_errors_before_any_launch(b):
     assert M(2, 4, 128, None, None, None, 3, None, None) == 1                  # dtype
     assert M(2, 4, 128, None, None, None, 1, None, None) == 1                  # null pointers
     assert M(2, 0, 128, None, None, None, 1, None, None) == 0                  # no rows: no-op
-    for mode in (2, 1, 0):
+    for mode in (3, 2, 1, 0):
         assert L.tp_mlp_set_splitk(h, mode) == 0
     assert L.tp_mlp_last_plan(h) == 1 and L.tp_mlp_last_launches(h) == 0        # the 0-token no-op
     b.tp_mlp_destroy(h)

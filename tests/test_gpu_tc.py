@@ -319,7 +319,7 @@ def test_tc_partials_integer_exact(plan, T):
 @pytest.mark.parametrize("T", [5, 16, 33, 100, 128])
 def test_tc_skinny_cluster_route_matches_reduction_kernel(act, T):
     """32 weight tiles per projection on 148 SMs: 4 CTAs share each tile.  The
-    default route adds their slots across a cluster of 4 (two launches, no
+    cluster route adds their slots across a cluster of 4 (two launches, no
     reduction kernel); it must give the reduction kernel's bits."""
     d, f, dout, tp = 512, 4096, 4096, 4
     p = inputs.generate(T, d, f, act, "bf16", seed=T + 17, init="fan_in", d_out=dout)
@@ -330,16 +330,17 @@ def test_tc_skinny_cluster_route_matches_reduction_kernel(act, T):
     packed = m.pack(Ad, Bd)
     x = dev(p.x, "bf16")
     outs, launches = {}, {}
-    for mode in ("auto", "separate"):
+    for mode in ("cluster", "separate", "auto"):
         m.set_splitk(mode)
         outs[mode] = m.forward_packed(x, packed)
         torch.cuda.synchronize()
         B().tp_mlp_get_device_status(m.h)
         launches[mode] = m.last_launches
-    assert launches["auto"] < launches["separate"], launches
+    assert launches["cluster"] < launches["separate"] == launches["auto"], launches
+    assert torch.equal(outs["cluster"], outs["separate"])
     assert torch.equal(outs["auto"], outs["separate"])
     rows = p.sample_rows(32)
-    assert_close(outs["auto"][torch.from_numpy(rows).cuda()], oracle.tp_mlp_sharded(p.x[rows], A, Bs, act),
+    assert_close(outs["cluster"][torch.from_numpy(rows).cuda()], oracle.tp_mlp_sharded(p.x[rows], A, Bs, act),
                  "bf16", f"cluster route T={T}")
 
 
@@ -355,7 +356,7 @@ def test_tc_cluster_route_shard_form_and_partials(T):
     m.set_plan("tc_skinny")
     x = dev(p.x, "bf16")
     res = {}
-    for mode in ("auto", "separate"):
+    for mode in ("cluster", "separate"):
         m.set_splitk(mode)
         out = m.forward(x, Ad, Bd)
         n_fwd = m.last_launches
@@ -363,13 +364,13 @@ def test_tc_cluster_route_shard_form_and_partials(T):
         torch.cuda.synchronize()
         B().tp_mlp_get_device_status(m.h)
         res[mode] = (out, parts, n_fwd, m.last_launches)
-    assert torch.equal(res["auto"][0], res["separate"][0])
-    assert torch.equal(res["auto"][1], res["separate"][1])
-    assert res["auto"][2] < res["separate"][2] and res["auto"][3] < res["separate"][3]
+    assert torch.equal(res["cluster"][0], res["separate"][0])
+    assert torch.equal(res["cluster"][1], res["separate"][1])
+    assert res["cluster"][2] < res["separate"][2] and res["cluster"][3] < res["separate"][3]
     ref, parts = oracle.tp_mlp_sharded(p.x, A, Bs, "swiglu", return_partials=True)
-    assert_close(res["auto"][0], ref, "bf16", "cluster route, shard form")
+    assert_close(res["cluster"][0], ref, "bf16", "cluster route, shard form")
     for i in range(tp):
-        assert_close(res["auto"][1][i], parts[i], "bf16", f"cluster route, partial {i}")
+        assert_close(res["cluster"][1][i], parts[i], "bf16", f"cluster route, partial {i}")
 
 
 def test_shard_form_falls_back_when_ranks_are_not_64_aligned():
