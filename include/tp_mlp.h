@@ -84,7 +84,10 @@ typedef enum {
                                   rows), 1..128 tokens as N; the weight stream split
                                   evenly over the SMs, or whole CTAs per tile when
                                   tiles are few                                       */
-    TP_MLP_PLAN_TC_WIDE256 = 6 /* tcgen05, tiles of 256 tokens x 256 weight rows      */
+    TP_MLP_PLAN_TC_WIDE256 = 6, /* tcgen05, tiles of 256 tokens x 256 weight rows     */
+    TP_MLP_PLAN_TC_PAIR = 7     /* packed bf16: tcgen05 on pairs of CTAs (cta_group::2),
+                                   256 tokens x 256 weight rows per pair, two TMEM
+                                   accumulators per CTA                               */
 } tp_mlp_plan;
 
 /*

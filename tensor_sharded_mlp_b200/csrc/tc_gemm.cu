@@ -505,6 +505,153 @@ done:
     teardown(s, tmem_base, a.status);
 }
 
+// ============ pair tiling: 256 tokens x 256 weight rows per pair of CTAs ============
+// A cluster of two CTAs computes each tile with cta_group::2 MMAs (M = 256
+// tokens, N = 256 weight rows).  CTA r of the pair loads tokens [128 r, 128 r
+// + 128) of the tile and weight rows [128 r, 128 r + 128) -- 32 KB per stage,
+// so 6 stages fit -- and holds its 128 tokens x 256 rows of the accumulator in
+// its own TMEM: two buffers in 512 columns, so one tile's epilogue overlaps the
+// next tile's MMAs (the 1-CTA 256-token tiling has room for one buffer only).
+// Per FLOP the operands cost the same L2 traffic as the 256-token tiling, and
+// each tensor core reads a third less shared memory.  The pair's first CTA
+// issues the MMAs and owns the mbarriers that both CTAs' loads complete on;
+// its commits arrive on the barriers of both CTAs, and both CTAs' epilogues
+// hand the accumulator back to it.  Packed weights only.
+constexpr int kPairStages = 6;
+
+__device__ __forceinline__ void pair_teardown(const Smem &s, uint32_t tmem_base, uint32_t rank, int *status) {
+    // The first CTA waits until its MMAs and their commits (which also arrive
+    // in the other CTA) are done; then neither CTA leaves while the other may
+    // still touch its shared memory or TMEM.
+    if (threadIdx.x == 32 && rank == 0) {
+        mma_commit_pair_local(smem_u32(s.drain));
+        volatile int never = 0;
+        mbar_wait(smem_u32(s.drain), 0, &never);
+    }
+    if (*s.abort && threadIdx.x == 0) {   // a bounded wait gave up: let copies in flight land
+        const unsigned long long t0 = globaltimer();
+        while (globaltimer() - t0 < 100000ull) {
+        }
+    }
+    tc_fence_before();
+    __syncwarp();
+    cluster_barrier();
+    if ((threadIdx.x >> 5) == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, 512);
+    }
+    if (threadIdx.x == 0 && *s.abort) atomicExch(status, 1);
+}
+
+template <int STAGES>
+__global__ void __launch_bounds__(NTHREADS, 1)
+    tc_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ WeightMaps wm, TcArgs a) {
+    constexpr uint32_t A_BYTES = 128 * BK * 2;   // this CTA's 128 tokens of a stage
+    constexpr uint32_t B_BYTES = 128 * BK * 2;   // this CTA's 128 weight rows of a stage
+    extern __shared__ uint8_t smem_raw[];
+    const Smem s = carve<STAGES>(smem_raw, A_BYTES, B_BYTES);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_rank();
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < STAGES; ++i) {
+            mbar_init(smem_u32(&s.full[i]), 1);
+            mbar_init(smem_u32(&s.empty[i]), 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(smem_u32(&s.tfull[i]), 1);
+            mbar_init(smem_u32(&s.tempty[i]), 8);   // 4 epilogue warps in each CTA
+        }
+        mbar_init(smem_u32(s.drain), 1);
+        *s.abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmX);
+        tma_prefetch_desc(&wm.map[0]);
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(smem_u32(s.tmem_slot), 512);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    cluster_barrier();   // both CTAs' barriers exist before anything arrives on them
+    tc_fence_after();
+    const uint32_t tmem_base = *s.tmem_slot;
+    pdl_allow_dependents();
+
+    const int MT = (a.rows_x + 255) / 256, NT = a.rows_w;   // rows_w: 256-row weight tiles
+    const int units = MT * NT;
+    const int pair = (int)(blockIdx.x >> 1), npairs = (int)(gridDim.x >> 1);
+    const int KB = a.KB;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            pdl_wait_previous();   // X / H come from the previous kernel
+            const uint32_t full0 = cluster_addr(smem_u32(&s.full[0]), 0);   // the first CTA's full[0]
+            int stage = 0;
+            uint32_t phase = 0;
+            for (int u = pair; u < units; u += npairs) {
+                int mt, nt;
+                wide_tile(u, MT, NT, mt, nt);
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!mbar_wait(smem_u32(&s.empty[stage]), phase ^ 1, s.abort)) goto done;
+                    if (rank == 0) mbar_arrive_expect_tx(smem_u32(&s.full[stage]), 2 * (A_BYTES + B_BYTES));
+                    const uint32_t fb = full0 + 8u * stage;
+                    tma_load_2d_pair(smem_u32(s.a + stage * A_BYTES), &tmX, kb * BK, mt * 256 + (int)rank * 128, fb);
+                    tma_load_2d_pair(smem_u32(s.b + stage * B_BYTES), &wm.map[0], 0,
+                                     (nt * KB + kb) * 256 + (int)rank * 128, fb);
+                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && rank == 0) {
+            const uint32_t idesc = idesc_bf16_f32(256, 256);
+            int stage = 0, acc = 0;
+            uint32_t phase = 0, acc_phase = 0;
+            for (int u = pair; u < units; u += npairs) {
+                if (!mbar_wait(smem_u32(&s.tempty[acc]), acc_phase ^ 1, s.abort)) goto done;
+                tc_fence_after();
+                const uint32_t d = tmem_base + acc * 256;
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!mbar_wait(smem_u32(&s.full[stage]), phase, s.abort)) goto done;
+                    tc_fence_after();
+                    const uint64_t da = smem_desc_kmajor_sw128(smem_u32(s.a + stage * A_BYTES));
+                    const uint64_t db = smem_desc_kmajor_sw128(smem_u32(s.b + stage * B_BYTES));
+#pragma unroll
+                    for (int k = 0; k < BK / 16; ++k) mma_bf16_pair(d, da + 2 * k, db + 2 * k, idesc, (kb | k) != 0);
+                    mma_commit_pair_both(smem_u32(&s.empty[stage]));
+                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                }
+                mma_commit_pair_both(smem_u32(&s.tfull[acc]));
+                if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+            }
+        }
+    } else {
+        // epilogue: TMEM lane quadrant q holds this CTA's tokens 32q..32q+31
+        pdl_wait_previous();   // outputs may still be read by the previous kernel
+        const int q = warp & 3;
+        const uint32_t tempty0 = cluster_addr(smem_u32(&s.tempty[0]), 0);
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int u = pair; u < units; u += npairs) {
+            int mt, nt;
+            wide_tile(u, MT, NT, mt, nt);
+            if (!mbar_wait(smem_u32(&s.tfull[acc]), acc_phase, s.abort)) break;
+            tc_fence_after();
+            wide_epilogue_half(a, mt * 256 + (int)rank * 128 + q * 32 + lane, nt,
+                               tmem_base + acc * 256 + ((uint32_t)(q * 32) << 16));
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_remote(tempty0 + 8u * acc);
+            if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+        }
+    }
+done:
+    pair_teardown(s, tmem_base, rank, a.status);
+}
+
 // ================== skinny tiling: 256 weight rows x BT tokens, stream-K ==================
 
 // Final epilogue of a skinny tile for 16 tokens t0..t0+15: v0 = rows r, v1 = rows 128 + r.
@@ -1451,6 +1598,35 @@ cudaError_t run_wide(const WeightOperand &w, const void *x, int T, int K, int ep
     return launch_pdl(kern, dim3(grid), dim3(NTHREADS), smem, st, mx, w.wm, a);
 }
 
+// The pair tiling (packed weights): clusters of 2 CTAs, one 256 x 256 tile per
+// pair at a time, persistent over the tiles.
+cudaError_t run_pair(const Problem &p, int proj, const void *wbase, const void *x, int T, int K, int epi,
+                     void *out, int out_cols, int *status, int num_sms, cudaStream_t st) {
+    WeightOperand w;
+    if (!weight_packed(&w, p, proj, wbase, true)) return cudaErrorInvalidValue;   // 128-row boxes
+    const long long rows_w = proj == 0 ? w1p_rows(p.d_ff, p.act) : p.d_out;
+    CUtensorMap mx;
+    if (!make_map(&mx, x, K, T, 128)) return cudaErrorInvalidValue;
+    TcArgs a{};
+    a.rows_x = T;
+    a.rows_w = (int)blk_tiles(rows_w);
+    a.K = K;
+    a.KB = w.KB;
+    a.epi = epi;
+    a.out = static_cast<__nv_bfloat16 *>(out);
+    a.ldo = out_cols;
+    a.out_cols = out_cols;
+    a.status = status;
+    const int units = ((T + 255) / 256) * a.rows_w;
+    const int pairs = std::max(1, std::min(units, num_sms / 2));
+    constexpr int S = kPairStages;
+    const size_t smem = smem_bytes<S>(128 * BK * 2, 128 * BK * 2);
+    auto kern = tc_pair_kernel<S>;
+    cudaError_t e = set_smem(kern, smem);
+    if (e != cudaSuccess) return e;
+    return launch_pdl_cluster(kern, dim3(2 * pairs), dim3(NTHREADS), smem, st, 2u, mx, w.wm, a);
+}
+
 int first_epi(int act) {
     return act == TP_MLP_ACT_SWIGLU ? EPI_H_SWIGLU : act == TP_MLP_ACT_TANH ? EPI_H_TANH : EPI_H_IDENT;
 }
@@ -1705,6 +1881,17 @@ cudaError_t launch_tc(const Problem &p, int tiling, const void *x, const void *w
     WeightOperand w1, w2;
     const bool raw = rawA != nullptr;
     if (partials && !raw) return cudaErrorInvalidValue;   // per-rank partials come from the shard form
+    if (tiling == kTilingPair) {   // packed weights only
+        if (raw || partials) return cudaErrorNotSupported;
+        marks.mark(0, st);
+        cudaError_t e = run_pair(p, 0, w1p, x, p.T, p.d_in, first_epi(p.act), h, p.d_ff, status, num_sms, st);
+        if (e != cudaSuccess) return e;
+        marks.mark(1, st);
+        e = run_pair(p, 1, w2p, h, p.T, p.d_ff, EPI_OUT, out, p.d_out, status, num_sms, st);
+        marks.mark(2, st);
+        *launches = 2;
+        return e;
+    }
     const bool skinny = tiling == kTilingSkinny;
     const int BT = skinny_bt(p.T);
     const bool half1 = skinny && skinny_half(0, p.act, BT, split_mode, raw);

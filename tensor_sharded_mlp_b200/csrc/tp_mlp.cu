@@ -285,7 +285,7 @@ static int run_shard_form(tp_mlp_t h, const void *x, int tokens, const void *con
         plan = tokens <= kTcSkinnyMaxTokens ? TP_MLP_PLAN_TC_SKINNY
                                             : tokens < kTcWide256MinTokens ? TP_MLP_PLAN_TC_WIDE : TP_MLP_PLAN_TC_WIDE256;
     const bool is_tc = plan == TP_MLP_PLAN_TC_WIDE || plan == TP_MLP_PLAN_TC_SKINNY || plan == TP_MLP_PLAN_TC_WIDE256;
-    if (plan != TP_MLP_PLAN_SIMT && !is_tc) return TP_MLP_ERR_UNSUPPORTED;
+    if (plan != TP_MLP_PLAN_SIMT && !is_tc) return TP_MLP_ERR_UNSUPPORTED;   // (the pair tiling needs packed weights)
     if (is_tc && tokens > 0 && (!tc_ok || (plan == TP_MLP_PLAN_TC_SKINNY && tokens > kTcSkinnyMaxTokens)))
         return TP_MLP_ERR_UNSUPPORTED;
     if (tokens == 0) {
@@ -369,12 +369,15 @@ int tp_mlp_forward_packed(tp_mlp_t h, const void *x, int tokens, const void *pac
     Problem p = problem_of(h, tokens);
     // plan choice (measured on B200 at d_model 8192, d_ff 28672): the CUDA-core
     // GEMV for 1 token; from 2 tokens on the tensor-core skinny tiling streams
-    // the weights as fast and its arithmetic stays hidden; wide beyond 128.
+    // the weights as fast and its arithmetic stays hidden; wide beyond 128,
+    // pairs of CTAs from 512 to 4096 tokens, 256-token tiles above.
     int plan = h->plan;
     const bool tc_ok = tc_supported(p);
     auto tc_tiling = [&](int t) {
         return t <= kTcSkinnyMaxTokens ? TP_MLP_PLAN_TC_SKINNY
-                                       : t < kTcWide256MinTokens ? TP_MLP_PLAN_TC_WIDE : TP_MLP_PLAN_TC_WIDE256;
+               : t < kTcPairMinTokens  ? TP_MLP_PLAN_TC_WIDE
+               : t <= kTcPairMaxTokens ? TP_MLP_PLAN_TC_PAIR
+                                       : TP_MLP_PLAN_TC_WIDE256;
     };
     if (plan == TP_MLP_PLAN_AUTO) {
         if (gemv_supported(p) && (tokens <= 1 || !tc_ok)) plan = TP_MLP_PLAN_GEMV;
@@ -383,7 +386,8 @@ int tp_mlp_forward_packed(tp_mlp_t h, const void *x, int tokens, const void *pac
     } else if (plan == TP_MLP_PLAN_TC) {
         plan = tc_tiling(tokens);
     }
-    const bool is_tc = plan == TP_MLP_PLAN_TC_WIDE || plan == TP_MLP_PLAN_TC_SKINNY || plan == TP_MLP_PLAN_TC_WIDE256;
+    const bool is_tc = plan == TP_MLP_PLAN_TC_WIDE || plan == TP_MLP_PLAN_TC_SKINNY ||
+                       plan == TP_MLP_PLAN_TC_WIDE256 || plan == TP_MLP_PLAN_TC_PAIR;
     if (tokens > 0) {
         if (plan == TP_MLP_PLAN_GEMV && !gemv_supported(p)) return TP_MLP_ERR_UNSUPPORTED;
         if (is_tc && !tc_ok) return TP_MLP_ERR_UNSUPPORTED;
@@ -414,7 +418,8 @@ int tp_mlp_forward_packed(tp_mlp_t h, const void *x, int tokens, const void *pac
                          &launches);
     } else if (is_tc) {
         const int tiling = plan == TP_MLP_PLAN_TC_SKINNY ? kTilingSkinny
-                           : plan == TP_MLP_PLAN_TC_WIDE ? kTilingWide128 : kTilingWide256;
+                           : plan == TP_MLP_PLAN_TC_WIDE ? kTilingWide128
+                           : plan == TP_MLP_PLAN_TC_PAIR ? kTilingPair : kTilingWide256;
         ce = launch_tc(p, tiling, x, w1p, w2p, nullptr, nullptr, hbuf, out, part, counters, status_word(h),
                        h->num_sms, st, h->marks, h->splitk, &launches);
     } else {
@@ -455,7 +460,7 @@ int tp_mlp_selftest_bounded_wait(tp_mlp_t h, unsigned wait_us, tp_mlp_stream_t s
 
 int tp_mlp_set_plan(tp_mlp_t h, int plan) {
     if (!h) return TP_MLP_ERR_INVALID_ARG;
-    if (plan < TP_MLP_PLAN_AUTO || plan > TP_MLP_PLAN_TC_WIDE256) return TP_MLP_ERR_INVALID_ARG;
+    if (plan < TP_MLP_PLAN_AUTO || plan > TP_MLP_PLAN_TC_PAIR) return TP_MLP_ERR_INVALID_ARG;
     h->plan = plan;
     return TP_MLP_OK;
 }
