@@ -61,7 +61,7 @@ FULL_METRICS = [
 
 def bench_cmd(config: str, extra: list[str]) -> str:
     return " ".join(["python", "bench.py", "--config", config, "--steps", "2", "--warmup", "3",
-                     "--no-e2e", "--no-cpu-baseline", "--no-graph"] + extra)
+                     "--no-e2e", "--no-cpu-baseline", "--no-graph", "--configs", "none"] + extra)
 
 
 def list_cmd(a) -> str:
