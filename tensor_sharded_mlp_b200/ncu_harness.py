@@ -88,13 +88,16 @@ def summarize_list(path: str, title: str, cmd: str) -> str:
     h = rows[0]
     ki, vi, ui = h.index("Kernel Name"), h.index("Metric Value"), h.index("Metric Unit")
     agg = collections.OrderedDict()
+    each = collections.defaultdict(list)
     for r in rows[1:]:
         if len(r) <= vi or r[h.index("Metric Name")] != "gpu__time_duration.sum":
             continue
         name = r[ki].split("(")[0].replace("void ", "").replace("tpmlp::", "").replace("<unnamed>::", "")
         a = agg.setdefault(name, [0, 0.0])
         a[0] += 1
-        a[1] += _to_ns(float(r[vi].replace(",", "")), r[ui])
+        t = _to_ns(float(r[vi].replace(",", "")), r[ui])
+        a[1] += t
+        each[name].append(t)
     total = sum(a[1] for a in agg.values())
     out = [f"# {title}", "", "Launch list from one ncu pass (`gpu__time_duration.sum` only).  Per-launch",
            "times here are serialised and cold-cache: compare shares, not absolute times.", "",
@@ -102,7 +105,27 @@ def summarize_list(path: str, title: str, cmd: str) -> str:
            "| kernel | launches | total µs | mean µs | share |", "|---|---:|---:|---:|---:|"]
     for k, (n, t) in sorted(agg.items(), key=lambda x: -x[1][1]):
         out.append(f"| `{k}` | {n} | {t / 1e3:.1f} | {t / n / 1e3:.1f} | {100 * t / total:.1f}% |")
+    # the kernels a forward launches (not the one-off pack or torch's input copies)
+    step = {k: v for k, v in agg.items() if k.startswith(STEP_KERNELS)}
+    st = sum(v[1] for v in step.values())
+    if step and st > 0:
+        out += ["", "Shares among the forward's own kernels (the timed region launches only these):", "",
+                "| kernel | launches | total µs | mean µs | share of the forward |", "|---|---:|---:|---:|---:|"]
+        for k, (n, t) in sorted(step.items(), key=lambda x: -x[1][1]):
+            out.append(f"| `{k}` | {n} | {t / 1e3:.1f} | {t / n / 1e3:.1f} | {100 * t / st:.1f}% |")
+        alt = {k: v for k, v in each.items() if k in step and len(v) % 2 == 0 and len(v) >= 2}
+        if alt:
+            out += ["", "A forward launches its first projection, then its second; where one kernel",
+                    "serves both, its launches alternate:", "",
+                    "| kernel | mean µs, 1st, 3rd, ... launch | mean µs, 2nd, 4th, ... launch |", "|---|---:|---:|"]
+            for k, v in alt.items():
+                out.append(f"| `{k}` | {sum(v[0::2]) / len(v[0::2]) / 1e3:.1f} | {sum(v[1::2]) / len(v[1::2]) / 1e3:.1f} |")
     return "\n".join(out) + "\n"
+
+
+STEP_KERNELS = ("gemv_kernel", "tc_skinny_kernel", "skinny_reduce_kernel", "tc_wide_kernel", "tc_pair_kernel",
+                "simt_", "allreduce_norm_kernel", "attn_merge_kernel", "unnamed>::tc_", "unnamed>::skinny",
+                "unnamed>::gemv")
 
 
 def _raw(report: str):
