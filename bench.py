@@ -3,7 +3,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--config decode_bs1|decode_bs32|prefill|sweep|tiny] [--tokens T] [--tp P]
-                    [--plan auto|simt|gemv|tc|tc_skinny|tc_wide|tc_wide256|tc_pair] [--api packed|shard]
+                    [--plan auto|simt|gemv|tc|tc_skinny|tc_wide|tc_wide256|tc_pair|tc_pair2] [--api packed|shard]
                     [--splitk auto|in_kernel|separate|cluster] [--no-e2e] [--no-cpu-baseline] [--no-graph]
                     [--configs auto|all|none]
     python bench.py --config fused_norm_decode_bs32|fused_norm_prefill|
@@ -716,7 +716,7 @@ class MlpRun:
         T, d, f, act, dt = c["tokens"], c["d_model"], c["d_ff"], c["act"], c["dtype"]
         j = int(np.argmax(kern_ms))
         extra = {}
-        if self.plan in ("tc_wide", "tc_wide256", "tc_pair"):
+        if self.plan in ("tc_wide", "tc_wide256", "tc_pair", "tc_pair2"):
             bound, unit = "tensor", "TFLOP/s"
             work = counts.gemm1_flops(T, d, f, act) if j == 0 else counts.gemm2_flops(T, f, d)
             achieved = work / (kern_ms[j] / 1e3) / 1e12

@@ -85,9 +85,11 @@ typedef enum {
                                   evenly over the SMs, or whole CTAs per tile when
                                   tiles are few                                       */
     TP_MLP_PLAN_TC_WIDE256 = 6, /* tcgen05, tiles of 256 tokens x 256 weight rows     */
-    TP_MLP_PLAN_TC_PAIR = 7     /* packed bf16: tcgen05 on pairs of CTAs (cta_group::2),
+    TP_MLP_PLAN_TC_PAIR = 7,    /* packed bf16: tcgen05 on pairs of CTAs (cta_group::2),
                                    256 tokens x 256 weight rows per pair, two TMEM
                                    accumulators per CTA                               */
+    TP_MLP_PLAN_TC_PAIR2 = 8    /* packed bf16: pairs of CTAs, 256 tokens x 512 weight
+                                   rows per pair (two weight tiles share each X stage) */
 } tp_mlp_plan;
 
 /*

@@ -517,7 +517,14 @@ done:
 // issues the MMAs and owns the mbarriers that both CTAs' loads complete on;
 // its commits arrive on the barriers of both CTAs, and both CTAs' epilogues
 // hand the accumulator back to it.  Packed weights only.
+// NB = 2: each unit is 256 tokens x 512 weight rows -- two weight tiles share
+// every X stage (two M=256 MMAs per 16-k step), so a CTA loads 48 KB per stage
+// for twice the FLOPs of 32 KB: a quarter less operand traffic per FLOP than
+// the 1-CTA 256-token tiling, which lowers the power a prefill-size GEMM draws
+// under the 1 kW cap.  Its two 256-column accumulators fill TMEM, so there is
+// one buffer and the epilogue does not overlap the MMAs.
 constexpr int kPairStages = 6;
+constexpr int kPair2Stages = 4;
 
 __device__ __forceinline__ void pair_teardown(const Smem &s, uint32_t tmem_base, uint32_t rank, int *status) {
     // The first CTA waits until its MMAs and their commits (which also arrive
@@ -544,11 +551,12 @@ __device__ __forceinline__ void pair_teardown(const Smem &s, uint32_t tmem_base,
     if (threadIdx.x == 0 && *s.abort) atomicExch(status, 1);
 }
 
-template <int STAGES>
+template <int STAGES, int NB>
 __global__ void __launch_bounds__(NTHREADS, 1)
     tc_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ WeightMaps wm, TcArgs a) {
-    constexpr uint32_t A_BYTES = 128 * BK * 2;   // this CTA's 128 tokens of a stage
-    constexpr uint32_t B_BYTES = 128 * BK * 2;   // this CTA's 128 weight rows of a stage
+    constexpr uint32_t A_BYTES = 128 * BK * 2;        // this CTA's 128 tokens of a stage
+    constexpr uint32_t B_BYTES = NB * 128 * BK * 2;   // this CTA's 128 rows of each of NB weight tiles
+    constexpr int NACC = NB == 1 ? 2 : 1;             // TMEM accumulator buffers (NB x 256 columns each)
     extern __shared__ uint8_t smem_raw[];
     const Smem s = carve<STAGES>(smem_raw, A_BYTES, B_BYTES);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -580,7 +588,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t tmem_base = *s.tmem_slot;
     pdl_allow_dependents();
 
-    const int MT = (a.rows_x + 255) / 256, NT = a.rows_w;   // rows_w: 256-row weight tiles
+    const int MT = (a.rows_x + 255) / 256;
+    const int NT = (a.rows_w + NB - 1) / NB;   // rows_w: 256-row weight tiles; a unit takes NB of them
     const int units = MT * NT;
     const int pair = (int)(blockIdx.x >> 1), npairs = (int)(gridDim.x >> 1);
     const int KB = a.KB;
@@ -599,8 +608,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     if (rank == 0) mbar_arrive_expect_tx(smem_u32(&s.full[stage]), 2 * (A_BYTES + B_BYTES));
                     const uint32_t fb = full0 + 8u * stage;
                     tma_load_2d_pair(smem_u32(s.a + stage * A_BYTES), &tmX, kb * BK, mt * 256 + (int)rank * 128, fb);
-                    tma_load_2d_pair(smem_u32(s.b + stage * B_BYTES), &wm.map[0], 0,
-                                     (nt * KB + kb) * 256 + (int)rank * 128, fb);
+#pragma unroll
+                    for (int j = 0; j < NB; ++j) {   // a tile past the end loads the last one again (discarded)
+                        const int wt = min(nt * NB + j, a.rows_w - 1);
+                        tma_load_2d_pair(smem_u32(s.b + stage * B_BYTES + j * 16384), &wm.map[0], 0,
+                                         (wt * KB + kb) * 256 + (int)rank * 128, fb);
+                    }
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
                 }
             }
@@ -613,19 +626,23 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             for (int u = pair; u < units; u += npairs) {
                 if (!mbar_wait(smem_u32(&s.tempty[acc]), acc_phase ^ 1, s.abort)) goto done;
                 tc_fence_after();
-                const uint32_t d = tmem_base + acc * 256;
+                const uint32_t d = tmem_base + acc * 256 * NB;
                 for (int kb = 0; kb < KB; ++kb) {
                     if (!mbar_wait(smem_u32(&s.full[stage]), phase, s.abort)) goto done;
                     tc_fence_after();
                     const uint64_t da = smem_desc_kmajor_sw128(smem_u32(s.a + stage * A_BYTES));
-                    const uint64_t db = smem_desc_kmajor_sw128(smem_u32(s.b + stage * B_BYTES));
 #pragma unroll
-                    for (int k = 0; k < BK / 16; ++k) mma_bf16_pair(d, da + 2 * k, db + 2 * k, idesc, (kb | k) != 0);
+                    for (int k = 0; k < BK / 16; ++k)
+#pragma unroll
+                        for (int j = 0; j < NB; ++j)
+                            mma_bf16_pair(d + 256 * j, da + 2 * k,
+                                          smem_desc_kmajor_sw128(smem_u32(s.b + stage * B_BYTES + j * 16384)) + 2 * k,
+                                          idesc, (kb | k) != 0);
                     mma_commit_pair_both(smem_u32(&s.empty[stage]));
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
                 }
                 mma_commit_pair_both(smem_u32(&s.tfull[acc]));
-                if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+                if (++acc == NACC) { acc = 0; acc_phase ^= 1; }
             }
         }
     } else {
@@ -640,12 +657,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             wide_tile(u, MT, NT, mt, nt);
             if (!mbar_wait(smem_u32(&s.tfull[acc]), acc_phase, s.abort)) break;
             tc_fence_after();
-            wide_epilogue_half(a, mt * 256 + (int)rank * 128 + q * 32 + lane, nt,
-                               tmem_base + acc * 256 + ((uint32_t)(q * 32) << 16));
+#pragma unroll 1
+            for (int j = 0; j < NB; ++j)
+                if (nt * NB + j < a.rows_w)
+                    wide_epilogue_half(a, mt * 256 + (int)rank * 128 + q * 32 + lane, nt * NB + j,
+                                       tmem_base + (acc * NB + j) * 256 + ((uint32_t)(q * 32) << 16));
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_remote(tempty0 + 8u * acc);
-            if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+            if (++acc == NACC) { acc = 0; acc_phase ^= 1; }
         }
     }
 done:
@@ -1600,6 +1620,7 @@ cudaError_t run_wide(const WeightOperand &w, const void *x, int T, int K, int ep
 
 // The pair tiling (packed weights): clusters of 2 CTAs, one 256 x 256 tile per
 // pair at a time, persistent over the tiles.
+template <int NB>
 cudaError_t run_pair(const Problem &p, int proj, const void *wbase, const void *x, int T, int K, int epi,
                      void *out, int out_cols, int *status, int num_sms, cudaStream_t st) {
     WeightOperand w;
@@ -1617,11 +1638,11 @@ cudaError_t run_pair(const Problem &p, int proj, const void *wbase, const void *
     a.ldo = out_cols;
     a.out_cols = out_cols;
     a.status = status;
-    const int units = ((T + 255) / 256) * a.rows_w;
+    const int units = ((T + 255) / 256) * ((a.rows_w + NB - 1) / NB);
     const int pairs = std::max(1, std::min(units, num_sms / 2));
-    constexpr int S = kPairStages;
-    const size_t smem = smem_bytes<S>(128 * BK * 2, 128 * BK * 2);
-    auto kern = tc_pair_kernel<S>;
+    constexpr int S = NB == 1 ? kPairStages : kPair2Stages;
+    const size_t smem = smem_bytes<S>(128 * BK * 2, NB * 128 * BK * 2);
+    auto kern = tc_pair_kernel<S, NB>;
     cudaError_t e = set_smem(kern, smem);
     if (e != cudaSuccess) return e;
     return launch_pdl_cluster(kern, dim3(2 * pairs), dim3(NTHREADS), smem, st, 2u, mx, w.wm, a);
@@ -1881,13 +1902,14 @@ cudaError_t launch_tc(const Problem &p, int tiling, const void *x, const void *w
     WeightOperand w1, w2;
     const bool raw = rawA != nullptr;
     if (partials && !raw) return cudaErrorInvalidValue;   // per-rank partials come from the shard form
-    if (tiling == kTilingPair) {   // packed weights only
+    if (tiling == kTilingPair || tiling == kTilingPair2) {   // packed weights only
         if (raw || partials) return cudaErrorNotSupported;
+        auto pair = tiling == kTilingPair ? run_pair<1> : run_pair<2>;
         marks.mark(0, st);
-        cudaError_t e = run_pair(p, 0, w1p, x, p.T, p.d_in, first_epi(p.act), h, p.d_ff, status, num_sms, st);
+        cudaError_t e = pair(p, 0, w1p, x, p.T, p.d_in, first_epi(p.act), h, p.d_ff, status, num_sms, st);
         if (e != cudaSuccess) return e;
         marks.mark(1, st);
-        e = run_pair(p, 1, w2p, h, p.T, p.d_ff, EPI_OUT, out, p.d_out, status, num_sms, st);
+        e = pair(p, 1, w2p, h, p.T, p.d_ff, EPI_OUT, out, p.d_out, status, num_sms, st);
         marks.mark(2, st);
         *launches = 2;
         return e;

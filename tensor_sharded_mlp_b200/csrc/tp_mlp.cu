@@ -370,14 +370,14 @@ int tp_mlp_forward_packed(tp_mlp_t h, const void *x, int tokens, const void *pac
     // plan choice (measured on B200 at d_model 8192, d_ff 28672): the CUDA-core
     // GEMV for 1 token; from 2 tokens on the tensor-core skinny tiling streams
     // the weights as fast and its arithmetic stays hidden; wide beyond 128,
-    // pairs of CTAs from 512 to 4096 tokens, 256-token tiles above.
+    // pairs of CTAs from 512 to 4096 tokens, two-tile pairs above.
     int plan = h->plan;
     const bool tc_ok = tc_supported(p);
     auto tc_tiling = [&](int t) {
         return t <= kTcSkinnyMaxTokens ? TP_MLP_PLAN_TC_SKINNY
                : t < kTcPairMinTokens  ? TP_MLP_PLAN_TC_WIDE
                : t <= kTcPairMaxTokens ? TP_MLP_PLAN_TC_PAIR
-                                       : TP_MLP_PLAN_TC_WIDE256;
+                                       : TP_MLP_PLAN_TC_PAIR2;
     };
     if (plan == TP_MLP_PLAN_AUTO) {
         if (gemv_supported(p) && (tokens <= 1 || !tc_ok)) plan = TP_MLP_PLAN_GEMV;
@@ -387,7 +387,7 @@ int tp_mlp_forward_packed(tp_mlp_t h, const void *x, int tokens, const void *pac
         plan = tc_tiling(tokens);
     }
     const bool is_tc = plan == TP_MLP_PLAN_TC_WIDE || plan == TP_MLP_PLAN_TC_SKINNY ||
-                       plan == TP_MLP_PLAN_TC_WIDE256 || plan == TP_MLP_PLAN_TC_PAIR;
+                       plan == TP_MLP_PLAN_TC_WIDE256 || plan == TP_MLP_PLAN_TC_PAIR || plan == TP_MLP_PLAN_TC_PAIR2;
     if (tokens > 0) {
         if (plan == TP_MLP_PLAN_GEMV && !gemv_supported(p)) return TP_MLP_ERR_UNSUPPORTED;
         if (is_tc && !tc_ok) return TP_MLP_ERR_UNSUPPORTED;
@@ -419,7 +419,8 @@ int tp_mlp_forward_packed(tp_mlp_t h, const void *x, int tokens, const void *pac
     } else if (is_tc) {
         const int tiling = plan == TP_MLP_PLAN_TC_SKINNY ? kTilingSkinny
                            : plan == TP_MLP_PLAN_TC_WIDE ? kTilingWide128
-                           : plan == TP_MLP_PLAN_TC_PAIR ? kTilingPair : kTilingWide256;
+                           : plan == TP_MLP_PLAN_TC_PAIR ? kTilingPair
+                           : plan == TP_MLP_PLAN_TC_PAIR2 ? kTilingPair2 : kTilingWide256;
         ce = launch_tc(p, tiling, x, w1p, w2p, nullptr, nullptr, hbuf, out, part, counters, status_word(h),
                        h->num_sms, st, h->marks, h->splitk, &launches);
     } else {
@@ -460,7 +461,7 @@ int tp_mlp_selftest_bounded_wait(tp_mlp_t h, unsigned wait_us, tp_mlp_stream_t s
 
 int tp_mlp_set_plan(tp_mlp_t h, int plan) {
     if (!h) return TP_MLP_ERR_INVALID_ARG;
-    if (plan < TP_MLP_PLAN_AUTO || plan > TP_MLP_PLAN_TC_PAIR) return TP_MLP_ERR_INVALID_ARG;
+    if (plan < TP_MLP_PLAN_AUTO || plan > TP_MLP_PLAN_TC_PAIR2) return TP_MLP_ERR_INVALID_ARG;
     h->plan = plan;
     return TP_MLP_OK;
 }

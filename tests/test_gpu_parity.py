@@ -78,7 +78,7 @@ def test_integer_inputs_fp32_bit_exact(act, tp):
     assert np.array_equal(m.forward_packed(x, packed).cpu().numpy().astype(np.float64), ref)
 
 
-@pytest.mark.parametrize("plan", ["simt", "gemv"])
+@pytest.mark.parametrize("plan", ["simt", "gemv", "tc_pair", "tc_pair2"])
 @pytest.mark.parametrize("T", [1, 3, 4])
 def test_integer_inputs_bf16_exact_rounding(plan, T):
     """bf16 with |H| <= 64 (exact in bf16) and fp32 sums that stay exact: the

@@ -192,26 +192,30 @@ def test_tc_wide256_parity(act, T, shape):
     assert_close(out[torch.from_numpy(rows).cuda()], ref, "bf16", f"wide256 T={T}")
 
 
+@pytest.mark.parametrize("plan", ["tc_pair", "tc_pair2"])
 @pytest.mark.parametrize("act", ["swiglu", "tanh", "identity"])
 @pytest.mark.parametrize("T", [1, 100, 255, 256, 257, 600, 2100])
 @pytest.mark.parametrize("shape", SHAPES[:3])
-def test_tc_pair_parity(act, T, shape):
-    """Pairs of CTAs (cta_group::2 MMAs, 256 tokens x 256 weight rows per pair,
-    two TMEM accumulators per CTA); ragged token and weight tails."""
+def test_tc_pair_parity(plan, act, T, shape):
+    """Pairs of CTAs (cta_group::2 MMAs): 256 tokens x 256 weight rows per pair
+    with two TMEM accumulators per CTA (tc_pair), or 256 x 512 with two weight
+    tiles per X stage (tc_pair2; an odd tile count leaves the last unit half
+    empty); ragged token and weight tails."""
     d, f, dout, tp = shape
     p = inputs.generate(T, d, f, act, "bf16", seed=T + 13 * d, init="fan_in", d_out=dout)
     A, Bs = p.shards(tp)
     rows = p.sample_rows(64)
     ref = oracle.tp_mlp_sharded(p.x[rows], A, Bs, act)
-    m, out, _, _, _ = _run(p, tp, "tc_pair")
-    assert m.last_plan == "tc_pair"
-    assert_close(out[torch.from_numpy(rows).cuda()], ref, "bf16", f"pair T={T}")
+    m, out, _, _, _ = _run(p, tp, plan)
+    assert m.last_plan == plan
+    assert_close(out[torch.from_numpy(rows).cuda()], ref, "bf16", f"{plan} T={T}")
 
 
+@pytest.mark.parametrize("plan", ["tc_pair", "tc_pair2"])
 @pytest.mark.parametrize("T", [3, 300, 1030])
-def test_tc_pair_integer_exact(T):
+def test_tc_pair_integer_exact(plan, T):
     p = inputs.integer_inputs(T, 64, 512, 264, "identity", seed=T + 5, lo=-1, hi=1)
-    m, out, A, Bs, _ = _run(p, 4, "tc_pair")
+    m, out, A, Bs, _ = _run(p, 4, plan)
     ref = oracle.tp_mlp_sharded(p.x, A, Bs, "identity")
     assert np.array_equal(out.float().cpu().numpy(), inputs.round_to_bf16(ref.astype(np.float32)))
 
@@ -221,22 +225,23 @@ def test_tc_pair_agrees_with_wide256():
     same k order; they agree within the bf16 bound (and with the oracle)."""
     p = inputs.generate(700, 512, 2048, "swiglu", "bf16", seed=77, init=0.02)
     outs = []
-    for plan in ("tc_pair", "tc_wide256"):
+    for plan in ("tc_pair", "tc_pair2", "tc_wide256"):
         _, out, _, _, _ = _run(p, 4, plan)
         outs.append(out)
-    assert_close(outs[0], outs[1].float().cpu().numpy(), "bf16", "pair vs wide256")
+    assert_close(outs[0], outs[2].float().cpu().numpy(), "bf16", "pair vs wide256")
+    assert_close(outs[1], outs[2].float().cpu().numpy(), "bf16", "pair2 vs wide256")
 
 
 def test_auto_plan_tiling_by_token_count():
     """Packed weights: 128-token tiles up to 511 tokens, pairs of CTAs from 512 to
-    4096, 256-token tiles above; the shard form keeps 256-token tiles from 2048."""
+    4096, two-tile pairs above; the shard form keeps 256-token tiles from 2048."""
     p = inputs.generate(4097, 256, 512, "swiglu", "bf16", seed=3)
     A, Bs = p.shards(2)
     Ad, Bd = [dev(a, "bf16") for a in A], [dev(b, "bf16") for b in Bs]
     m = B().TpMlp(256, 512, 2, "swiglu", "bf16", max_tokens=4097)
     packed = m.pack(Ad, Bd)
     x = dev(p.x, "bf16")
-    for T, plan in ((511, "tc_wide"), (512, "tc_pair"), (4096, "tc_pair"), (4097, "tc_wide256")):
+    for T, plan in ((511, "tc_wide"), (512, "tc_pair"), (4096, "tc_pair"), (4097, "tc_pair2")):
         m.forward_packed(x[:T], packed)
         assert m.last_plan == plan, (T, m.last_plan)
     for T, plan in ((2047, "tc_wide"), (2048, "tc_wide256")):
