@@ -8,6 +8,7 @@
                     [--configs auto|all|none]
     python bench.py --config fused_norm_decode_bs32|fused_norm_prefill|
                              attn_merge_decode_bs32|attn_merge_decode_bs256 [...]
+    torchrun --nproc-per-node N bench.py --config xgpu_decode_bs32 [...]
 
 One step = one forward of the whole hot path (first projection + activation,
 second projection with the ranks' partial sums reduced on the device) over one
@@ -33,6 +34,10 @@ The fused_norm_* and attn_merge_* configs time the two other operators (the
 all-reduce fused with residual add and RMSNorm; the merge of attention
 partials across KV shards): one launch per step, the K steps captured in a
 CUDA graph, inputs smaller than L2 rotated through enough copies to exceed it.
+
+The xgpu_decode_bs32 config runs tensor parallelism across GPUs (one rank per
+GPU under torchrun, tp = the number of ranks) and times the fused one-shot
+all-reduce step against each rank's partial followed by NCCL's all_reduce.
 """
 from __future__ import annotations
 
@@ -62,7 +67,7 @@ def parse():
     ap.add_argument("--config", default="decode_bs1",
                     help="MLP: tiny, decode_bs1, decode_bs32, sweep, prefill; other operators: "
                          "fused_norm_decode_bs32, fused_norm_prefill, attn_merge_decode_bs32, "
-                         "attn_merge_decode_bs256")
+                         "attn_merge_decode_bs256; across GPUs (torchrun): xgpu_decode_bs32")
     ap.add_argument("--tokens", type=int, default=None)
     ap.add_argument("--tp", type=int, default=None)
     ap.add_argument("--plan", default="auto")
@@ -786,8 +791,85 @@ def measure_extra(name, tokens, tp, args, peaks, src, barrier, cpu):
     return key, e
 
 
+XGPU_METRIC = "cross-GPU tensor-parallel MLP step (one rank per GPU): tokens/s, fused one-shot all-reduce vs NCCL"
+
+
+def run_xgpu(args):
+    """--config xgpu_decode_bs32: the decode batch-32 MLP (bf16 SwiGLU, d 8192,
+    f 28672) with tp = the number of ranks, one rank per GPU.  Times the fused
+    step (tp_mlp_xgpu_forward: the one-shot all-reduce inside the second
+    projection) against the unfused one (each rank's fp32 partial from the
+    library, then the process group's NCCL all_reduce), max over ranks.  The
+    weights are random on the device (seeded per rank); correctness is the tests'
+    business.  The whole job processes T tokens per step: strong scaling."""
+    import torch
+
+    from tensor_sharded_mlp_b200 import replicas, xgpu
+    rank, world, local = replicas.rank_env()
+    torch.cuda.set_device(local)
+    replicas.init("nccl", torch.device("cuda", local), timeout_s=120)
+    d, f, T = 8192, 28672, args.tokens or 32
+    tp = world
+    fs = f // tp
+    g = torch.Generator(device="cuda")
+    g.manual_seed(1000 + rank)
+    A_r = (torch.randn(d, 2 * fs, device="cuda", generator=g) * 0.02).to(torch.bfloat16)
+    B_r = (torch.randn(fs, d, device="cuda", generator=g) * 0.02).to(torch.bfloat16)
+    g.manual_seed(7)                                   # the same tokens on every rank
+    x = torch.randn(T, d, device="cuda", generator=g).to(torch.bfloat16)
+    fused = xgpu.CrossGpuMlp(d, f, tp, "swiglu", T, rank, A_r, B_r)
+    unfused = xgpu.LibraryAllReduceMlp(d, f, tp, "swiglu", T, A_r, B_r)
+    out = torch.empty(T, d, dtype=torch.bfloat16, device="cuda")
+    K, W = args.steps, max(3, args.warmup)
+
+    def timed(fn):
+        for _ in range(W):
+            fn()
+        replicas.barrier()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(K):
+            fn()
+        b.record()
+        b.synchronize()
+        replicas.barrier()
+        return replicas.max_over_ranks(a.elapsed_time(b))
+
+    sampler = ClockSampler(torch.cuda.current_device())
+    sampler.start()
+    ms_fused = timed(lambda: fused.forward(x, out))
+    ms_nccl = timed(lambda: unfused.forward(x))
+    sampler.stop()
+    agree = float((fused.forward(x, out).float() - unfused.forward(x).float()).abs().max())
+    torch.cuda.synchronize()
+    fused.close()
+    if rank == 0:
+        line = {"metric": XGPU_METRIC, "value": T * K / (ms_fused / 1e3), "unit": "tokens/s", "n_gpus": world,
+                "steps": K, "warmup": W, "ms_per_step": ms_fused / K, "higher_is_better": True,
+                "scaling": "strong", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": f"xgpu_decode_bs32: bf16 SwiGLU MLP, tokens={T}, d_model={d}, d_ff={f}, "
+                                       f"tp={tp} (one rank per GPU), random weights N(0,0.02^2)",
+                           "tokens": T, "d_model": d, "d_ff": f, "tp": tp, "parallelism": f"tp{tp}"},
+                "nccl_allreduce_arm": {"ms_per_step": ms_nccl / K, "value": T * K / (ms_nccl / 1e3),
+                                       "unit": "tokens/s",
+                                       "what": "library fp32 partial per rank + torch.distributed all_reduce"},
+                "max_abs_difference_between_arms": agree, "gpu_launches": K * 2, "clocks": sampler.summary(),
+                "note": "n_gpus=1 has no exchange partner (tp 1)" if world == 1 else ""}
+        print(json.dumps(line), flush=True)
+    replicas.finish()
+    return 0
+
+
 def main():
     args = parse()
+    if args.config == "xgpu_decode_bs32":
+        if args.impl == "reference":
+            if int(os.environ.get("RANK", 0)) == 0:
+                print(json.dumps({"impl": "reference", "unavailable": "the cross-GPU mode has no oracle arm; "
+                                  "its correctness is in tests/test_gpu_xgpu.py"}), flush=True)
+            return 0
+        return run_xgpu(args)
     op = small_op(args)
     if op is not None:
         return run_small_op_reference(args, op) if args.impl == "reference" else run_small_op(args, op)

@@ -234,7 +234,21 @@ int tp_mlp_create(tp_mlp_t *handle, int d_model, int d_ff, int d_out, int tp_deg
     const int widths[4] = {16, 32, 64, 128};
     for (int i = 0; i < 4; ++i) {
         const int t = widths[i] < max_tokens ? widths[i] : max_tokens;
-        h->tc_part[i] = (i == 0 || max_tokens > widths[i - 1]) ? tc_workspace_bytes(problem_of(h, t), h->num_sms) : 0;
+        if (i > 0 && max_tokens <= widths[i - 1]) {
+            h->tc_part[i] = 0;
+            continue;
+        }
+        Problem p = problem_of(h, t);
+        size_t m = tc_workspace_bytes(p, h->num_sms);
+        // the cross-GPU step runs one rank's shards alone (tp 1, d_ff / tp features)
+        Problem p1 = p;
+        p1.tp = 1;
+        p1.d_ff = p.fs;
+        if (p.fs % 64 == 0) {
+            const size_t m1 = tc_workspace_bytes(p1, h->num_sms);
+            m = m1 > m ? m1 : m;
+        }
+        h->tc_part[i] = m;
     }
     *handle = h;
     return TP_MLP_OK;

@@ -32,7 +32,10 @@ Handle = Tuple[bytes, int]   # (64-byte CUDA IPC handle, offset of the buffer in
 
 
 def exchange_handles(local: Handle, group=None) -> List[Handle]:
-    """Every rank's (handle, offset), in rank order, on every rank."""
+    """Every rank's (handle, offset), in rank order, on every rank (a single
+    process without a process group has only its own)."""
+    if not dist.is_initialized():
+        return [(bytes(local[0]), int(local[1]))]
     world = dist.get_world_size(group)
     out: List[Optional[Handle]] = [None] * world
     dist.all_gather_object(out, (bytes(local[0]), int(local[1])), group=group)
@@ -99,7 +102,8 @@ class CrossGpuMlp:
 def allreduce_partial(z: torch.Tensor, group=None) -> torch.Tensor:
     """The comparison arm's exchange: the process group's all_reduce (sum) of
     this rank's partial, in place (NCCL for CUDA tensors, gloo on the CPU)."""
-    dist.all_reduce(z, op=dist.ReduceOp.SUM, group=group)
+    if dist.is_initialized():
+        dist.all_reduce(z, op=dist.ReduceOp.SUM, group=group)
     return z
 
 
