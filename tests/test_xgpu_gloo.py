@@ -71,29 +71,44 @@ def test_exchange_and_library_allreduce_on_two_gloo_ranks(tmp_path):
         assert r["err"] <= 1e-5                                   # rank sum == unsharded MLP (fp32 sum)
 
 
-def _worker_leaves(rank, world, port, out_dir):
+def _worker_leaves(rank, world, port, out_dir, when):
     _env(rank, world, port)
     import datetime
     import time
+    import torch
     import torch.distributed as dist
     from tensor_sharded_mlp_b200 import xgpu
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=5))
     dist.barrier()
-    if rank == 1:
+    if when == "before_exchange" and rank == 1:
         return                              # leaves before the handle exchange, nothing in flight
+    steps_done = 0
+    if when == "between_steps":
+        xgpu.exchange_handles((bytes([rank + 1]) * 64, 0))
+        for _ in range(2):                  # two steps of the comparison arm's exchange
+            xgpu.allreduce_partial(torch.ones(4, 8))
+            steps_done += 1
+        if rank == 1:
+            return                          # leaves between steps, nothing in flight
     t0 = time.time()
     outcome = "no error"
     try:
-        xgpu.exchange_handles((bytes(64), 0))
+        if when == "before_exchange":
+            xgpu.exchange_handles((bytes(64), 0))
+        else:
+            xgpu.allreduce_partial(torch.ones(4, 8))
     except Exception as e:
         outcome = type(e).__name__
     with open(os.path.join(out_dir, "survivor.json"), "w") as f:
-        json.dump({"outcome": outcome, "seconds": time.time() - t0}, f)
+        json.dump({"outcome": outcome, "seconds": time.time() - t0, "steps_done": steps_done}, f)
 
 
-def test_a_rank_that_leaves_before_the_exchange_is_detected(tmp_path):
+@pytest.mark.parametrize("when", ["before_exchange", "between_steps"])
+def test_a_rank_that_leaves_is_detected(tmp_path, when):
     port = _free_port()
-    mp.start_processes(_worker_leaves, args=(2, port, str(tmp_path)), nprocs=2, start_method="spawn", join=True)
+    mp.start_processes(_worker_leaves, args=(2, port, str(tmp_path), when), nprocs=2, start_method="spawn",
+                       join=True)
     r = json.load(open(tmp_path / "survivor.json"))
     assert r["outcome"] != "no error"
     assert r["seconds"] < 60
+    assert r["steps_done"] == (2 if when == "between_steps" else 0)
