@@ -675,12 +675,25 @@ class MlpRun:
         b.synchronize()
         return a.elapsed_time(b) / n
 
-    def timed(self, K, barrier):
+    TENSOR_PLANS = ("tc_wide", "tc_wide256", "tc_pair", "tc_pair2")
+
+    def timed(self, K, barrier, kernel_events=False):
         """K clean steps back to back (each may overlap the previous one's tail
         through programmatic dependent launch), CUDA events on the launch stream,
-        NVML clocks sampled over the window.  Returns (ms, clock summary)."""
+        NVML clocks sampled over the window.  Returns (ms, clock summary, mean ms
+        per phase or None).  kernel_events: the library also records events
+        before, between and after its kernels inside this timed region -- for
+        the tensor-bound tilings, whose millisecond kernels gain nothing from
+        launch overlap, so each kernel is timed under the same clocks as the step."""
         torch = self.torch
         stream = torch.cuda.current_stream()
+        ev = None
+        if kernel_events:
+            ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+            for row in ev:
+                for e in row:
+                    e.record(stream)
+            torch.cuda.synchronize()
         sampler = ClockSampler(torch.cuda.current_device())
         sampler.start()
         time.sleep(0.1)
@@ -688,13 +701,19 @@ class MlpRun:
         barrier()
         t0 = time.perf_counter()
         start.record(stream)
-        for _ in range(K):
+        for i in range(K):
+            if ev is not None:
+                self.binding.tp_mlp_set_profile_events(self.m.h, ev[i])
             self.fwd()
         end.record(stream)
         barrier()
         sampler.mark(t0, time.perf_counter())
         sampler.stop()
-        return start.elapsed_time(end), sampler.summary()
+        phases = None
+        if ev is not None:
+            self.binding.tp_mlp_set_profile_events(self.m.h, None)
+            phases = [statistics.fmean(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(K)) for j in range(2)]
+        return start.elapsed_time(end), sampler.summary(), phases
 
     def phases(self, K, barrier):
         """The same K steps again with the library recording events before, between
@@ -721,7 +740,7 @@ class MlpRun:
         T, d, f, act, dt = c["tokens"], c["d_model"], c["d_ff"], c["act"], c["dtype"]
         j = int(np.argmax(kern_ms))
         extra = {}
-        if self.plan in ("tc_wide", "tc_wide256", "tc_pair", "tc_pair2"):
+        if self.plan in self.TENSOR_PLANS:
             bound, unit = "tensor", "TFLOP/s"
             work = counts.gemm1_flops(T, d, f, act) if j == 0 else counts.gemm2_flops(T, f, d)
             achieved = work / (kern_ms[j] / 1e3) / 1e12
@@ -741,7 +760,11 @@ class MlpRun:
         r = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
              "traffic": recorded_traffic(kname, workload_key), "kernel": PHASE_NAMES[j] + split,
              "kernel_ms": kern_ms[j], "algorithmic_per_launch": work, "peak_source": peak_note,
-             "kernel_ms_all": kern_ms}
+             "kernel_ms_all": kern_ms,
+             "kernel_timer": ("CUDA events around each kernel inside the timed region"
+                              if self.plan in self.TENSOR_PLANS else
+                              "CUDA events around each kernel in a second pass of the same steps (an event "
+                              "between two kernels would stop their launch overlap in the timed region)")}
         r.update(extra)
         return r
 
@@ -769,8 +792,9 @@ def measure_extra(name, tokens, tp, args, peaks, src, barrier, cpu):
     run.warm(W)
     est = run.estimate_ms()
     K = max(args.steps, int(np.ceil(EXTRA_MIN_TIMED_S * 1e3 / max(est, 1e-3))))
-    ms_total, clocks = run.timed(K, barrier)
-    kern_ms = run.phases(min(K, 200), barrier)
+    ms_total, clocks, kern_ms = run.timed(K, barrier, kernel_events=run.plan in MlpRun.TENSOR_PLANS)
+    if kern_ms is None:
+        kern_ms = run.phases(min(K, 200), barrier)
     ms = ms_total / K
     rates, step_bytes = run.step_rates(ms)
     key = name if tokens is None else f"{name}_T{tokens}"
@@ -895,8 +919,9 @@ def main():
     K, W = args.steps, max(3, args.warmup)
     run.warm(W)
     nk, plan = run.nk, run.plan
-    elapsed_ms, clocks = run.timed(K, barrier)
-    kern_ms = run.phases(K, barrier)
+    elapsed_ms, clocks, kern_ms = run.timed(K, barrier, kernel_events=plan in MlpRun.TENSOR_PLANS)
+    if kern_ms is None:
+        kern_ms = run.phases(K, barrier)
     elapsed_ms = replicas.max_over_ranks(elapsed_ms)
     graph_steps = None
     if not args.no_graph:
