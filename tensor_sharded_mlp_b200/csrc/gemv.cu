@@ -8,6 +8,11 @@
 //     reads one contiguous run of 32 KB blocks (256 rows x 64 k);
 //   * one producer thread moves the blocks into a ring of shared-memory
 //     stages with bulk copies (cp.async.bulk, 128 KB in flight per SM);
+//   * the activations a CTA needs (the k-blocks of its share: at most one
+//     tile's K, as a cyclic window) are bulk-copied into shared memory once,
+//     as soon as the previous kernel is done, instead of being read per block
+//     from L2 (whose latency, under a full weight stream, held back the CTAs
+//     that saw the most of it: the step took 9 % longer);
 //   * eight compute warps take 32 rows each; per step a lane reads one
 //     16-byte granule (8 weights) of one row, so a warp reads 512 contiguous
 //     bytes, and multiplies it with the matching 8 activations of each token;
@@ -50,6 +55,7 @@ struct GemvArgs {
     float *part;              // [tile][slot][T][256] fp32
     unsigned *tile_cnt;       // k-blocks done per tile, zero between launches
     int *status;
+    int xwin;                 // k-blocks of X staged in shared memory per token (0: read X from L2)
 };
 
 struct GemvSmem {
@@ -58,7 +64,12 @@ struct GemvSmem {
     float *rowsum;            // [T][256]
     volatile int *abort;
     int *flag;
+    uint64_t *xbar;           // completes when the staged X has landed
+    __nv_bfloat16 *xs;        // [T][xwin][64] staged X, k-block kb at slot (kb - first kb) mod KB
 };
+
+constexpr size_t kSmemFixed = 128 + STAGES * (size_t)BLK_BYTES + 2 * STAGES * 8 + 16 + 128;
+constexpr size_t kSmemOptin = 227 * 1024;   // largest dynamic shared memory of one CTA on sm_100
 
 template <int T>
 __device__ __forceinline__ GemvSmem gemv_carve(uint8_t *raw) {
@@ -70,12 +81,33 @@ __device__ __forceinline__ GemvSmem gemv_carve(uint8_t *raw) {
     s.rowsum = reinterpret_cast<float *>(s.empty + STAGES);
     s.abort = reinterpret_cast<volatile int *>(s.rowsum + T * kTileRows);
     s.flag = const_cast<int *>(s.abort) + 1;
+    s.xbar = reinterpret_cast<uint64_t *>(reinterpret_cast<uint8_t *>(s.flag) + 12);
+    s.xs = reinterpret_cast<__nv_bfloat16 *>(reinterpret_cast<uint8_t *>(s.xbar) + 128);
     return s;
 }
 
+size_t gemv_smem_bytes(int T, int xwin) {
+    return kSmemFixed + (size_t)T * kTileRows * 4 + (size_t)T * xwin * kKBlock * 2;
+}
+
+// Thread 0 of the compute warps: bulk-copy the X this CTA's share reads into
+// s.xs.  The share's k-blocks form the cyclic window [kbs, kbs + W) mod KB, at
+// most two contiguous runs of every token's row of X.  The last block of a row
+// may be partial (K % 64 != 0); the readers skip k >= K.
 template <int T>
-constexpr size_t gemv_smem_bytes() {
-    return 128 + STAGES * (size_t)BLK_BYTES + 2 * STAGES * 8 + T * kTileRows * 4 + 16;
+__device__ __forceinline__ void stage_x(const GemvArgs &a, const GemvSmem &s, int kbs, int W) {
+    const int r1e = min(a.KB, kbs + W);
+    const int r2e = kbs + W - a.KB;   // > 0: the window wraps to k-block 0
+    const uint32_t n1 = (uint32_t)(min(r1e * kKBlock, a.K) - kbs * kKBlock) * 2;
+    const uint32_t n2 = r2e > 0 ? (uint32_t)min(r2e * kKBlock, a.K) * 2 : 0u;
+    const uint32_t xb = smem_u32(s.xbar);
+    mbar_arrive_expect_tx(xb, T * (n1 + n2));
+#pragma unroll
+    for (int t = 0; t < T; ++t) {
+        __nv_bfloat16 *row = s.xs + (size_t)t * a.xwin * kKBlock;
+        bulk_load(smem_u32(row), a.x + (long)t * a.K + kbs * kKBlock, n1, xb);
+        if (n2) bulk_load(smem_u32(row + (size_t)(a.KB - kbs) * kKBlock), a.x + (long)t * a.K, n2, xb);
+    }
 }
 
 // Final value of row `row` of tile `tile` for all tokens, from s.rowsum.
@@ -101,7 +133,7 @@ __device__ __forceinline__ void finish_row(const GemvArgs &a, const GemvSmem &s,
     }
 }
 
-template <int T>
+template <int T, bool XS>
 __global__ void __launch_bounds__(NTHR, 1) gemv_kernel(GemvArgs a) {
     extern __shared__ uint8_t smem_raw[];
     const GemvSmem s = gemv_carve<T>(smem_raw);
@@ -111,6 +143,7 @@ __global__ void __launch_bounds__(NTHR, 1) gemv_kernel(GemvArgs a) {
             mbar_init(smem_u32(&s.full[i]), 1);
             mbar_init(smem_u32(&s.empty[i]), CWARPS);
         }
+        mbar_init(smem_u32(s.xbar), 1);
         *s.abort = 0;
         fence_barrier_init();
     }
@@ -138,11 +171,17 @@ __global__ void __launch_bounds__(NTHR, 1) gemv_kernel(GemvArgs a) {
         }
     } else {
         pdl_wait_previous();   // X and the outputs belong to the previous kernel until it is done
+        const int kbs = (int)(it_b % KB);
+        bool xok = true;
+        if (XS) {
+            if (threadIdx.x == 0) stage_x<T>(a, s, kbs, (int)min((long long)KB, it_e - it_b));
+            xok = mbar_wait(smem_u32(s.xbar), 0, s.abort);
+        }
         const int g = lane & 7;                         // granule (8 k) of the row
         const int rbase = warp * 32 + (lane >> 3);      // rows rbase + 4j, j = 0..7
         int stage = 0;
         uint32_t phase = 0;
-        for (long long it = it_b; it < it_e;) {
+        for (long long it = it_b; xok && it < it_e;) {
             const int tile = (int)(it / KB);
             const int kb0 = (int)(it - (long long)tile * KB);
             const int kb1 = (int)min((long long)KB, it_e - (long long)tile * KB);
@@ -157,10 +196,13 @@ __global__ void __launch_bounds__(NTHR, 1) gemv_kernel(GemvArgs a) {
                 // this lane's 8 activations of every token for k = kb*64 + 8g ..
                 float xv[T][8];
                 const int k = kb * kKBlock + g * 8;
+                const int slot = kb - kbs + (kb < kbs ? KB : 0);
 #pragma unroll
                 for (int t = 0; t < T; ++t) {
                     if (k < a.K) {   // K is a multiple of 8: a granule is all in or all out
-                        const uint4 w4 = __ldg(reinterpret_cast<const uint4 *>(a.x + (long)t * a.K + k));
+                        const uint4 w4 =
+                            XS ? *reinterpret_cast<const uint4 *>(s.xs + ((size_t)t * a.xwin + slot) * kKBlock + g * 8)
+                               : __ldg(reinterpret_cast<const uint4 *>(a.x + (long)t * a.K + k));
                         xv[t][0] = bf16lo(w4.x); xv[t][1] = bf16hi(w4.x);
                         xv[t][2] = bf16lo(w4.y); xv[t][3] = bf16hi(w4.y);
                         xv[t][4] = bf16lo(w4.z); xv[t][5] = bf16hi(w4.z);
@@ -260,13 +302,18 @@ StreamKGeom gemv_geom(long long rows, int K, int num_sms) {
     return streamk_geom(blk_tiles(rows), blk_kblocks(K), num_sms);
 }
 
-template <int T>
+template <int T, bool XS>
 cudaError_t launch_one(const GemvArgs &a, int grid, cudaStream_t st) {
-    constexpr size_t smem = gemv_smem_bytes<T>();
-    auto kern = gemv_kernel<T>;
-    cudaError_t e = ensure_smem_attr(kern, smem);
+    const size_t smem = gemv_smem_bytes(T, XS ? a.xwin : 0);
+    auto kern = gemv_kernel<T, XS>;
+    cudaError_t e = ensure_smem_attr(kern, kSmemOptin);
     if (e != cudaSuccess) return e;
     return launch_pdl(kern, dim3(grid), dim3(NTHR), smem, st, a);
+}
+
+template <int T>
+cudaError_t launch_one(const GemvArgs &a, int grid, cudaStream_t st) {
+    return a.xwin > 0 ? launch_one<T, true>(a, grid, st) : launch_one<T, false>(a, grid, st);
 }
 
 cudaError_t launch_T(int T, const GemvArgs &a, int grid, cudaStream_t st) {
@@ -296,6 +343,9 @@ cudaError_t run_part(const void *w, long long rows, int K, const void *x, int T,
     a.part = part;
     a.tile_cnt = cnt;
     a.status = status;
+    // a share spans at most ceil(total / grid) k-blocks, and the window never more than one tile's K
+    a.xwin = (int)std::min<long long>(g.KB, (g.total + g.grid - 1) / g.grid);
+    if (gemv_smem_bytes(T, a.xwin) > kSmemOptin) a.xwin = 0;
     return launch_T(T, a, g.grid, st);
 }
 

@@ -161,6 +161,7 @@ GEMV_SHAPES = [  # (d_in, d_ff, d_out, tp)
     (520, 400, 264, 4),      # K not a multiple of 256, ragged 128-blocks
     (8192, 1024, 256, 2),    # long K: split-K in the first projection at T >= 3
     (256, 4096, 128, 8),     # few output rows: split-K in the second projection
+    (136, 38400, 200, 4),    # K of 3 blocks, the last ragged: shares longer than K, staged X windows wrap
 ]
 
 
@@ -181,6 +182,23 @@ def test_gemv_decode_parity(act, T, shape):
     assert_close(got, ref, "bf16", "gemv")
     again = m.forward_packed(x, packed)           # split-K counters were reset
     assert torch.equal(got, again)
+
+
+@pytest.mark.slow
+def test_gemv_window_too_large_for_shared_memory():
+    """4 tokens, K = 12160 and 148 tiles of the first projection: a CTA's share
+    is a whole tile's K (190 blocks), whose X (4 x 190 x 128 B) no longer fits
+    beside the weight ring, so that projection reads X from L2 instead."""
+    T, d, f, dout, tp = 4, 12160, 37888, 256, 4
+    p = inputs.generate(T, d, f, "tanh", "bf16", seed=11, init="fan_in", d_out=dout)
+    Ad, Bd, A, Bs = _upload(p, tp, "bf16")
+    ref = oracle.tp_mlp_sharded(p.x, A, Bs, "tanh")
+    del A, Bs
+    m = _mlp(p, tp, "bf16", max_tokens=T)
+    m.set_plan("gemv")
+    got = m.forward_packed(dev(p.x, "bf16"), m.pack(Ad, Bd))
+    assert m.last_plan == "gemv"
+    assert_close(got, ref, "bf16", "gemv, X read from L2")
 
 
 @pytest.mark.parametrize("act", ["tanh", "swiglu"])
