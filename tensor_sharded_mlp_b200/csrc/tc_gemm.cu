@@ -1364,7 +1364,12 @@ int skinny_bt(int T) { return T <= 16 ? 16 : T <= 32 ? 32 : T <= 64 ? 64 : 128; 
 
 // Ring depth of the skinny kernel per token width: 128-row tiles (SKH) and
 // 256-row tiles (SK).  Each stage holds one weight block and one X box, so the
-// wider the token tile, the fewer stages fit in shared memory.
+// wider the token tile, the fewer stages fit in shared memory.  More is not
+// better on a grid of every SM: with 148 CTAs of 6 x 36 KB in flight (decode,
+// 32 tokens) HBM is oversubscribed and serves the SMs unevenly -- equal shares
+// finished 102-142 us after the start -- while 4 stages (21 MB in flight over
+// the GPU) finished in 121-135 us: 3 % off the step at 2-32 tokens.  Fewer
+// than 4 lets two CTAs share an SM, which was far slower.
 #ifndef TPMLP_SKH_S16
 #define TPMLP_SKH_S16 8
 #endif
@@ -1378,13 +1383,13 @@ int skinny_bt(int T) { return T <= 16 ? 16 : T <= 32 ? 32 : T <= 64 ? 64 : 128; 
 #define TPMLP_SKH_S128 6
 #endif
 #ifndef TPMLP_SK_S16
-#define TPMLP_SK_S16 6
+#define TPMLP_SK_S16 4
 #endif
 #ifndef TPMLP_SK_S32
-#define TPMLP_SK_S32 6
+#define TPMLP_SK_S32 4
 #endif
 #ifndef TPMLP_SK_S64
-#define TPMLP_SK_S64 5
+#define TPMLP_SK_S64 4
 #endif
 #ifndef TPMLP_SK_S128
 #define TPMLP_SK_S128 4
