@@ -3,7 +3,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--config decode_bs1|decode_bs32|prefill|sweep|tiny] [--tokens T] [--tp P]
-                    [--plan auto|simt|gemv|tc|tc_skinny|tc_wide|tc_wide256|tc_pair|tc_pair2] [--api packed|shard]
+                    [--plan auto|simt|gemv|tc|tc_skinny|tc_fused|tc_wide|tc_wide256|tc_pair|tc_pair2] [--api packed|shard]
                     [--splitk auto|in_kernel|separate|cluster] [--no-e2e] [--no-cpu-baseline] [--no-graph]
                     [--configs auto|all|none]
     python bench.py --config fused_norm_decode_bs32|fused_norm_prefill|
@@ -613,6 +613,9 @@ EXTRA_CONFIGS = (("decode_bs32", None, None), ("prefill", None, 8), ("sweep", 16
 EXTRA_MIN_TIMED_S = 0.25     # timed window of each extra workload (room for clock samples)
 EXTRA_ORACLE_BUDGET_S = 4.0  # CPU-baseline budget of each extra workload (at least one call)
 PHASE_NAMES = ["first projection + activation", "second projection + rank sum"]
+# tc_fused: one persistent kernel runs both projections; the second projection's
+# split tiles are added by a reduction kernel behind it.
+FUSED_PHASE_NAMES = ["both projections (one persistent kernel)", "split-tile reduction of the second projection"]
 
 
 def config_of(name, tokens=None, tp=None):
@@ -739,6 +742,9 @@ class MlpRun:
         c = self.c
         T, d, f, act, dt = c["tokens"], c["d_model"], c["d_ff"], c["act"], c["dtype"]
         j = int(np.argmax(kern_ms))
+        fused = self.plan == "tc_fused"
+        if fused:
+            j = 0   # the kernel that streams both projections' weights
         extra = {}
         if self.plan in self.TENSOR_PLANS:
             bound, unit = "tensor", "TFLOP/s"
@@ -751,14 +757,18 @@ class MlpRun:
                 extra = {"peak_sustained": sus, "frac_sustained": achieved / sus}
         else:
             bound, unit = "hbm", "GB/s"
-            work = counts.gemm1_bytes(T, d, f, act, dt) if j == 0 else counts.gemm2_bytes(T, f, d, dt)
+            if fused:
+                work = counts.gemm1_bytes(T, d, f, act, dt) + counts.gemm2_bytes(T, f, d, dt)
+            else:
+                work = counts.gemm1_bytes(T, d, f, act, dt) if j == 0 else counts.gemm2_bytes(T, f, d, dt)
             achieved = work / (kern_ms[j] / 1e3) / 1e9
             peak = peaks["hbm_gbs"]
             peak_note = f"hbm_gbs ({src})"
-        kname = f"{self.plan}:{'first' if j == 0 else 'second'}"
+        kname = f"{self.plan}:{'first' if j == 0 else 'second'}" if not fused else "tc_fused:both"
         split = " (GEMM + split-tile reduction kernel)" if self.nk > 2 and self.plan == "tc_skinny" else ""
         r = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
-             "traffic": recorded_traffic(kname, workload_key), "kernel": PHASE_NAMES[j] + split,
+             "traffic": recorded_traffic(kname, workload_key),
+             "kernel": (FUSED_PHASE_NAMES if fused else PHASE_NAMES)[j] + split,
              "kernel_ms": kern_ms[j], "algorithmic_per_launch": work, "peak_source": peak_note,
              "kernel_ms_all": kern_ms,
              "kernel_timer": ("CUDA events around each kernel inside the timed region"

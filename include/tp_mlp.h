@@ -88,8 +88,16 @@ typedef enum {
     TP_MLP_PLAN_TC_PAIR = 7,    /* packed bf16: tcgen05 on pairs of CTAs (cta_group::2),
                                    256 tokens x 256 weight rows per pair, two TMEM
                                    accumulators per CTA                               */
-    TP_MLP_PLAN_TC_PAIR2 = 8    /* packed bf16: pairs of CTAs, 256 tokens x 512 weight
+    TP_MLP_PLAN_TC_PAIR2 = 8,   /* packed bf16: pairs of CTAs, 256 tokens x 512 weight
                                    rows per pair (two weight tiles share each X stage) */
+    TP_MLP_PLAN_TC_FUSED = 9    /* packed bf16, 1..128 tokens: the skinny tiling with
+                                   both projections in one persistent launch (the
+                                   second projection's weights stream in while the
+                                   first finishes; its H loads wait on a device
+                                   counter).  Needs every CTA of the grid (one per
+                                   SM) resident at once: a GPU shared with other work
+                                   can make the bounded wait run out, reported as
+                                   TP_MLP_ERR_TIMEOUT by tp_mlp_get_device_status. */
 } tp_mlp_plan;
 
 /*

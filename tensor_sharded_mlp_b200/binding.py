@@ -27,7 +27,7 @@ ACT = {"tanh": 0, "swiglu": 1, "identity": 2}
 DTYPE = {"f32": 0, "bf16": 1}
 TORCH_DTYPE = {"f32": torch.float32, "bf16": torch.bfloat16}
 PLAN = {"auto": 0, "simt": 1, "gemv": 2, "tc": 3, "tc_wide": 4, "tc_skinny": 5, "tc_wide256": 6, "tc_pair": 7,
-        "tc_pair2": 8}
+        "tc_pair2": 8, "tc_fused": 9}
 PLAN_NAME = {v: k for k, v in PLAN.items()}
 STATUS = {0: "OK", 1: "ERR_INVALID_ARG", 2: "ERR_SHAPE", 3: "ERR_ALIGNMENT", 4: "ERR_UNSUPPORTED",
           5: "ERR_CUDA", 6: "ERR_TIMEOUT", 7: "ERR_WORKSPACE"}

@@ -105,6 +105,7 @@ _KERNEL_SOURCES = {
     "tc_wide256": ["tc_gemm.cu", "common.cuh", "streamk.cuh", "tc_ptx.cuh"],
     "tc_pair": ["tc_gemm.cu", "common.cuh", "streamk.cuh", "tc_ptx.cuh"],
     "tc_pair2": ["tc_gemm.cu", "common.cuh", "streamk.cuh", "tc_ptx.cuh"],
+    "tc_fused": ["tc_gemm.cu", "common.cuh", "streamk.cuh", "tc_ptx.cuh"],
     "simt": ["simt.cu", "common.cuh"],
 }
 

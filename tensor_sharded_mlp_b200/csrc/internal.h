@@ -56,6 +56,7 @@ cudaError_t launch_attn_merge(int P, int rows, int D, const float *maximum, cons
 // Split-tile counters the GEMV and tcgen05 skinny kernels need (one per
 // weight tile of both parts; first part's tiles first).
 size_t tile_counter_slots(const Problem &p);
+size_t fused_counter_offset(const Problem &p);   // the fused skinny kernel's two words
 
 // gemv.cu: decode path, packed bf16, 1..kGemvMaxTokens tokens.
 constexpr int kGemvMaxTokens = 4;
@@ -76,8 +77,11 @@ constexpr int kTcWide256MinTokens = 2048;   // auto, shard form: 256-token tiles
 // 8.56-8.58 ms, 1-CTA 256-token tiles 8.69-8.74, one-tile pairs 8.88-8.93).
 constexpr int kTcPairMinTokens = 512;
 constexpr int kTcPairMaxTokens = 4096;
-enum { kTilingSkinny = 0, kTilingWide128 = 1, kTilingWide256 = 2, kTilingPair = 3, kTilingPair2 = 4 };
+// kTilingFused: the skinny tiling with both projections in one persistent
+// launch (packed weights, 1..kTcSkinnyMaxTokens tokens; fused_supported).
+enum { kTilingSkinny = 0, kTilingWide128 = 1, kTilingWide256 = 2, kTilingPair = 3, kTilingPair2 = 4, kTilingFused = 5 };
 bool tc_supported(const Problem &p);
+bool fused_supported(const Problem &p, int num_sms);
 bool tc_raw_supported(const Problem &p);   // also needs f_s % 64 == 0
 size_t tc_workspace_bytes(const Problem &p, int num_sms);
 // Split tiles of the skinny tiling (values of tp_mlp_splitk): finished by the

@@ -1219,6 +1219,342 @@ __global__ void __launch_bounds__(128) skinny_reduce_kernel(TcArgs a, int BT) {
     }
 }
 
+// ===== fused skinny tiling: both projections in one persistent launch =====
+// A skinny projection is a weight stream of 20-140 us.  Run as two kernels,
+// the second projection's CTAs can start only when the first one's leave
+// their SMs (each holds most of an SM's shared memory), refill their rings
+// from nothing (~3.5 us before the first MMA at 16-128 tokens) and wait for a
+// kernel that adds split tiles in between.  Here every CTA streams its share
+// of the first projection's weights and then, in the same ring, its share of
+// the second's: those blocks do not depend on H and arrive while the first
+// projection's last tiles finish.  Only the X operand of the second
+// projection (H) waits -- for a device counter that reaches the number of
+// first-projection tiles once each tile's H is stored: a whole tile by its
+// CTA, a split tile by the last of its CTAs to arrive, which adds the slots
+// (in slot order, as skinny_reduce_kernel does).  Split tiles of the second
+// projection go to skinny_reduce_kernel, launched behind: finished inside the
+// kernel, by the last CTA of each tile, they left those few CTAs a long
+// latency-bound tail (sweep, 128 tokens: 64.9 against 54.3 us).  Every
+// CTA of the grid (one per SM at most) must be resident at once for the
+// counter to be reached; the wait is bounded, so a grid that cannot be fails
+// with a status instead of hanging.  The last CTA past the wait resets it.
+struct FusedMaps {
+    CUtensorMap w1, w2;   // packed parts: boxes of 256 (or 128) rows x 64 k
+    CUtensorMap x, h;     // X (T x d_in) and H (T x d_ff): boxes of BT rows x 64 k
+    unsigned *h_done;     // first-projection tiles whose H is stored, this launch
+    unsigned *exits;      // CTAs past their wait on h_done, this launch
+    unsigned h_tiles;     // first-projection tiles
+};
+
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned *p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Last CTA of a split tile: add its n slots in slot order (the order of
+// skinny_reduce_kernel, so both routes give the same bits) and apply the
+// epilogue.  Each thread walks whole float4 positions (row r, 4 tokens), U of
+// them at a time, so the loads of several positions and slots are in flight
+// together.  Runs on the 128 epilogue threads.
+template <int BT, bool HALF>
+__device__ __forceinline__ void fixup_tile(const TcArgs &a, int tile, int n) {
+    constexpr int ROWS = HALF ? 128 : 256;
+    constexpr long SLOT4 = (long)ROWS * BT / 4;   // float4s per slot
+    constexpr int NPOS = (BT / 4) * 128;           // (token quad, row) positions
+    constexpr int U = 4;
+    const float4 *tb = reinterpret_cast<const float4 *>(a.part + (long long)tile * a.slots * ROWS * BT);
+#pragma unroll 1
+    for (int p0 = threadIdx.x - 64; p0 < NPOS; p0 += 128 * U) {
+        float4 s0[U], s1[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) s0[u] = s1[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 2
+        for (int sl = 0; sl < n; ++sl) {
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int pos = p0 + u * 128;
+                if (pos < NPOS) {
+                    const long o = sl * SLOT4 + (long)(pos >> 7) * ROWS + (pos & 127);
+                    const float4 g = __ldcg(tb + o);
+                    s0[u].x += g.x; s0[u].y += g.y; s0[u].z += g.z; s0[u].w += g.w;
+                    if (!HALF) {
+                        const float4 h = __ldcg(tb + o + 128);
+                        s1[u].x += h.x; s1[u].y += h.y; s1[u].z += h.z; s1[u].w += h.w;
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int pos = p0 + u * 128;
+            if (pos >= NPOS) continue;
+            if (HALF)
+                skinny_final_half4(a, tile, pos & 127, (pos >> 7) * 4, s0[u]);
+            else
+                skinny_final4(a, tile, pos & 127, (pos >> 7) * 4, s0[u], s1[u]);
+        }
+    }
+}
+
+// One unit of the fused kernel's epilogue (this CTA's k-blocks kb0..kb1 of
+// weight tile `tile`), on the 128 epilogue threads.  h_done != nullptr: a
+// first-projection unit, whose tile is counted once its H is final.  Returns
+// false if a wait gave up.
+template <int BT, bool HALF>
+__device__ __forceinline__ bool fused_unit(const TcArgs &a, const Smem &s, __nv_bfloat16 *stage_out,
+                                           uint32_t tmem_base, int tile, int kb0, int kb1, int &acc,
+                                           uint32_t &acc_phase, int c, unsigned *h_done) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int q = warp & 3;
+    const int r = q * 32 + lane;   // row within each 128-row half
+    constexpr int ROWS = HALF ? 128 : 256;
+    if (!mbar_wait(smem_u32(&s.tfull[acc]), acc_phase, s.abort)) return false;
+    tc_fence_after();
+    const uint32_t taddr = tmem_base + acc * (2 * BT) + ((uint32_t)(q * 32) << 16);
+    bool final_here = true;   // this CTA wrote the tile's final values
+    if (kb0 == 0 && kb1 == a.KB) {
+#pragma unroll 1
+        for (int t0 = 0; t0 < BT; t0 += 16) {
+            float v0[16], v1[16];
+            tmem_ld16(taddr + t0, v0);
+            if (!HALF) tmem_ld16(taddr + BT + t0, v1);
+            tmem_ld_wait();
+            if (HALF) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) stage_out[(t0 + i) * 128 + r] = __float2bfloat16_rn(act_out(a.epi, v0[i]));
+            } else {
+                skinny_final16(a, tile, r, t0, v0, v1);
+            }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&s.tempty[acc]));
+        if (HALF) {
+            named_bar(1, 128);   // the whole tile is staged
+            skinny_store_staged(a, tile, BT, stage_out);
+        }
+    } else {
+        // this CTA's share of the tile -> its slot, [token/4][row][token%4]
+        const long long it0 = (long long)tile * a.KB;
+        const int c_first = share_owner(it0, a.total_iters, a.grid);
+        float4 *base = reinterpret_cast<float4 *>(a.part + ((long long)tile * a.slots + (c - c_first)) * ROWS * BT);
+#pragma unroll 1
+        for (int t0 = 0; t0 < BT; t0 += 16) {
+            float v0[16], v1[16];
+            tmem_ld16(taddr + t0, v0);
+            if (!HALF) tmem_ld16(taddr + BT + t0, v1);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int qd = t0 / 4 + j;
+                base[qd * ROWS + r] = make_float4(v0[4 * j], v0[4 * j + 1], v0[4 * j + 2], v0[4 * j + 3]);
+                if (!HALF)
+                    base[qd * ROWS + 128 + r] = make_float4(v1[4 * j], v1[4 * j + 1], v1[4 * j + 2], v1[4 * j + 3]);
+            }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&s.tempty[acc]));
+        if (a.split_mode != kSplitInKernel) {
+            final_here = false;   // skinny_reduce_kernel adds the slots
+        } else {
+            // the last CTA of the tile to arrive adds its n slots in slot order
+            __threadfence();
+            named_bar(1, 128);
+            if (threadIdx.x == 64) {
+                const unsigned done_kb = atomicAdd(&a.tile_cnt[tile], (unsigned)(kb1 - kb0)) + (kb1 - kb0);
+                *s.flag = (done_kb == (unsigned)a.KB);
+            }
+            named_bar(1, 128);
+            final_here = *s.flag != 0;
+            if (final_here) {
+                __threadfence();
+                fixup_tile<BT, HALF>(a, tile, share_owner(it0 + a.KB - 1, a.total_iters, a.grid) - c_first + 1);
+                if (threadIdx.x == 64) a.tile_cnt[tile] = 0u;
+            }
+        }
+    }
+    if (h_done) __threadfence();   // H of this tile before the count that publishes it
+    named_bar(1, 128);             // staging and the flag are free for the next unit
+    if (h_done && final_here && threadIdx.x == 64) atomicAdd(h_done, 1u);
+    acc ^= 1;
+    if (acc == 0) acc_phase ^= 1;
+    return true;
+}
+
+template <bool HALF>
+__device__ __forceinline__ void load_w_packed(uint32_t dst, const CUtensorMap *m, int tile, int kb, int KB,
+                                              uint32_t bar) {
+    if (HALF)
+        tma_load_2d(dst, m, 0, ((tile >> 1) * KB + kb) * 256 + (tile & 1) * 128, bar);
+    else
+        tma_load_2d(dst, m, 0, (tile * KB + kb) * 256, bar);
+}
+
+// HALF: 128-row tiles in both projections (tanh / identity); otherwise 256.
+template <int BT, int STAGES, bool HALF>
+__global__ void __launch_bounds__(NTHREADS, 1)
+    tc_fused_kernel(const __grid_constant__ FusedMaps m, const __grid_constant__ TcArgs a1,
+                    const __grid_constant__ TcArgs a2) {
+    constexpr uint32_t W_BYTES = (HALF ? 128 : 256) * BK * 2;
+    constexpr uint32_t X_BYTES = BT * BK * 2;
+    extern __shared__ uint8_t smem_raw[];
+    const Smem s = carve<STAGES>(smem_raw, W_BYTES, X_BYTES);
+    __nv_bfloat16 *stage_out = reinterpret_cast<__nv_bfloat16 *>(
+        (reinterpret_cast<uintptr_t>(s.tmem_slot) + 16 + 15) & ~uintptr_t(15));
+    const uint32_t tmem_base = setup<STAGES>(s, &m.w1, &m.x);
+    pdl_allow_dependents();
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int c = blockIdx.x;
+    const long long b1 = share_begin(c, a1.total_iters, a1.grid), e1 = share_begin(c + 1, a1.total_iters, a1.grid);
+    long long b2 = 0, e2 = 0;   // CTAs beyond the second projection's grid have no share of it
+    if (c < a2.grid) {
+        b2 = share_begin(c, a2.total_iters, a2.grid);
+        e2 = share_begin(c + 1, a2.total_iters, a2.grid);
+    }
+
+    if (warp == 0) {
+        if (lane == 0) {
+            tma_prefetch_desc(&m.w2);
+            tma_prefetch_desc(&m.h);
+            // first projection: the weights of the first stages before the
+            // wait on the previous kernel, then X
+            const int npre = (int)min((long long)STAGES, e1 - b1);
+            for (int i = 0; i < npre; ++i) {
+                const long long it = b1 + i;
+                const int tile = (int)(it / a1.KB), kb = (int)(it - (long long)tile * a1.KB);
+                const uint32_t fb = smem_u32(&s.full[i]);
+                mbar_arrive_expect_tx(fb, W_BYTES + X_BYTES);
+                load_w_packed<HALF>(smem_u32(s.a + i * W_BYTES), &m.w1, tile, kb, a1.KB, fb);
+            }
+            pdl_wait_previous();
+            for (int i = 0; i < npre; ++i) {
+                const long long it = b1 + i;
+                const int kb = (int)(it - it / a1.KB * a1.KB);
+                tma_load_2d(smem_u32(s.b + i * X_BYTES), &m.x, kb * BK, 0, smem_u32(&s.full[i]));
+            }
+            int stage = npre % STAGES;
+            uint32_t phase = npre == STAGES ? 1u : 0u;
+            for (long long it = b1 + npre; it < e1; ++it) {
+                const int tile = (int)(it / a1.KB), kb = (int)(it - (long long)tile * a1.KB);
+                if (!mbar_wait(smem_u32(&s.empty[stage]), phase ^ 1, s.abort)) goto done;
+                const uint32_t fb = smem_u32(&s.full[stage]);
+                mbar_arrive_expect_tx(fb, W_BYTES + X_BYTES);
+                load_w_packed<HALF>(smem_u32(s.a + stage * W_BYTES), &m.w1, tile, kb, a1.KB, fb);
+                tma_load_2d(smem_u32(s.b + stage * X_BYTES), &m.x, kb * BK, 0, fb);
+                if (++stage == STAGES) { stage = 0; phase ^= 1; }
+            }
+            // second projection: weights into the stages as they free up, H
+            // once every first-projection tile has been stored
+            const int npre2 = (int)min((long long)STAGES, e2 - b2);
+            const int stage0 = stage;
+            for (int i = 0; i < npre2; ++i) {
+                const long long it = b2 + i;
+                const int tile = (int)(it / a2.KB), kb = (int)(it - (long long)tile * a2.KB);
+                if (!mbar_wait(smem_u32(&s.empty[stage]), phase ^ 1, s.abort)) goto done;
+                const uint32_t fb = smem_u32(&s.full[stage]);
+                mbar_arrive_expect_tx(fb, W_BYTES + X_BYTES);
+                load_w_packed<HALF>(smem_u32(s.a + stage * W_BYTES), &m.w2, tile, kb, a2.KB, fb);
+                if (++stage == STAGES) { stage = 0; phase ^= 1; }
+            }
+            {
+                // every CTA waits (also one without a share of the second
+                // projection), so that the last to pass can reset both words
+                const unsigned long long t0 = globaltimer();
+                while (ld_acquire_gpu(m.h_done) < m.h_tiles) {
+                    if (*s.abort) goto done;
+                    if (globaltimer() - t0 > kWaitLimitNs) {
+                        *s.abort = 1;
+                        goto done;
+                    }
+                }
+                if (atomicAdd(m.exits, 1u) == gridDim.x - 1) {   // every CTA is past the wait
+                    atomicExch(m.h_done, 0u);
+                    atomicExch(m.exits, 0u);
+                }
+            }
+            if (npre2 > 0) {
+                // H was written with generic stores: order them before this thread's TMA reads
+                asm volatile("fence.proxy.async.global;" ::: "memory");
+                int sx = stage0;
+                for (int i = 0; i < npre2; ++i) {
+                    const long long it = b2 + i;
+                    const int kb = (int)(it - it / a2.KB * a2.KB);
+                    tma_load_2d(smem_u32(s.b + sx * X_BYTES), &m.h, kb * BK, 0, smem_u32(&s.full[sx]));
+                    if (++sx == STAGES) sx = 0;
+                }
+            }
+            for (long long it = b2 + npre2; it < e2; ++it) {
+                const int tile = (int)(it / a2.KB), kb = (int)(it - (long long)tile * a2.KB);
+                if (!mbar_wait(smem_u32(&s.empty[stage]), phase ^ 1, s.abort)) goto done;
+                const uint32_t fb = smem_u32(&s.full[stage]);
+                mbar_arrive_expect_tx(fb, W_BYTES + X_BYTES);
+                load_w_packed<HALF>(smem_u32(s.a + stage * W_BYTES), &m.w2, tile, kb, a2.KB, fb);
+                tma_load_2d(smem_u32(s.b + stage * X_BYTES), &m.h, kb * BK, 0, fb);
+                if (++stage == STAGES) { stage = 0; phase ^= 1; }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t idesc = idesc_bf16_f32(128, BT);
+            int stage = 0, acc = 0;
+            uint32_t phase = 0, acc_phase = 0;
+            for (int ph = 0; ph < 2; ++ph) {
+                const int KB = ph ? a2.KB : a1.KB;
+                const long long ie = ph ? e2 : e1;
+                for (long long it = ph ? b2 : b1; it < ie;) {
+                    const int tile = (int)(it / KB);
+                    const int kb0 = (int)(it - (long long)tile * KB);
+                    const int kb1 = (int)min((long long)KB, ie - (long long)tile * KB);
+                    if (!mbar_wait(smem_u32(&s.tempty[acc]), acc_phase ^ 1, s.abort)) goto done;
+                    tc_fence_after();
+                    const uint32_t d0 = tmem_base + acc * (2 * BT), d1 = d0 + BT;
+                    for (int kb = kb0; kb < kb1; ++kb) {
+                        if (!mbar_wait(smem_u32(&s.full[stage]), phase, s.abort)) goto done;
+                        tc_fence_after();
+                        const uint32_t wa = smem_u32(s.a + stage * W_BYTES);
+                        const uint64_t dw0 = smem_desc_kmajor_sw128(wa), dw1 = smem_desc_kmajor_sw128(wa + 128 * 128);
+                        const uint64_t dx = smem_desc_kmajor_sw128(smem_u32(s.b + stage * X_BYTES));
+#pragma unroll
+                        for (int k = 0; k < BK / 16; ++k) {
+                            const uint32_t accum = (kb != kb0 || k != 0) ? 1u : 0u;
+                            mma_bf16(d0, dw0 + 2 * k, dx + 2 * k, idesc, accum);
+                            if (!HALF) mma_bf16(d1, dw1 + 2 * k, dx + 2 * k, idesc, accum);
+                        }
+                        mma_commit(smem_u32(&s.empty[stage]));
+                        if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                    }
+                    mma_commit(smem_u32(&s.tfull[acc]));
+                    acc ^= 1;
+                    if (acc == 0) acc_phase ^= 1;
+                    it = (long long)tile * KB + kb1;
+                }
+            }
+        }
+    } else {
+        pdl_wait_previous();
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        bool ok = true;
+        for (int ph = 0; ph < 2 && ok; ++ph) {
+            const TcArgs &a = ph ? a2 : a1;
+            const long long ie = ph ? e2 : e1;
+            for (long long it = ph ? b2 : b1; it < ie && ok;) {
+                const int tile = (int)(it / a.KB);
+                const int kb0 = (int)(it - (long long)tile * a.KB);
+                const int kb1 = (int)min((long long)a.KB, ie - (long long)tile * a.KB);
+                it = (long long)tile * a.KB + kb1;
+                ok = fused_unit<BT, HALF>(a, s, stage_out, tmem_base, tile, kb0, kb1, acc, acc_phase, c,
+                                          ph ? nullptr : m.h_done);
+            }
+        }
+    }
+done:
+    teardown(s, tmem_base, a1.status);
+}
+
 // ======================================= host side =======================================
 
 typedef CUresult (*PFN_encodeTiled)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
@@ -1657,6 +1993,144 @@ int first_epi(int act) {
     return act == TP_MLP_ACT_SWIGLU ? EPI_H_SWIGLU : act == TP_MLP_ACT_TANH ? EPI_H_TANH : EPI_H_IDENT;
 }
 
+// Ring depth of the fused kernel (defaults: the skinny kernel's).
+#ifndef TPMLP_FZH_S16
+#define TPMLP_FZH_S16 TPMLP_SKH_S16
+#endif
+#ifndef TPMLP_FZH_S32
+#define TPMLP_FZH_S32 TPMLP_SKH_S32
+#endif
+#ifndef TPMLP_FZH_S64
+#define TPMLP_FZH_S64 TPMLP_SKH_S64
+#endif
+#ifndef TPMLP_FZH_S128
+#define TPMLP_FZH_S128 TPMLP_SKH_S128
+#endif
+#ifndef TPMLP_FZ_S16
+#define TPMLP_FZ_S16 TPMLP_SK_S16
+#endif
+#ifndef TPMLP_FZ_S32
+#define TPMLP_FZ_S32 TPMLP_SK_S32
+#endif
+#ifndef TPMLP_FZ_S64
+#define TPMLP_FZ_S64 TPMLP_SK_S64
+#endif
+#ifndef TPMLP_FZ_S128
+#define TPMLP_FZ_S128 TPMLP_SK_S128
+#endif
+
+// Fused skinny tiling: one grid for both projections, the first projection's
+// (skinny_grid); the second is split evenly over the same CTAs.
+struct FusedGeom {
+    StreamKGeom g1, g2;
+};
+FusedGeom fused_geom(const Problem &p, bool half, int num_sms) {
+    const int BT = skinny_bt(p.T);
+    FusedGeom f;
+    f.g1 = skinny_geom((int)skinny_tiles(p, 0, false, half), (int)blk_kblocks(p.d_in), BT, num_sms);
+    f.g2 = streamk_geom(skinny_tiles(p, 1, false, half), blk_kblocks(p.d_ff), f.g1.grid);
+    return f;
+}
+// 128-row tiles for tanh / identity when no first-projection tile is split
+// (a split 128-row tile has no in-kernel finish); 256 otherwise, and always for
+// SwiGLU (gate and up share a tile).
+bool fused_half(const Problem &p, int num_sms) {
+    return p.act != TP_MLP_ACT_SWIGLU && skinny_bt(p.T) >= TPMLP_SKINNY_HALF_MIN_BT &&
+           fused_geom(p, true, num_sms).g1.slots == 1;
+}
+
+bool fused_ok(const Problem &p, int num_sms) {
+    (void)num_sms;
+    return tc_supported(p) && p.T >= 1 && p.T <= kTcSkinnyMaxTokens;
+}
+
+template <int BT, int STAGES, bool HALF>
+cudaError_t launch_fused_kern(const FusedMaps &m, const TcArgs &a1, const TcArgs &a2, cudaStream_t st) {
+    const size_t smem = smem_bytes<STAGES>((HALF ? 128 : 256) * BK * 2, BT * BK * 2) + (HALF ? BT * 256 + 16 : 0);
+    auto kern = tc_fused_kernel<BT, STAGES, HALF>;
+    cudaError_t e = set_smem(kern, smem);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(kern, dim3(a1.grid), dim3(NTHREADS), smem, st, m, a1, a2);
+}
+
+// Both projections of the skinny tiling in one launch (packed weights), then
+// skinny_reduce_kernel for the second projection's split tiles.  Marks: 0
+// before, 1 after the fused kernel, 2 after the reduction.
+cudaError_t run_fused(const Problem &p, const void *x, const void *w1p, const void *w2p, void *h, void *out,
+                      float *part, unsigned *counters, int *status, int num_sms, cudaStream_t st,
+                      const Marks &marks, int *launches) {
+    *launches = 0;
+    if (!fused_ok(p, num_sms)) return cudaErrorNotSupported;
+    const int BT = skinny_bt(p.T);
+    const bool half = fused_half(p, num_sms);
+    const FusedGeom f = fused_geom(p, half, num_sms);
+    WeightOperand w1, w2;
+    if (!weight_packed(&w1, p, 0, w1p, half) || !weight_packed(&w2, p, 1, w2p, half)) return cudaErrorInvalidValue;
+    FusedMaps m;
+    memset(&m, 0, sizeof(m));
+    m.w1 = w1.wm.map[0];
+    m.w2 = w2.wm.map[0];
+    if (!make_map(&m.x, x, p.d_in, p.T, BT) || !make_map(&m.h, h, p.d_ff, p.T, BT)) return cudaErrorInvalidValue;
+    m.h_done = counters + fused_counter_offset(p);
+    m.exits = m.h_done + 1;
+    m.h_tiles = (unsigned)f.g1.tiles;
+    TcArgs a1{}, a2{};
+    for (TcArgs *a : {&a1, &a2}) {
+        a->rows_x = p.T;
+        a->part = part;
+        a->status = status;
+    }
+    a1.rows_w = f.g1.tiles;
+    a1.K = p.d_in;
+    a1.KB = f.g1.KB;
+    a1.epi = first_epi(p.act);
+    a1.out = static_cast<__nv_bfloat16 *>(h);
+    a1.ldo = a1.out_cols = p.d_ff;
+    a1.total_iters = f.g1.total;
+    a1.slots = f.g1.slots;
+    a1.tile_cnt = counters;
+    a1.split_mode = kSplitInKernel;
+    a1.grid = f.g1.grid;
+    a2.rows_w = f.g2.tiles;
+    a2.K = p.d_ff;
+    a2.KB = f.g2.KB;
+    a2.epi = EPI_OUT;
+    a2.out = static_cast<__nv_bfloat16 *>(out);
+    a2.ldo = a2.out_cols = p.d_out;
+    a2.total_iters = f.g2.total;
+    a2.slots = f.g2.slots;
+    a2.split_mode = kSplitSeparate;
+    a2.grid = f.g2.grid;
+    marks.mark(0, st);
+    cudaError_t e;
+    if (half) {
+        switch (BT) {
+            case 16: e = launch_fused_kern<16, TPMLP_FZH_S16, true>(m, a1, a2, st); break;
+            case 32: e = launch_fused_kern<32, TPMLP_FZH_S32, true>(m, a1, a2, st); break;
+            case 64: e = launch_fused_kern<64, TPMLP_FZH_S64, true>(m, a1, a2, st); break;
+            default: e = launch_fused_kern<128, TPMLP_FZH_S128, true>(m, a1, a2, st); break;
+        }
+    } else {
+        switch (BT) {
+            case 16: e = launch_fused_kern<16, TPMLP_FZ_S16, false>(m, a1, a2, st); break;
+            case 32: e = launch_fused_kern<32, TPMLP_FZ_S32, false>(m, a1, a2, st); break;
+            case 64: e = launch_fused_kern<64, TPMLP_FZ_S64, false>(m, a1, a2, st); break;
+            default: e = launch_fused_kern<128, TPMLP_FZ_S128, false>(m, a1, a2, st); break;
+        }
+    }
+    if (e != cudaSuccess) return e;
+    ++*launches;
+    marks.mark(1, st);
+    if (f.g2.slots > 1) {
+        const dim3 rgrid(f.g2.tiles * (BT / 4));
+        e = half ? launch_pdl(skinny_reduce_kernel<true>, rgrid, dim3(128), 0, st, a2, BT)
+                 : launch_pdl(skinny_reduce_kernel<false>, rgrid, dim3(128), 0, st, a2, BT);
+        if (e == cudaSuccess) ++*launches;
+    }
+    marks.mark(2, st);
+    return e;
+}
+
 // Launch with thread-block clusters and without programmatic overlap.
 template <typename... KArgs, typename... Args>
 cudaError_t launch_cluster(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
@@ -1859,6 +2333,8 @@ cudaError_t launch_xgpu(const Problem &p, int rank0, int nranks, const void *x, 
     return e;
 }
 
+bool fused_supported(const Problem &p, int num_sms) { return fused_ok(p, num_sms); }
+
 size_t xgpu_header_bytes(const Problem &p) {
     return kArControlBytes + align256((size_t)p.tp * blk_tiles(p.d_out) * 8 * 4);
 }
@@ -1870,12 +2346,15 @@ bool tc_supported(const Problem &p) {
 
 bool tc_raw_supported(const Problem &p) { return tc_supported(p) && p.fs % BK == 0; }
 
-// Counters serve the in-kernel fixup, which only runs 256-row tiles: the first
-// projection's tiles (either layout) then the second's.
-size_t tile_counter_slots(const Problem &p) {
+// Counters serve the in-kernel fixup of the skinny kernel, which only runs
+// 256-row tiles: the first projection's tiles (either layout) then the
+// second's; then the fused kernel's two words (stored H tiles, CTAs past the
+// wait).
+size_t fused_counter_offset(const Problem &p) {
     return (size_t)(std::max(skinny_tiles(p, 0, false, false), skinny_tiles(p, 0, true, false)) +
                     blk_tiles(p.d_out));
 }
+size_t tile_counter_slots(const Problem &p) { return fused_counter_offset(p) + 2; }
 
 // Split-tile scratch: the largest over both layouts, both projections and both
 // tile heights, since the split mode may change after the workspace is sized.
@@ -1896,6 +2375,10 @@ size_t tc_workspace_bytes(const Problem &p, int num_sms) {
         const StreamKGeom g = skinny_geom((int)tiles, p.fs / BK, BT, num_sms);
         m = std::max(m, (size_t)g.tiles * g.slots * 256 * BT * 4);
     }
+    for (int half = 0; half < 2; ++half) {   // fused: the second projection on the first one's grid
+        const FusedGeom f = fused_geom(p, half != 0, num_sms);
+        m = std::max(m, (size_t)f.g2.tiles * f.g2.slots * (half ? 128 : 256) * BT * 4);
+    }
     return align256(m);
 }
 
@@ -1907,6 +2390,10 @@ cudaError_t launch_tc(const Problem &p, int tiling, const void *x, const void *w
     WeightOperand w1, w2;
     const bool raw = rawA != nullptr;
     if (partials && !raw) return cudaErrorInvalidValue;   // per-rank partials come from the shard form
+    if (tiling == kTilingFused) {   // packed weights only
+        if (raw || partials) return cudaErrorNotSupported;
+        return run_fused(p, x, w1p, w2p, h, out, part, counters, status, num_sms, st, marks, launches);
+    }
     if (tiling == kTilingPair || tiling == kTilingPair2) {   // packed weights only
         if (raw || partials) return cudaErrorNotSupported;
         auto pair = tiling == kTilingPair ? run_pair<1> : run_pair<2>;

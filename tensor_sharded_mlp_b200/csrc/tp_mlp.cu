@@ -383,12 +383,14 @@ int tp_mlp_forward_packed(tp_mlp_t h, const void *x, int tokens, const void *pac
     Problem p = problem_of(h, tokens);
     // plan choice (measured on B200 at d_model 8192, d_ff 28672): the CUDA-core
     // GEMV for 1 token; from 2 tokens on the tensor-core skinny tiling streams
-    // the weights as fast and its arithmetic stays hidden; wide beyond 128,
-    // pairs of CTAs from 512 to 4096 tokens, two-tile pairs above.
+    // the weights as fast and its arithmetic stays hidden -- both projections
+    // in one persistent launch, which measured 1-4 % faster than two kernels
+    // at 2-128 tokens (decode and the d 4096 / f 16384 sweep); wide beyond
+    // 128, pairs of CTAs from 512 to 4096 tokens, two-tile pairs above.
     int plan = h->plan;
     const bool tc_ok = tc_supported(p);
     auto tc_tiling = [&](int t) {
-        return t <= kTcSkinnyMaxTokens ? TP_MLP_PLAN_TC_SKINNY
+        return t <= kTcSkinnyMaxTokens ? (fused_supported(p, h->num_sms) ? TP_MLP_PLAN_TC_FUSED : TP_MLP_PLAN_TC_SKINNY)
                : t < kTcPairMinTokens  ? TP_MLP_PLAN_TC_WIDE
                : t <= kTcPairMaxTokens ? TP_MLP_PLAN_TC_PAIR
                                        : TP_MLP_PLAN_TC_PAIR2;
@@ -401,9 +403,11 @@ int tp_mlp_forward_packed(tp_mlp_t h, const void *x, int tokens, const void *pac
         plan = tc_tiling(tokens);
     }
     const bool is_tc = plan == TP_MLP_PLAN_TC_WIDE || plan == TP_MLP_PLAN_TC_SKINNY ||
-                       plan == TP_MLP_PLAN_TC_WIDE256 || plan == TP_MLP_PLAN_TC_PAIR || plan == TP_MLP_PLAN_TC_PAIR2;
+                       plan == TP_MLP_PLAN_TC_WIDE256 || plan == TP_MLP_PLAN_TC_PAIR || plan == TP_MLP_PLAN_TC_PAIR2 ||
+                       plan == TP_MLP_PLAN_TC_FUSED;
     if (tokens > 0) {
         if (plan == TP_MLP_PLAN_GEMV && !gemv_supported(p)) return TP_MLP_ERR_UNSUPPORTED;
+        if (plan == TP_MLP_PLAN_TC_FUSED && !fused_supported(p, h->num_sms)) return TP_MLP_ERR_UNSUPPORTED;
         if (is_tc && !tc_ok) return TP_MLP_ERR_UNSUPPORTED;
         if (plan == TP_MLP_PLAN_TC_SKINNY && tokens > kTcSkinnyMaxTokens) return TP_MLP_ERR_UNSUPPORTED;
     }
@@ -434,7 +438,8 @@ int tp_mlp_forward_packed(tp_mlp_t h, const void *x, int tokens, const void *pac
         const int tiling = plan == TP_MLP_PLAN_TC_SKINNY ? kTilingSkinny
                            : plan == TP_MLP_PLAN_TC_WIDE ? kTilingWide128
                            : plan == TP_MLP_PLAN_TC_PAIR ? kTilingPair
-                           : plan == TP_MLP_PLAN_TC_PAIR2 ? kTilingPair2 : kTilingWide256;
+                           : plan == TP_MLP_PLAN_TC_PAIR2 ? kTilingPair2
+                           : plan == TP_MLP_PLAN_TC_FUSED ? kTilingFused : kTilingWide256;
         ce = launch_tc(p, tiling, x, w1p, w2p, nullptr, nullptr, hbuf, out, part, counters, status_word(h),
                        h->num_sms, st, h->marks, h->splitk, &launches);
     } else {
@@ -475,7 +480,7 @@ int tp_mlp_selftest_bounded_wait(tp_mlp_t h, unsigned wait_us, tp_mlp_stream_t s
 
 int tp_mlp_set_plan(tp_mlp_t h, int plan) {
     if (!h) return TP_MLP_ERR_INVALID_ARG;
-    if (plan < TP_MLP_PLAN_AUTO || plan > TP_MLP_PLAN_TC_PAIR2) return TP_MLP_ERR_INVALID_ARG;
+    if (plan < TP_MLP_PLAN_AUTO || plan > TP_MLP_PLAN_TC_FUSED) return TP_MLP_ERR_INVALID_ARG;
     h->plan = plan;
     return TP_MLP_OK;
 }

@@ -123,7 +123,7 @@ def summarize_list(path: str, title: str, cmd: str) -> str:
     return "\n".join(out) + "\n"
 
 
-STEP_KERNELS = ("gemv_kernel", "tc_skinny_kernel", "skinny_reduce_kernel", "tc_wide_kernel", "tc_pair_kernel",
+STEP_KERNELS = ("gemv_kernel", "tc_fused_kernel", "tc_skinny_kernel", "skinny_reduce_kernel", "tc_wide_kernel", "tc_pair_kernel",
                 "simt_", "allreduce_norm_kernel", "attn_merge_kernel", "unnamed>::tc_", "unnamed>::skinny",
                 "unnamed>::gemv")
 

@@ -131,7 +131,8 @@ def test_call_argument_errors_before_any_launch(b):
     assert L.tp_mlp_forward_packed(h, ok_ptr, 5, ok_ptr, ok_ptr, None) == 2
     assert L.tp_mlp_forward_packed(h, bad_ptr, 1, ok_ptr, ok_ptr, None) == 3
     assert L.tp_mlp_pack(None, A, A, ok_ptr, None) == 1
-    assert L.tp_mlp_set_plan(h, 9) == 1
+    assert L.tp_mlp_set_plan(h, 10) == 1
+    assert L.tp_mlp_set_plan(h, 9) == 0          # the fused skinny plan
     assert L.tp_mlp_set_plan(h, 3) == 0
     assert L.tp_mlp_forward_packed(h, ok_ptr, 1, ok_ptr, ok_ptr, None) == 4     # tcgen05 needs bf16
     assert L.tp_mlp_set_plan(h, 2) == 0

@@ -224,7 +224,7 @@ def test_auto_plan_choice():
     m.forward_packed(dev(p.x[:1], "bf16"), packed)
     assert m.last_plan == "gemv"
     m.forward_packed(dev(p.x[:3], "bf16"), packed)
-    assert m.last_plan == "tc_skinny"
+    assert m.last_plan == "tc_fused"
 
 
 # --- the named workloads at full size ---------------------------------------------------
@@ -241,6 +241,10 @@ def test_decode_configs_full_size(name):
     packed = m.pack(Ad, Bd)
     del A, Bs
     assert_close(m.forward_packed(x, packed), ref, "bf16", f"{name} packed/{m.last_plan}")
+    if c["tokens"] > 1:   # the two-kernel skinny tiling (auto takes the fused one)
+        m.set_plan("tc_skinny")
+        assert_close(m.forward_packed(x, packed), ref, "bf16", f"{name} packed/tc_skinny")
+        m.set_plan("auto")
     out = m.forward(x, Ad, Bd)
     assert_close(out, ref, "bf16", f"{name} shard form")
     # the per-rank partials (tensor cores, each rank's K loop apart) and their sum
@@ -265,8 +269,14 @@ def test_sweep_config(T):
             ref = oracle.tp_mlp_sharded(p.x[rows], A, Bs, "tanh")
         m = _mlp(p, tp, "bf16", max_tokens=T)
         x = dev(p.x, "bf16")
-        out = m.forward_packed(x, m.pack(Ad, Bd))
+        packed = m.pack(Ad, Bd)
+        out = m.forward_packed(x, packed)
         assert_close(out[torch.from_numpy(rows).cuda()], ref, "bf16", f"sweep T={T} tp={tp}")
+        if 1 < T <= 128:   # the two-kernel skinny tiling (auto takes the fused one)
+            m.set_plan("tc_skinny")
+            out = m.forward_packed(x, packed)
+            assert_close(out[torch.from_numpy(rows).cuda()], ref, "bf16", f"sweep T={T} tp={tp} skinny")
+            m.set_plan("auto")
         out = m.forward(x, Ad, Bd)          # the shard form (its own tiling and grid)
         assert_close(out[torch.from_numpy(rows).cuda()], ref, "bf16", f"sweep T={T} tp={tp} shard form")
         del Ad, Bd, m

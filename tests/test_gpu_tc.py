@@ -168,11 +168,15 @@ def test_auto_plan_uses_tensor_cores():
     packed = m.pack([dev(a, "bf16") for a in A], [dev(b, "bf16") for b in Bs])
     x = dev(p.x, "bf16")
     m.forward_packed(x[:32], packed)
-    assert m.last_plan == "tc_skinny"
+    assert m.last_plan == "tc_fused"
     m.forward_packed(x, packed)
     assert m.last_plan == "tc_wide"
     m.forward_packed(x[:2], packed)
-    assert m.last_plan == "tc_skinny"
+    assert m.last_plan == "tc_fused"
+    m.set_plan("tc")                   # tensor cores, tiling by token count
+    m.forward_packed(x[:2], packed)
+    assert m.last_plan == "tc_fused"
+    m.set_plan("auto")
     m.forward_packed(x[:1], packed)
     assert m.last_plan == "gemv"
 
@@ -230,6 +234,82 @@ def test_tc_pair_agrees_with_wide256():
         outs.append(out)
     assert_close(outs[0], outs[2].float().cpu().numpy(), "bf16", "pair vs wide256")
     assert_close(outs[1], outs[2].float().cpu().numpy(), "bf16", "pair2 vs wide256")
+
+
+FUSED_SHAPES = SHAPES + [
+    (512, 16384, 512, 8),   # 128 first-projection tiles of 128 rows: one whole tile per CTA
+]
+
+
+@pytest.mark.parametrize("act", ["swiglu", "tanh", "identity"])
+@pytest.mark.parametrize("T", [1, 5, 17, 33, 100, 128])
+@pytest.mark.parametrize("shape", FUSED_SHAPES)
+def test_tc_fused_parity(act, T, shape):
+    """Both skinny projections in one persistent launch: the second projection's
+    H loads wait on a device count of stored first-projection tiles (whole
+    tiles, or split tiles finished inside the kernel by their last CTA).  The
+    last CTA resets the count, so repeated calls agree bit for bit."""
+    d, f, dout, tp = shape
+    p = inputs.generate(T, d, f, act, "bf16", seed=3 * T + f, init="fan_in", d_out=dout)
+    A, Bs = p.shards(tp)
+    ref = oracle.tp_mlp_sharded(p.x, A, Bs, act)
+    m, out, _, _, packed = _run(p, tp, "tc_fused")
+    assert m.last_plan == "tc_fused"
+    assert_close(out, ref, "bf16", f"fused T={T}")
+    x = dev(p.x, "bf16")
+    for _ in range(3):
+        assert torch.equal(m.forward_packed(x, packed), out)
+    torch.cuda.synchronize()
+    B().tp_mlp_get_device_status(m.h)
+
+
+@pytest.mark.parametrize("T", [3, 33, 128])
+def test_tc_fused_integer_exact(T):
+    p = inputs.integer_inputs(T, 64, 256, 264, "identity", seed=T + 9, lo=-1, hi=1)
+    m, out, A, Bs, _ = _run(p, 4, "tc_fused")
+    ref = oracle.tp_mlp_sharded(p.x, A, Bs, "identity")
+    assert np.array_equal(out.float().cpu().numpy(), inputs.round_to_bf16(ref.astype(np.float32)))
+
+
+def test_tc_fused_token_counts_and_graph_replay():
+    """Calls of different token counts in turn on one handle, then the same
+    calls captured in a CUDA graph and replayed with new inputs: the counters
+    the kernel waits on live on the device and come back to zero after every
+    launch."""
+    d, f, dout, tp = 1024, 4096, 1024, 4
+    Ts = (64, 7, 33)
+    m = B().TpMlp(d, f, tp, "swiglu", "bf16", max(Ts), d_out=dout)
+    m.set_plan("tc_fused")
+    p = inputs.generate(max(Ts), d, f, "swiglu", "bf16", seed=21, init="fan_in", d_out=dout)
+    A, Bs = p.shards(tp)
+    packed = m.pack([dev(a, "bf16") for a in A], [dev(b, "bf16") for b in Bs])
+    x = dev(p.x, "bf16")
+    for T in Ts + Ts[:1]:
+        out = m.forward_packed(x[:T], packed)
+        assert m.last_plan == "tc_fused"
+        assert_close(out, oracle.tp_mlp_sharded(p.x[:T], A, Bs, "swiglu"), "bf16", f"fused T={T}")
+    outs = [torch.empty(T, dout, dtype=torch.bfloat16, device="cuda") for T in Ts]
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for o, T in zip(outs, Ts):
+            m.forward_packed(x[:T], packed, out=o)
+    s.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        for o, T in zip(outs, Ts):
+            m.forward_packed(x[:T], packed, out=o)
+    for step in range(2):
+        q = inputs.generate(max(Ts), d, f, "swiglu", "bf16", seed=40 + step, init="fan_in", d_out=dout)
+        x.copy_(dev(q.x, "bf16"))
+        torch.cuda.synchronize()
+        with torch.cuda.stream(s):
+            g.replay()
+        s.synchronize()
+        for o, T in zip(outs, Ts):
+            assert_close(o, oracle.tp_mlp_sharded(q.x[:T], A, Bs, "swiglu"), "bf16", f"graph step {step} T={T}")
+    B().tp_mlp_get_device_status(m.h)
+    del g
 
 
 def test_auto_plan_tiling_by_token_count():
