@@ -1299,8 +1299,10 @@ __device__ __forceinline__ void fixup_tile(const TcArgs &a, int tile, int n) {
 
 // One unit of the fused kernel's epilogue (this CTA's k-blocks kb0..kb1 of
 // weight tile `tile`), on the 128 epilogue threads.  h_done != nullptr: a
-// first-projection unit, whose tile is counted once its H is final.  Returns
-// false if a wait gave up.
+// first-projection unit, whose tile is counted once its H is final.
+// stage_out: where a whole 128-row tile is staged for 16-byte stores, or
+// nullptr (2-byte stores straight from the accumulator).  Returns false if a
+// wait gave up.
 template <int BT, bool HALF>
 __device__ __forceinline__ bool fused_unit(const TcArgs &a, const Smem &s, __nv_bfloat16 *stage_out,
                                            uint32_t tmem_base, int tile, int kb0, int kb1, int &acc,
@@ -1320,9 +1322,15 @@ __device__ __forceinline__ bool fused_unit(const TcArgs &a, const Smem &s, __nv_
             tmem_ld16(taddr + t0, v0);
             if (!HALF) tmem_ld16(taddr + BT + t0, v1);
             tmem_ld_wait();
-            if (HALF) {
+            if (HALF && stage_out) {
 #pragma unroll
                 for (int i = 0; i < 16; ++i) stage_out[(t0 + i) * 128 + r] = __float2bfloat16_rn(act_out(a.epi, v0[i]));
+            } else if (HALF) {
+                const int n = tile_col(a, tile, r, 128);
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    if (n >= 0 && t0 + i < a.rows_x)
+                        a.out[(long)(t0 + i) * a.ldo + n] = __float2bfloat16_rn(act_out(a.epi, v0[i]));
             } else {
                 skinny_final16(a, tile, r, t0, v0, v1);
             }
@@ -1330,9 +1338,11 @@ __device__ __forceinline__ bool fused_unit(const TcArgs &a, const Smem &s, __nv_
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&s.tempty[acc]));
-        if (HALF) {
+        if (HALF && stage_out) {
             named_bar(1, 128);   // the whole tile is staged
             skinny_store_staged(a, tile, BT, stage_out);
+            // the staging area is a ring stage's X box, which TMA fills next
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         }
     } else {
         // this CTA's share of the tile -> its slot, [token/4][row][token%4]
@@ -1401,8 +1411,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     constexpr uint32_t X_BYTES = BT * BK * 2;
     extern __shared__ uint8_t smem_raw[];
     const Smem s = carve<STAGES>(smem_raw, W_BYTES, X_BYTES);
-    __nv_bfloat16 *stage_out = reinterpret_cast<__nv_bfloat16 *>(
-        (reinterpret_cast<uintptr_t>(s.tmem_slot) + 16 + 15) & ~uintptr_t(15));
+    // A whole 128-row tile is staged for its stores in the ring's X boxes
+    // (BT x 128 bf16 = two of them): only for the CTA's last first-projection
+    // unit, after which no X box is read or filled until that unit's H is
+    // published.  Other whole 128-row tiles are stored straight from TMEM.
+    static_assert(STAGES >= 2, "staging needs two X boxes");
+    __nv_bfloat16 *const stage_x = reinterpret_cast<__nv_bfloat16 *>(s.b);
     const uint32_t tmem_base = setup<STAGES>(s, &m.w1, &m.x);
     pdl_allow_dependents();
 
@@ -1546,8 +1560,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 const int kb0 = (int)(it - (long long)tile * a.KB);
                 const int kb1 = (int)min((long long)a.KB, ie - (long long)tile * a.KB);
                 it = (long long)tile * a.KB + kb1;
-                ok = fused_unit<BT, HALF>(a, s, stage_out, tmem_base, tile, kb0, kb1, acc, acc_phase, c,
-                                          ph ? nullptr : m.h_done);
+                ok = fused_unit<BT, HALF>(a, s, ph == 0 && it == ie ? stage_x : nullptr, tmem_base, tile, kb0, kb1,
+                                          acc, acc_phase, c, ph ? nullptr : m.h_done);
             }
         }
     }
@@ -1993,7 +2007,11 @@ int first_epi(int act) {
     return act == TP_MLP_ACT_SWIGLU ? EPI_H_SWIGLU : act == TP_MLP_ACT_TANH ? EPI_H_TANH : EPI_H_IDENT;
 }
 
-// Ring depth of the fused kernel (defaults: the skinny kernel's).
+// Ring depth of the fused kernel: the skinny kernel's, except at 128 tokens,
+// where the fused kernel's epilogue staging leaves room for a seventh stage
+// (sweep d 4096 / f 16384, 128 tokens: 54.5 against 54.9 us with six).  More
+// stages at 16-64 tokens measured no faster (8 -> 10-11 at 16 and 32, 8 -> 9
+// at 64), and deeper 256-row rings slower (decode, 2-32 tokens: +9-12 us).
 #ifndef TPMLP_FZH_S16
 #define TPMLP_FZH_S16 TPMLP_SKH_S16
 #endif
@@ -2004,7 +2022,7 @@ int first_epi(int act) {
 #define TPMLP_FZH_S64 TPMLP_SKH_S64
 #endif
 #ifndef TPMLP_FZH_S128
-#define TPMLP_FZH_S128 TPMLP_SKH_S128
+#define TPMLP_FZH_S128 7
 #endif
 #ifndef TPMLP_FZ_S16
 #define TPMLP_FZ_S16 TPMLP_SK_S16
@@ -2046,7 +2064,7 @@ bool fused_ok(const Problem &p, int num_sms) {
 
 template <int BT, int STAGES, bool HALF>
 cudaError_t launch_fused_kern(const FusedMaps &m, const TcArgs &a1, const TcArgs &a2, cudaStream_t st) {
-    const size_t smem = smem_bytes<STAGES>((HALF ? 128 : 256) * BK * 2, BT * BK * 2) + (HALF ? BT * 256 + 16 : 0);
+    const size_t smem = smem_bytes<STAGES>((HALF ? 128 : 256) * BK * 2, BT * BK * 2);
     auto kern = tc_fused_kernel<BT, STAGES, HALF>;
     cudaError_t e = set_smem(kern, smem);
     if (e != cudaSuccess) return e;
