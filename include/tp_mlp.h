@@ -90,14 +90,16 @@ typedef enum {
                                    accumulators per CTA                               */
     TP_MLP_PLAN_TC_PAIR2 = 8,   /* packed bf16: pairs of CTAs, 256 tokens x 512 weight
                                    rows per pair (two weight tiles share each X stage) */
-    TP_MLP_PLAN_TC_FUSED = 9    /* packed bf16, 1..128 tokens: the skinny tiling with
-                                   both projections in one persistent launch (the
+    TP_MLP_PLAN_TC_FUSED = 9    /* bf16, 1..128 tokens: the skinny tiling with both
+                                   projections in one persistent launch (the
                                    second projection's weights stream in while the
                                    first finishes; its H loads wait on a device
                                    counter).  Needs every CTA of the grid (one per
                                    SM) resident at once: a GPU shared with other work
                                    can make the bounded wait run out, reported as
-                                   TP_MLP_ERR_TIMEOUT by tp_mlp_get_device_status. */
+                                   TP_MLP_ERR_TIMEOUT by tp_mlp_get_device_status.
+                                   Auto takes it for packed weights; the shard form
+                                   (tp_mlp_forward) runs it when chosen.       */
 } tp_mlp_plan;
 
 /*

@@ -78,10 +78,11 @@ constexpr int kTcWide256MinTokens = 2048;   // auto, shard form: 256-token tiles
 constexpr int kTcPairMinTokens = 512;
 constexpr int kTcPairMaxTokens = 4096;
 // kTilingFused: the skinny tiling with both projections in one persistent
-// launch (packed weights, 1..kTcSkinnyMaxTokens tokens; fused_supported).
+// launch (packed weights or the shard form, 1..kTcSkinnyMaxTokens tokens;
+// fused_supported).
 enum { kTilingSkinny = 0, kTilingWide128 = 1, kTilingWide256 = 2, kTilingPair = 3, kTilingPair2 = 4, kTilingFused = 5 };
 bool tc_supported(const Problem &p);
-bool fused_supported(const Problem &p, int num_sms);
+bool fused_supported(const Problem &p, bool raw);   // raw: the shard form
 bool tc_raw_supported(const Problem &p);   // also needs f_s % 64 == 0
 size_t tc_workspace_bytes(const Problem &p, int num_sms);
 // Split tiles of the skinny tiling (values of tp_mlp_splitk): finished by the

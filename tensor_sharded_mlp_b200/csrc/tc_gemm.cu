@@ -1239,7 +1239,7 @@ __global__ void __launch_bounds__(128) skinny_reduce_kernel(TcArgs a, int BT) {
 // counter to be reached; the wait is bounded, so a grid that cannot be fails
 // with a status instead of hanging.  The last CTA past the wait resets it.
 struct FusedMaps {
-    CUtensorMap w1, w2;   // packed parts: boxes of 256 (or 128) rows x 64 k
+    WeightMaps w1, w2;    // packed parts (map[0]) or the per-rank shards (RAW), as for the skinny kernel
     CUtensorMap x, h;     // X (T x d_in) and H (T x d_ff): boxes of BT rows x 64 k
     unsigned *h_done;     // first-projection tiles whose H is stored, this launch
     unsigned *exits;      // CTAs past their wait on h_done, this launch
@@ -1393,17 +1393,9 @@ __device__ __forceinline__ bool fused_unit(const TcArgs &a, const Smem &s, __nv_
     return true;
 }
 
-template <bool HALF>
-__device__ __forceinline__ void load_w_packed(uint32_t dst, const CUtensorMap *m, int tile, int kb, int KB,
-                                              uint32_t bar) {
-    if (HALF)
-        tma_load_2d(dst, m, 0, ((tile >> 1) * KB + kb) * 256 + (tile & 1) * 128, bar);
-    else
-        tma_load_2d(dst, m, 0, (tile * KB + kb) * 256, bar);
-}
-
 // HALF: 128-row tiles in both projections (tanh / identity); otherwise 256.
-template <int BT, int STAGES, bool HALF>
+// RAW: the shard form, per-rank tensors read MN-major (always 256-row tiles).
+template <int BT, int STAGES, bool HALF, bool RAW>
 __global__ void __launch_bounds__(NTHREADS, 1)
     tc_fused_kernel(const __grid_constant__ FusedMaps m, const __grid_constant__ TcArgs a1,
                     const __grid_constant__ TcArgs a2) {
@@ -1417,7 +1409,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     // published.  Other whole 128-row tiles are stored straight from TMEM.
     static_assert(STAGES >= 2, "staging needs two X boxes");
     __nv_bfloat16 *const stage_x = reinterpret_cast<__nv_bfloat16 *>(s.b);
-    const uint32_t tmem_base = setup<STAGES>(s, &m.w1, &m.x);
+    const uint32_t tmem_base = setup<STAGES>(s, &m.w1.map[0], &m.x);
     pdl_allow_dependents();
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -1431,7 +1423,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
     if (warp == 0) {
         if (lane == 0) {
-            tma_prefetch_desc(&m.w2);
+            tma_prefetch_desc(&m.w2.map[0]);
             tma_prefetch_desc(&m.h);
             // first projection: the weights of the first stages before the
             // wait on the previous kernel, then X
@@ -1441,7 +1433,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 const int tile = (int)(it / a1.KB), kb = (int)(it - (long long)tile * a1.KB);
                 const uint32_t fb = smem_u32(&s.full[i]);
                 mbar_arrive_expect_tx(fb, W_BYTES + X_BYTES);
-                load_w_packed<HALF>(smem_u32(s.a + i * W_BYTES), &m.w1, tile, kb, a1.KB, fb);
+                load_w_tile<RAW, HALF>(smem_u32(s.a + i * W_BYTES), m.w1, tile, kb, a1.KB, fb);
             }
             pdl_wait_previous();
             for (int i = 0; i < npre; ++i) {
@@ -1456,7 +1448,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 if (!mbar_wait(smem_u32(&s.empty[stage]), phase ^ 1, s.abort)) goto done;
                 const uint32_t fb = smem_u32(&s.full[stage]);
                 mbar_arrive_expect_tx(fb, W_BYTES + X_BYTES);
-                load_w_packed<HALF>(smem_u32(s.a + stage * W_BYTES), &m.w1, tile, kb, a1.KB, fb);
+                load_w_tile<RAW, HALF>(smem_u32(s.a + stage * W_BYTES), m.w1, tile, kb, a1.KB, fb);
                 tma_load_2d(smem_u32(s.b + stage * X_BYTES), &m.x, kb * BK, 0, fb);
                 if (++stage == STAGES) { stage = 0; phase ^= 1; }
             }
@@ -1470,7 +1462,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 if (!mbar_wait(smem_u32(&s.empty[stage]), phase ^ 1, s.abort)) goto done;
                 const uint32_t fb = smem_u32(&s.full[stage]);
                 mbar_arrive_expect_tx(fb, W_BYTES + X_BYTES);
-                load_w_packed<HALF>(smem_u32(s.a + stage * W_BYTES), &m.w2, tile, kb, a2.KB, fb);
+                load_w_tile<RAW, HALF>(smem_u32(s.a + stage * W_BYTES), m.w2, tile, kb, a2.KB, fb);
                 if (++stage == STAGES) { stage = 0; phase ^= 1; }
             }
             {
@@ -1505,14 +1497,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 if (!mbar_wait(smem_u32(&s.empty[stage]), phase ^ 1, s.abort)) goto done;
                 const uint32_t fb = smem_u32(&s.full[stage]);
                 mbar_arrive_expect_tx(fb, W_BYTES + X_BYTES);
-                load_w_packed<HALF>(smem_u32(s.a + stage * W_BYTES), &m.w2, tile, kb, a2.KB, fb);
+                load_w_tile<RAW, HALF>(smem_u32(s.a + stage * W_BYTES), m.w2, tile, kb, a2.KB, fb);
                 tma_load_2d(smem_u32(s.b + stage * X_BYTES), &m.h, kb * BK, 0, fb);
                 if (++stage == STAGES) { stage = 0; phase ^= 1; }
             }
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            const uint32_t idesc = idesc_bf16_f32(128, BT);
+            const uint32_t idesc = idesc_bf16_f32(128, BT) | (RAW ? kIdescAMajorMN : 0u);
             int stage = 0, acc = 0;
             uint32_t phase = 0, acc_phase = 0;
             for (int ph = 0; ph < 2; ++ph) {
@@ -1529,13 +1521,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         if (!mbar_wait(smem_u32(&s.full[stage]), phase, s.abort)) goto done;
                         tc_fence_after();
                         const uint32_t wa = smem_u32(s.a + stage * W_BYTES);
-                        const uint64_t dw0 = smem_desc_kmajor_sw128(wa), dw1 = smem_desc_kmajor_sw128(wa + 128 * 128);
+                        // rows 128..255 of the tile: K-major 16 KB in; MN-major atoms 2-3, 16 KB in
+                        const uint64_t dw0 = RAW ? smem_desc_mnmajor_sw128(wa) : smem_desc_kmajor_sw128(wa);
+                        const uint64_t dw1 =
+                            RAW ? smem_desc_mnmajor_sw128(wa + 16384) : smem_desc_kmajor_sw128(wa + 128 * 128);
+                        constexpr uint32_t kstep_w = RAW ? 128 : 2;
                         const uint64_t dx = smem_desc_kmajor_sw128(smem_u32(s.b + stage * X_BYTES));
 #pragma unroll
                         for (int k = 0; k < BK / 16; ++k) {
                             const uint32_t accum = (kb != kb0 || k != 0) ? 1u : 0u;
-                            mma_bf16(d0, dw0 + 2 * k, dx + 2 * k, idesc, accum);
-                            if (!HALF) mma_bf16(d1, dw1 + 2 * k, dx + 2 * k, idesc, accum);
+                            mma_bf16(d0, dw0 + kstep_w * k, dx + 2 * k, idesc, accum);
+                            if (!HALF) mma_bf16(d1, dw1 + kstep_w * k, dx + 2 * k, idesc, accum);
                         }
                         mma_commit(smem_u32(&s.empty[stage]));
                         if (++stage == STAGES) { stage = 0; phase ^= 1; }
@@ -2042,11 +2038,11 @@ int first_epi(int act) {
 struct FusedGeom {
     StreamKGeom g1, g2;
 };
-FusedGeom fused_geom(const Problem &p, bool half, int num_sms) {
+FusedGeom fused_geom(const Problem &p, bool half, bool raw, int num_sms) {
     const int BT = skinny_bt(p.T);
     FusedGeom f;
-    f.g1 = skinny_geom((int)skinny_tiles(p, 0, false, half), (int)blk_kblocks(p.d_in), BT, num_sms);
-    f.g2 = streamk_geom(skinny_tiles(p, 1, false, half), blk_kblocks(p.d_ff), f.g1.grid);
+    f.g1 = skinny_geom((int)skinny_tiles(p, 0, raw, half), (int)blk_kblocks(p.d_in), BT, num_sms);
+    f.g2 = streamk_geom(skinny_tiles(p, 1, raw, half), blk_kblocks(p.d_ff), f.g1.grid);
     return f;
 }
 // 128-row tiles for tanh / identity when no first-projection tile is split
@@ -2054,40 +2050,49 @@ FusedGeom fused_geom(const Problem &p, bool half, int num_sms) {
 // SwiGLU (gate and up share a tile).
 bool fused_half(const Problem &p, int num_sms) {
     return p.act != TP_MLP_ACT_SWIGLU && skinny_bt(p.T) >= TPMLP_SKINNY_HALF_MIN_BT &&
-           fused_geom(p, true, num_sms).g1.slots == 1;
+           fused_geom(p, true, false, num_sms).g1.slots == 1;
 }
 
-bool fused_ok(const Problem &p, int num_sms) {
-    (void)num_sms;
-    return tc_supported(p) && p.T >= 1 && p.T <= kTcSkinnyMaxTokens;
+// raw: the shard form (256-row tiles, f_s % 64 == 0, as for the skinny kernel).
+bool fused_ok(const Problem &p, bool raw) {
+    return (raw ? tc_raw_supported(p) : tc_supported(p)) && p.T >= 1 && p.T <= kTcSkinnyMaxTokens;
 }
 
-template <int BT, int STAGES, bool HALF>
+template <int BT, int STAGES, bool HALF, bool RAW = false>
 cudaError_t launch_fused_kern(const FusedMaps &m, const TcArgs &a1, const TcArgs &a2, cudaStream_t st) {
     const size_t smem = smem_bytes<STAGES>((HALF ? 128 : 256) * BK * 2, BT * BK * 2);
-    auto kern = tc_fused_kernel<BT, STAGES, HALF>;
+    auto kern = tc_fused_kernel<BT, STAGES, HALF, RAW>;
     cudaError_t e = set_smem(kern, smem);
     if (e != cudaSuccess) return e;
     return launch_pdl(kern, dim3(a1.grid), dim3(NTHREADS), smem, st, m, a1, a2);
 }
 
-// Both projections of the skinny tiling in one launch (packed weights), then
-// skinny_reduce_kernel for the second projection's split tiles.  Marks: 0
-// before, 1 after the fused kernel, 2 after the reduction.
-cudaError_t run_fused(const Problem &p, const void *x, const void *w1p, const void *w2p, void *h, void *out,
-                      float *part, unsigned *counters, int *status, int num_sms, cudaStream_t st,
-                      const Marks &marks, int *launches) {
+// Both projections of the skinny tiling in one launch (packed weights, or the
+// per-rank shards when rawA / rawB are given), then skinny_reduce_kernel for
+// the second projection's split tiles.  Marks: 0 before, 1 after the fused
+// kernel, 2 after the reduction.
+cudaError_t run_fused(const Problem &p, const void *x, const void *w1p, const void *w2p, const ShardPtrs *rawA,
+                      const ShardPtrs *rawB, void *h, void *out, float *part, unsigned *counters, int *status,
+                      int num_sms, cudaStream_t st, const Marks &marks, int *launches) {
     *launches = 0;
-    if (!fused_ok(p, num_sms)) return cudaErrorNotSupported;
+    const bool raw = rawA != nullptr;
+    if (!fused_ok(p, raw)) return cudaErrorNotSupported;
     const int BT = skinny_bt(p.T);
-    const bool half = fused_half(p, num_sms);
-    const FusedGeom f = fused_geom(p, half, num_sms);
+    const bool half = !raw && fused_half(p, num_sms);
+    const FusedGeom f = fused_geom(p, half, raw, num_sms);
     WeightOperand w1, w2;
-    if (!weight_packed(&w1, p, 0, w1p, half) || !weight_packed(&w2, p, 1, w2p, half)) return cudaErrorInvalidValue;
+    if (raw) {
+        if (!weight_raw_first(&w1, p, *rawA, false) || !weight_raw_second(&w2, p, *rawB, false, false))
+            return cudaErrorInvalidValue;
+    } else if (!weight_packed(&w1, p, 0, w1p, half) || !weight_packed(&w2, p, 1, w2p, half)) {
+        return cudaErrorInvalidValue;
+    }
+    if (w1.tiles != f.g1.tiles || w1.KB != f.g1.KB || w2.tiles != f.g2.tiles || w2.KB != f.g2.KB)
+        return cudaErrorInvalidValue;   // the operands' tiling must be the geometry's
     FusedMaps m;
     memset(&m, 0, sizeof(m));
-    m.w1 = w1.wm.map[0];
-    m.w2 = w2.wm.map[0];
+    m.w1 = w1.wm;
+    m.w2 = w2.wm;
     if (!make_map(&m.x, x, p.d_in, p.T, BT) || !make_map(&m.h, h, p.d_ff, p.T, BT)) return cudaErrorInvalidValue;
     m.h_done = counters + fused_counter_offset(p);
     m.exits = m.h_done + 1;
@@ -2101,6 +2106,9 @@ cudaError_t run_fused(const Problem &p, const void *x, const void *w1p, const vo
     a1.rows_w = f.g1.tiles;
     a1.K = p.d_in;
     a1.KB = f.g1.KB;
+    a1.raw_first = w1.raw_first;   // the shard form's tiles map to features per rank
+    a1.tps = w1.tps;
+    a1.fs = w1.fs;
     a1.epi = first_epi(p.act);
     a1.out = static_cast<__nv_bfloat16 *>(h);
     a1.ldo = a1.out_cols = p.d_ff;
@@ -2121,7 +2129,14 @@ cudaError_t run_fused(const Problem &p, const void *x, const void *w1p, const vo
     a2.grid = f.g2.grid;
     marks.mark(0, st);
     cudaError_t e;
-    if (half) {
+    if (raw) {
+        switch (BT) {
+            case 16: e = launch_fused_kern<16, TPMLP_FZ_S16, false, true>(m, a1, a2, st); break;
+            case 32: e = launch_fused_kern<32, TPMLP_FZ_S32, false, true>(m, a1, a2, st); break;
+            case 64: e = launch_fused_kern<64, TPMLP_FZ_S64, false, true>(m, a1, a2, st); break;
+            default: e = launch_fused_kern<128, TPMLP_FZ_S128, false, true>(m, a1, a2, st); break;
+        }
+    } else if (half) {
         switch (BT) {
             case 16: e = launch_fused_kern<16, TPMLP_FZH_S16, true>(m, a1, a2, st); break;
             case 32: e = launch_fused_kern<32, TPMLP_FZH_S32, true>(m, a1, a2, st); break;
@@ -2351,7 +2366,7 @@ cudaError_t launch_xgpu(const Problem &p, int rank0, int nranks, const void *x, 
     return e;
 }
 
-bool fused_supported(const Problem &p, int num_sms) { return fused_ok(p, num_sms); }
+bool fused_supported(const Problem &p, bool raw) { return fused_ok(p, raw); }
 
 size_t xgpu_header_bytes(const Problem &p) {
     return kArControlBytes + align256((size_t)p.tp * blk_tiles(p.d_out) * 8 * 4);
@@ -2393,8 +2408,10 @@ size_t tc_workspace_bytes(const Problem &p, int num_sms) {
         const StreamKGeom g = skinny_geom((int)tiles, p.fs / BK, BT, num_sms);
         m = std::max(m, (size_t)g.tiles * g.slots * 256 * BT * 4);
     }
-    for (int half = 0; half < 2; ++half) {   // fused: the second projection on the first one's grid
-        const FusedGeom f = fused_geom(p, half != 0, num_sms);
+    for (int v = 0; v < 3; ++v) {   // fused: the second projection on the first one's grid
+        const bool half = v == 1, raw = v == 2;
+        if (raw && p.fs % BK) continue;
+        const FusedGeom f = fused_geom(p, half, raw, num_sms);
         m = std::max(m, (size_t)f.g2.tiles * f.g2.slots * (half ? 128 : 256) * BT * 4);
     }
     return align256(m);
@@ -2408,9 +2425,9 @@ cudaError_t launch_tc(const Problem &p, int tiling, const void *x, const void *w
     WeightOperand w1, w2;
     const bool raw = rawA != nullptr;
     if (partials && !raw) return cudaErrorInvalidValue;   // per-rank partials come from the shard form
-    if (tiling == kTilingFused) {   // packed weights only
-        if (raw || partials) return cudaErrorNotSupported;
-        return run_fused(p, x, w1p, w2p, h, out, part, counters, status, num_sms, st, marks, launches);
+    if (tiling == kTilingFused) {   // the forward only (no per-rank partials)
+        if (partials) return cudaErrorNotSupported;
+        return run_fused(p, x, w1p, w2p, rawA, rawB, h, out, part, counters, status, num_sms, st, marks, launches);
     }
     if (tiling == kTilingPair || tiling == kTilingPair2) {   // packed weights only
         if (raw || partials) return cudaErrorNotSupported;

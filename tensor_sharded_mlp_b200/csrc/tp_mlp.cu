@@ -295,12 +295,23 @@ static int run_shard_form(tp_mlp_t h, const void *x, int tokens, const void *con
     const bool tc_ok = tc_raw_supported(p);
     int plan = h->plan;
     if (plan == TP_MLP_PLAN_AUTO) plan = tc_ok ? TP_MLP_PLAN_TC : TP_MLP_PLAN_SIMT;
+    // Up to 128 tokens: the two-kernel skinny tiling.  The fused kernel also
+    // takes the shard form (TP_MLP_PLAN_TC_FUSED) but measured slower on it:
+    // its 256-row first-projection tiles are split, and inside the fused
+    // kernel their slots must be added at the end of the first projection,
+    // where the reduction kernel spreads that work over the GPU (sweep d 4096 /
+    // f 16384, tp 8, 16 / 64 / 128 tokens: 53.5 / 66.8 / 81.8 against 52.6 /
+    // 57.6 / 67.2 us; decode bs32 231 against 225).
     if (plan == TP_MLP_PLAN_TC)
         plan = tokens <= kTcSkinnyMaxTokens ? TP_MLP_PLAN_TC_SKINNY
-                                            : tokens < kTcWide256MinTokens ? TP_MLP_PLAN_TC_WIDE : TP_MLP_PLAN_TC_WIDE256;
-    const bool is_tc = plan == TP_MLP_PLAN_TC_WIDE || plan == TP_MLP_PLAN_TC_SKINNY || plan == TP_MLP_PLAN_TC_WIDE256;
+               : tokens < kTcWide256MinTokens ? TP_MLP_PLAN_TC_WIDE
+                                              : TP_MLP_PLAN_TC_WIDE256;
+    const bool is_tc = plan == TP_MLP_PLAN_TC_WIDE || plan == TP_MLP_PLAN_TC_SKINNY || plan == TP_MLP_PLAN_TC_WIDE256 ||
+                       (plan == TP_MLP_PLAN_TC_FUSED && !partials);
     if (plan != TP_MLP_PLAN_SIMT && !is_tc) return TP_MLP_ERR_UNSUPPORTED;   // (the pair tiling needs packed weights)
-    if (is_tc && tokens > 0 && (!tc_ok || (plan == TP_MLP_PLAN_TC_SKINNY && tokens > kTcSkinnyMaxTokens)))
+    if (is_tc && tokens > 0 &&
+        (!tc_ok || (plan == TP_MLP_PLAN_TC_SKINNY && tokens > kTcSkinnyMaxTokens) ||
+         (plan == TP_MLP_PLAN_TC_FUSED && !fused_supported(p, true))))
         return TP_MLP_ERR_UNSUPPORTED;
     if (tokens == 0) {
         h->last_plan = plan;
@@ -323,8 +334,10 @@ static int run_shard_form(tp_mlp_t h, const void *x, int tokens, const void *con
     cudaError_t ce;
     int launches = 2;
     if (is_tc) {
-        const int tiling = plan == TP_MLP_PLAN_TC_SKINNY ? kTilingSkinny
-                           : plan == TP_MLP_PLAN_TC_WIDE ? kTilingWide128 : kTilingWide256;
+        const int tiling = plan == TP_MLP_PLAN_TC_SKINNY  ? kTilingSkinny
+                           : plan == TP_MLP_PLAN_TC_FUSED ? kTilingFused
+                           : plan == TP_MLP_PLAN_TC_WIDE  ? kTilingWide128
+                                                          : kTilingWide256;
         float *part = reinterpret_cast<float *>(ws + counters_bytes(h) + h_bytes(h, tokens));
         ce = launch_tc(p, tiling, x, nullptr, nullptr, &a, &b, hbuf, out, part, reinterpret_cast<unsigned *>(ws),
                        status_word(h), h->num_sms, st, h->marks, h->splitk, &launches, partials);
@@ -390,7 +403,7 @@ int tp_mlp_forward_packed(tp_mlp_t h, const void *x, int tokens, const void *pac
     int plan = h->plan;
     const bool tc_ok = tc_supported(p);
     auto tc_tiling = [&](int t) {
-        return t <= kTcSkinnyMaxTokens ? (fused_supported(p, h->num_sms) ? TP_MLP_PLAN_TC_FUSED : TP_MLP_PLAN_TC_SKINNY)
+        return t <= kTcSkinnyMaxTokens ? (fused_supported(p, false) ? TP_MLP_PLAN_TC_FUSED : TP_MLP_PLAN_TC_SKINNY)
                : t < kTcPairMinTokens  ? TP_MLP_PLAN_TC_WIDE
                : t <= kTcPairMaxTokens ? TP_MLP_PLAN_TC_PAIR
                                        : TP_MLP_PLAN_TC_PAIR2;
@@ -407,7 +420,7 @@ int tp_mlp_forward_packed(tp_mlp_t h, const void *x, int tokens, const void *pac
                        plan == TP_MLP_PLAN_TC_FUSED;
     if (tokens > 0) {
         if (plan == TP_MLP_PLAN_GEMV && !gemv_supported(p)) return TP_MLP_ERR_UNSUPPORTED;
-        if (plan == TP_MLP_PLAN_TC_FUSED && !fused_supported(p, h->num_sms)) return TP_MLP_ERR_UNSUPPORTED;
+        if (plan == TP_MLP_PLAN_TC_FUSED && !fused_supported(p, false)) return TP_MLP_ERR_UNSUPPORTED;
         if (is_tc && !tc_ok) return TP_MLP_ERR_UNSUPPORTED;
         if (plan == TP_MLP_PLAN_TC_SKINNY && tokens > kTcSkinnyMaxTokens) return TP_MLP_ERR_UNSUPPORTED;
     }

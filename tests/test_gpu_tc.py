@@ -363,6 +363,32 @@ def test_tc_shard_form_parity(act, plan, T, shape):
     assert_close(out[torch.from_numpy(rows).cuda()], ref, "bf16", f"shard form {plan} T={T}")
 
 
+@pytest.mark.parametrize("act", ["swiglu", "tanh", "identity"])
+@pytest.mark.parametrize("T", [1, 5, 33, 100, 128])
+@pytest.mark.parametrize("shape", RAW_SHAPES)
+def test_tc_fused_shard_form_parity(act, T, shape):
+    """The fused kernel on the per-rank shards (MN-major weight boxes, 256-row
+    tiles, first-projection split tiles finished in the kernel), chosen
+    explicitly; repeated calls agree bit for bit."""
+    d, f, dout, tp = shape
+    p = inputs.generate(T, d, f, act, "bf16", seed=7 * T + f + dout, init="fan_in", d_out=dout)
+    A, Bs = p.shards(tp)
+    ref = oracle.tp_mlp_sharded(p.x, A, Bs, act)
+    m = B().TpMlp(d, f, tp, act, "bf16", T, d_out=dout)
+    Ad, Bd = [dev(a, "bf16") for a in A], [dev(b, "bf16") for b in Bs]
+    x = dev(p.x, "bf16")
+    m.set_plan("tc_fused")
+    out = m.forward(x, Ad, Bd)
+    assert m.last_plan == "tc_fused"
+    assert_close(out, ref, "bf16", f"fused shard form T={T}")
+    for _ in range(2):
+        assert torch.equal(m.forward(x, Ad, Bd), out)
+    m.set_plan("tc_skinny")                     # the two-kernel tiling agrees with the oracle too
+    assert_close(m.forward(x, Ad, Bd), ref, "bf16", f"skinny shard form T={T}")
+    torch.cuda.synchronize()
+    B().tp_mlp_get_device_status(m.h)
+
+
 @pytest.mark.parametrize("T", [9, 64, 128])
 def test_tc_shard_form_split_finish_modes_agree(T):
     d, f, dout, tp = RAW_SHAPES[0]
