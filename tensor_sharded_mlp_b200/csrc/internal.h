@@ -69,12 +69,14 @@ cudaError_t launch_gemv(const Problem &p, const void *x, const void *w1p, const 
 // tc_gemm.cu: tcgen05 path, packed bf16.  skinny: tokens <= kTcSkinnyMaxTokens.
 constexpr int kTcSkinnyMaxTokens = 128;
 constexpr int kTcWide256MinTokens = 2048;   // auto, shard form: 256-token tiles from here on
-// auto, packed weights: pairs of CTAs (cta_group::2, 256 x 256 per pair) from
-// kTcPairMinTokens to kTcPairMaxTokens tokens, pairs with two weight tiles per
-// X stage (256 x 512) above (measured on B200, sweep d 4096 / f 16384: T=1024
-// 198-205 us pair vs 228 us 128-token tiles and 264 us two-tile pairs; prefill
-// d 8192 / f 28672, T=8192, power-capped at ~1.2 GHz: two-tile pairs
-// 8.56-8.58 ms, 1-CTA 256-token tiles 8.69-8.74, one-tile pairs 8.88-8.93).
+// auto, packed weights: pairs of CTAs (cta_group::2) from kTcPairMinTokens to
+// kTcPairMaxTokens tokens, one or two 256-row weight tiles per unit chosen per
+// projection by wave efficiency (tc_gemm.cu, pair_tiles_per_unit), and two
+// tiles per unit (256 x 512) above (measured on B200, sweep d 4096 / f 16384:
+// T=1024 198-205 us pair vs 228 us 128-token tiles and 264 us two-tile pairs
+// on both projections; prefill d 8192 / f 28672, T=8192, power-capped at ~1.2
+// GHz: two-tile pairs 8.56-8.58 ms, 1-CTA 256-token tiles 8.69-8.74, one-tile
+// pairs 8.88-8.93).
 constexpr int kTcPairMinTokens = 512;
 constexpr int kTcPairMaxTokens = 4096;
 // kTilingFused: the skinny tiling with both projections in one persistent

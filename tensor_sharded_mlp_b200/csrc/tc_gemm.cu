@@ -1999,6 +1999,26 @@ cudaError_t run_pair(const Problem &p, int proj, const void *wbase, const void *
     return launch_pdl_cluster(kern, dim3(2 * pairs), dim3(NTHREADS), smem, st, 2u, mx, w.wm, a);
 }
 
+// Weight tiles per pair unit for one projection of the pair tiling: two
+// (tc_pair_kernel<NB = 2>: each X stage feeds two 256-row tiles, a third less
+// operand traffic per FLOP) unless the units then fill the pairs' waves worse:
+// wave efficiency units / (waves x pairs) at least that of one tile per unit,
+// less 2 %.  Sweep d 4096 / f 16384, tp 8: 2100 / 4096 tokens 400 / 857 us
+// against 409 / 873 with one tile per unit (4096: 0.4 s windows); equal at
+// 512-1024 tokens, where the rule keeps one tile for the second projection
+// (two-tile units would leave 42 of 74 pairs idle: 171 against 117 us).
+#ifndef TPMLP_PAIR_AUTO_NB
+#define TPMLP_PAIR_AUTO_NB 1
+#endif
+int pair_tiles_per_unit(const Problem &p, int proj, int num_sms) {
+    if (!TPMLP_PAIR_AUTO_NB) return 1;
+    const long long MT = (p.T + 255) / 256;
+    const long long tiles = blk_tiles(proj == 0 ? w1p_rows(p.d_ff, p.act) : p.d_out);
+    const long long pairs = std::max(1, num_sms / 2);
+    auto eff = [&](long long units) { return (double)units / (double)(((units + pairs - 1) / pairs) * pairs); };
+    return eff(MT * ((tiles + 1) / 2)) >= eff(MT * tiles) - 0.02 ? 2 : 1;
+}
+
 int first_epi(int act) {
     return act == TP_MLP_ACT_SWIGLU ? EPI_H_SWIGLU : act == TP_MLP_ACT_TANH ? EPI_H_TANH : EPI_H_IDENT;
 }
@@ -2431,12 +2451,14 @@ cudaError_t launch_tc(const Problem &p, int tiling, const void *x, const void *w
     }
     if (tiling == kTilingPair || tiling == kTilingPair2) {   // packed weights only
         if (raw || partials) return cudaErrorNotSupported;
-        auto pair = tiling == kTilingPair ? run_pair<1> : run_pair<2>;
+        auto nb = [&](int proj) { return tiling == kTilingPair2 ? 2 : pair_tiles_per_unit(p, proj, num_sms); };
         marks.mark(0, st);
-        cudaError_t e = pair(p, 0, w1p, x, p.T, p.d_in, first_epi(p.act), h, p.d_ff, status, num_sms, st);
+        cudaError_t e = (nb(0) == 2 ? run_pair<2> : run_pair<1>)(p, 0, w1p, x, p.T, p.d_in, first_epi(p.act), h,
+                                                                   p.d_ff, status, num_sms, st);
         if (e != cudaSuccess) return e;
         marks.mark(1, st);
-        e = pair(p, 1, w2p, h, p.T, p.d_ff, EPI_OUT, out, p.d_out, status, num_sms, st);
+        e = (nb(1) == 2 ? run_pair<2> : run_pair<1>)(p, 1, w2p, h, p.T, p.d_ff, EPI_OUT, out, p.d_out, status,
+                                                     num_sms, st);
         marks.mark(2, st);
         *launches = 2;
         return e;
