@@ -176,6 +176,7 @@ __global__ void __launch_bounds__(NTHR, 1) gemv_kernel(GemvArgs a) {
         if (XS) {
             if (threadIdx.x == 0) stage_x<T>(a, s, kbs, (int)min((long long)KB, it_e - it_b));
             xok = mbar_wait(smem_u32(s.xbar), 0, s.abort);
+            xok = !named_bar_or(1, CWARPS * 32, !xok);   // all compute threads alike
         }
         const int g = lane & 7;                         // granule (8 k) of the row
         const int rbase = warp * 32 + (lane >> 3);      // rows rbase + 4j, j = 0..7
@@ -233,7 +234,8 @@ __global__ void __launch_bounds__(NTHR, 1) gemv_kernel(GemvArgs a) {
                 if (lane == 0) mbar_arrive(smem_u32(&s.empty[stage]));
                 if (++stage == STAGES) { stage = 0; phase ^= 1; }
             }
-            if (!ok) break;
+            // leave together if a wait gave up in any warp (the barriers below need all)
+            if (named_bar_or(1, CWARPS * 32, !ok)) break;
             // the 8 lanes of a row hold partial sums of its 8 granules
 #pragma unroll
             for (int j = 0; j < 8; ++j)

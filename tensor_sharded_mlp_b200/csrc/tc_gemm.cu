@@ -995,7 +995,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const int kb0 = (int)(it - (long long)tile * KB);
             const int kb1 = (int)min((long long)KB, it_e - (long long)tile * KB);
             it = (long long)tile * KB + kb1;
-            if (!mbar_wait(smem_u32(&s.tfull[acc]), acc_phase, s.abort)) break;
+            // all 128 epilogue threads leave alike if the wait gave up in any
+            if (named_bar_or(1, 128, !mbar_wait(smem_u32(&s.tfull[acc]), acc_phase, s.abort))) break;
             tc_fence_after();
             const uint32_t taddr = tmem_base + acc * (2 * BT) + ((uint32_t)(q * 32) << 16);
             // (the cluster route stages even a whole tile: the all-reduce needs it there)
@@ -1311,7 +1312,8 @@ __device__ __forceinline__ bool fused_unit(const TcArgs &a, const Smem &s, __nv_
     const int q = warp & 3;
     const int r = q * 32 + lane;   // row within each 128-row half
     constexpr int ROWS = HALF ? 128 : 256;
-    if (!mbar_wait(smem_u32(&s.tfull[acc]), acc_phase, s.abort)) return false;
+    // all 128 threads leave alike if the wait gave up in any (the barriers below need all)
+    if (named_bar_or(1, 128, !mbar_wait(smem_u32(&s.tfull[acc]), acc_phase, s.abort))) return false;
     tc_fence_after();
     const uint32_t taddr = tmem_base + acc * (2 * BT) + ((uint32_t)(q * 32) << 16);
     bool final_here = true;   // this CTA wrote the tile's final values

@@ -226,6 +226,18 @@ __device__ __forceinline__ void mbar_arrive_remote(uint32_t bar) {
 __device__ __forceinline__ void named_bar(int id, int count) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
+// The same, returning whether `pred` held in any of the threads: a decision
+// every thread of the group takes alike (e.g. to leave a loop after a bounded
+// wait gave up in some of them, so that no thread is left at a later barrier).
+__device__ __forceinline__ bool named_bar_or(int id, int count, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.or.pred q, %2, %3, p;\n selp.u32 %0, 1, 0, q;\n}\n"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "r"(id), "r"(count)
+        : "memory");
+    return r != 0;
+}
 
 }  // namespace tc
 }  // namespace tpmlp
