@@ -1235,7 +1235,10 @@ __global__ void __launch_bounds__(128) skinny_reduce_kernel(TcArgs a, int BT) {
 // (in slot order, as skinny_reduce_kernel does).  Split tiles of the second
 // projection go to skinny_reduce_kernel, launched behind: finished inside the
 // kernel, by the last CTA of each tile, they left those few CTAs a long
-// latency-bound tail (sweep, 128 tokens: 64.9 against 54.3 us).  Every
+// latency-bound tail (sweep, 128 tokens: 64.9 against 54.3 us); added by the
+// whole grid after a grid-wide count, they kept every SM busy to the end,
+// where the reduction kernel lets the next launch's CTAs start streaming
+// (60.7 against 54.9 us).  Every
 // CTA of the grid (one per SM at most) must be resident at once for the
 // counter to be reached; the wait is bounded, so a grid that cannot be fails
 // with a status instead of hanging.  The last CTA past the wait resets it.
