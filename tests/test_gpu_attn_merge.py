@@ -4,8 +4,10 @@
 parallelism.  Partials come from the oracle's rank-local step over random
 q, K, V (so the merge must also reproduce attention over the whole history)
 and from the seeded generator; edge cases cover empty ranks, rows with every
-rank empty, maxima near +-1000, head sizes that are not a multiple of the
-warp's 128-element stride and the largest head size the kernel takes.
+rank empty, maxima near +-1000, head sizes that share a warp between rows
+(with a ragged last warp), that leave some of a row's lanes idle or give
+them one group more than the others, that rule out 16-byte bf16 loads
+(head_dim % 8 != 0), and the largest head size the kernel takes.
 """
 import numpy as np
 import pytest
@@ -55,7 +57,8 @@ def test_merge_reproduces_attention_over_the_whole_history(cuts):
     assert_close(got, oracle.attention_full(q, k, v, sc), "f32", "merge vs full attention")
 
 
-SHAPES = [(1, 1, 4), (2, 3, 64), (3, 5, 68), (8, 2048, 128), (5, 33, 132), (8, 100, 4096), (7, 9, 256)]
+SHAPES = [(1, 1, 4), (2, 3, 64), (3, 5, 68), (8, 2048, 128), (5, 33, 132), (8, 100, 4096), (7, 9, 256),
+          (4, 37, 8), (6, 50, 24), (2, 300, 40), (8, 65, 12)]
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
