@@ -960,7 +960,8 @@ def main():
         e2e = {"value": replicas.whole_job_rate(T, K, world, e2e_ms), "unit": "tokens/s",
                "h2d_bytes_per_step": step.x_host.numel() * step.x_host.element_size(),
                "d2h_bytes_per_step": step.out_host.numel() * step.out_host.element_size(),
-               "api": "binding.GraphStep (CUDA graph: H2D x, tp_mlp_forward_packed, D2H out, synchronize)",
+               "api": "binding.GraphStep (CUDA graph: tp_mlp_copy_async H2D x, tp_mlp_forward_packed, "
+                      "tp_mlp_copy_async D2H out; synchronize)",
                "timer": "CUDA events on the step's stream around K steps, host waits included",
                "matches_device_result": e2e_ok}
         del step

@@ -479,6 +479,33 @@ int tp_mlp_ipc_get_handle(const void *dev_ptr, void *handle, size_t *offset);
 int tp_mlp_ipc_open_handle(const void *handle, size_t offset, void **dev_ptr);
 int tp_mlp_ipc_close_handle(void *dev_ptr, size_t offset);
 
+/*
+ * Copy `bytes` bytes from src to dst on `stream`, for a step's host<->device
+ * transfers (no counterpart in the pages, which count a decode step's fixed
+ * costs per launch, "7.4 推理侧并行" §7.4.2: a decode step's input and output
+ * are a few kilobytes, so the transfer's setup, not its bytes, is what costs).
+ * Up to 1 MiB the copy is a library kernel that reads or writes the host side
+ * directly over the bus, so it needs no copy-engine setup, can be captured in
+ * a CUDA graph with the forward, and hands over to the next library kernel by
+ * programmatic dependent launch; larger copies go to the copy engine
+ * (cudaMemcpyAsync).
+ *
+ *   dst, src  each either device memory of the current device or page-locked
+ *             host memory mapped into its address space (cudaHostAlloc /
+ *             cudaMallocHost, or cudaHostRegister with mapping, under unified
+ *             addressing); 16-byte aligned; each inside one allocation of at
+ *             least `bytes` from the pointer on.  The two ranges must not
+ *             overlap.
+ *   bytes     any count; 0 is a no-op.
+ * Errors (nothing is launched): TP_MLP_ERR_INVALID_ARG for a null pointer,
+ * memory CUDA does not know (pageable host memory), host memory not mapped
+ * for this device, device memory of another context, or overlapping ranges;
+ * TP_MLP_ERR_ALIGNMENT; TP_MLP_ERR_SHAPE if `bytes` runs past the allocation.
+ * Asynchronous on `stream`: a host destination holds the data once the
+ * stream's work up to this call has completed.
+ */
+int tp_mlp_copy_async(void *dst, const void *src, size_t bytes, tp_mlp_stream_t stream);
+
 /* Human-readable name of a status code (static string; no counterpart in the pages). */
 const char *tp_mlp_status_string(int status);
 

@@ -66,6 +66,7 @@ _SIGS = {
     "tp_mlp_ipc_get_handle": (_i, [_vp, _vp, ctypes.POINTER(_sz)]),
     "tp_mlp_ipc_open_handle": (_i, [_vp, _sz, ctypes.POINTER(_vp)]),
     "tp_mlp_ipc_close_handle": (_i, [_vp, _sz]),
+    "tp_mlp_copy_async": (_i, [_vp, _vp, _sz, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -365,6 +366,20 @@ def tp_mlp_merge_attention_partials(maximum: torch.Tensor, exp_sum: torch.Tensor
     return out
 
 
+def tp_mlp_copy_async(dst: torch.Tensor, src: torch.Tensor, stream=None) -> torch.Tensor:
+    """Copy src's bytes into dst on the stream.  Each may be a CUDA tensor of the
+    current device or a pinned host tensor; both contiguous, the same size in
+    bytes, not overlapping.  Decode-sized copies run as a library kernel."""
+    n = src.numel() * src.element_size()
+    if not src.is_contiguous() or not dst.is_contiguous() or dst.numel() * dst.element_size() != n:
+        raise ValueError("src and dst must be contiguous tensors of the same size in bytes")
+    for t in (src, dst):
+        if not t.is_cuda and not t.is_pinned():
+            raise ValueError("host tensors must be pinned (page-locked)")
+    _check("tp_mlp_copy_async", _lib.tp_mlp_copy_async(_ptr(dst), _ptr(src), n, _stream(stream)))
+    return dst
+
+
 # --- convenience wrapper -----------------------------------------------------------
 
 class TpMlp:
@@ -383,7 +398,7 @@ class TpMlp:
 
     def __del__(self):
         h = getattr(self, "h", None)
-        if h is not None:
+        if h is not None and _lib is not None:   # module globals are gone at interpreter exit
             _lib.tp_mlp_destroy(h)
             self.h = None
 
@@ -465,10 +480,11 @@ class GraphStep:
     """A whole decode/prefill step replayed as one CUDA graph.
 
     Per call: copy the step's input from a pinned host buffer to the device,
-    run tp_mlp_forward_packed, copy the result back to a pinned host buffer,
-    and wait for it.  Capturing these into a graph once removes the per-kernel
-    launch cost from every later step (the pages put it at 5-10 us per kernel
-    in a decode step, "7.4 推理侧并行" §7.4.2).  The library's calls allocate
+    run tp_mlp_forward_packed, copy the result back to a pinned host buffer
+    (both copies by tp_mlp_copy_async: a kernel at decode sizes), and wait for
+    it.  Capturing these into a graph once removes the per-kernel launch cost
+    from every later step (the pages put it at 5-10 us per kernel in a decode
+    step, "7.4 推理侧并行" §7.4.2).  The library's calls allocate
     nothing and take no host-side decisions that change between replays, so
     they are safe to capture; the handle's workspace and the packed weights
     must outlive the step.
@@ -496,9 +512,9 @@ class GraphStep:
         self.launches = mlp.last_launches
 
     def _body(self):
-        self.x_dev.copy_(self.x_host, non_blocking=True)
+        tp_mlp_copy_async(self.x_dev, self.x_host)
         self.mlp.forward_packed(self.x_dev, self.packed, out=self.out_dev)
-        self.out_host.copy_(self.out_dev, non_blocking=True)
+        tp_mlp_copy_async(self.out_host, self.out_dev)
 
     def __call__(self, x: Optional[torch.Tensor] = None) -> torch.Tensor:
         if x is not None:

@@ -53,6 +53,12 @@ constexpr int kMergeMaxHeadDim = 4096;
 cudaError_t launch_attn_merge(int P, int rows, int D, const float *maximum, const float *exp_sum,
                               const void *weighted, int dtype, void *out, cudaStream_t st);
 
+// copy.cu: `bytes` from src to dst by a kernel (either side may be page-locked
+// host memory mapped into the device's address space); copies above
+// kCopyKernelMaxBytes go to the copy engine instead.
+constexpr size_t kCopyKernelMaxBytes = 1u << 20;
+cudaError_t launch_copy(void *dst, const void *src, size_t bytes, int num_sms, cudaStream_t st);
+
 // Split-tile counters the GEMV and tcgen05 skinny kernels need (one per
 // weight tile of both parts; first part's tiles first).
 size_t tile_counter_slots(const Problem &p);

@@ -98,6 +98,51 @@ int check_dev(const void *p, size_t bytes) {
     return TP_MLP_OK;
 }
 
+typedef CUresult (*PFN_pointerGetAttribute)(void *, CUpointer_attribute, CUdeviceptr);
+
+static PFN_pointerGetAttribute pointer_attribute_fn() {
+    static PFN_pointerGetAttribute fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuPointerGetAttribute", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_pointerGetAttribute>(p);
+    });
+    return fn;
+}
+
+// A pointer a kernel of the current device may read or write `bytes` from:
+// device memory of the current context (check_dev), or page-locked host
+// memory mapped into the device's address space.  *dev is the address the
+// kernel uses.
+int check_reachable(const void *p, size_t bytes, const void **dev) {
+    if (!p) return TP_MLP_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(p) & 15u) return TP_MLP_ERR_ALIGNMENT;
+    PFN_pointerGetAttribute fn = pointer_attribute_fn();
+    if (!fn) return TP_MLP_ERR_CUDA;
+    const CUdeviceptr ptr = reinterpret_cast<CUdeviceptr>(p);
+    unsigned type = 0;
+    if (fn(&type, CU_POINTER_ATTRIBUTE_MEMORY_TYPE, ptr) != CUDA_SUCCESS)
+        return TP_MLP_ERR_INVALID_ARG;   // memory CUDA does not know (pageable host memory)
+    if (type != CU_MEMORYTYPE_HOST) {
+        *dev = p;
+        return check_dev(p, bytes);
+    }
+    CUdeviceptr alias = 0, start = 0;
+    size_t size = 0;
+    if (fn(&alias, CU_POINTER_ATTRIBUTE_DEVICE_POINTER, ptr) != CUDA_SUCCESS ||
+        fn(&start, CU_POINTER_ATTRIBUTE_RANGE_START_ADDR, ptr) != CUDA_SUCCESS ||
+        fn(&size, CU_POINTER_ATTRIBUTE_RANGE_SIZE, ptr) != CUDA_SUCCESS)
+        return TP_MLP_ERR_INVALID_ARG;   // not mapped for this device
+    if (ptr < start || ptr + bytes > start + size) return TP_MLP_ERR_SHAPE;
+    if (alias & 15u) return TP_MLP_ERR_ALIGNMENT;
+    *dev = reinterpret_cast<const void *>(alias);
+    return TP_MLP_OK;
+}
+
 }  // namespace tpmlp
 
 namespace {
@@ -538,6 +583,25 @@ int tp_mlp_merge_attention_partials(int tp_degree, int rows, int head_dim, const
     if ((s = check_dev(out, (size_t)rows * head_dim * e))) return s;
     return from_cuda(launch_attn_merge(tp_degree, rows, head_dim, maximum, exp_sum, weighted, dtype, out,
                                        reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int tp_mlp_copy_async(void *dst, const void *src, size_t bytes, tp_mlp_stream_t stream) {
+    if (bytes == 0) return TP_MLP_OK;
+    if (!dst || !src) return TP_MLP_ERR_INVALID_ARG;
+    const uintptr_t a = reinterpret_cast<uintptr_t>(src), b = reinterpret_cast<uintptr_t>(dst);
+    if ((a | b) & 15u) return TP_MLP_ERR_ALIGNMENT;
+    const void *s_dev = nullptr, *d_dev = nullptr;
+    int s;
+    if ((s = check_reachable(src, bytes, &s_dev))) return s;
+    if ((s = check_reachable(dst, bytes, &d_dev))) return s;
+    if (a < b + bytes && b < a + bytes) return TP_MLP_ERR_INVALID_ARG;   // overlapping ranges
+    const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (bytes > kCopyKernelMaxBytes) return from_cuda(cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDefault, st));
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
+        return TP_MLP_ERR_CUDA;
+    return from_cuda(launch_copy(const_cast<void *>(d_dev), s_dev, bytes, sms, st));
 }
 
 // Exchange buffer: [control + flags | receive rows | gathered rows (sequence parallelism)].

@@ -160,6 +160,11 @@ def test_call_argument_errors_before_any_launch(b):
     assert M(2, 4, 128, None, None, None, 3, None, None) == 1                  # dtype
     assert M(2, 4, 128, None, None, None, 1, None, None) == 1                  # null pointers
     assert M(2, 0, 128, None, None, None, 1, None, None) == 0                  # no rows: no-op
+    # host<->device copy: these checks come before any driver query
+    C = L.tp_mlp_copy_async
+    assert C(ok_ptr, bad_ptr, 0, None) == 0                                    # no bytes: no-op
+    assert C(ok_ptr, None, 64, None) == 1 and C(None, ok_ptr, 64, None) == 1   # null pointers
+    assert C(ok_ptr, bad_ptr, 64, None) == 3 and C(bad_ptr, ok_ptr, 64, None) == 3
     for mode in (3, 2, 1, 0):
         assert L.tp_mlp_set_splitk(h, mode) == 0
     assert L.tp_mlp_last_plan(h) == 1 and L.tp_mlp_last_launches(h) == 0        # the 0-token no-op
