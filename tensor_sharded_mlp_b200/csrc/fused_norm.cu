@@ -38,6 +38,12 @@ __device__ __forceinline__ uint32_t cluster_ctarank() {
 __device__ __forceinline__ void cluster_sync() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
+// a cluster barrier that publishes nothing: the arrive does not wait for this
+// thread's earlier stores to complete (its earlier loads have completed, since
+// their values were used before it)
+__device__ __forceinline__ void cluster_sync_relaxed() {
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;\n\tbarrier.cluster.wait.aligned;" ::: "memory");
+}
 // float at the same shared-memory address in CTA `rank` of this cluster
 __device__ __forceinline__ float ld_dsmem(const float *local, uint32_t rank) {
     uint32_t remote;
@@ -106,7 +112,7 @@ __global__ void __launch_bounds__(kNormThreads)
                                               h.w * scale * g.w));
         store4(res_out + row + 4LL * q, h);
     }
-    cluster_sync();   // no CTA leaves while another may still read its cta_sq
+    cluster_sync_relaxed();   // no CTA leaves while another may still read its cta_sq
 }
 
 template <typename T, int P>
