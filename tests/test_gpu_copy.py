@@ -66,10 +66,11 @@ def test_copies_in_a_graph_replay_with_new_host_data():
         assert torch.equal(back, src)
 
 
-@pytest.mark.parametrize("act,tokens", [("swiglu", 1), ("swiglu", 3), ("tanh", 16)])
-def test_graph_step_matches_the_forward(act, tokens):
-    d, f, tp = 256, 1024, 4
-    m = B().TpMlp(d, f, tp, act, "bf16", max_tokens=16)
+@pytest.mark.parametrize("act,tokens,d", [("swiglu", 1, 256), ("swiglu", 3, 256), ("tanh", 16, 256),
+                                          ("tanh", 160, 4096)])   # x and out of 1.25 MiB: copy-engine copies
+def test_graph_step_matches_the_forward(act, tokens, d):
+    f, tp = 1024, 4
+    m = B().TpMlp(d, f, tp, act, "bf16", max_tokens=max(16, tokens))
     fs = f // tp
     wa = 2 * fs if act == "swiglu" else fs
     g = torch.Generator().manual_seed(tokens)
