@@ -7,7 +7,8 @@ and from the seeded generator; edge cases cover empty ranks, rows with every
 rank empty, maxima near +-1000, head sizes that share a warp between rows
 (with a ragged last warp), that leave some of a row's lanes idle or give
 them one group more than the others, that rule out 16-byte bf16 loads
-(head_dim % 8 != 0), and the largest head size the kernel takes.
+(head_dim % 8 != 0), the largest head size the kernel takes, and row counts
+of several waves of CTAs with a ragged last one.
 """
 import numpy as np
 import pytest
@@ -65,6 +66,19 @@ SHAPES = [(1, 1, 4), (2, 3, 64), (3, 5, 68), (8, 2048, 128), (5, 33, 132), (8, 1
 @pytest.mark.parametrize("P,rows,D", SHAPES)
 def test_merge_parity(P, rows, D, dtype):
     a = inputs.generate_attn_merge(P, rows, D, dtype, seed=P * 100 + rows + D)
+    got = _merge(a.maximum, a.exp_sum, a.weighted, dtype)
+    assert_close(got, oracle.merge_attention_partials(a.maximum, a.exp_sum, a.weighted), dtype,
+                 f"merge P={P} rows={rows} D={D}")
+
+
+# many rows: several waves of CTAs, ragged last CTAs
+MANY_ROWS = [(8, 16384 + 5, 128), (2, 40000, 64), (4, 77777, 136), (8, 9999, 256), (1, 300001, 16)]
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("P,rows,D", MANY_ROWS)
+def test_merge_parity_many_rows(P, rows, D, dtype):
+    a = inputs.generate_attn_merge(P, rows, D, dtype, seed=P + rows + D)
     got = _merge(a.maximum, a.exp_sum, a.weighted, dtype)
     assert_close(got, oracle.merge_attention_partials(a.maximum, a.exp_sum, a.weighted), dtype,
                  f"merge P={P} rows={rows} D={D}")
