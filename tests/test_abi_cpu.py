@@ -183,6 +183,18 @@ def test_binding_pairs_shards_strictly(b):
     b.tp_mlp_destroy(h)
 
 
+def test_binding_copy_checks_before_the_library(b):
+    """The copy wrapper refuses mismatched sizes, strided tensors and pageable
+    host tensors before calling the library (no device is present here)."""
+    import torch
+    with pytest.raises(ValueError):
+        b.tp_mlp_copy_async(torch.zeros(16, dtype=torch.uint8), torch.zeros(32, dtype=torch.uint8))
+    with pytest.raises(ValueError):
+        b.tp_mlp_copy_async(torch.zeros(4, 4)[:, :2], torch.zeros(4, 2))
+    with pytest.raises(ValueError):   # pageable (not pinned) host memory
+        b.tp_mlp_copy_async(torch.zeros(64, dtype=torch.uint8), torch.zeros(64, dtype=torch.uint8))
+
+
 def _model_slots(tiles, KB, BT, sms=148):
     """Split pieces per tile under the documented grid rule: floor(sms / tiles)
     CTAs per tile when that keeps 80 % of the SMs busy, else equal contiguous
