@@ -950,10 +950,10 @@ def main():
             step()
         barrier()
         s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        s2.record(step.stream)
+        s2.record(torch.cuda.current_stream())
         for _ in range(K):
             step()                    # replay + wait for the result on the host
-        e2.record(step.stream)
+        e2.record(torch.cuda.current_stream())
         e2.synchronize()
         e2e_ms = replicas.max_over_ranks(s2.elapsed_time(e2))
         ref_out = out.cpu()
@@ -963,7 +963,7 @@ def main():
                "d2h_bytes_per_step": step.out_host.numel() * step.out_host.element_size(),
                "api": "binding.GraphStep (CUDA graph: tp_mlp_copy_async H2D x, tp_mlp_forward_packed, "
                       "tp_mlp_copy_async D2H out; synchronize)",
-               "timer": "CUDA events on the step's stream around K steps, host waits included",
+               "timer": "CUDA events on the replay stream around K steps, host waits included",
                "matches_device_result": e2e_ok}
         del step
 

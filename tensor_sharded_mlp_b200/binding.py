@@ -492,6 +492,8 @@ class GraphStep:
         step = GraphStep(mlp, packed, tokens)
         step.x_host.copy_(x)          # or step(x) to copy and run
         out = step()                  # pinned host tensor, valid until the next call
+
+    A call replays the graph on the caller's current CUDA stream and waits for it.
     """
 
     def __init__(self, mlp: "TpMlp", packed: torch.Tensor, tokens: int):
@@ -519,7 +521,7 @@ class GraphStep:
     def __call__(self, x: Optional[torch.Tensor] = None) -> torch.Tensor:
         if x is not None:
             self.x_host.copy_(x)
-        with torch.cuda.stream(self.stream):   # replay() launches on the current stream
-            self.graph.replay()
-        self.stream.synchronize()
+        stream = torch.cuda.current_stream(self.mlp.device)
+        self.graph.replay()      # on the caller's current stream, after its earlier work
+        stream.synchronize()
         return self.out_host
