@@ -499,8 +499,9 @@ int tp_mlp_ipc_close_handle(void *dev_ptr, size_t offset);
  *   bytes     any count; 0 is a no-op.
  * Errors (nothing is launched): TP_MLP_ERR_INVALID_ARG for a null pointer,
  * memory CUDA does not know (pageable host memory), host memory not mapped
- * for this device, device memory of another context, or overlapping ranges;
- * TP_MLP_ERR_ALIGNMENT; TP_MLP_ERR_SHAPE if `bytes` runs past the allocation.
+ * for this device, device memory of another device or context, or
+ * overlapping ranges; TP_MLP_ERR_ALIGNMENT; TP_MLP_ERR_SHAPE if `bytes` runs
+ * past the allocation.
  * Asynchronous on `stream`: a host destination holds the data once the
  * stream's work up to this call has completed.
  */

@@ -128,6 +128,11 @@ int check_reachable(const void *p, size_t bytes, const void **dev) {
     if (fn(&type, CU_POINTER_ATTRIBUTE_MEMORY_TYPE, ptr) != CUDA_SUCCESS)
         return TP_MLP_ERR_INVALID_ARG;   // memory CUDA does not know (pageable host memory)
     if (type != CU_MEMORYTYPE_HOST) {
+        // device memory: of this device (another GPU's would need peer access)
+        int ordinal = -1, cur = -1;
+        if (fn(&ordinal, CU_POINTER_ATTRIBUTE_DEVICE_ORDINAL, ptr) == CUDA_SUCCESS && ordinal >= 0 &&
+            (cudaGetDevice(&cur) != cudaSuccess || ordinal != cur))
+            return TP_MLP_ERR_INVALID_ARG;
         *dev = p;
         return check_dev(p, bytes);
     }
